@@ -1,0 +1,161 @@
+/*
+ * favor.h -- C ABI of libfavor.so, the FAVOR+ attention hot path for NVIDIA B200 (sm_100a).
+ *
+ * FAVOR+ ("Fast Attention Via Positive Orthogonal Random Features", the attention of the
+ * Performer, "Rethinking Attention with Performers", arXiv 2009.14794) replaces the L x L
+ * softmax attention matrix A(i,j) = K(q_i, k_j) by random features phi with
+ * K(x, y) = E[phi(x)^T phi(y)] ("Fast Attention Via Positive Orthogonal Random Features",
+ * codewithpapers.app/method/favor, the FA-part equations), and evaluates
+ *
+ *     out = D^-1 (Q' ((K')^T V)),   D = diag(Q' ((K')^T 1_L)),   Q' = phi(Q), K' = phi(K),
+ *
+ * in time linear in L. This library uses the positive map phi(x) = exp(W x - |x|^2/2) / sqrt(m)
+ * with block-orthogonal Gaussian W (m x d), a causal (masked, j <= i) variant by prefix sums
+ * ("Random Features for Efficient Attention Approximation", thesis abstract: masked
+ * self-attention), and the backward pass with W held fixed.
+ *
+ * Conventions for every call:
+ *   - Tensors are contiguous row-major [B, H, L, d] (d innermost); W is row-major [m, d].
+ *   - Device pointers are CUDA global-memory pointers owned by the caller; the library never
+ *     frees or retains them. Host pointers are marked "host".
+ *   - Q and K are used as given: any d^-1/4 scaling belongs to the caller.
+ *   - Outputs and gradients are fp32. With bf16 inputs a bf16 output would by itself exceed a
+ *     2e-2 * RMS(out) max-error budget (outputs are averages whose largest entries are ~10x
+ *     their RMS), so the output precision is fixed at fp32.
+ *   - Calls that take a stream are asynchronous on that stream (a cudaStream_t passed as
+ *     void*; NULL is the legacy default stream). Argument errors are reported before any launch.
+ *     Device-side conditions (a bounded wait that ran out) are recorded in a device status word
+ *     read by favor_sync_status().
+ *   - No call allocates device memory: scratch comes from the caller's workspace.
+ *   - Nothing aborts, throws or prints; every call returns a favor_status.
+ */
+#ifndef FAVOR_H
+#define FAVOR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FAVOR_API __attribute__((visibility("default")))
+#else
+#define FAVOR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FAVOR_OK = 0,
+    FAVOR_ERR_INVALID_ARG = 1,  /* null pointer, non-positive or inconsistent size         */
+    FAVOR_ERR_UNSUPPORTED = 2,  /* valid arguments outside what the kernels implement       */
+    FAVOR_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, tensor map)   */
+    FAVOR_ERR_TIMEOUT = 4,      /* a device-side bounded wait gave up (see favor_sync_status) */
+    FAVOR_ERR_WORKSPACE = 5     /* workspace or ctx pointer null or smaller than required   */
+} favor_status;
+
+typedef enum {
+    FAVOR_F32 = 0,   /* fp32 Q, K, V, W, dO: CUDA-core fp32 path                           */
+    FAVOR_BF16 = 1   /* bf16 Q, K, V, W, dO: tcgen05 tensor-core path, fp32 accumulation   */
+} favor_dtype;
+
+/* Problem shape. L >= 1; d in {64, 128}; m a multiple of 16 (fp32 path: 16..512;
+ * bf16 path: 64..256, multiple of 64). */
+typedef struct {
+    int B, H, L, d, m;
+    favor_dtype dtype;
+} favor_shape;
+
+/* Tuning knobs; pass NULL for defaults. Zero fields take their defaults too.
+ *   split_tiles : 128-token tiles per CTA for the key-side reduction (and per causal segment)
+ *   exp_poly_pct: percent (0..100) of feature exponentials evaluated by the FMA-pipe
+ *                 polynomial instead of the MUFU ex2 unit (bf16 path). */
+typedef struct {
+    int split_tiles;
+    int exp_poly_pct;
+    int reserved[6];
+} favor_opts;
+
+/*
+ * favor_draw_features -- draw the block-orthogonal random feature matrix W (host only).
+ *
+ * Positive *orthogonal* random features ("Rethinking Attention with Performers" abstract; the
+ * summary page's limitations: orthogonality holds within blocks of at most d rows). W has
+ * ceil(m/d) independent blocks; block b is a d x d Gaussian matrix from Philox4x64-10 keyed by
+ * (seed, 0), counter (n/4, b, 0, 0), Box-Muller pairs; its rows are orthonormalised by modified
+ * Gram-Schmidt with one re-orthogonalisation pass, then each row i is scaled by an independent
+ * chi(d) norm sqrt(sum of d squared Gaussians from counter (n/4, b, 1, 0)). The last block is
+ * truncated to its first rows. Every step is one IEEE double operation in a fixed order, so the
+ * result is reproducible bit for bit.
+ *
+ *   seed   : any 64-bit value
+ *   m, d   : W is m x d; 1 <= m, 1 <= d <= 1024
+ *   W_host : host, caller-owned, m*d doubles, row-major; written on FAVOR_OK only
+ * Returns FAVOR_ERR_INVALID_ARG on a null pointer or bad size.
+ */
+FAVOR_API favor_status favor_draw_features(uint64_t seed, int m, int d, double *W_host);
+
+/*
+ * favor_workspace_size -- bytes of device workspace favor_fwd (backward = 0) or favor_bwd
+ * (backward = 1) needs for this shape, causal flag and options (NULL = defaults).
+ * Returns 0 for an invalid or unsupported shape.
+ */
+FAVOR_API size_t favor_workspace_size(const favor_shape *shape, int causal, int backward, const favor_opts *opts);
+
+/*
+ * favor_ctx_size -- bytes of the forward-to-backward context (per-head key stabiliser,
+ * per-key norms and the fp32 state (K')^T [V | 1_L]). Returns 0 for an invalid shape.
+ */
+FAVOR_API size_t favor_ctx_size(const favor_shape *shape, int causal);
+
+/*
+ * favor_fwd -- FAVOR+ forward: out = D^-1 (Q' ((K')^T V)) (causal = 0, the bidirectional
+ * FA-part) or out_i = phi(q_i)^T S_i / phi(q_i)^T z_i with prefix sums S_i, z_i over j <= i
+ * (causal = 1).
+ *
+ *   shape        : host pointer
+ *   Q, K, V      : device, [B,H,L,d] in shape->dtype
+ *   W            : device, [m,d] in shape->dtype (the caller rounds the fp64 draw)
+ *   causal       : 0 or 1
+ *   out          : device, fp32 [B,H,L,d]; fully written
+ *   ctx          : device, favor_ctx_size bytes, or NULL when no backward will follow
+ *   workspace    : device, >= favor_workspace_size(shape, causal, 0, opts) bytes, 256-B aligned
+ *   stream       : cudaStream_t as void*
+ * Numerics: features are stabilised by a per-row max for queries and the per-(batch, head)
+ * max over keys; both cancel exactly in D^-1. Inputs Q, K, V, W, out must be 16-byte aligned.
+ */
+FAVOR_API favor_status favor_fwd(const favor_shape *shape, const void *Q, const void *K, const void *V,
+                       const void *W, int causal, float *out, void *ctx, void *workspace,
+                       size_t ws_bytes, const favor_opts *opts, void *stream);
+
+/*
+ * favor_bwd -- gradients of sum(dout * out) with respect to Q, K, V, with W fixed.
+ * (Derived by the chain rule from the forward definition; the pages print no backward.)
+ *
+ *   Q, K, V, W   : as passed to favor_fwd
+ *   out          : device, fp32 [B,H,L,d], the forward output
+ *   dout         : device, [B,H,L,d] in shape->dtype, upstream gradient
+ *   ctx          : device, the context written by favor_fwd with the same inputs
+ *   dQ, dK, dV   : device, fp32 [B,H,L,d]; fully written
+ *   workspace    : device, >= favor_workspace_size(shape, causal, 1, opts) bytes
+ */
+FAVOR_API favor_status favor_bwd(const favor_shape *shape, const void *Q, const void *K, const void *V,
+                       const void *W, const float *out, const void *dout, const void *ctx,
+                       int causal, float *dQ, float *dK, float *dV, void *workspace,
+                       size_t ws_bytes, const favor_opts *opts, void *stream);
+
+/*
+ * favor_sync_status -- synchronise the stream, then return and clear the device status word
+ * (FAVOR_ERR_TIMEOUT if a bounded wait inside a kernel gave up since the last call), or
+ * FAVOR_ERR_CUDA if the stream reports an error.
+ */
+FAVOR_API favor_status favor_sync_status(void *stream);
+
+/* favor_status_string -- static, never-NULL description of a status code. */
+FAVOR_API const char *favor_status_string(favor_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FAVOR_H */

@@ -1,0 +1,249 @@
+// C ABI of libfavor.so (declared in include/favor.h). Single translation unit: the kernel files
+// are included here so the device status word has one definition without relocatable code.
+//
+// Host responsibilities: argument validation before any launch, workspace carving, TMA tensor
+// maps, and the launch sequence per call. Every step of the computation runs in the kernels.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+
+#include "k_fp32.cu"
+#include "k_keys.cu"
+#include "k_query.cu"
+
+namespace favor {
+namespace {
+
+// ------------------------------------------------------------------------------- validation
+
+bool shape_ok(const favor_shape *s) {
+    if (s == nullptr) return false;
+    if (s->B <= 0 || s->H <= 0 || s->L <= 0 || s->d <= 0 || s->m <= 0) return false;
+    if (s->dtype != FAVOR_F32 && s->dtype != FAVOR_BF16) return false;
+    if ((long long)s->B * s->H * s->L > (1ll << 31)) return false;
+    return true;
+}
+
+// What the kernels implement for this shape (FAVOR_OK or FAVOR_ERR_UNSUPPORTED).
+favor_status shape_supported(const favor_shape *s, int causal, int backward) {
+    if (s->d != 64 && s->d != 128) return FAVOR_ERR_UNSUPPORTED;
+    if ((long long)s->B * s->H > 65535) return FAVOR_ERR_UNSUPPORTED;
+    if (s->dtype == FAVOR_F32) {
+        if (s->m % 16 != 0 || s->m > 512) return FAVOR_ERR_UNSUPPORTED;
+        return FAVOR_OK;
+    }
+    if (s->m != 128 && s->m != 256) return FAVOR_ERR_UNSUPPORTED;
+    if (causal || backward) return FAVOR_ERR_UNSUPPORTED;
+    return FAVOR_OK;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+int opt_split_tiles(const favor_opts *o) {
+    const int v = o ? o->split_tiles : 0;
+    return v > 0 ? std::min(v, 64) : 8;
+}
+
+// -------------------------------------------------------------------------------- workspace
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Bf16Layout {
+    int BH, n_tiles, tiles_per_split, n_split;
+    size_t off_bias, off_split_max, off_head_max, off_part_S, off_part_z, off_state, total;
+};
+
+Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_ws) {
+    Bf16Layout l{};
+    l.BH = s->B * s->H;
+    l.n_tiles = (s->L + kTile - 1) / kTile;
+    l.tiles_per_split = opt_split_tiles(o);
+    l.n_split = (l.n_tiles + l.tiles_per_split - 1) / l.tiles_per_split;
+    size_t off = 0;
+    l.off_bias = off;
+    off += align256((size_t)l.BH * s->L * 4);
+    l.off_split_max = off;
+    off += align256((size_t)l.BH * l.n_split * 4);
+    l.off_head_max = off;
+    off += align256((size_t)l.BH * 4);
+    l.off_part_S = off;
+    off += align256((size_t)l.BH * l.n_split * s->m * s->d * 4);
+    l.off_part_z = off;
+    off += align256((size_t)l.BH * l.n_split * s->m * 4);
+    l.off_state = off;
+    if (state_in_ws) off += align256((size_t)l.BH * state_floats(s->m, s->d) * 4);
+    l.total = off;
+    return l;
+}
+
+size_t ctx_bytes(const favor_shape *s) {
+    return align256((size_t)s->B * s->H * state_floats(s->m, s->d) * 4) + align256((size_t)s->B * s->H * s->L * 4);
+}
+
+// ------------------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+// [BH, L, d] bf16 tensor as a 3-D map (d, L, BH) with 64 x 128 x 1 boxes, 128-byte swizzle;
+// rows past L read as zeros.
+bool make_token_map(CUtensorMap *map, const void *base, int BH, int L, int d) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)L * d * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [m, d] bf16 W as a 2-D map (d, m) with 64 x m boxes, 128-byte swizzle.
+bool make_w_map(CUtensorMap *map, const void *base, int m, int d) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)m};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)m};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+favor_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA; }
+
+// ---------------------------------------------------------------------------- bf16 forward
+
+favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W, float *out,
+                      void *ctx, uint8_t *ws, size_t ws_bytes, const favor_opts *o, cudaStream_t st) {
+    const Bf16Layout l = bf16_layout(s, o, ctx == nullptr);
+    if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
+    CUtensorMap mQ, mK, mW;
+    if (!make_token_map(&mQ, Q, l.BH, s->L, s->d) || !make_token_map(&mK, K, l.BH, s->L, s->d) ||
+        !make_w_map(&mW, W, s->m, s->d))
+        return FAVOR_ERR_CUDA;
+    // Per-key -|k|^2/2 goes straight into the context (after the state blocks) when one is kept.
+    float *bias = ctx ? (float *)((uint8_t *)ctx + align256((size_t)l.BH * state_floats(s->m, s->d) * 4))
+                      : (float *)(ws + l.off_bias);
+    float *split_max = (float *)(ws + l.off_split_max);
+    float *head_max = (float *)(ws + l.off_head_max);
+    float *part_S = (float *)(ws + l.off_part_S);
+    float *part_z = (float *)(ws + l.off_part_z);
+    float *state = ctx ? (float *)ctx : (float *)(ws + l.off_state);
+
+    KeyMaxParams km{s->L, s->d, s->m, l.n_split, l.tiles_per_split, bias, split_max};
+    cudaError_t e = launch_key_logit_max(mK, mW, km, l.BH, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    KeyStateParams ks{s->L, s->d, s->m, l.n_split, l.tiles_per_split, (const uint16_t *)V, bias, split_max,
+                      part_S, part_z, head_max};
+    if ((e = launch_key_state(mK, mW, ks, l.BH, st)) != cudaSuccess) return FAVOR_ERR_CUDA;
+    FinalizeParams fp{s->m, s->d, l.n_split, part_S, part_z, head_max, state};
+    if ((e = launch_state_finalize(fp, l.BH, st)) != cudaSuccess) return FAVOR_ERR_CUDA;
+    QueryParams qp{s->L, s->d, s->m, opt_split_tiles(o), state, out};
+    if ((e = launch_query_out(mQ, mW, qp, l.BH, st)) != cudaSuccess) return FAVOR_ERR_CUDA;
+    return FAVOR_OK;
+}
+
+}  // namespace
+}  // namespace favor
+
+using namespace favor;
+
+extern "C" const char *favor_status_string(favor_status st) {
+    switch (st) {
+        case FAVOR_OK: return "FAVOR_OK";
+        case FAVOR_ERR_INVALID_ARG: return "FAVOR_ERR_INVALID_ARG: null pointer or invalid size";
+        case FAVOR_ERR_UNSUPPORTED: return "FAVOR_ERR_UNSUPPORTED: valid arguments outside the implemented cases";
+        case FAVOR_ERR_CUDA: return "FAVOR_ERR_CUDA: a CUDA runtime or driver call failed";
+        case FAVOR_ERR_TIMEOUT: return "FAVOR_ERR_TIMEOUT: a bounded device-side wait gave up";
+        case FAVOR_ERR_WORKSPACE: return "FAVOR_ERR_WORKSPACE: workspace or ctx missing or too small";
+    }
+    return "FAVOR: unknown status";
+}
+
+extern "C" size_t favor_workspace_size(const favor_shape *s, int causal, int backward, const favor_opts *o) {
+    if (!shape_ok(s) || (causal != 0 && causal != 1)) return 0;
+    if (shape_supported(s, causal, backward) != FAVOR_OK) return 0;
+    if (s->dtype == FAVOR_F32) return align256(f32_workspace_floats(s->B * s->H, s->L, s->d, s->m) * 4);
+    return bf16_layout(s, o, true).total;
+}
+
+extern "C" size_t favor_ctx_size(const favor_shape *s, int causal) {
+    if (!shape_ok(s) || (causal != 0 && causal != 1)) return 0;
+    return ctx_bytes(s);
+}
+
+extern "C" favor_status favor_fwd(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W,
+                                  int causal, float *out, void *ctx, void *workspace, size_t ws_bytes,
+                                  const favor_opts *o, void *stream) {
+    if (!shape_ok(s) || Q == nullptr || K == nullptr || V == nullptr || W == nullptr || out == nullptr ||
+        (causal != 0 && causal != 1))
+        return FAVOR_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(W) || !aligned16(out))
+        return FAVOR_ERR_INVALID_ARG;
+    const favor_status sup = shape_supported(s, causal, 0);
+    if (sup != FAVOR_OK) return sup;
+    if (workspace == nullptr || ((uintptr_t)workspace & 255u) != 0) return FAVOR_ERR_WORKSPACE;
+    if (ctx != nullptr && ((uintptr_t)ctx & 255u) != 0) return FAVOR_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (s->dtype == FAVOR_F32) {
+        if (ws_bytes < favor_workspace_size(s, causal, 0, o)) return FAVOR_ERR_WORKSPACE;
+        F32Params p{s->L, s->d, s->m, (const float *)Q, (const float *)K, (const float *)V, (const float *)W,
+                    nullptr, nullptr, out, nullptr, nullptr, nullptr, (float *)workspace};
+        return cuda_status(launch_f32(p, s->B * s->H, causal != 0, false, st));
+    }
+    return fwd_bf16(s, Q, K, V, W, out, ctx, (uint8_t *)workspace, ws_bytes, o, st);
+}
+
+extern "C" favor_status favor_bwd(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W,
+                                  const float *out, const void *dout, const void *ctx, int causal, float *dQ,
+                                  float *dK, float *dV, void *workspace, size_t ws_bytes, const favor_opts *o,
+                                  void *stream) {
+    if (!shape_ok(s) || Q == nullptr || K == nullptr || V == nullptr || W == nullptr || out == nullptr ||
+        dout == nullptr || dQ == nullptr || dK == nullptr || dV == nullptr || (causal != 0 && causal != 1))
+        return FAVOR_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(W) || !aligned16(out) || !aligned16(dout) ||
+        !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+        return FAVOR_ERR_INVALID_ARG;
+    const favor_status sup = shape_supported(s, causal, 1);
+    if (sup != FAVOR_OK) return sup;
+    if (workspace == nullptr || ((uintptr_t)workspace & 255u) != 0) return FAVOR_ERR_WORKSPACE;
+    if (ws_bytes < favor_workspace_size(s, causal, 1, o)) return FAVOR_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    (void)ctx;
+    F32Params p{s->L, s->d, s->m, (const float *)Q, (const float *)K, (const float *)V, (const float *)W,
+                out, (const float *)dout, nullptr, dQ, dK, dV, (float *)workspace};
+    return cuda_status(launch_f32(p, s->B * s->H, causal != 0, true, st));
+}
+
+extern "C" favor_status favor_sync_status(void *stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FAVOR_ERR_CUDA;
+    int v = FAVOR_OK;
+    if (cudaMemcpyFromSymbol(&v, favor::g_status, sizeof(int)) != cudaSuccess) return FAVOR_ERR_CUDA;
+    if (v != FAVOR_OK) {
+        const int zero = FAVOR_OK;
+        if (cudaMemcpyToSymbol(favor::g_status, &zero, sizeof(int)) != cudaSuccess) return FAVOR_ERR_CUDA;
+    }
+    return (favor_status)v;
+}

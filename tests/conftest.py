@@ -11,3 +11,31 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: long CPU-side oracle work")
+
+
+@pytest.fixture(scope="session")
+def favor_lib():
+    """The built C-ABI library (built here with nvcc if absent; nvcc cross-compiles without a GPU)."""
+    from linear_attention_positive_b200 import api, build
+
+    if not os.path.exists(api.LIB_PATH):
+        build.build()
+    return api.library()
+
+
+def gpu_available():
+    try:
+        import torch
+
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+@pytest.fixture(scope="session")
+def cuda_device(favor_lib):
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.fail("gpu test selected but no CUDA device is visible")
+    return torch.device("cuda:0")

@@ -1,0 +1,90 @@
+"""The C-ABI library on the CPU: it loads, exports every entry point include/favor.h declares,
+draws W bit for bit like the oracle, sizes workspaces, and rejects bad arguments before any
+launch (no compute call runs here)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from linear_attention_positive_b200 import api
+from oracle import features
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_entry_points():
+    with open(os.path.join(ROOT, "include", "favor.h")) as f:
+        text = f.read()
+    return re.findall(r"FAVOR_API\s+[^;(]*?\b(favor_\w+)\s*\(", text)
+
+
+def test_exports_match_header(favor_lib):
+    declared = header_entry_points()
+    assert set(declared) >= set(api.EXPORTS)
+    for name in declared:
+        assert hasattr(favor_lib, name), name
+
+
+@pytest.mark.parametrize("seed,m,d", [(1, 64, 64), (2, 256, 64), (5, 256, 128), (3, 100, 32),
+                                      (2**64 - 1, 16, 64), (0, 1, 1)])
+def test_draw_features_bit_exact_with_oracle(favor_lib, seed, m, d):
+    assert np.array_equal(api.draw_features(seed, m, d), features.draw_W(seed, m, d))
+
+
+def test_draw_features_matches_golden_fixture(favor_lib):
+    vals = []
+    with open(os.path.join(ROOT, "tests", "golden", "W_seed1_m64_d64.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                vals.extend(float.fromhex(t) for t in line.split())
+    assert np.array_equal(api.draw_features(1, 64, 64), np.array(vals).reshape(64, 64))
+
+
+def test_draw_features_rejects_bad_args(favor_lib):
+    buf = (ctypes.c_double * 4)()
+    assert favor_lib.favor_draw_features(1, 0, 4, buf) == api.FAVOR_ERR_INVALID_ARG
+    assert favor_lib.favor_draw_features(1, 4, 0, buf) == api.FAVOR_ERR_INVALID_ARG
+    assert favor_lib.favor_draw_features(1, 4, 4, None) == api.FAVOR_ERR_INVALID_ARG
+
+
+def test_workspace_and_ctx_sizes(favor_lib):
+    ok = api.make_shape(8, 8, 4096, 64, 256, api.FAVOR_BF16)
+    assert api.workspace_size(ok) > 8 * 8 * 4096 * 4
+    assert api.workspace_size(ok) % 256 == 0
+    assert api.ctx_size(ok) >= 64 * (256 * 64 + 256) * 4
+    f32 = api.make_shape(1, 1, 256, 64, 64, api.FAVOR_F32)
+    assert api.workspace_size(f32) > 0 and api.workspace_size(f32, causal=True, backward=True) > 0
+    # invalid or unsupported shapes size to zero
+    for bad in (api.make_shape(0, 1, 256, 64, 64, 0), api.make_shape(1, 1, 256, 96, 64, 0),
+                api.make_shape(1, 1, 256, 64, 192, api.FAVOR_BF16), api.make_shape(1, 1, 256, 64, 64, 7)):
+        assert api.workspace_size(bad) == 0
+    assert favor_lib.favor_workspace_size(None, 0, 0, None) == 0
+    assert favor_lib.favor_workspace_size(ctypes.byref(ok), 2, 0, None) == 0
+
+
+def test_fwd_bwd_argument_errors_return_before_launch(favor_lib):
+    sh = api.make_shape(1, 1, 256, 64, 64, api.FAVOR_F32)
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    null = None
+    fwd = favor_lib.favor_fwd
+    assert fwd(None, p, p, p, p, 0, p, null, p, 1 << 20, null, null) == api.FAVOR_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(sh), null, p, p, p, 0, p, null, p, 1 << 20, null, null) == api.FAVOR_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(sh), p, p, p, p, 3, p, null, p, 1 << 20, null, null) == api.FAVOR_ERR_INVALID_ARG
+    unaligned = ctypes.c_void_p(258)
+    assert fwd(ctypes.byref(sh), unaligned, p, p, p, 0, p, null, p, 1 << 20, null, null) == api.FAVOR_ERR_INVALID_ARG
+    assert fwd(ctypes.byref(sh), p, p, p, p, 0, p, null, null, 1 << 20, null, null) == api.FAVOR_ERR_WORKSPACE
+    assert fwd(ctypes.byref(sh), p, p, p, p, 0, p, null, p, 16, null, null) == api.FAVOR_ERR_WORKSPACE
+    odd = api.make_shape(1, 1, 256, 96, 64, api.FAVOR_F32)
+    assert fwd(ctypes.byref(odd), p, p, p, p, 0, p, null, p, 1 << 20, null, null) == api.FAVOR_ERR_UNSUPPORTED
+    bwd = favor_lib.favor_bwd
+    assert bwd(ctypes.byref(sh), p, p, p, p, p, null, null, 0, p, p, p, p, 1 << 20, null, null) == api.FAVOR_ERR_INVALID_ARG
+    assert bwd(ctypes.byref(sh), p, p, p, p, p, p, null, 0, p, p, p, p, 16, null, null) == api.FAVOR_ERR_WORKSPACE
+
+
+def test_status_strings(favor_lib):
+    for code in range(6):
+        assert api.status_string(code).startswith("FAVOR_")
+    assert "unknown" in api.status_string(99)
