@@ -1,0 +1,397 @@
+"""FAVOR+ benchmark: tokens/s (B*H*L) of one pass of the hot path, and its roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2|3|4|5] [--impl ours|reference]
+
+A step is one pass of the whole hot path (every kernel favor_fwd launches, plus favor_bwd for the
+forward+backward workload) over one batch of seeded synthetic input already resident in HBM.
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a device synchronise;
+each step is timed with CUDA events on the launching stream and the L2 cache is flushed (a
+256 MB write) between steps outside the timed events; the job time is the max over ranks. One
+JSON line is printed by rank 0. Under torchrun each rank runs its own replica of the workload
+(independent heads; weak scaling, no data-path collective).
+
+--impl reference times the fp64 oracle (the method's plain CPU definition) on the host cores on a
+bounded sample of the same workload; under torchrun only rank 0 runs it.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_positive_b200.inputs import WORKLOADS, make_inputs, round_to_bf16  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor rate
+L2_FLUSH_BYTES = 256 << 20
+
+# Kernels favor_fwd launches for the bf16 bidirectional path, in launch order.
+FWD_STAGES = ["k_key_logit_max", "k_key_state", "k_state_finalize", "k_query_out"]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def stage_work(name, w):
+    """Algorithmic HBM bytes and tensor FLOPs (bf16, tf32) of one launch of a stage."""
+    t, d, m = w.tokens, w.d, w.m
+    if name == "k_key_logit_max":      # read K; write -|k|^2/2
+        return t * (2 * d + 4), 2 * m * d * t, 0
+    if name == "k_key_state":          # read K, V, -|k|^2/2
+        return t * (4 * d + 4), 2 * m * d * t, 2 * m * d * t
+    if name == "k_query_out":          # read Q; write fp32 out
+        return t * (2 * d + 4 * d), 2 * m * d * t, 2 * m * d * t
+    if name == "k_state_finalize":
+        BH = w.B * w.H
+        n_split = -(-(-(-w.L // 128)) // 8)
+        return BH * n_split * m * (d + 1) * 4 + BH * m * (d + 1) * 4, 0, 0
+    return 0, 0, 0
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_positive_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel, workload_name):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or rec.get("source_sha") != source_hash() or rec.get("workload") != workload_name:
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"favor_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.remove(self.path)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------ oracle arm
+
+def oracle_sample(w, x, W64, heads):
+    """Runs the fp64 oracle over ``heads`` (b, h) pairs of the workload; returns tokens done."""
+    from oracle import favor
+
+    for b, h in heads:
+        X = {k: x[k][b, h].astype(np.float64) for k in x}
+        if w.backward:
+            favor.fwd(X["Q"][None, None], X["K"][None, None], X["V"][None, None], W64, causal=w.causal)
+            favor.bwd(X["Q"][None, None], X["K"][None, None], X["V"][None, None], W64, X["dO"][None, None],
+                      causal=w.causal)
+        else:
+            favor.fwd(X["Q"][None, None], X["K"][None, None], X["V"][None, None], W64, causal=w.causal)
+    return len(heads) * w.L
+
+
+def pick_sample(w, x, W64, budget_s):
+    """Number of heads whose oracle run takes about budget_s seconds (at least one)."""
+    t0 = time.perf_counter()
+    oracle_sample(w, x, W64, [(0, 0)])
+    per_head = time.perf_counter() - t0
+    return max(1, min(w.B * w.H, int(budget_s / max(per_head, 1e-6))))
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    x = make_inputs(w)
+    W64 = round_to_bf16(api_draw(w).astype(np.float32)).astype(np.float64) if w.dtype == "bf16" else \
+        api_draw(w).astype(np.float32).astype(np.float64)
+    n_heads = pick_sample(w, x, W64, budget_s=max(1.0, 60.0 / max(args.steps + args.warmup, 1)))
+    heads = [(i // w.H, i % w.H) for i in range(n_heads)]
+    for _ in range(args.warmup):
+        oracle_sample(w, x, W64, heads[:1])
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        toks = oracle_sample(w, x, W64, heads)
+        times.append(time.perf_counter() - t0)
+    sec = statistics.mean(times)
+    value = toks / sec
+    sample = f"{n_heads} of {w.B * w.H} heads (L={w.L}) per step, fp64 numpy oracle"
+    line = {
+        "impl": "reference", "metric": metric_name(w), "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def api_draw(w):
+    from linear_attention_positive_b200 import api
+
+    return api.draw_features(w.w_seed, w.m, w.d)
+
+
+def metric_name(w):
+    kind = "fwd+bwd" if w.backward else "fwd"
+    return f"FAVOR+ {kind} tokens/s (B*H*L)"
+
+
+def workload_config(w, n):
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "m": w.m, "causal": w.causal,
+            "backward": w.backward, "global_batch": w.B * n, "seq_len": w.L, "parallelism": f"replicas{n}",
+            "l2": "flushed between steps (256 MB write, outside the timed events)"}
+
+
+# ------------------------------------------------------------------------------------ GPU arm
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from linear_attention_positive_b200 import api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    x = make_inputs(w)
+    Wf = api_draw(w).astype(np.float32)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    T = {k: torch.from_numpy(x[k]).to(tdt).to(dev) for k in x}
+    Wt = torch.from_numpy(round_to_bf16(Wf) if w.dtype == "bf16" else Wf).to(tdt).to(dev)
+    shape = api.make_shape(w.B, w.H, w.L, w.d, w.m, api.FAVOR_BF16 if w.dtype == "bf16" else api.FAVOR_F32)
+    n_stage = len(FWD_STAGES) if w.dtype == "bf16" else 1
+    ws = torch.empty(max(api.workspace_size(shape, w.causal, False), api.workspace_size(shape, w.causal, w.backward)),
+                     dtype=torch.uint8, device=dev)
+    ctx = torch.empty(api.ctx_size(shape, w.causal), dtype=torch.uint8, device=dev) if w.backward else None
+    out = torch.empty(T["Q"].shape, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def new_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record()
+        return evs
+
+    def step(opts=None):
+        api.fwd(T["Q"], T["K"], T["V"], Wt, causal=w.causal, out=out, ctx=ctx, workspace=ws, opts=opts)
+        if w.backward:
+            api.bwd(T["Q"], T["K"], T["V"], Wt, out, T["dO"], ctx=ctx, causal=w.causal, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if api.sync_status() != api.FAVOR_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    step_ev = [new_events(2) for _ in range(args.steps)]
+    stage_ev = [new_events(2 * api.FAVOR_MAX_STAGES) for _ in range(args.steps)]
+    opts = [api.make_opts(stage_events=stage_ev[k]) for k in range(args.steps)]
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.zero_()
+        step_ev[k][0].record(stream)
+        step(opts[k])
+        step_ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    status = api.sync_status()
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    stage_ms = [[stage_ev[k][2 * i].elapsed_time(stage_ev[k][2 * i + 1]) for k in range(args.steps)]
+                for i in range(n_stage)]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    job_ms = float(t.item())
+    ms_per_step = job_ms / args.steps
+    value = w.tokens * world / (ms_per_step * 1e-3)
+
+    # End to end through the public API: pinned host inputs in, fp32 output back, every step.
+    pin = {k: torch.from_numpy(x[k]).to(tdt).pin_memory() for k in x}
+    out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    dT = {k: torch.empty_like(T[k]) for k in T}
+    e2e_ev = [new_events(2) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    for k in range(args.steps):
+        flush.zero_()
+        e2e_ev[k][0].record(stream)
+        for name in dT:
+            dT[name].copy_(pin[name], non_blocking=True)
+        api.fwd(dT["Q"], dT["K"], dT["V"], Wt, causal=w.causal, out=out, ctx=ctx, workspace=ws)
+        if w.backward:
+            dq, dk, dv = api.bwd(dT["Q"], dT["K"], dT["V"], Wt, out, dT["dO"], ctx=ctx, causal=w.causal, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+        e2e_ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    h2d = sum(pin[k].numel() * pin[k].element_size() for k in pin)
+    d2h = out_h.numel() * 4
+
+    peaks, peak_src = load_peaks()
+    line = {
+        "metric": metric_name(w), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": workload_config(w, world),
+        "e2e": {"value": w.tokens * world / (float(e2e_ms.item()) * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": n_stage * args.steps if w.dtype == "bf16" else args.steps,
+        "device_status": api.status_string(status),
+    }
+    if w.dtype == "bf16" and not w.backward:
+        avg = {FWD_STAGES[i]: statistics.mean(stage_ms[i]) for i in range(n_stage)}
+        line["stage_ms"] = {k: round(v, 5) for k, v in avg.items()}
+        dom = max(avg, key=avg.get)
+        nbytes, f_bf16, f_tf32 = stage_work(dom, w)
+        sec = avg[dom] * 1e-3
+        hbm_peak = peaks["hbm_gbs"]
+        tc_peak = peaks["bf16_tflops"]
+        t_hbm = nbytes / (hbm_peak * 1e9)
+        t_tc = f_bf16 / (tc_peak * 1e12) + f_tf32 / (tc_peak * TF32_PER_BF16 * 1e12)
+        if t_tc > t_hbm:
+            eq = f_bf16 + f_tf32 / TF32_PER_BF16
+            line["roofline"] = {"kernel": dom, "bound": "tensor", "achieved": eq / sec / 1e12, "peak": tc_peak,
+                                "unit": "TFLOP/s", "frac": (eq / sec / 1e12) / tc_peak,
+                                "traffic": measured_traffic(dom, w.name),
+                                "note": f"bf16-equivalent FLOPs (tf32 counted at the nominal {TF32_PER_BF16:.3f}x rate); "
+                                        f"peak {peak_src} burst bf16"}
+        else:
+            line["roofline"] = {"kernel": dom, "bound": "hbm", "achieved": nbytes / sec / 1e9, "peak": hbm_peak,
+                                "unit": "GB/s", "frac": (nbytes / sec / 1e9) / hbm_peak,
+                                "traffic": measured_traffic(dom, w.name), "note": f"peak {peak_src} copy bandwidth"}
+        path_bytes = w.tokens * (6 * w.d + 4 * w.d)
+        line["path_roofline"] = {"hbm_bytes_per_step": path_bytes,
+                                 "hbm_frac": path_bytes / (ms_per_step * 1e-3) / (hbm_peak * 1e9)}
+    if clk is not None:
+        line["clocks"] = clk
+    if world == 1:
+        try:
+            W64 = (round_to_bf16(Wf) if w.dtype == "bf16" else Wf).astype(np.float64)
+            n_heads = pick_sample(w, x, W64, budget_s=15.0)
+            t0 = time.perf_counter()
+            toks = oracle_sample(w, x, W64, [(i // w.H, i % w.H) for i in range(n_heads)])
+            sec = time.perf_counter() - t0
+            line["cpu_baseline"] = {"value": toks / sec, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                                    "sample": f"{n_heads} of {w.B * w.H} heads (L={w.L}), fp64 numpy oracle"}
+        except Exception as exc:  # the baseline is reported, never required
+            line["cpu_baseline"] = {"value": None, "error": str(exc)[:200]}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=2, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -66,14 +66,21 @@ typedef struct {
     favor_dtype dtype;
 } favor_shape;
 
+/* Most kernel launches one call makes (the length of a stage_events array is 2x this). */
+#define FAVOR_MAX_STAGES 8
+
 /* Tuning knobs; pass NULL for defaults. Zero fields take their defaults too.
  *   split_tiles : 128-token tiles per CTA for the key-side reduction (and per causal segment)
  *   exp_poly_pct: percent (0..100) of feature exponentials evaluated by the FMA-pipe
- *                 polynomial instead of the MUFU ex2 unit (bf16 path). */
+ *                 polynomial instead of the MUFU ex2 unit (bf16 path)
+ *   stage_events: NULL, or 2 * FAVOR_MAX_STAGES caller-created cudaEvent_t handles (as void*);
+ *                 the call records events[2k] before and events[2k+1] after its k-th kernel
+ *                 launch on the call's stream (NULL entries are skipped). For timing. */
 typedef struct {
     int split_tiles;
     int exp_poly_pct;
     int reserved[6];
+    void **stage_events;
 } favor_opts;
 
 /*

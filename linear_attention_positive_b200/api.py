@@ -46,8 +46,12 @@ class Shape(ctypes.Structure):
                 ("m", ctypes.c_int), ("dtype", ctypes.c_int)]
 
 
+FAVOR_MAX_STAGES = 8
+
+
 class Opts(ctypes.Structure):
-    _fields_ = [("split_tiles", ctypes.c_int), ("exp_poly_pct", ctypes.c_int), ("reserved", ctypes.c_int * 6)]
+    _fields_ = [("split_tiles", ctypes.c_int), ("exp_poly_pct", ctypes.c_int), ("reserved", ctypes.c_int * 6),
+                ("stage_events", ctypes.POINTER(ctypes.c_void_p))]
 
 
 _LIB = None
@@ -94,8 +98,17 @@ def make_shape(B, H, L, d, m, dtype):
     return Shape(B, H, L, d, m, dtype)
 
 
-def make_opts(split_tiles=0, exp_poly_pct=0):
-    return Opts(split_tiles, exp_poly_pct, (ctypes.c_int * 6)())
+def make_opts(split_tiles=0, exp_poly_pct=0, stage_events=None):
+    """Options struct. ``stage_events``: optional list of 2*FAVOR_MAX_STAGES torch.cuda.Event
+    (enable_timing=True, already recorded once so their handles exist) or None entries."""
+    o = Opts(split_tiles, exp_poly_pct, (ctypes.c_int * 6)(), None)
+    if stage_events is not None:
+        arr = (ctypes.c_void_p * (2 * FAVOR_MAX_STAGES))()
+        for i, ev in enumerate(stage_events[: 2 * FAVOR_MAX_STAGES]):
+            arr[i] = ev.cuda_event if ev is not None else None
+        o._events_keepalive = arr
+        o.stage_events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    return o
 
 
 def draw_features(seed, m, d):

@@ -261,4 +261,15 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 __device__ __forceinline__ uint32_t elect_lane0() { return (threadIdx.x & 31u) == 0u; }
 
+// The tensor core reads a tf32 operand as the fp32 value with its low 13 mantissa bits dropped
+// (truncation). Sums taken on CUDA cores that must agree with an MMA over the same operand use the
+// same truncated value, so both sides carry the same rounding.
+__device__ __forceinline__ float tf32_trunc(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
+
+// Stored form of an fp32 value in an MMA operand image: half a tf32 ulp added to the bit pattern,
+// so the hardware's truncation yields the value rounded to nearest (ties away). The exact fp32
+// value is recovered by subtracting the same integer.
+__device__ __forceinline__ float tf32_store(float x) { return __uint_as_float(__float_as_uint(x) + 0x1000u); }
+__device__ __forceinline__ float tf32_load(float y) { return __uint_as_float(__float_as_uint(y) - 0x1000u); }
+
 }  // namespace favor

@@ -16,6 +16,7 @@
 #include "k_fp32.cu"
 #include "k_keys.cu"
 #include "k_query.cu"
+#include "k_causal.cu"
 
 namespace favor {
 namespace {
@@ -39,7 +40,8 @@ favor_status shape_supported(const favor_shape *s, int causal, int backward) {
         return FAVOR_OK;
     }
     if (s->m != 128 && s->m != 256) return FAVOR_ERR_UNSUPPORTED;
-    if (causal || backward) return FAVOR_ERR_UNSUPPORTED;
+    if (causal && s->d != 64) return FAVOR_ERR_UNSUPPORTED;
+    if (backward) return FAVOR_ERR_UNSUPPORTED;
     return FAVOR_OK;
 }
 
@@ -54,12 +56,15 @@ int opt_split_tiles(const favor_opts *o) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Tokens per head that the causal path recomputes exactly in fp32 (see k_causal.cu).
+constexpr int kCausalExactPrefix = 512;
+
 struct Bf16Layout {
-    int BH, n_tiles, tiles_per_split, n_split;
-    size_t off_bias, off_split_max, off_head_max, off_part_S, off_part_z, off_state, total;
+    int BH, n_tiles, tiles_per_split, n_split, P_exact;
+    size_t off_bias, off_split_max, off_head_max, off_part_S, off_part_z, off_state, off_seg, off_phi, total;
 };
 
-Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_ws) {
+Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_ws, int causal = 0) {
     Bf16Layout l{};
     l.BH = s->B * s->H;
     l.n_tiles = (s->L + kTile - 1) / kTile;
@@ -78,6 +83,11 @@ Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_
     off += align256((size_t)l.BH * l.n_split * s->m * 4);
     l.off_state = off;
     if (state_in_ws) off += align256((size_t)l.BH * state_floats(s->m, s->d) * 4);
+    l.P_exact = causal ? std::min(s->L, kCausalExactPrefix) : 0;
+    l.off_seg = off;
+    if (causal) off += align256((size_t)l.BH * l.n_split * state_floats(s->m, s->d) * 4);
+    l.off_phi = off;
+    if (causal) off += align256((size_t)2 * l.BH * l.P_exact * s->m * 4);
     l.total = off;
     return l;
 }
@@ -133,11 +143,17 @@ bool make_w_map(CUtensorMap *map, const void *base, int m, int d) {
 
 favor_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA; }
 
+// Records the caller's timing event (2k before / 2k+1 after launch k), if one was supplied.
+void record_stage(const favor_opts *o, int slot, cudaStream_t st) {
+    if (o != nullptr && o->stage_events != nullptr && slot < 2 * FAVOR_MAX_STAGES && o->stage_events[slot] != nullptr)
+        cudaEventRecord((cudaEvent_t)o->stage_events[slot], st);
+}
+
 // ---------------------------------------------------------------------------- bf16 forward
 
 favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W, float *out,
-                      void *ctx, uint8_t *ws, size_t ws_bytes, const favor_opts *o, cudaStream_t st) {
-    const Bf16Layout l = bf16_layout(s, o, ctx == nullptr);
+                      void *ctx, uint8_t *ws, size_t ws_bytes, const favor_opts *o, cudaStream_t st, int causal) {
+    const Bf16Layout l = bf16_layout(s, o, ctx == nullptr, causal);
     if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
     CUtensorMap mQ, mK, mW;
     if (!make_token_map(&mQ, Q, l.BH, s->L, s->d) || !make_token_map(&mK, K, l.BH, s->L, s->d) ||
@@ -153,15 +169,46 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     float *state = ctx ? (float *)ctx : (float *)(ws + l.off_state);
 
     KeyMaxParams km{s->L, s->d, s->m, l.n_split, l.tiles_per_split, bias, split_max};
+    record_stage(o, 0, st);
     cudaError_t e = launch_key_logit_max(mK, mW, km, l.BH, st);
+    record_stage(o, 1, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     KeyStateParams ks{s->L, s->d, s->m, l.n_split, l.tiles_per_split, (const uint16_t *)V, bias, split_max,
                       part_S, part_z, head_max};
-    if ((e = launch_key_state(mK, mW, ks, l.BH, st)) != cudaSuccess) return FAVOR_ERR_CUDA;
+    record_stage(o, 2, st);
+    e = launch_key_state(mK, mW, ks, l.BH, st);
+    record_stage(o, 3, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    if (causal) {
+        ScanParams sp{s->m, s->d, l.n_split, part_S, part_z, head_max, (float *)(ws + l.off_seg)};
+        record_stage(o, 4, st);
+        e = launch_state_scan(sp, l.BH, st);
+        record_stage(o, 5, st);
+        if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+        CausalParams cp{s->L, s->d, s->m, l.tiles_per_split, l.P_exact, (const uint16_t *)V, bias,
+                        (const float *)(ws + l.off_seg), l.n_split, out};
+        record_stage(o, 6, st);
+        e = launch_causal_out(mQ, mK, mW, cp, l.BH, st);
+        record_stage(o, 7, st);
+        if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+        float *phi = (float *)(ws + l.off_phi);
+        PrefixParams pp{s->L, s->d, s->m, l.P_exact, (const uint16_t *)Q, (const uint16_t *)K, (const uint16_t *)V,
+                        (const uint16_t *)W, bias, head_max, phi, phi + (size_t)l.BH * l.P_exact * s->m, out};
+        record_stage(o, 8, st);
+        e = launch_causal_prefix(pp, l.BH, st);
+        record_stage(o, 9, st);
+        return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+    }
     FinalizeParams fp{s->m, s->d, l.n_split, part_S, part_z, head_max, state};
-    if ((e = launch_state_finalize(fp, l.BH, st)) != cudaSuccess) return FAVOR_ERR_CUDA;
+    record_stage(o, 4, st);
+    e = launch_state_finalize(fp, l.BH, st);
+    record_stage(o, 5, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     QueryParams qp{s->L, s->d, s->m, opt_split_tiles(o), state, out};
-    if ((e = launch_query_out(mQ, mW, qp, l.BH, st)) != cudaSuccess) return FAVOR_ERR_CUDA;
+    record_stage(o, 6, st);
+    e = launch_query_out(mQ, mW, qp, l.BH, st);
+    record_stage(o, 7, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     return FAVOR_OK;
 }
 
@@ -186,7 +233,7 @@ extern "C" size_t favor_workspace_size(const favor_shape *s, int causal, int bac
     if (!shape_ok(s) || (causal != 0 && causal != 1)) return 0;
     if (shape_supported(s, causal, backward) != FAVOR_OK) return 0;
     if (s->dtype == FAVOR_F32) return align256(f32_workspace_floats(s->B * s->H, s->L, s->d, s->m) * 4);
-    return bf16_layout(s, o, true).total;
+    return bf16_layout(s, o, true, causal).total;
 }
 
 extern "C" size_t favor_ctx_size(const favor_shape *s, int causal) {
@@ -213,7 +260,7 @@ extern "C" favor_status favor_fwd(const favor_shape *s, const void *Q, const voi
                     nullptr, nullptr, out, nullptr, nullptr, nullptr, (float *)workspace};
         return cuda_status(launch_f32(p, s->B * s->H, causal != 0, false, st));
     }
-    return fwd_bf16(s, Q, K, V, W, out, ctx, (uint8_t *)workspace, ws_bytes, o, st);
+    return fwd_bf16(s, Q, K, V, W, out, ctx, (uint8_t *)workspace, ws_bytes, o, st, causal);
 }
 
 extern "C" favor_status favor_bwd(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W,

@@ -185,7 +185,9 @@ k_key_logit_max(const __grid_constant__ CUtensorMap mapK, const __grid_constant_
 // Per 64-token sub-tile: D2[r, j] = W . K_sub^T (bf16, M = 128 features per half, N = 64 tokens);
 // the epilogue (thread <-> feature r) overwrites D2 in place with phi = 2^(D2 log2e + b_j) where
 // b_j = (-|k_j|^2/2 - C) log2e, and sums phi into z_r; then S[r, :] += phi(TMEM, tf32) x V_sub
-// (fp32 copy of V in shared memory, tf32 MMA, M = 128 features, N = d, K = 8 tokens per step).
+// (fp32 V^T in shared memory as the K-major B operand, tf32 MMA, M = 128 features, N = d,
+// K = 8 tokens per step). tf32 keeps phi and V to 11 significant bits, which the 2e-2 * RMS
+// output budget needs; bf16 features would use most of it.
 
 struct KeyStateParams {
     int L, d, m, n_split, tiles_per_split;
@@ -201,7 +203,7 @@ template <int D>
 struct KeyStateSmem {
     static constexpr int KB = D / 64;
     static constexpr uint32_t K_TILE = KB * kTile * 128;         // bf16 K tile
-    static constexpr uint32_t V32_SUB = (D / 32) * 64 * 128;     // fp32 V, 64 tokens
+    static constexpr uint32_t V32_SUB = 2 * D * 128;             // fp32 V^T, 64 tokens
     static constexpr int STAGES = D == 64 ? 3 : 2;
 };
 
@@ -296,7 +298,7 @@ k_key_state(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CU
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc_p = make_idesc(128, 64, kFmtBF16, 0, 0);
-            const uint32_t idesc_s = make_idesc(128, D, kFmtTF32, 0, 1);
+            const uint32_t idesc_s = make_idesc(128, D, kFmtTF32, 0, 0);
             bool ok = mbar_wait(w_full, 0, abort_flag);
             // Projection of sub-tile u into D2 buffer u&1.
             auto project = [&](int u) -> bool {
@@ -328,7 +330,8 @@ k_key_state(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CU
                 const uint32_t vb = smem_u32(sV + b * SM::V32_SUB);
                 for (int h = 0; h < halves; ++h) {
                     for (int ks = 0; ks < 8; ++ks) {
-                        const uint64_t bd = make_sdesc(vb + ks * 8 * 128, 64 * 128, 1024);
+                        // K-step of 8 tokens: block ks/4 of V^T, 32-byte offset inside its rows.
+                        const uint64_t bd = make_sdesc(vb + (ks >> 2) * (D * 128) + (ks & 3) * 32, 16, 1024);
                         mma_tf32_ts(tmem + s_col + h * D, tmem + b * d2_cols + h * 64 + ks * 8, bd, idesc_s,
                                     (u > 0 || ks > 0) ? 1u : 0u);
                     }
@@ -342,36 +345,30 @@ k_key_state(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CU
             mbar_wait(drain, 0, &no_abort);
         }
     } else if (warp == 2 || warp == 3) {
-        // V converter: bf16 V rows of a 64-token sub-tile -> fp32, MN-major 128-byte-swizzled
-        // layout [d/32 blocks][64 tokens][32 fp32]; also b_j = (-|k_j|^2/2 - C) log2e.
-        const int t = threadIdx.x - 64;  // 0..63
+        // V converter: the bf16 V rows of a 64-token sub-tile become the K-major tf32 operand
+        // V^T: [2 blocks of 32 tokens][D value rows][32 fp32], 128-byte swizzled. Lane <-> token,
+        // so the transposing 4-byte stores of a warp fill one 128-byte row without bank conflicts.
+        // Also b_j = (-|k_j|^2/2 - C) log2e for the sub-tile's tokens.
+        const int tok = threadIdx.x - 64;  // 0..63
+        const int kb = tok >> 5, ch = (tok & 31) >> 2, pos = tok & 3;
         for (int u = 0; u < n_sub; ++u) {
             const int b = u & 1;
             if (!mbar_wait(&v_empty[b], ((u >> 1) & 1) ^ 1, abort_flag)) break;
-            const int j0 = (t0 + (u >> 1)) * kTile + (u & 1) * 64;
-            uint8_t *dst = sV + b * SM::V32_SUB;
-            constexpr int CHUNKS = 64 * D / 8;  // 16-byte chunks of bf16 source
-            for (int c = t; c < CHUNKS; c += 64) {
-                const int tok = c / (D / 8), e0 = (c % (D / 8)) * 8;
-                const int j = j0 + tok;
+            const int j = (t0 + (u >> 1)) * kTile + (u & 1) * 64 + tok;
+            uint8_t *dst = sV + b * SM::V32_SUB + kb * (D * 128) + pos * 4;
+            const uint4 *src = (const uint4 *)(p.V + ((size_t)bh * p.L + j) * D);
+#pragma unroll 4
+            for (int e0 = 0; e0 < D; e0 += 8) {
                 uint4 v = make_uint4(0, 0, 0, 0);
-                if (j < p.L) v = __ldg((const uint4 *)(p.V + ((size_t)bh * p.L + j) * D + e0));
+                if (j < p.L) v = __ldg(src + e0 / 8);
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                float f[8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    f[2 * e] = __uint_as_float(w4[e] << 16);
-                    f[2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+                    *(float *)(dst + sw128_offset(e0 + 2 * e, ch)) = __uint_as_float(w4[e] << 16);
+                    *(float *)(dst + sw128_offset(e0 + 2 * e + 1, ch)) = __uint_as_float(w4[e] & 0xFFFF0000u);
                 }
-                const int blk = e0 / 32, ch = (e0 % 32) / 4;
-                uint8_t *base = dst + blk * 64 * 128;
-                *(float4 *)(base + sw128_offset(tok, ch)) = make_float4(f[0], f[1], f[2], f[3]);
-                *(float4 *)(base + sw128_offset(tok, ch + 1)) = make_float4(f[4], f[5], f[6], f[7]);
             }
-            {
-                const int j = j0 + t;
-                sBB[b * 64 + t] = j < p.L ? (p.bias[(size_t)bh * p.L + j] * kLog2e - Clog2) : -INFINITY;
-            }
+            sBB[b * 64 + tok] = j < p.L ? (p.bias[(size_t)bh * p.L + j] * kLog2e - Clog2) : -INFINITY;
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&v_full[b]);
@@ -397,7 +394,7 @@ k_key_state(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CU
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const float ph = ex2_approx(fmaf(v[e], kLog2e, bb[c0 + e]));
-                        zsum += ph;
+                        zsum += tf32_trunc(ph);
                         v[e] = ph;
                     }
                     tmem_st32(ta, v);

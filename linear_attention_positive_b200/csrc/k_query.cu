@@ -8,7 +8,7 @@
 //                      normaliser), with Q' = exp(Q W^T - rowmax) formed in TMEM.
 //
 // Per-head state block (floats): [ image (m*d) | z (m) | C, 0, 0, 0 ]. The image holds S[r, c]
-// at  (c/64)*(m*64*4) + (r/32)*(64*128) + swizzle128(row c%64, chunk (r%32)/4) + (r%4)*4  bytes:
+// (in the tf32_store form) at  (c/64)*(m*64*4) + (r/32)*(64*128) + swizzle128(row c%64, chunk (r%32)/4) + (r%4)*4  bytes:
 // for each half of the value columns, m/32 blocks of 64 rows x 128 bytes.
 
 #include "common.cuh"
@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(256) k_state_finalize(FinalizeParams p) {
         const int r = (int)(i / p.d), c = (int)(i % p.d);
         float s = 0.f;
         for (int k = 0; k < p.n_split; ++k) s += p.part_S[((size_t)bh * p.n_split + k) * md + i];
-        *(float *)(img + state_image_offset(r, c, p.m)) = s;
+        *(float *)(img + state_image_offset(r, c, p.m)) = tf32_store(s);
     }
     for (int r = threadIdx.x; r < p.m; r += blockDim.x) {
         float z = 0.f;
@@ -258,7 +258,7 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const float ph = ex2_approx(fmaf(v[e], kLog2e, -cl));
-                        den = fmaf(ph, z[e], den);
+                        den = fmaf(tf32_trunc(ph), z[e], den);
                         v[e] = ph;
                     }
                     tmem_st32(ta, v);

@@ -112,3 +112,79 @@ def test_bf16_config2_full_size_sampled_rows(cuda_device):
             refs.append(ref)
     rms = np.sqrt(np.mean(np.concatenate(refs) ** 2))
     assert max(errs) / rms <= TOL["bf16"]
+
+
+CAUSAL_SHAPES = [
+    (1, 1, 128, 64, 256),
+    (1, 2, 1000, 64, 256),
+    (1, 1, 2200, 64, 256),   # three segments of 8 tiles
+    (2, 1, 700, 64, 128),
+    (1, 1, 1, 64, 256),
+    (1, 1, 520, 64, 256),    # just past the exact prefix
+]
+
+
+@pytest.mark.parametrize("B,H,L,d,m", CAUSAL_SHAPES)
+def test_bf16_causal_shapes(cuda_device, B, H, L, d, m):
+    w = Workload("t", B, H, L, d, m, True, "bf16", False, 3, 30 + L)
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, m, d, "bf16")
+    out = run_fwd(w, x, Wr, cuda_device, causal=True)
+    assert np.isfinite(out).all()
+    assert rel_max_err(out, oracle_fwd(x, W64, True)) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("split_tiles", [1, 2, 5])
+def test_bf16_causal_segment_choice(cuda_device, split_tiles):
+    w = Workload("t", 1, 2, 1700, 64, 256, True, "bf16", False, 3, 37)
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    out = run_fwd(w, x, Wr, cuda_device, True, opts=api.make_opts(split_tiles=split_tiles))
+    assert rel_max_err(out, oracle_fwd(x, W64, True)) <= TOL["bf16"]
+
+
+def test_bf16_causal_config3_prefix_slice_against_brute_force(cuda_device):
+    """Full causal workload (B=4, H=8, L=8192); the first 512 outputs of every head depend only on
+    the first 512 inputs and are checked against the explicit masked 512 x 512 matrix."""
+    w = WORKLOADS[3]
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    out = run_fwd(w, x, Wr, cuda_device, True)
+    assert np.isfinite(out).all()
+    errs, refs = [], []
+    for b in range(w.B):
+        for h in range(w.H):
+            X = {k: x[k][b, h, :512].astype(np.float64) for k in "QKV"}
+            ref, _ = favor.attention_brute(X["Q"], X["K"], X["V"], W64, causal=True)
+            errs.append(np.abs(out[b, h, :512] - ref).max())
+            refs.append(ref)
+    # RMS of the whole output (linear-form oracle on two heads) sets the scale of the bound.
+    full = [favor.fwd_causal(*(x[k][0, h].astype(np.float64) for k in "QKV"), W64) for h in range(2)]
+    rms = np.sqrt(np.mean(np.concatenate(full) ** 2))
+    assert max(errs) / rms <= TOL["bf16"]
+    # and the rest of the sequence on the two heads
+    for h in range(2):
+        assert np.abs(out[0, h] - full[h]).max() / rms <= TOL["bf16"]
+
+
+def test_bf16_causal_config4_full_size_sampled_rows(cuda_device):
+    """Long causal workload (B=1, H=16, L=65536, rotated 0.5-scaled inputs) in the benchmark's
+    launch configuration; per head 40 sampled rows including the first, the last and the
+    exact-prefix boundary."""
+    w = WORKLOADS[4]
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    out = run_fwd(w, x, Wr, cuda_device, True)
+    assert np.isfinite(out).all()
+    rng = np.random.default_rng(1)
+    errs, refs = [], []
+    for h in range(w.H):
+        rows = np.unique(np.concatenate([[0, 1, 127, 128, 511, 512, 513, w.L - 1], rng.integers(0, w.L, 32)]))
+        X = {k: x[k][0, h].astype(np.float64) for k in "QKV"}
+        ref = favor.fwd_causal_rows(X["Q"], X["K"], X["V"], W64, rows)
+        errs.append(np.abs(out[0, h, rows] - ref).max())
+        refs.append(ref)
+    # RMS(out) from the full oracle output of one head (sampled rows over-weight the first rows)
+    full = favor.fwd_causal(*(x[k][0, 0].astype(np.float64) for k in "QKV"), W64)
+    rms = np.sqrt(np.mean(full ** 2))
+    assert max(errs) / rms <= TOL["bf16"]
