@@ -34,8 +34,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor rate
 L2_FLUSH_BYTES = 256 << 20
 
-# Kernels favor_fwd launches for the bf16 bidirectional path, in launch order.
+# Kernels favor_fwd launches for the bf16 path, in launch order (stage k <-> events 2k, 2k+1).
 FWD_STAGES = ["k_key_logit_max", "k_key_state", "k_state_finalize", "k_query_out"]
+CAUSAL_STAGES = ["k_key_logit_max", "k_key_state", "k_state_scan", "k_causal_out", "k_causal_prefix"]
 
 
 def load_peaks():
@@ -56,6 +57,8 @@ def stage_work(name, w):
         return t * (4 * d + 4), 2 * m * d * t, 2 * m * d * t
     if name == "k_query_out":          # read Q; write fp32 out
         return t * (2 * d + 4 * d), 2 * m * d * t, 2 * m * d * t
+    if name == "k_causal_out":         # read Q, K, V, -|k|^2/2; write fp32 out
+        return t * (10 * d + 4), 6 * m * d * t, (4 * m * d + 2 * 128 * m + 2 * 128 * d) * t
     if name == "k_state_finalize":
         BH = w.B * w.H
         n_split = -(-(-(-w.L // 128)) // 8)
@@ -240,7 +243,8 @@ def run_ours(args, w):
     T = {k: torch.from_numpy(x[k]).to(tdt).to(dev) for k in x}
     Wt = torch.from_numpy(round_to_bf16(Wf) if w.dtype == "bf16" else Wf).to(tdt).to(dev)
     shape = api.make_shape(w.B, w.H, w.L, w.d, w.m, api.FAVOR_BF16 if w.dtype == "bf16" else api.FAVOR_F32)
-    n_stage = len(FWD_STAGES) if w.dtype == "bf16" else 1
+    stages = (CAUSAL_STAGES if w.causal else FWD_STAGES) if w.dtype == "bf16" else ["k_f32_head"]
+    n_stage = len(stages)
     ws = torch.empty(max(api.workspace_size(shape, w.causal, False), api.workspace_size(shape, w.causal, w.backward)),
                      dtype=torch.uint8, device=dev)
     ctx = torch.empty(api.ctx_size(shape, w.causal), dtype=torch.uint8, device=dev) if w.backward else None
@@ -333,11 +337,11 @@ def run_ours(args, w):
         "config": workload_config(w, world),
         "e2e": {"value": w.tokens * world / (float(e2e_ms.item()) * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": n_stage * args.steps if w.dtype == "bf16" else args.steps,
+        "gpu_launches": (n_stage + (1 if w.causal else 0)) * args.steps if w.dtype == "bf16" else args.steps,
         "device_status": api.status_string(status),
     }
     if w.dtype == "bf16" and not w.backward:
-        avg = {FWD_STAGES[i]: statistics.mean(stage_ms[i]) for i in range(n_stage)}
+        avg = {stages[i]: statistics.mean(stage_ms[i]) for i in range(n_stage)}
         line["stage_ms"] = {k: round(v, 5) for k, v in avg.items()}
         dom = max(avg, key=avg.get)
         nbytes, f_bf16, f_tf32 = stage_work(dom, w)
