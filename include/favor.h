@@ -161,6 +161,36 @@ FAVOR_API favor_status favor_sync_status(void *stream);
 /* favor_status_string -- static, never-NULL description of a status code. */
 FAVOR_API const char *favor_status_string(favor_status status);
 
+/* Size of the library's own fixed scratch array used by favor_fwd_static_scratch (32 MiB). */
+#define FAVOR_STATIC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * favor_fwd_static_scratch -- bidirectional bf16 forward that allocates nothing and takes no
+ * workspace. (The paper has no counterpart: this is an interface for callers that cannot
+ * allocate device memory -- code running inside another allocator's callback, where a nested
+ * cudaMalloc would recurse, or in a process whose device memory is fully reserved by a
+ * framework's caching allocator.)
+ *
+ * Computes exactly what favor_fwd(shape, Q, K, V, W, causal = 0, out, ctx = NULL, ...) computes,
+ * with the same kernels; the scratch comes from a fixed array of FAVOR_STATIC_SCRATCH_BYTES in
+ * the library's device memory, which every GPU that loads the library holds until process exit.
+ *
+ *   shape        : host pointer; dtype must be FAVOR_BF16
+ *   Q, K, V, W   : device, as for favor_fwd (16-byte aligned)
+ *   out          : device, fp32 [B,H,L,d]; fully written
+ *   stream       : cudaStream_t as void*
+ * Returns FAVOR_ERR_WORKSPACE when favor_workspace_size(shape, 0, 0, NULL) exceeds
+ * FAVOR_STATIC_SCRATCH_BYTES, FAVOR_ERR_UNSUPPORTED for fp32 or unsupported shapes.
+ *
+ * The first call on a device (with that device current) looks up the array's device address
+ * with cudaGetSymbolAddress; make that first call before any stream capture. Every call on a
+ * device shares the one array: calls that overlap on the GPU (different streams, no ordering
+ * between them) race on it. No part of the array has to start at zero; each call overwrites
+ * everything it reads. Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+FAVOR_API favor_status favor_fwd_static_scratch(const favor_shape *shape, const void *Q, const void *K,
+                                                const void *V, const void *W, float *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,6 +31,7 @@ EXPORTS = (
     "favor_bwd",
     "favor_sync_status",
     "favor_status_string",
+    "favor_fwd_static_scratch",
 )
 
 
@@ -81,6 +82,8 @@ def library():
     lib.favor_sync_status.restype = I
     lib.favor_status_string.argtypes = [I]
     lib.favor_status_string.restype = ctypes.c_char_p
+    lib.favor_fwd_static_scratch.argtypes = [SP, P, P, P, P, P, P]
+    lib.favor_fwd_static_scratch.restype = I
     _LIB = lib
     return lib
 
@@ -213,3 +216,20 @@ def bwd(Q, K, V, W, out, dout, ctx=None, causal=False, workspace=None, opts=None
 def sync_status(stream=None):
     """Synchronise the stream and return (and clear) the device status word."""
     return library().favor_sync_status(_stream_ptr(stream))
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def fwd_static_scratch(Q, K, V, W, out=None, stream=None):
+    """Bidirectional bf16 forward through favor_fwd_static_scratch: no workspace is passed, the
+    library uses its own fixed device array (for callers that cannot allocate device memory)."""
+    torch = _torch()
+    _check_inputs((Q, K, V, W), Q)
+    shape = _shape_of(Q, W)
+    if out is None:
+        out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    st = library().favor_fwd_static_scratch(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(W), _ptr(out),
+                                            _stream_ptr(stream))
+    _check(st, "favor_fwd_static_scratch")
+    return out

@@ -294,3 +294,6 @@ extern "C" favor_status favor_sync_status(void *stream) {
     }
     return (favor_status)v;
 }
+
+// The no-allocation variant of the bidirectional forward (uses the definitions above).
+#include "favor_static.cu"
