@@ -140,7 +140,8 @@ FAVOR_API favor_status favor_fwd(const favor_shape *shape, const void *Q, const 
  * (Derived by the chain rule from the forward definition; the pages print no backward.)
  *
  *   Q, K, V, W   : as passed to favor_fwd
- *   out          : device, fp32 [B,H,L,d], the forward output
+ *   out          : device, fp32 [B,H,L,d], the forward output (validated; the kernels recompute
+ *                  out_i from the features and state they differentiate through)
  *   dout         : device, [B,H,L,d] in shape->dtype, upstream gradient
  *   ctx          : device, the context written by favor_fwd with the same inputs
  *   dQ, dK, dV   : device, fp32 [B,H,L,d]; fully written

@@ -266,6 +266,15 @@ __device__ __forceinline__ uint32_t elect_lane0() { return (threadIdx.x & 31u) =
 // same truncated value, so both sides carry the same rounding.
 __device__ __forceinline__ float tf32_trunc(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
 
+// Rounds an MMA operand to tf32 (nearest, ties away from zero): returns the value to store (the
+// bits plus half a tf32 ulp, which the tensor core's truncation turns into the rounded value) and
+// sets `used` to that rounded value for sums on CUDA cores that must match the MMA.
+__device__ __forceinline__ float tf32_round_store(float x, float &used) {
+    const uint32_t u = __float_as_uint(x) + 0x1000u;
+    used = __uint_as_float(u & 0xFFFFE000u);
+    return __uint_as_float(u);
+}
+
 // Stored form of an fp32 value in an MMA operand image: half a tf32 ulp added to the bit pattern,
 // so the hardware's truncation yields the value rounded to nearest (ties away). The exact fp32
 // value is recovered by subtracting the same integer.

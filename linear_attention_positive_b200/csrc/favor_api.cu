@@ -40,8 +40,8 @@ favor_status shape_supported(const favor_shape *s, int causal, int backward) {
         return FAVOR_OK;
     }
     if (s->m != 128 && s->m != 256) return FAVOR_ERR_UNSUPPORTED;
-    if (causal && s->d != 64) return FAVOR_ERR_UNSUPPORTED;
-    if (backward) return FAVOR_ERR_UNSUPPORTED;
+    if (causal && !backward && s->d != 64) return FAVOR_ERR_UNSUPPORTED;
+    if (backward && s->m > 512) return FAVOR_ERR_UNSUPPORTED;
     return FAVOR_OK;
 }
 
@@ -90,6 +90,13 @@ Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_
     if (causal) off += align256((size_t)2 * l.BH * l.P_exact * s->m * 4);
     l.total = off;
     return l;
+}
+
+// bf16 backward (current route): Q, K, V, dO and W widened to fp32, then the fp32 kernels.
+size_t bf16_bwd_bytes(const favor_shape *s) {
+    const size_t n = (size_t)s->B * s->H * s->L * s->d;
+    return 4 * align256(n * 4) + align256((size_t)s->m * s->d * 4) +
+           align256(f32_workspace_floats(s->B * s->H, s->L, s->d, s->m) * 4);
 }
 
 size_t ctx_bytes(const favor_shape *s) {
@@ -204,9 +211,9 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     e = launch_state_finalize(fp, l.BH, st);
     record_stage(o, 5, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-    QueryParams qp{s->L, s->d, s->m, opt_split_tiles(o), state, out};
+    QueryParams qp{s->L, s->d, s->m, l.BH, 0, state, out};
     record_stage(o, 6, st);
-    e = launch_query_out(mQ, mW, qp, l.BH, st);
+    e = launch_query_out(mQ, mW, qp, st);
     record_stage(o, 7, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     return FAVOR_OK;
@@ -233,6 +240,7 @@ extern "C" size_t favor_workspace_size(const favor_shape *s, int causal, int bac
     if (!shape_ok(s) || (causal != 0 && causal != 1)) return 0;
     if (shape_supported(s, causal, backward) != FAVOR_OK) return 0;
     if (s->dtype == FAVOR_F32) return align256(f32_workspace_floats(s->B * s->H, s->L, s->d, s->m) * 4);
+    if (backward) return bf16_bwd_bytes(s);
     return bf16_layout(s, o, true, causal).total;
 }
 
@@ -279,6 +287,26 @@ extern "C" favor_status favor_bwd(const favor_shape *s, const void *Q, const voi
     if (ws_bytes < favor_workspace_size(s, causal, 1, o)) return FAVOR_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     (void)ctx;
+    if (s->dtype == FAVOR_BF16) {
+        const size_t n = (size_t)s->B * s->H * s->L * s->d;
+        uint8_t *ws = (uint8_t *)workspace;
+        float *q = (float *)ws, *k = (float *)(ws + align256(n * 4)), *v = (float *)(ws + 2 * align256(n * 4));
+        float *g = (float *)(ws + 3 * align256(n * 4)), *w = (float *)(ws + 4 * align256(n * 4));
+        float *fws = (float *)(ws + 4 * align256(n * 4) + align256((size_t)s->m * s->d * 4));
+        const void *src[5] = {Q, K, V, dout, W};
+        float *dst[5] = {q, k, v, g, w};
+        for (int i = 0; i < 5; ++i) {
+            record_stage(o, 2 * i, st);
+            const cudaError_t e = launch_widen(src[i], dst[i], i == 4 ? (size_t)s->m * s->d : n, st);
+            record_stage(o, 2 * i + 1, st);
+            if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+        }
+        F32Params p{s->L, s->d, s->m, q, k, v, w, out, g, nullptr, dQ, dK, dV, fws};
+        record_stage(o, 10, st);
+        const cudaError_t e = launch_f32(p, s->B * s->H, causal != 0, true, st);
+        record_stage(o, 11, st);
+        return cuda_status(e);
+    }
     F32Params p{s->L, s->d, s->m, (const float *)Q, (const float *)K, (const float *)V, (const float *)W,
                 out, (const float *)dout, nullptr, dQ, dK, dV, (float *)workspace};
     return cuda_status(launch_f32(p, s->B * s->H, causal != 0, true, st));

@@ -29,28 +29,31 @@ struct ScanParams {
     float *seg_state;       // [BH, n_split, state_floats]: exclusive prefix per segment
 };
 
+// One thread per state element, walking the segments in order (grid: element blocks x heads).
 __global__ void __launch_bounds__(256) k_state_scan(ScanParams p) {
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.y;
     const size_t md = (size_t)p.m * p.d, sf = state_floats(p.m, p.d);
     float *base = p.seg_state + (size_t)bh * p.n_split * sf;
-    for (size_t i = threadIdx.x; i < md; i += blockDim.x) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < md) {
         const int r = (int)(i / p.d), c = (int)(i % p.d);
         const uint32_t off = state_image_offset(r, c, p.m);
+        const float *src = p.part_S + (size_t)bh * p.n_split * md + i;
         float run = 0.f;
         for (int s = 0; s < p.n_split; ++s) {
             *(float *)((uint8_t *)(base + (size_t)s * sf) + off) = tf32_store(run);
-            run += p.part_S[((size_t)bh * p.n_split + s) * md + i];
+            run += src[(size_t)s * md];
         }
-    }
-    for (int r = threadIdx.x; r < p.m; r += blockDim.x) {
+    } else if (i < md + p.m) {
+        const int r = (int)(i - md);
+        const float *src = p.part_z + (size_t)bh * p.n_split * p.m + r;
         float run = 0.f;
         for (int s = 0; s < p.n_split; ++s) {
             base[(size_t)s * sf + md + r] = run;
-            run += p.part_z[((size_t)bh * p.n_split + s) * p.m + r];
+            run += src[(size_t)s * p.m];
         }
-    }
-    if (threadIdx.x < p.n_split) {
-        float *t = base + (size_t)threadIdx.x * sf + md + p.m;
+    } else if (i < md + p.m + p.n_split) {
+        float *t = base + (i - md - p.m) * sf + md + p.m;
         t[0] = p.head_max[bh];
         t[1] = t[2] = t[3] = 0.f;
     }
@@ -355,8 +358,9 @@ k_causal_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
                     const float *z = sZ + h * 128 + c0;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        v[e] = ex2_approx(fmaf(v[e], kLog2e, -cl));
-                        den = fmaf(tf32_trunc(v[e]), z[e], den);
+                        float used;
+                        v[e] = tf32_round_store(ex2_approx(fmaf(v[e], kLog2e, -cl)), used);
+                        den = fmaf(used, z[e], den);
                     }
                     tmem_st32(ta, v);
                 }
@@ -371,8 +375,9 @@ k_causal_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
                     tmem_ld32(ta, v);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        v[e] = ex2_approx(fmaf(v[e], kLog2e, sBB[c0 + e]));
-                        zs += tf32_trunc(v[e]);
+                        float used;
+                        v[e] = tf32_round_store(ex2_approx(fmaf(v[e], kLog2e, sBB[c0 + e])), used);
+                        zs += used;
                     }
                     tmem_st32(ta, v);
                 }
@@ -465,8 +470,9 @@ k_causal_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ C
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int kj = c0 + e;
-                    v[e] = (kj <= qi && j0 + kj < p.L) ? v[e] : 0.f;
-                    rs += tf32_trunc(v[e]);
+                    float used;
+                    v[e] = tf32_round_store((kj <= qi && j0 + kj < p.L) ? v[e] : 0.f, used);
+                    rs += used;
                 }
                 tmem_st32(ta, v);
             }
@@ -526,7 +532,8 @@ static size_t causal_smem() {
 }
 
 cudaError_t launch_state_scan(const ScanParams &p, int BH, cudaStream_t st) {
-    k_state_scan<<<BH, 256, 0, st>>>(p);
+    const size_t n = (size_t)p.m * p.d + p.m + p.n_split;
+    k_state_scan<<<dim3((unsigned)((n + 255) / 256), BH), 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kF32Threads) k_f32_head(F32Params p) {
     }
 
     // ---------------------------------------------------------------- backward
-    const float *O = p.out + off, *dO = p.dout + off;
+    const float *dO = p.dout + off;
     if (!CAUSAL)
         for (int j = 0; j < L; ++j) add_key(j);
     // Query pass (forward order): dq_i, and g_i, s_i, c_i saved for the G, h sums.
@@ -154,11 +154,16 @@ __global__ void __launch_bounds__(kF32Threads) k_f32_head(F32Params p) {
         if (CAUSAL) add_key(i);
         const float den = query_features(i);
         const float c = red[31];
+        // s_i uses out_i recomputed from the same features and state the gradient runs through
+        // (a caller's output from a lower-precision forward would break the cancellation
+        // sum_r phi(q)_r dphi(q)_r = 0 that the query gradient relies on).
         float sp = 0.f;
         for (int e = tid; e < d; e += blockDim.x) {
+            float num = 0.f;
+            for (int r = 0; r < m; ++r) num = fmaf(ph[r], S[(size_t)r * d + e], num);
             const float go = dO[(size_t)i * d + e];
             g[e] = go / den;
-            sp = fmaf(go, O[(size_t)i * d + e], sp);
+            sp = fmaf(go, num / den, sp);
         }
         const float s = -block_reduce_sum(sp, red) / den;
         float ysum = 0.f;
@@ -230,6 +235,17 @@ __global__ void __launch_bounds__(kF32Threads) k_f32_head(F32Params p) {
         }
         __syncthreads();
     }
+}
+
+// bf16 -> fp32 widening (exact), for running bf16 operands through the fp32 kernels.
+__global__ void k_widen_bf16(const uint16_t *__restrict__ src, float *__restrict__ dst, size_t n) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        dst[i] = __uint_as_float((uint32_t)src[i] << 16);
+}
+
+cudaError_t launch_widen(const void *src, float *dst, size_t n, cudaStream_t st) {
+    k_widen_bf16<<<592, 256, 0, st>>>((const uint16_t *)src, dst, n);
+    return cudaGetLastError();
 }
 
 size_t f32_workspace_floats(int BH, int L, int d, int m) {

@@ -393,9 +393,9 @@ k_key_state(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CU
                     tmem_ld32(ta, v);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const float ph = ex2_approx(fmaf(v[e], kLog2e, bb[c0 + e]));
-                        zsum += tf32_trunc(ph);
-                        v[e] = ph;
+                        float used;
+                        v[e] = tf32_round_store(ex2_approx(fmaf(v[e], kLog2e, bb[c0 + e])), used);
+                        zsum += used;
                     }
                     tmem_st32(ta, v);
                 }

@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 
 from linear_attention_positive_b200 import api
-from linear_attention_positive_b200.inputs import WORKLOADS, Workload, make_inputs
+from linear_attention_positive_b200.inputs import WORKLOADS, Workload, make_inputs, round_to_bf16
 from oracle import favor
 from tests.helpers import features_for, rel_max_err, to_torch
 
@@ -87,6 +87,9 @@ def test_bf16_stabilisers_handle_large_logits(cuda_device):
     x = make_inputs(w)
     x["K"][0, 0, 100] *= 12.0
     x["Q"][0, 0, 7] *= 12.0
+    # keep the inputs exactly representable in bf16, so kernel and oracle read the same values
+    x["K"] = round_to_bf16(x["K"])
+    x["Q"] = round_to_bf16(x["Q"])
     Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
     out = run_fwd(w, x, Wr, cuda_device, False)
     assert np.isfinite(out).all()
@@ -158,33 +161,31 @@ def test_bf16_causal_config3_prefix_slice_against_brute_force(cuda_device):
             ref, _ = favor.attention_brute(X["Q"], X["K"], X["V"], W64, causal=True)
             errs.append(np.abs(out[b, h, :512] - ref).max())
             refs.append(ref)
-    # RMS of the whole output (linear-form oracle on two heads) sets the scale of the bound.
-    full = [favor.fwd_causal(*(x[k][0, h].astype(np.float64) for k in "QKV"), W64) for h in range(2)]
-    rms = np.sqrt(np.mean(np.concatenate(full) ** 2))
+    # every row of every head against the linear-form (prefix-sum) oracle, which also sets RMS(out)
+    full_err, sq = [], 0.0
+    for b in range(w.B):
+        for h in range(w.H):
+            ref = favor.fwd_causal(*(x[k][b, h].astype(np.float64) for k in "QKV"), W64)
+            full_err.append(np.abs(out[b, h] - ref).max())
+            sq += float(np.sum(ref * ref))
+    rms = np.sqrt(sq / (w.B * w.H * w.L * w.d))
     assert max(errs) / rms <= TOL["bf16"]
-    # and the rest of the sequence on the two heads
-    for h in range(2):
-        assert np.abs(out[0, h] - full[h]).max() / rms <= TOL["bf16"]
+    assert max(full_err) / rms <= TOL["bf16"]
 
 
-def test_bf16_causal_config4_full_size_sampled_rows(cuda_device):
+def test_bf16_causal_config4_full_size_all_rows(cuda_device):
     """Long causal workload (B=1, H=16, L=65536, rotated 0.5-scaled inputs) in the benchmark's
-    launch configuration; per head 40 sampled rows including the first, the last and the
-    exact-prefix boundary."""
+    launch configuration, every row of every head against the fp64 prefix-sum oracle. (Rows just
+    past the exact fp32 prefix carry the largest errors: there |out| is still ~40x RMS(out).)"""
     w = WORKLOADS[4]
     x = make_inputs(w)
     Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
     out = run_fwd(w, x, Wr, cuda_device, True)
     assert np.isfinite(out).all()
-    rng = np.random.default_rng(1)
-    errs, refs = [], []
+    errs, sq = [], 0.0
     for h in range(w.H):
-        rows = np.unique(np.concatenate([[0, 1, 127, 128, 511, 512, 513, w.L - 1], rng.integers(0, w.L, 32)]))
-        X = {k: x[k][0, h].astype(np.float64) for k in "QKV"}
-        ref = favor.fwd_causal_rows(X["Q"], X["K"], X["V"], W64, rows)
-        errs.append(np.abs(out[0, h, rows] - ref).max())
-        refs.append(ref)
-    # RMS(out) from the full oracle output of one head (sampled rows over-weight the first rows)
-    full = favor.fwd_causal(*(x[k][0, 0].astype(np.float64) for k in "QKV"), W64)
-    rms = np.sqrt(np.mean(full ** 2))
+        ref = favor.fwd_causal(*(x[k][0, h].astype(np.float64) for k in "QKV"), W64)
+        errs.append(np.abs(out[0, h] - ref).max())
+        sq += float(np.sum(ref * ref))
+    rms = np.sqrt(sq / (w.H * w.L * w.d))
     assert max(errs) / rms <= TOL["bf16"]
