@@ -19,8 +19,8 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -35,7 +35,7 @@ TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor rate
 L2_FLUSH_BYTES = 256 << 20
 
 # Kernels favor_fwd launches for the bf16 path, in launch order (stage k <-> events 2k, 2k+1).
-FWD_STAGES = ["k_key_logit_max", "k_key_state", "k_state_finalize", "k_query_out"]
+FWD_STAGES = ["k_key_max", "k_key_partials", "k_state_image", "k_query_out"]
 CAUSAL_STAGES = ["k_key_logit_max", "k_key_state", "k_state_scan", "k_causal_out", "k_causal_prefix"]
 
 
@@ -48,21 +48,25 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def stage_work(name, w):
-    """Algorithmic HBM bytes and tensor FLOPs (bf16, tf32) of one launch of a stage."""
+def stage_work(name, w, n_sms=148):
+    """Algorithmic HBM bytes and tensor FLOPs (bf16/fp16 rate, tf32 rate) of one launch of a stage."""
     t, d, m = w.tokens, w.d, w.m
+    BH = w.B * w.H
+    if name == "k_key_max":            # read K
+        return t * 2 * d, 2 * m * d * t, 0
+    if name == "k_key_partials":       # read K, V; MMAs K W^T and phi'(K)^T [V | 1]
+        return t * 4 * d, 2 * m * d * t + 2 * m * (d + 1) * t, 0
+    if name == "k_state_image":        # read the per-run partial states, write the fp16 images
+        runs = n_sms + BH - 1
+        return runs * (d + 1) * m * 4 + BH * (d // 64) * (m // 128) * 20480, 0, 0
+    if name == "k_query_out":          # read Q; write fp32 out; MMAs Q W^T and phi(Q) [S | z]
+        return t * (2 * d + 4 * d), 2 * m * d * t + 2 * m * (d + 1) * t, 0
     if name == "k_key_logit_max":      # read K; write -|k|^2/2
         return t * (2 * d + 4), 2 * m * d * t, 0
     if name == "k_key_state":          # read K, V, -|k|^2/2
         return t * (4 * d + 4), 2 * m * d * t, 2 * m * d * t
-    if name == "k_query_out":          # read Q; write fp32 out
-        return t * (2 * d + 4 * d), 2 * m * d * t, 2 * m * d * t
     if name == "k_causal_out":         # read Q, K, V, -|k|^2/2; write fp32 out
         return t * (10 * d + 4), 6 * m * d * t, (4 * m * d + 2 * 128 * m + 2 * 128 * d) * t
-    if name == "k_state_finalize":
-        BH = w.B * w.H
-        n_split = -(-(-(-w.L // 128)) // 8)
-        return BH * n_split * m * (d + 1) * 4 + BH * m * (d + 1) * 4, 0, 0
     return 0, 0, 0
 
 
@@ -88,56 +92,58 @@ def measured_traffic(kernel, workload_name):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled every ~0.5 ms through NVML while the timed
+    region runs (a background thread; the timed steps themselves take a few milliseconds)."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"favor_clocks_{os.getpid()}.csv")
+    def __init__(self, device):
+        self.device = device
+        self.samples = []
+        self.thread = None
+        self.stop_flag = threading.Event()
+
+    def _handle(self, pynvml):
+        try:
+            p = torch.cuda.get_device_properties(self.device)
+            bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.device)
+
+    def _run(self, pynvml, h):
+        while not self.stop_flag.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, mx, rs))
+            except Exception:
+                return
+            time.sleep(0.0005)
 
     def start(self):
         try:
-            self.out = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            h = self._handle(pynvml)
         except Exception:
-            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._run, args=(pynvml, h), daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.out.close()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
-        os.remove(self.path)
-        if not sm:
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        if not self.samples:
             return None
-        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sm = [a for a, _, _ in self.samples]
+        loaded = [x for x in sm if x > 0.5 * max(sm)] or sm
+        reasons = sorted({name for _, _, r in self.samples for bit, name in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(m for _, m, _ in self.samples),
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
 
 # ------------------------------------------------------------------------------------ oracle arm
@@ -263,18 +269,19 @@ def run_ours(args, w):
         if w.backward:
             api.bwd(T["Q"], T["K"], T["V"], Wt, out, T["dO"], ctx=ctx, causal=w.causal, workspace=ws)
 
+    base_opts = api.make_opts(exp_poly_pct=args.exp_poly_pct)
     for _ in range(args.warmup):
         flush.zero_()
-        step()
+        step(base_opts)
     torch.cuda.synchronize()
     if api.sync_status() != api.FAVOR_OK:
         raise RuntimeError("device status not OK after warm-up")
 
     step_ev = [new_events(2) for _ in range(args.steps)]
     stage_ev = [new_events(2 * api.FAVOR_MAX_STAGES) for _ in range(args.steps)]
-    opts = [api.make_opts(stage_events=stage_ev[k]) for k in range(args.steps)]
+    opts = [api.make_opts(exp_poly_pct=args.exp_poly_pct, stage_events=stage_ev[k]) for k in range(args.steps)]
     torch.cuda.synchronize()
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev.index if dev.index is not None else local)
     clocks.start()
     if world > 1:
         dist.barrier()
@@ -313,7 +320,7 @@ def run_ours(args, w):
         e2e_ev[k][0].record(stream)
         for name in dT:
             dT[name].copy_(pin[name], non_blocking=True)
-        api.fwd(dT["Q"], dT["K"], dT["V"], Wt, causal=w.causal, out=out, ctx=ctx, workspace=ws)
+        api.fwd(dT["Q"], dT["K"], dT["V"], Wt, causal=w.causal, out=out, ctx=ctx, workspace=ws, opts=base_opts)
         if w.backward:
             dq, dk, dv = api.bwd(dT["Q"], dT["K"], dT["V"], Wt, out, dT["dO"], ctx=ctx, causal=w.causal, workspace=ws)
         out_h.copy_(out, non_blocking=True)
@@ -344,7 +351,7 @@ def run_ours(args, w):
         avg = {stages[i]: statistics.mean(stage_ms[i]) for i in range(n_stage)}
         line["stage_ms"] = {k: round(v, 5) for k, v in avg.items()}
         dom = max(avg, key=avg.get)
-        nbytes, f_bf16, f_tf32 = stage_work(dom, w)
+        nbytes, f_bf16, f_tf32 = stage_work(dom, w, torch.cuda.get_device_properties(dev).multi_processor_count)
         sec = avg[dom] * 1e-3
         hbm_peak = peaks["hbm_gbs"]
         tc_peak = peaks["bf16_tflops"]
@@ -366,7 +373,7 @@ def run_ours(args, w):
                                  "hbm_frac": path_bytes / (ms_per_step * 1e-3) / (hbm_peak * 1e9)}
     if clk is not None:
         line["clocks"] = clk
-    if world == 1:
+    if world == 1 and not args.no_cpu_baseline:
         try:
             W64 = (round_to_bf16(Wf) if w.dtype == "bf16" else Wf).astype(np.float64)
             n_heads = pick_sample(w, x, W64, budget_s=15.0)
@@ -387,6 +394,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", type=int, default=2, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--exp-poly-pct", type=int, default=0,
+                    help="percent of feature exponentials on the FMA-pipe polynomial (0: library default)")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle sample after the timed region (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -87,6 +87,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// mbar_wait for all lanes of a converged warp, with a warp-uniform result.
+__device__ __forceinline__ bool mbar_wait_all(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
 // -------------------------------------------------------------------------------- TMA / bulk copy
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
@@ -145,6 +150,50 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d, uint64_t a, uint64_t b, u
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]; kind::f16 with fp16 operands (A packed two per TMEM column,
+// the lower K index in the low half), fp32 accumulation.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// Chains of kind::f16 MMAs issued from one asm block, so the issuing thread spends a few
+// instructions per MMA. Descriptors advance by a fixed number of 16-byte units per K-step of 16
+// (the start-address field is the descriptor's low bits; no step crosses its range).
+// D (+)= sum_k A_k B_k with A and B in shared memory: 4 K-steps, A/B advancing by a_step/b_step.
+__device__ __forceinline__ void mma_ss_x4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                          uint32_t a_step, uint32_t b_step) {
+    const uint64_t a1 = a + a_step, b1 = b + b_step, a2 = a1 + a_step, b2 = b1 + b_step, a3 = a2 + a_step,
+                   b3 = b2 + b_step;
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\tsetp.ne.b32 p, %9, 0;\n\tsetp.eq.b32 t, %9, %9;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %8, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %8, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %8, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %10, %8, t;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "l"(a1), "l"(b1), "l"(a2), "l"(b2), "l"(a3), "r"(idesc), "r"(acc), "l"(b3)
+        : "memory");
+}
+
+// D (+)= sum_k A_k B_k with A in TMEM (8 columns per K-step of 16 fp16) and B in shared memory:
+// 4 K-steps, B advancing by b_step.
+__device__ __forceinline__ void mma_ts_x4(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc,
+                                          uint32_t b_step) {
+    const uint64_t b1 = b + b_step, b2 = b1 + b_step, b3 = b2 + b_step;
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\tsetp.ne.b32 p, %6, 0;\n\tsetp.eq.b32 t, %6, %6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %5, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %3, %5, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %4, %5, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%9], %10, %5, t;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "l"(b1), "l"(b2), "r"(idesc), "r"(acc), "r"(a_tmem + 8), "r"(a_tmem + 16),
+        "r"(a_tmem + 24), "l"(b3)
+        : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]; kind::tf32, fp32 accumulation.
 __device__ __forceinline__ void mma_tf32_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
@@ -175,6 +224,7 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N, uint32_t fmt, ui
     return (1u << 4) | (fmt << 7) | (fmt << 10) | (a_mn << 15) | (b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
 }
+constexpr uint32_t kFmtF16 = 0;
 constexpr uint32_t kFmtBF16 = 1;
 constexpr uint32_t kFmtTF32 = 2;
 
@@ -237,6 +287,123 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Stores columns [OFF, OFF + 32) of a 128-value register row to 32 consecutive TMEM columns
+// (compile-time offset, so the row stays in registers).
+template <int OFF>
+__device__ __forceinline__ void tmem_st32_at(uint32_t taddr, const float (&v)[128]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "f"(v[OFF + 0]), "f"(v[OFF + 1]), "f"(v[OFF + 2]), "f"(v[OFF + 3]), "f"(v[OFF + 4]), "f"(v[OFF + 5]),
+        "f"(v[OFF + 6]), "f"(v[OFF + 7]), "f"(v[OFF + 8]), "f"(v[OFF + 9]), "f"(v[OFF + 10]), "f"(v[OFF + 11]),
+        "f"(v[OFF + 12]), "f"(v[OFF + 13]), "f"(v[OFF + 14]), "f"(v[OFF + 15]), "f"(v[OFF + 16]), "f"(v[OFF + 17]),
+        "f"(v[OFF + 18]), "f"(v[OFF + 19]), "f"(v[OFF + 20]), "f"(v[OFF + 21]), "f"(v[OFF + 22]), "f"(v[OFF + 23]),
+        "f"(v[OFF + 24]), "f"(v[OFF + 25]), "f"(v[OFF + 26]), "f"(v[OFF + 27]), "f"(v[OFF + 28]), "f"(v[OFF + 29]),
+        "f"(v[OFF + 30]), "f"(v[OFF + 31])
+        : "memory");
+}
+
+#define FAVOR_REG128(v) FAVOR_REG32((&v[0])), FAVOR_REG32((&v[32])), FAVOR_REG32((&v[64])), FAVOR_REG32((&v[96]))
+
+// Loads 128 consecutive fp32 columns of this thread's TMEM lane (two 64-column loads, so that no
+// single instruction needs more than 64 destination registers) and waits for them.
+#define FAVOR_REG64(v) FAVOR_REG32((&v[0])), FAVOR_REG32((&v[32]))
+__device__ __forceinline__ void tmem_ld64_nowait(uint32_t taddr, float *v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+        "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, "
+        "%51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+        : FAVOR_REG64(v)
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
+    tmem_ld64_nowait(taddr, &v[0]);
+    tmem_ld64_nowait(taddr + 64, &v[64]);
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&v[0])), FAVOR_RW32((&v[32])), FAVOR_RW32((&v[64])),
+                 FAVOR_RW32((&v[96]))::"memory");
+}
+
+// Loads one fp32 column of this thread's TMEM lane and waits for it.
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+    float v;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=f"(v) : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+f"(v)::"memory");
+    return v;
+}
+
+#define FAVOR_U16(h, o)                                                                                        \
+    "r"(h[o + 0]), "r"(h[o + 1]), "r"(h[o + 2]), "r"(h[o + 3]), "r"(h[o + 4]), "r"(h[o + 5]), "r"(h[o + 6]),   \
+        "r"(h[o + 7]), "r"(h[o + 8]), "r"(h[o + 9]), "r"(h[o + 10]), "r"(h[o + 11]), "r"(h[o + 12]),           \
+        "r"(h[o + 13]), "r"(h[o + 14]), "r"(h[o + 15])
+
+// Stores 64 consecutive 32-bit columns of this thread's TMEM lane (warp-collective; not waited).
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&h)[64]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, "
+        "%35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, "
+        "%56, %57, %58, %59, %60, %61, %62, %63, %64};" ::"r"(taddr),
+        FAVOR_U16(h, 0), FAVOR_U16(h, 16), FAVOR_U16(h, 32), FAVOR_U16(h, 48)
+        : "memory");
+}
+
+// Two fp32 values rounded to fp16 (nearest even) and packed, `lo` in the low 16 bits.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// {a0, a1} * {b0, b1} + {c0, c1} on the FMA pipe as one paired instruction.
+__device__ __forceinline__ void ffma2(float a0, float a1, float b0, float b1, float c0, float c1, float &r0,
+                                      float &r1) {
+    uint64_t a, b, c, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(c0), "f"(c1));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
+}
+
+// Non-blocking test of an mbarrier phase (true once the phase with this parity has completed).
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Tiled TMA store shared -> global (bulk async-group completion).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until at most N committed bulk groups of this thread still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Waits until every committed bulk group of this thread has completed.
+__device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Per-warpgroup register budget changes (all four warps of a warpgroup execute the same one).
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // TMEM address of (lane quarter of this warp, column).
 __device__ __forceinline__ uint32_t tmem_lane_addr(uint32_t base, uint32_t warp_idx, uint32_t col) {
     return base + (((warp_idx & 3u) * 32u) << 16) + col;
@@ -260,6 +427,43 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 __device__ __forceinline__ uint32_t elect_lane0() { return (threadIdx.x & 31u) == 0u; }
+
+// One lane of a converged warp (elect.sync): the warp runs a producer loop together, so its
+// descriptor arithmetic stays warp-uniform, and the elected lane issues the TMA / MMA instruction.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r));
+    return r != 0;
+}
+
+// 2^t for a pair of values on the FMA pipe (no MUFU), t <= 0: Cody-Waite split t = n + f with
+// n = round(t) taken from the low bits of t + 1.5*2^23, |f| <= 1/2, a degree-3 polynomial for 2^f
+// (this library's own relative-minimax fit on [-1/2, 1/2], max relative error 7.5e-5, below the
+// 2^-12 tf32 rounding applied afterwards) and n added to the exponent field. t is clamped at -126
+// (results below 2^-126 come out as ~2^-126 instead of 0).
+__device__ __forceinline__ void exp2_poly_pair(float t0, float t1, float &r0, float &r1) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    t0 = fmaxf(t0, -126.0f);
+    t1 = fmaxf(t1, -126.0f);
+    uint64_t t, j, n, f, p;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(t) : "f"(t0), "f"(t1));
+    const uint64_t sh = 0x4B4000004B400000ull, nsh = 0xCB400000CB400000ull;   // {kShift}, {-kShift}
+    const uint64_t m1 = 0xBF800000BF800000ull;                                   // {-1}
+    const uint64_t c3 = 0x3D61FBAF3D61FBAFull, c2 = 0x3E786F0D3E786F0Dull;      // 2^f ~ c0 + f(c1 + f(c2 + f c3))
+    const uint64_t c1 = 0x3F31798D3F31798Dull, c0 = 0x3F7FFB493F7FFB49ull;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(j) : "l"(t), "l"(sh));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(n) : "l"(j), "l"(nsh));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(f) : "l"(n), "l"(m1), "l"(t));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(c3), "l"(f), "l"(c2));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c1));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c0));
+    const uint32_t j0 = (uint32_t)j, j1 = (uint32_t)(j >> 32);
+    const uint32_t p0 = (uint32_t)p, p1 = (uint32_t)(p >> 32);
+    r0 = __uint_as_float(p0 + (j0 << 23));
+    r1 = __uint_as_float(p1 + (j1 << 23));
+}
 
 // The tensor core reads a tf32 operand as the fp32 value with its low 13 mantissa bits dropped
 // (truncation). Sums taken on CUDA cores that must agree with an MMA over the same operand use the

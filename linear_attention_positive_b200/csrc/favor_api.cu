@@ -15,6 +15,7 @@
 
 #include "k_fp32.cu"
 #include "k_keys.cu"
+#include "k_keys_bidir.cu"
 #include "k_query.cu"
 #include "k_causal.cu"
 
@@ -46,6 +47,12 @@ favor_status shape_supported(const favor_shape *s, int causal, int backward) {
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Share of feature exponentials on the FMA-pipe polynomial (percent); 0 takes the default.
+int opt_poly_pct(const favor_opts *o) {
+    const int v = o ? o->exp_poly_pct : 0;
+    return v > 0 ? std::min(v, 100) : 37;
+}
 
 int opt_split_tiles(const favor_opts *o) {
     const int v = o ? o->split_tiles : 0;
@@ -92,6 +99,33 @@ Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_
     return l;
 }
 
+// Bidirectional bf16 forward: per-run key maxima, per-run partial states [S | z] (feature-major
+// columns), their largest magnitudes, and the per-head fp16 state images (unless a ctx holds them).
+struct BidirLayout {
+    Flat f_max, f;  // 128-token tiles of k_key_max, 64-token tiles of k_key_partials
+    int BH;
+    size_t off_run_max, off_part, off_amax, off_state, total;
+};
+
+BidirLayout bidir_layout(const favor_shape *s, bool state_in_ws) {
+    BidirLayout l{};
+    l.BH = s->B * s->H;
+    l.f_max = make_flat(l.BH, s->L, num_sms(), kTile);
+    l.f = make_flat(l.BH, s->L, num_sms(), kKeyTile);
+    const size_t slots = (size_t)flat_slots(l.f, l.BH);
+    size_t off = 0;
+    l.off_run_max = off;
+    off += align256((size_t)flat_slots(l.f_max, l.BH) * 8 * 4);
+    l.off_part = off;
+    off += align256(slots * (s->d + 1) * s->m * 4);
+    l.off_amax = off;
+    off += align256(slots * 8 * 4);
+    l.off_state = off;
+    if (state_in_ws) off += align256((size_t)l.BH * state_floats(s->m, s->d) * 4);
+    l.total = off;
+    return l;
+}
+
 // bf16 backward (current route): Q, K, V, dO and W widened to fp32, then the fp32 kernels.
 size_t bf16_bwd_bytes(const favor_shape *s) {
     const size_t n = (size_t)s->B * s->H * s->L * s->d;
@@ -121,14 +155,14 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [BH, L, d] bf16 tensor as a 3-D map (d, L, BH) with 64 x 128 x 1 boxes, 128-byte swizzle;
+// [BH, L, d] bf16 tensor as a 3-D map (d, L, BH) with 64 x rows x 1 boxes, 128-byte swizzle;
 // rows past L read as zeros.
-bool make_token_map(CUtensorMap *map, const void *base, int BH, int L, int d) {
+bool make_token_map(CUtensorMap *map, const void *base, int BH, int L, int d, int rows = kTile) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)BH};
     const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)L * d * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+    const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -148,6 +182,20 @@ bool make_w_map(CUtensorMap *map, const void *base, int m, int d) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 [BH, L, d] output as a 3-D map (d, L, BH) with 32 x 32 x 1 boxes, 128-byte swizzle (the
+// staging layout of the output epilogue); rows past L are not written.
+bool make_out_map(CUtensorMap *map, void *base, int BH, int L, int d) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)L * d * 4};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 favor_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA; }
 
 // Records the caller's timing event (2k before / 2k+1 after launch k), if one was supplied.
@@ -158,8 +206,46 @@ void record_stage(const favor_opts *o, int slot, cudaStream_t st) {
 
 // ---------------------------------------------------------------------------- bf16 forward
 
+favor_status fwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W,
+                            float *out, void *ctx, uint8_t *ws, size_t ws_bytes, const favor_opts *o, cudaStream_t st) {
+    const BidirLayout l = bidir_layout(s, ctx == nullptr);
+    if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
+    CUtensorMap mQ, mK, mK64, mV64, mW, mO;
+    if (!make_token_map(&mQ, Q, l.BH, s->L, s->d) || !make_token_map(&mK, K, l.BH, s->L, s->d) ||
+        !make_token_map(&mK64, K, l.BH, s->L, s->d, kKeyTile) || !make_token_map(&mV64, V, l.BH, s->L, s->d, kKeyTile) ||
+        !make_w_map(&mW, W, s->m, s->d) || !make_out_map(&mO, out, l.BH, s->L, s->d))
+        return FAVOR_ERR_CUDA;
+    float *run_max = (float *)(ws + l.off_run_max);
+    float *part = (float *)(ws + l.off_part);
+    float *amax = (float *)(ws + l.off_amax);
+    uint8_t *state = ctx ? (uint8_t *)ctx : ws + l.off_state;
+    const size_t stride = state_floats(s->m, s->d) * 4;
+
+    KeyMaxParams2 km{s->L, s->m, l.f_max, run_max};
+    record_stage(o, 0, st);
+    cudaError_t e = launch_key_max(mK, mW, km, s->d, st);
+    record_stage(o, 1, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    KeyStateParams2 ks{s->L, s->m, l.f, l.f_max, run_max, part, amax};
+    record_stage(o, 2, st);
+    e = launch_key_partials(mK64, mV64, mW, ks, s->d, opt_poly_pct(o), st);
+    record_stage(o, 3, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    ImageParams ip{s->m, s->d, l.f, part, amax, state, stride};
+    record_stage(o, 4, st);
+    e = launch_state_image(ip, l.BH, st);
+    record_stage(o, 5, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    QueryParams qp{s->L, s->d, s->m, l.BH, 0, state, stride};
+    record_stage(o, 6, st);
+    e = launch_query_out(mQ, mW, mO, qp, opt_poly_pct(o), st);
+    record_stage(o, 7, st);
+    return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
 favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W, float *out,
                       void *ctx, uint8_t *ws, size_t ws_bytes, const favor_opts *o, cudaStream_t st, int causal) {
+    if (!causal) return fwd_bf16_bidir(s, Q, K, V, W, out, ctx, ws, ws_bytes, o, st);
     const Bf16Layout l = bf16_layout(s, o, ctx == nullptr, causal);
     if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
     CUtensorMap mQ, mK, mW;
@@ -206,17 +292,7 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
         record_stage(o, 9, st);
         return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
     }
-    FinalizeParams fp{s->m, s->d, l.n_split, part_S, part_z, head_max, state};
-    record_stage(o, 4, st);
-    e = launch_state_finalize(fp, l.BH, st);
-    record_stage(o, 5, st);
-    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-    QueryParams qp{s->L, s->d, s->m, l.BH, 0, state, out};
-    record_stage(o, 6, st);
-    e = launch_query_out(mQ, mW, qp, st);
-    record_stage(o, 7, st);
-    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-    return FAVOR_OK;
+    return FAVOR_ERR_INVALID_ARG;
 }
 
 }  // namespace
@@ -241,6 +317,7 @@ extern "C" size_t favor_workspace_size(const favor_shape *s, int causal, int bac
     if (shape_supported(s, causal, backward) != FAVOR_OK) return 0;
     if (s->dtype == FAVOR_F32) return align256(f32_workspace_floats(s->B * s->H, s->L, s->d, s->m) * 4);
     if (backward) return bf16_bwd_bytes(s);
+    if (!causal) return bidir_layout(s, true).total;
     return bf16_layout(s, o, true, causal).total;
 }
 

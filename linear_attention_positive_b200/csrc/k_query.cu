@@ -1,15 +1,21 @@
-// Bidirectional state finalisation and query-side output of the bf16 tensor-core path.
+// Bidirectional state image and query-side output of the bf16 tensor-core path.
 //
-//   k_state_finalize : sums the per-split partial states in split order into the per-head
-//                      state [S | z] = (K')^T [V | 1_L] and writes it in the layout the output MMA
-//                      reads (tf32, K-major, 128-byte swizzled), plus z and the key stabiliser C.
-//   k_query_out      : out = D^-1 (Q' S), D = diag(Q' z) ("Fast Attention Via Positive Orthogonal
-//                      Random Features", codewithpapers.app/method/favor, the FA-part and its
-//                      normaliser), with Q' = exp(Q W^T - rowmax) formed in TMEM.
+//   k_state_image : sums the per-run partial states in run order into the per-head state
+//                   [S | z] = (K')^T [V | 1_L], scales it by a power of two so that its largest
+//                   magnitude lies in [2^14, 2^15), and writes it as fp16 in the layout the output
+//                   MMA reads (the scale cancels between numerator and denominator).
+//   k_query_out   : out = D^-1 (Q' S), D = diag(Q' z) ("Fast Attention Via Positive Orthogonal
+//                   Random Features", codewithpapers.app/method/favor, the FA-part and its
+//                   normaliser), with Q' = exp(Q W^T - rowmax) formed in TMEM and z riding along
+//                   as one more column of the output MMA.
 //
-// Per-head state block (floats): [ image (m*d) | z (m) | C, 0, 0, 0 ]. The image holds S[r, c]
-// (in the tf32_store form) at  (c/64)*(m*64*4) + (r/32)*(64*128) + swizzle128(row c%64, chunk (r%32)/4) + (r%4)*4  bytes:
-// for each half of the value columns, m/32 blocks of 64 rows x 128 bytes.
+// State image of one head (fp16, B operand of the output MMA, K-major, 128-byte swizzle): for each
+// value half nh (64 columns of d) and feature half h (128 features), two k-blocks of 64 features,
+// each 80 rows x 128 bytes: row n < 64 holds S[., nh*64 + n], row 64 holds z, rows 65..79 are zero.
+// Byte offset of (nh, h, kb, row n, 16-byte chunk p) = (((nh*H + h)*2 + kb)*80 + n)*128 + p*16,
+// and chunk p holds features kb*64 + 8*(p ^ (n & 7)) + [0, 8) of the half.
+//
+// The causal path keeps the fp32 per-segment state blocks below (state_floats, state_image_offset).
 
 #include "common.cuh"
 
@@ -22,101 +28,184 @@ __device__ __forceinline__ uint32_t state_image_offset(int r, int c, int m) {
     return (uint32_t)nh * (m * 64 * 4) + (uint32_t)kb * (64 * 128) + sw128_offset(cc, ch) + pos * 4;
 }
 
-struct FinalizeParams {
-    int m, d, n_split;
-    const float *part_S;     // [BH, n_split, m, d]
-    const float *part_z;     // [BH, n_split, m]
-    const float *head_max;   // [BH]
-    float *state;            // [BH, state_floats]
+constexpr int kImgRows = 80;                          // 64 value columns + z + 15 zero rows
+constexpr uint32_t kImgKBlock = kImgRows * 128;       // bytes of one 64-feature k-block
+constexpr uint32_t kImgHalf = 2 * kImgKBlock;         // bytes of one 128-feature half
+
+// Bytes of one head's image (all value halves and feature halves).
+__host__ __device__ inline size_t image_bytes(int m, int d) { return (size_t)(d / 64) * (m / 128) * kImgHalf; }
+
+// ============================================================================ k_state_image
+
+struct ImageParams {
+    int m, d;
+    Flat f;                  // partition of the key tiles (runs and their slots)
+    const float *part;       // [slots][d+1][m]
+    const float *part_amax;  // [slots][8]
+    uint8_t *image;          // per head at image + bh * image_stride
+    size_t image_stride;     // bytes
 };
 
-// One thread per state element, summing the splits in order (grid: element blocks x heads).
-__global__ void __launch_bounds__(256) k_state_finalize(FinalizeParams p) {
+constexpr int kImageThreads = 128;
+
+// One thread per 16-byte image chunk (8 features of one row): the head's runs summed in CTA
+// order, times 2^(15 - e) where 2^e exceeds (number of runs) x (largest run magnitude), which
+// bounds the sums, rounded to fp16. Grid: (chunks / 128, heads).
+__global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
     const int bh = blockIdx.y;
-    float *st = p.state + (size_t)bh * state_floats(p.m, p.d);
-    const size_t md = (size_t)p.m * p.d;
-    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < md) {
-        const int r = (int)(i / p.d), c = (int)(i % p.d);
-        const float *src = p.part_S + (size_t)bh * p.n_split * md + i;
-        float s = 0.f;
-        for (int k = 0; k < p.n_split; ++k) s += src[(size_t)k * md];
-        *(float *)((uint8_t *)st + state_image_offset(r, c, p.m)) = tf32_store(s);
-    } else if (i < md + p.m) {
-        const int r = (int)(i - md);
-        const float *src = p.part_z + (size_t)bh * p.n_split * p.m + r;
-        float z = 0.f;
-        for (int k = 0; k < p.n_split; ++k) z += src[(size_t)k * p.m];
-        st[md + r] = z;
-    } else if (i == md + p.m) {
-        st[md + p.m] = p.head_max[bh];
-        st[md + p.m + 1] = 0.f;
-        st[md + p.m + 2] = 0.f;
-        st[md + p.m + 3] = 0.f;
+    const int c_first = flat_first_cta(p.f, bh), c_last = flat_last_cta(p.f, bh);
+    const int halves = p.m / 128, nhs = p.d / 64;
+    float amax = 0.f;
+    for (int c = c_first; c <= c_last; ++c)
+        for (int w = 0; w < 4 * halves; ++w) amax = fmaxf(amax, p.part_amax[(size_t)(c + bh) * 8 + w]);
+    const float bound = amax * (float)(c_last - c_first + 1);
+    int ex = 0;
+    frexpf(bound, &ex);  // bound < 2^ex
+    const float scale = bound > 0.f ? ldexpf(1.f, 15 - ex) : 1.f;
+
+    const int chunks = nhs * halves * 2 * kImgRows * 8;
+    const int q = blockIdx.x * kImageThreads + threadIdx.x;
+    if (q >= chunks) return;
+    const int pch = q & 7, row = (q >> 3) % kImgRows, blk = (q >> 3) / kImgRows;  // blk = (nh*H + h)*2 + kb
+    const int kb = blk & 1, h = (blk >> 1) % halves, nh = (blk >> 1) / halves;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (row <= 64) {
+        const int col = row < 64 ? nh * 64 + row : p.d;
+        const int r0 = h * 128 + kb * 64 + 8 * (pch ^ (row & 7));
+        for (int c = c_first; c <= c_last; ++c) {
+            const float4 *src = (const float4 *)(p.part + ((size_t)(c + bh) * (p.d + 1) + col) * p.m + r0);
+            const float4 a = src[0], b = src[1];
+            v[0] += a.x;
+            v[1] += a.y;
+            v[2] += a.z;
+            v[3] += a.w;
+            v[4] += b.x;
+            v[5] += b.y;
+            v[6] += b.z;
+            v[7] += b.w;
+        }
     }
+    uint4 u;
+    u.x = pack_f16x2(v[0] * scale, v[1] * scale);
+    u.y = pack_f16x2(v[2] * scale, v[3] * scale);
+    u.z = pack_f16x2(v[4] * scale, v[5] * scale);
+    u.w = pack_f16x2(v[6] * scale, v[7] * scale);
+    *(uint4 *)(p.image + (size_t)bh * p.image_stride + ((size_t)blk * kImgRows + row) * 128 + pch * 16) = u;
 }
 
 // ============================================================================ k_query_out
 //
-// Persistent CTAs over a flat, head-major range of (head, 128-token tile) items. Per item the 256
-// features are handled as two 128-feature halves; warpgroup h owns half h end to end:
-//   P[h] = Q W_h^T (bf16 MMA, N = 128) -> row max c_h over the half -> phi_h = 2^(P log2e - c_h)
-//   in place (tf32 operand) and den_h = phi_h . z_h on CUDA cores -> O_h = phi_h S_h (tf32 MMA).
-// The output warpgroup combines the halves exactly: with c = max(c_0, c_1) and a_h = 2^(c_h - c),
-//   out = (a_0 O_0 + a_1 O_1) / (a_0 den_0 + a_1 den_1),
-// i.e. the stabiliser is the exact per-row maximum. The half buffers let the projection of one
-// half overlap the exponentials of the other.
-// TMEM: P[0] [0,128), P[1] [128,256), O[tile parity][half] at 256 + (2 parity + half) * 64.
+// Persistent CTAs over a flat, head-major range of (head, value half, 128-query tile) items. The
+// m features are split into 128-feature halves h, one per exponent warpgroup, each with its own
+// TMEM buffers, so the halves never wait on each other's MMAs:
+//   P_h = Q W_h^T (bf16 MMA into TMEM)
+//   -> warpgroup h: row max of P_h, exchanged with the other half through shared memory, so both
+//      use the row max over all m features, c; phi_h = 2^(P_h log2e - c) rounded to fp16, into TMEM
+//   -> [O | den] = sum_h phi_h [S_h | z_h] (fp16 MMA, A from TMEM, N = 80: z rides along as one
+//      more column of the state image)
+//   -> epilogue warpgroup: out = O / den, staged in shared memory and written by TMA stores.
+// Warp roles (16 warps): 0-3 epilogue, 4-7 / 8-11 exponentials of feature half 0 / 1, 12 TMA loads
+// of Q and W, 13 MMA issue, 14 state image loads, 15 idle. Exponentials: per 32 columns, POLY go
+// through the FMA-pipe polynomial and the rest through MUFU ex2, to balance the two pipes.
+// TMEM columns: P_h [128h, +128), phi_h [256 + 64h, +64) (fp16 pairs), [O | den] [384, +80).
 
 struct QueryParams {
     int L, d, m, BH, tiles_per_cta;
-    const float *state;  // [BH, state_floats]
-    float *out;          // fp32 [BH, L, d]
+    const uint8_t *image;  // per head at image + bh * image_stride
+    size_t image_stride;
 };
 
+constexpr int kQueryThreads = 512;
+constexpr uint32_t kTmemPhi = 256, kTmemO = 384, kOCols = 80;
+
 template <int D>
-struct QuerySmem {
+struct QueryCfg {
     static constexpr int KB = D / 64, NH = D / 64;
     static constexpr uint32_t Q_TILE = KB * kTile * 128;
     static constexpr int STAGES = D == 64 ? 3 : 2;
+    static constexpr int OUT_BUFS = D == 64 ? 2 : 1;
+    static constexpr uint32_t OUT_BUF = 4 * 2 * 32 * 128;  // 4 warps x two 32-column blocks x 32 rows
 };
 
-// Loads 64 consecutive fp32 TMEM columns of this thread's lane and waits.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&a)[32], float (&b)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : FAVOR_REG32(a)
-        : "r"(taddr));
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : FAVOR_REG32(b)
-        : "r"(taddr + 32));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32(a), FAVOR_RW32(b)::"memory");
+// One item's place in the CTA's range: head, value half, tile, and its (head, value half) group.
+struct ItemInfo {
+    int bh, nh, t, first_of_group, last_of_group, group;
+};
+
+template <int NH>
+__device__ __forceinline__ ItemInfo item_info(int g, int f0, int f1, int nt) {
+    ItemInfo it{};
+    int group = 0;
+    for (int bh = f0 / nt;; ++bh) {
+        const int lo = max(f0, bh * nt) - bh * nt, hi = min(f1, (bh + 1) * nt) - bh * nt;
+        const int n = hi - lo;
+        if (g < NH * n) {
+            it.bh = bh;
+            it.nh = g / n;
+            it.t = lo + g % n;
+            it.first_of_group = (g % n) == 0;
+            it.last_of_group = (g % n) == n - 1;
+            it.group = group + it.nh;
+            return it;
+        }
+        g -= NH * n;
+        group += NH;
+    }
 }
 
-template <int D>
-__global__ void __launch_bounds__(512, 1)
-k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapW, QueryParams p) {
-    using SM = QuerySmem<D>;
-    constexpr int KB = SM::KB, NH = SM::NH, STAGES = SM::STAGES;
+// Row maximum of 128 values (four independent chains).
+__device__ __forceinline__ float row_max128(const float (&v)[128]) {
+    float a = -INFINITY, b = -INFINITY, c = -INFINITY, d = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 128; e += 8) {
+        a = fmax3(a, v[e], v[e + 1]);
+        b = fmax3(b, v[e + 2], v[e + 3]);
+        c = fmax3(c, v[e + 4], v[e + 5]);
+        d = fmax3(d, v[e + 6], v[e + 7]);
+    }
+    return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+// phi = 2^(v log2e - cl) for a row of 128 logits, rounded to fp16 pairs. Per 32 columns the first
+// 32 - POLY exponentials go to MUFU ex2, the last POLY to the FMA-pipe polynomial.
+template <int POLY>
+__device__ __forceinline__ void query_features(float (&v)[128], float cl, uint32_t (&hv)[64]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int e = c * 32; e < c * 32 + 32; ++e) v[e] = fmaf(v[e], kLog2e, -cl);
+#pragma unroll
+        for (int e = c * 32; e < c * 32 + 32 - POLY; ++e) v[e] = ex2_approx(v[e]);
+#pragma unroll
+        for (int e = c * 32 + 32 - POLY; e < c * 32 + 32; e += 2) exp2_poly_pair(v[e], v[e + 1], v[e], v[e + 1]);
+#pragma unroll
+        for (int e = c * 32; e < c * 32 + 32; e += 2) hv[e >> 1] = pack_f16x2(v[e], v[e + 1]);
+    }
+}
+
+template <int D, int POLY>
+__global__ void __launch_bounds__(kQueryThreads, 1)
+k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapW,
+            const __grid_constant__ CUtensorMap mapO, QueryParams p) {
+    using C = QueryCfg<D>;
+    constexpr int KB = C::KB, NH = C::NH, STAGES = C::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const uint32_t img_half_bytes = (uint32_t)p.m * 64 * 4;
-    uint8_t *sW = smem;                                          // KB x m x 128
-    uint8_t *sImg = sW + (size_t)KB * p.m * 128;                 // m x 64 x 4 (one value half)
-    float *sZ = (float *)(sImg + img_half_bytes);                // m (<= 256) in a 1024-byte slot
-    uint8_t *sQ = (uint8_t *)sZ + 1024;                          // STAGES x Q_TILE
-    float *sDen = (float *)(sQ + (size_t)STAGES * SM::Q_TILE);  // [2 parity][2 half][128]
-    float *sCl = sDen + 512;                                     // [2 parity][2 half][128]
-    uint64_t *bars = (uint64_t *)(sCl + 512);
+    const int halves = p.m / 128;
+    const uint32_t img_bytes = (uint32_t)halves * kImgHalf;
+    uint8_t *sW = smem;                                              // KB x m x 128
+    uint8_t *sImg = sW + (size_t)KB * p.m * 128;                     // halves x kImgHalf
+    uint8_t *sQ = sImg + 2 * kImgHalf;                               // STAGES x Q_TILE
+    uint8_t *sOut = sQ + (size_t)STAGES * C::Q_TILE;                 // OUT_BUFS x OUT_BUF
+    float *sMax = (float *)(sOut + (size_t)C::OUT_BUFS * C::OUT_BUF);  // [2 parity][2 half][128]
+    uint64_t *bars = (uint64_t *)(sMax + 512);
     uint64_t *full = bars, *empty = bars + STAGES;
     uint64_t *w_full = empty + STAGES, *img_full = w_full + 1, *img_empty = img_full + 1;
-    uint64_t *p_full = img_empty + 1, *p_free = p_full + 2;      // per half buffer
-    uint64_t *chunk_full = p_free + 2;                           // [2 half][4 chunk]
-    uint64_t *o_full = chunk_full + 8, *o_empty = o_full + 2;
-    uint64_t *den_full = o_empty + 2, *den_empty = den_full + 2, *drain = den_empty + 2;
+    uint64_t *p_full = img_empty + 1, *p_free = p_full + 1;
+    uint64_t *xchg = p_free + 1;                                   // per item parity
+    uint64_t *phi_full = xchg + 2, *phi_free = phi_full + 1;
+    uint64_t *o_full = phi_free + 1, *o_empty = o_full + 1;
+    uint64_t *drain = o_empty + 1;
     uint32_t *tmem_slot = (uint32_t *)(drain + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
 
@@ -126,8 +215,6 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     const int f0 = blockIdx.x * p.tiles_per_cta;
     const int f1 = min(f0 + p.tiles_per_cta, total);
     const int n_items = NH * max(f1 - f0, 0);
-    const int halves = p.m / 128;
-    const uint32_t tO = 256;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -137,22 +224,19 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
         mbar_init(w_full, 1);
         mbar_init(img_full, 1);
         mbar_init(img_empty, 1);
-        for (int h = 0; h < 2; ++h) {
-            mbar_init(&p_full[h], 1);
-            mbar_init(&p_free[h], 1);
-        }
-        for (int c = 0; c < 8; ++c) mbar_init(&chunk_full[c], 4);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&o_full[b], 1);
-            mbar_init(&o_empty[b], 4);
-            mbar_init(&den_full[b], 4 * halves);
-            mbar_init(&den_empty[b], 4);
-        }
+        mbar_init(p_full, 1);
+        mbar_init(p_free, 128 * halves);
+        mbar_init(&xchg[0], 128 * halves);
+        mbar_init(&xchg[1], 128 * halves);
+        mbar_init(phi_full, 128 * halves);
+        mbar_init(phi_free, 1);
+        mbar_init(o_full, 1);
+        mbar_init(o_empty, 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 1) {
+    if (warp == 13) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -161,202 +245,212 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // Item order: head runs inside [f0, f1), then value halves nh, then tiles.
-    const int bh_first = f0 / nt, bh_last = (f1 - 1) / nt;
-
-    if (warp == 0) {
-        if (lane == 0 && n_items > 0) {
-            prefetch_tensormap(&mapQ);
-            prefetch_tensormap(&mapW);
-            mbar_arrive_expect_tx(w_full, KB * p.m * 128);
-            for (int kb = 0; kb < KB; ++kb) tma_load_2d(sW + (size_t)kb * p.m * 128, &mapW, w_full, kb * 64, 0);
-            int g = 0, grp = 0, issued = 0;
-            bool ok = true;
-            for (int bh = bh_first; ok && bh <= bh_last; ++bh) {
-                const int lo = max(f0, bh * nt) - bh * nt, hi = min(f1, (bh + 1) * nt) - bh * nt;
-                const float *st = p.state + (size_t)bh * state_floats(p.m, D);
-                for (int nh = 0; ok && nh < NH; ++nh, ++grp) {
-                    if (!mbar_wait(img_empty, (grp & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    mbar_arrive_expect_tx(img_full, img_half_bytes + p.m * 4);
-                    const uint8_t *src = (const uint8_t *)st + (size_t)nh * img_half_bytes;
-                    for (uint32_t off = 0; off < img_half_bytes; off += 32768)
-                        bulk_load(sImg + off, src + off, min(32768u, img_half_bytes - off), img_full);
-                    bulk_load(sZ, st + (size_t)p.m * D, p.m * 4, img_full);
-                    for (int t = lo; t < hi; ++t, ++g) {
-                        const int s = g % STAGES;
-                        if (!mbar_wait(&empty[s], ((g / STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                        mbar_arrive_expect_tx(&full[s], SM::Q_TILE);
-                        for (int kb = 0; kb < KB; ++kb)
-                            tma_load_3d(sQ + (size_t)s * SM::Q_TILE + kb * kTile * 128, &mapQ, &full[s], kb * 64,
-                                        t * kTile, bh);
-                        ++issued;
-                    }
+    if (warp >= 12) {
+        regs_dec<56>();
+        if (warp == 12 && n_items > 0) {
+            // Q tiles (and W once).
+            if (elect_one()) {
+                prefetch_tensormap(&mapQ);
+                prefetch_tensormap(&mapW);
+                prefetch_tensormap(&mapO);
+                mbar_arrive_expect_tx(w_full, KB * p.m * 128);
+                for (int kb = 0; kb < KB; ++kb) tma_load_2d(sW + (size_t)kb * p.m * 128, &mapW, w_full, kb * 64, 0);
+            }
+            __syncwarp();
+            int issued = 0;
+            for (int g = 0; g < n_items; ++g) {
+                const ItemInfo it = item_info<NH>(g, f0, f1, nt);
+                const int s = g % STAGES;
+                if (!mbar_wait_all(&empty[s], ((g / STAGES) & 1) ^ 1, abort_flag)) break;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&full[s], C::Q_TILE);
+                    for (int kb = 0; kb < KB; ++kb)
+                        tma_load_3d(sQ + (size_t)s * C::Q_TILE + kb * kTile * 128, &mapQ, &full[s], kb * 64,
+                                    it.t * kTile, it.bh);
                 }
+                __syncwarp();
+                ++issued;
             }
             volatile int no_abort = 0;
             for (int i = max(issued - STAGES, 0); i < issued; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, &no_abort);
             mbar_wait(w_full, 0, &no_abort);
-            if (grp > 0) mbar_wait(img_full, (grp - 1) & 1, &no_abort);
-        }
-    } else if (warp == 1) {
-        if (lane == 0 && n_items > 0) {
-            const uint32_t idesc1 = make_idesc(kTile, 128, kFmtBF16, 0, 0);
-            const uint32_t idesc2 = make_idesc(kTile, 64, kFmtTF32, 0, 0);
-            bool ok = mbar_wait(w_full, 0, abort_flag);
-            int g = 0, grp = 0;
-            for (int bh = bh_first; ok && bh <= bh_last; ++bh) {
-                const int lo = max(f0, bh * nt) - bh * nt, hi = min(f1, (bh + 1) * nt) - bh * nt;
-                for (int nh = 0; ok && nh < NH; ++nh, ++grp) {
-                    if (!mbar_wait(img_full, grp & 1, abort_flag)) { ok = false; break; }
-                    for (int t = lo; ok && t < hi; ++t, ++g) {
-                        const int s = g % STAGES, ob = g & 1;
-                        if (!mbar_wait(&full[s], (g / STAGES) & 1, abort_flag)) { ok = false; break; }
-                        const uint32_t a0 = smem_u32(sQ + (size_t)s * SM::Q_TILE), b0 = smem_u32(sW);
-                        for (int h = 0; h < halves; ++h) {
-                            if (!mbar_wait(&p_free[h], (g & 1) ^ 1, abort_flag)) { ok = false; break; }
-                            tc_fence_after();
-                            for (int k = 0; k < D / 16; ++k) {
-                                const int kb = k >> 2, kk = k & 3;
-                                mma_f16_ss(tmem + h * 128, make_sdesc(a0 + kb * kTile * 128 + kk * 32, 16, 1024),
-                                           make_sdesc(b0 + kb * p.m * 128 + h * 128 * 128 + kk * 32, 16, 1024), idesc1,
-                                           k > 0);
-                            }
-                            mma_commit(&p_full[h]);
-                        }
-                        if (!ok) break;
-                        mma_commit(&empty[s]);
-                        if (!mbar_wait(&o_empty[ob], ((g >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                        for (int h = 0; ok && h < halves; ++h) {
-                            for (int c = 0; c < 4; ++c) {
-                                if (!mbar_wait(&chunk_full[h * 4 + c], g & 1, abort_flag)) { ok = false; break; }
-                                tc_fence_after();
-                                const uint32_t ib = smem_u32(sImg) + (h * 4 + c) * 64 * 128;
-                                for (int kk = 0; kk < 4; ++kk)
-                                    mma_tf32_ts(tmem + tO + (ob * 2 + h) * 64, tmem + h * 128 + c * 32 + kk * 8,
-                                                make_sdesc(ib + kk * 32, 16, 1024), idesc2, (c > 0 || kk > 0) ? 1u : 0u);
-                            }
-                            if (ok) mma_commit(&p_free[h]);
-                        }
-                        if (!ok) break;
-                        mma_commit(&o_full[ob]);
+        } else if (warp == 14 && n_items > 0) {
+            // State image of each (head, value half) group, once the previous group's output
+            // MMAs have finished with it.
+            int groups = 0;
+            for (int g = 0; g < n_items; ++g) {
+                const ItemInfo it = item_info<NH>(g, f0, f1, nt);
+                if (!it.first_of_group) continue;
+                if (!mbar_wait_all(img_empty, (it.group & 1) ^ 1, abort_flag)) break;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(img_full, img_bytes);
+                    const uint8_t *src = p.image + (size_t)it.bh * p.image_stride + (size_t)it.nh * img_bytes;
+                    for (int h = 0; h < halves; ++h)
+                        bulk_load(sImg + h * kImgHalf, src + h * kImgHalf, kImgHalf, img_full);
+                }
+                __syncwarp();
+                ++groups;
+            }
+            volatile int no_abort = 0;
+            if (groups > 0) mbar_wait(img_full, (groups - 1) & 1, &no_abort);
+        } else if (warp == 13 && n_items > 0) {
+            // MMA issue in a fixed order: the projection of item g+1 (both halves, N = m) as soon
+            // as both halves' P have been read, then the output MMAs of item g once phi is in TMEM.
+            const uint32_t idesc1 = make_idesc(kTile, p.m, kFmtBF16, 0, 0);
+            const uint32_t idesc2 = make_idesc(kTile, kOCols, kFmtF16, 0, 0);
+            const uint64_t dQ = make_sdesc(smem_u32(sQ), 16, 1024), dW = make_sdesc(smem_u32(sW), 16, 1024);
+            const uint64_t dI = make_sdesc(smem_u32(sImg), 16, 1024);
+            const uint32_t w_kb = (uint32_t)p.m * 128 / 16;  // W k-block stride, 16-byte units
+            auto project = [&](int g) {
+                const uint64_t a = dQ + (uint32_t)(g % STAGES) * (C::Q_TILE / 16);
+                if (elect_one()) {
+                    mma_ss_x4(tmem, a, dW, idesc1, 0u, 2, 2);
+                    if (KB == 2) mma_ss_x4(tmem, a + kTile * 128 / 16, dW + w_kb, idesc1, 1u, 2, 2);
+                    mma_commit(p_full);
+                }
+                __syncwarp();
+            };
+            bool ok = mbar_wait_all(w_full, 0, abort_flag) && mbar_wait_all(&full[0], 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                project(0);
+                if (elect_one()) mma_commit(&empty[0]);
+                __syncwarp();
+            }
+            int bh = f0 / nt, nh = 0, t = f0 - bh * nt, group = 0;  // item g's place, advanced per item
+            int run_end = min(f1, (bh + 1) * nt) - bh * nt;          // one past the last tile of this group
+            int run_begin = t;
+            for (int g = 0; ok && g < n_items; ++g) {
+                const bool first = t == run_begin, last = t == run_end - 1;
+                if (g + 1 < n_items) {
+                    const int s1 = (g + 1) % STAGES;
+                    if (!mbar_wait_all(&full[s1], ((g + 1) / STAGES) & 1, abort_flag)) break;
+                    if (!mbar_wait_all(p_free, g & 1, abort_flag)) break;
+                    tc_fence_after();
+                    project(g + 1);
+                    if (elect_one()) mma_commit(&empty[s1]);
+                    __syncwarp();
+                }
+                if (first && !mbar_wait_all(img_full, group & 1, abort_flag)) break;
+                if (g > 0 && !mbar_wait_all(o_empty, (g - 1) & 1, abort_flag)) break;
+                if (!mbar_wait_all(phi_full, g & 1, abort_flag)) break;
+                tc_fence_after();
+                if (elect_one()) {
+                    for (int h = 0; h < halves; ++h) {
+                        const uint64_t b = dI + (uint32_t)h * (kImgHalf / 16);
+                        mma_ts_x4(tmem + kTmemO, tmem + kTmemPhi + h * 64, b, idesc2, h > 0 ? 1u : 0u, 2);
+                        mma_ts_x4(tmem + kTmemO, tmem + kTmemPhi + h * 64 + 32, b + kImgKBlock / 16, idesc2, 1u, 2);
                     }
-                    mma_commit(img_empty);
+                    mma_commit(phi_free);
+                    mma_commit(o_full);
+                    if (last) mma_commit(img_empty);
+                }
+                __syncwarp();
+                // advance to item g + 1
+                if (!last) {
+                    ++t;
+                } else if (nh + 1 < NH) {
+                    ++nh;
+                    ++group;
+                    t = run_begin;
+                } else {
+                    ++bh;
+                    nh = 0;
+                    ++group;
+                    run_begin = t = 0;
+                    run_end = min(f1, (bh + 1) * nt) - bh * nt;
                 }
             }
-            mma_commit(drain);
+            if (elect_one()) mma_commit(drain);
+            __syncwarp();
             volatile int no_abort = 0;
             mbar_wait(drain, 0, &no_abort);
         }
-    } else if (warp >= 4 && warp < 12) {
-        // Exponent warpgroup h: thread <-> token row, the 128 feature columns of half h.
+    } else if (warp >= 4) {
+        regs_inc<184>();
+        // Warpgroup h: feature half h of every item (TMEM lane quarter = warp & 3).
         const int h = (warp - 4) >> 2, row = (warp & 3) * 32 + lane;
         if (h < halves) {
-            const uint32_t base = tmem + h * 128;
+            const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
             for (int g = 0; g < n_items; ++g) {
-                const int ob = g & 1;
-                if (!mbar_wait(&p_full[h], g & 1, abort_flag)) break;
+                if (!mbar_wait_all(p_full, g & 1, abort_flag)) break;
                 tc_fence_after();
-                float rmax = -INFINITY;
-#pragma unroll 1
-                for (int c0 = 0; c0 < 128; c0 += 64) {
-                    float a[32], b[32];
-                    tmem_ld64(tmem_lane_addr(base, warp, c0), a, b);
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) rmax = fmax3(rmax, fmax3(a[e], a[e + 1], b[e]), b[e + 1]);
+                float v[128];
+                tmem_ld128(tmem + lane_off + h * 128, v);
+                tc_fence_before();
+                mbar_arrive(p_free);
+                float rmax = row_max128(v);
+                if (halves == 2) {
+                    const int pb = g & 1;
+                    sMax[(pb * 2 + h) * 128 + row] = rmax;
+                    mbar_arrive(&xchg[pb]);
+                    if (!mbar_wait_all(&xchg[pb], (g >> 1) & 1, abort_flag)) break;
+                    rmax = fmaxf(rmax, sMax[(pb * 2 + (h ^ 1)) * 128 + row]);
                 }
-                const float cl = rmax * kLog2e;
-                float den = 0.f;
-#pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    const uint32_t ta = tmem_lane_addr(base, warp, cc * 32);
-                    float v[32];
-                    tmem_ld32(ta, v);
-                    const float *z = sZ + h * 128 + cc * 32;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        float used;
-                        v[e] = tf32_round_store(ex2_approx(fmaf(v[e], kLog2e, -cl)), used);
-                        den = fmaf(used, z[e], den);
-                    }
-                    tmem_st32(ta, v);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&chunk_full[h * 4 + cc]);
-                }
-                if (!mbar_wait(&den_empty[ob], ((g >> 1) & 1) ^ 1, abort_flag)) break;
-                sDen[(ob * 2 + h) * 128 + row] = den;
-                sCl[(ob * 2 + h) * 128 + row] = cl;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&den_full[ob]);
+                uint32_t hv[64];
+                query_features<POLY>(v, rmax * kLog2e, hv);
+                if (g > 0 && !mbar_wait_all(phi_free, (g - 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                tmem_st64(tmem + lane_off + kTmemPhi + h * 64, hv);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(phi_full);
             }
         }
-    } else if (warp >= 12) {
-        // Output warpgroup: combine the halves and write fp32 rows.
-        const int row = (warp & 3) * 32 + lane;
-        int g = 0;
-        bool ok = true;
-        for (int bh = bh_first; ok && n_items > 0 && bh <= bh_last; ++bh) {
-            const int lo = max(f0, bh * nt) - bh * nt, hi = min(f1, (bh + 1) * nt) - bh * nt;
-            for (int nh = 0; ok && nh < NH; ++nh) {
-                for (int t = lo; t < hi; ++t, ++g) {
-                    const int ob = g & 1;
-                    if (!mbar_wait(&o_full[ob], (g >> 1) & 1, abort_flag) ||
-                        !mbar_wait(&den_full[ob], (g >> 1) & 1, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    float a0 = 1.f, a1 = 0.f, den = sDen[(ob * 2) * 128 + row];
-                    if (halves == 2) {
-                        const float c0 = sCl[(ob * 2) * 128 + row], c1 = sCl[(ob * 2 + 1) * 128 + row];
-                        const float c = fmaxf(c0, c1);
-                        a0 = ex2_approx(c0 - c);
-                        a1 = ex2_approx(c1 - c);
-                        den = a0 * den + a1 * sDen[(ob * 2 + 1) * 128 + row];
-                    }
-                    const float inv = 1.0f / den;
-                    a0 *= inv;
-                    a1 *= inv;
-                    const int j = t * kTile + row;
-                    float *dst = p.out + ((size_t)bh * p.L + j) * D + nh * 64;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < 64; c0 += 32) {
-                        float v0[32], v1[32];
-                        tmem_ld32(tmem_lane_addr(tmem + tO + (ob * 2) * 64, warp, c0), v0);
-                        if (halves == 2) tmem_ld32(tmem_lane_addr(tmem + tO + (ob * 2 + 1) * 64, warp, c0), v1);
-                        else {
+    } else {
+        regs_dec<88>();
+        // Epilogue warpgroup: rows (warp)*32 + lane of every item.
+        const uint32_t lane_off = ((uint32_t)warp * 32u) << 16;
+        uint8_t *stage0 = sOut + warp * (2 * 32 * 128);
+        for (int g = 0; g < n_items; ++g) {
+            if (!mbar_wait_all(o_full, g & 1, abort_flag)) break;
+            tc_fence_after();
+            float o[64];
+            tmem_ld64_nowait(tmem + lane_off + kTmemO, o);
+            float den;
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=f"(den) : "r"(tmem + lane_off + kTmemO + 64));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&o[0])), FAVOR_RW32((&o[32])), "+f"(den)::"memory");
+            tc_fence_before();
+            mbar_arrive(o_empty);
+            const float inv = 1.0f / den;
+            uint8_t *stage = stage0 + (size_t)(g % C::OUT_BUFS) * C::OUT_BUF;
+            if (lane == 0 && g >= C::OUT_BUFS) bulk_wait_group_read<C::OUT_BUFS - 1>();
+            __syncwarp();
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) v1[e] = 0.f;
-                        }
-                        if (j < p.L) {
+            for (int cb = 0; cb < 2; ++cb) {
+                uint8_t *rowp = stage + cb * (32 * 128) + lane * 128;
 #pragma unroll
-                            for (int e = 0; e < 32; e += 4)
-                                *(float4 *)(dst + c0 + e) =
-                                    make_float4(a0 * v0[e] + a1 * v1[e], a0 * v0[e + 1] + a1 * v1[e + 1],
-                                                a0 * v0[e + 2] + a1 * v1[e + 2], a0 * v0[e + 3] + a1 * v1[e + 3]);
-                        }
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(&o_empty[ob]);
-                        mbar_arrive(&den_empty[ob]);
-                    }
+                for (int ch = 0; ch < 8; ++ch) {
+                    const float *q = &o[cb * 32 + 4 * ch];
+                    *(float4 *)(rowp + ((ch ^ (lane & 7)) << 4)) = make_float4(q[0] * inv, q[1] * inv, q[2] * inv, q[3] * inv);
                 }
             }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const ItemInfo it = item_info<NH>(g, f0, f1, nt);
+                const int y = it.t * kTile + warp * 32;
+                tma_store_3d(&mapO, stage, it.nh * 64, y, it.bh);
+                tma_store_3d(&mapO, stage + 32 * 128, it.nh * 64 + 32, y, it.bh);
+                bulk_commit_group();
+            }
         }
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (warp == 13) tmem_dealloc(tmem, 512);
 }
 
 // ============================================================================ host launchers
 
 template <int D>
 static size_t query_smem(int m) {
-    using SM = QuerySmem<D>;
-    return 1024 + (size_t)SM::KB * m * 128 + (size_t)m * 64 * 4 + 1024 + (size_t)SM::STAGES * SM::Q_TILE +
-           (512 + 512) * 4 + 512;
+    using C = QueryCfg<D>;
+    return 1024 + (size_t)C::KB * m * 128 + 2 * kImgHalf + (size_t)C::STAGES * C::Q_TILE +
+           (size_t)C::OUT_BUFS * C::OUT_BUF + 512 * 4 + 256;
 }
 
 int num_sms() {
@@ -369,27 +463,56 @@ int num_sms() {
     return n;
 }
 
-cudaError_t launch_state_finalize(const FinalizeParams &p, int BH, cudaStream_t st) {
-    const size_t n = (size_t)p.m * p.d + p.m + 1;
-    k_state_finalize<<<dim3((unsigned)((n + 255) / 256), BH), 256, 0, st>>>(p);
+cudaError_t launch_state_image(const ImageParams &p, int BH, cudaStream_t st) {
+    const int chunks = (p.d / 64) * (p.m / 128) * 2 * kImgRows * 8;
+    k_state_image<<<dim3((chunks + kImageThreads - 1) / kImageThreads, BH), kImageThreads, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+// The register split of k_query_out (88 + 2 x 184 + 56 per warpgroup lane) adds up to the 128 per
+// thread it is launched with; a build that launched with fewer would leave setmaxnreg waiting, so
+// the launch is refused unless the kernel carries exactly 128.
+template <typename Kern>
+static bool query_regs_ok(Kern k) {
+    cudaFuncAttributes a{};
+    return cudaFuncGetAttributes(&a, k) == cudaSuccess && a.numRegs == 128;
+}
+
+template <int D, int POLY>
+static cudaError_t launch_query_t(const CUtensorMap &mQ, const CUtensorMap &mW, const CUtensorMap &mO,
+                                  const QueryParams &p, dim3 grid, cudaStream_t st) {
+    static int checked = 0;  // 1 ok, -1 refused
+    if (checked == 0) checked = query_regs_ok(k_query_out<D, POLY>) ? 1 : -1;
+    if (checked < 0) return cudaErrorInvalidConfiguration;
+    const size_t sm = query_smem<D>(p.m);
+    cudaFuncSetAttribute(k_query_out<D, POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_query_out<D, POLY><<<grid, kQueryThreads, sm, st>>>(mQ, mW, mO, p);
     return cudaGetLastError();
 }
 
 // Persistent launch: at most one CTA per SM, each over a contiguous head-major range of tiles.
-cudaError_t launch_query_out(const CUtensorMap &mQ, const CUtensorMap &mW, QueryParams p, cudaStream_t st) {
+// poly_pct: share of exponentials taken by the FMA-pipe polynomial, rounded to 0, 25, 37.5 or 50
+// percent (0, 8, 12 or 16 of every 32).
+cudaError_t launch_query_out(const CUtensorMap &mQ, const CUtensorMap &mW, const CUtensorMap &mO, QueryParams p,
+                             int poly_pct, cudaStream_t st) {
     const int total = p.BH * ((p.L + kTile - 1) / kTile);
     p.tiles_per_cta = (total + num_sms() - 1) / num_sms();
     const dim3 grid((total + p.tiles_per_cta - 1) / p.tiles_per_cta);
+    const int poly = poly_pct < 13 ? 0 : poly_pct < 31 ? 8 : poly_pct < 44 ? 12 : 16;
     if (p.d == 64) {
-        const size_t sm = query_smem<64>(p.m);
-        cudaFuncSetAttribute(k_query_out<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        k_query_out<64><<<grid, 512, sm, st>>>(mQ, mW, p);
-    } else {
-        const size_t sm = query_smem<128>(p.m);
-        cudaFuncSetAttribute(k_query_out<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        k_query_out<128><<<grid, 512, sm, st>>>(mQ, mW, p);
+        switch (poly) {
+            case 0: return launch_query_t<64, 0>(mQ, mW, mO, p, grid, st);
+            case 8: return launch_query_t<64, 8>(mQ, mW, mO, p, grid, st);
+            case 12: return launch_query_t<64, 12>(mQ, mW, mO, p, grid, st);
+            default: return launch_query_t<64, 16>(mQ, mW, mO, p, grid, st);
+        }
     }
-    return cudaGetLastError();
+    switch (poly) {
+        case 0: return launch_query_t<128, 0>(mQ, mW, mO, p, grid, st);
+        case 8: return launch_query_t<128, 8>(mQ, mW, mO, p, grid, st);
+        case 12: return launch_query_t<128, 12>(mQ, mW, mO, p, grid, st);
+        default: return launch_query_t<128, 16>(mQ, mW, mO, p, grid, st);
+    }
 }
 
 }  // namespace favor

@@ -71,6 +71,46 @@ def test_bf16_bidirectional_shapes(cuda_device, B, H, L, d, m):
     assert rel_max_err(out, oracle_fwd(x, W64, False)) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("d,m", [(64, 256), (128, 256), (128, 128), (64, 128)])
+def test_bf16_bidirectional_ranges_crossing_heads(cuda_device, d, m):
+    # 24 heads x 13 tiles = 312 tiles over at most 148 persistent CTAs (3 tiles each): most CTA
+    # ranges end inside one head and start inside the next.
+    w = Workload("t", 2, 12, 1600, d, m, False, "bf16", False, 2, 55)
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, m, d, "bf16")
+    out = run_fwd(w, x, Wr, cuda_device, causal=False)
+    assert rel_max_err(out, oracle_fwd(x, W64, False)) <= TOL["bf16"]
+
+
+def test_bf16_many_short_heads(cuda_device):
+    # 300 one-tile heads over at most 148 CTAs: every CTA range holds several whole heads.
+    w = Workload("t", 3, 100, 60, 64, 256, False, "bf16", False, 2, 56)
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    out = run_fwd(w, x, Wr, cuda_device, causal=False)
+    assert rel_max_err(out, oracle_fwd(x, W64, False)) <= TOL["bf16"]
+
+
+def test_bf16_value_tiles_of_very_different_magnitude(cuda_device):
+    # One key tile's values near 3e4 and another's near 1e-5: the per-tile power-of-two scaling
+    # of V keeps both inside fp16's normal range.
+    w = Workload("t", 1, 1, 640, 64, 256, False, "bf16", False, 2, 57)
+    x = make_inputs(w)
+    x["V"][0, 0, :128] *= 3.0e4
+    x["V"][0, 0, 256:384] *= 1.0e-5
+    x["V"] = round_to_bf16(x["V"])
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    out = run_fwd(w, x, Wr, cuda_device, causal=False)
+    assert np.isfinite(out).all()
+    assert rel_max_err(out, oracle_fwd(x, W64, False)) <= TOL["bf16"]
+    # the small tile alone: the same keys with every other value zeroed
+    x2 = dict(x)
+    x2["V"] = np.zeros_like(x["V"])
+    x2["V"][0, 0, 256:384] = x["V"][0, 0, 256:384]
+    out2 = run_fwd(w, x2, Wr, cuda_device, causal=False)
+    assert rel_max_err(out2, oracle_fwd(x2, W64, False)) <= TOL["bf16"]
+
+
 @pytest.mark.parametrize("split_tiles", [1, 3, 64])
 def test_bf16_split_choice_does_not_change_result(cuda_device, split_tiles):
     w = Workload("t", 1, 2, 1500, 64, 256, False, "bf16", False, 2, 33)
