@@ -35,7 +35,7 @@ TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor rate
 L2_FLUSH_BYTES = 256 << 20
 
 # Kernels favor_fwd launches for the bf16 path, in launch order (stage k <-> events 2k, 2k+1).
-FWD_STAGES = ["k_key_max", "k_key_partials", "k_state_image", "k_query_out"]
+FWD_STAGES = ["k_key_partials", "k_state_image", "k_query_out"]
 CAUSAL_STAGES = ["k_key_logit_max", "k_key_state", "k_state_scan", "k_causal_out", "k_causal_prefix"]
 
 
@@ -56,9 +56,9 @@ def stage_work(name, w, n_sms=148):
         return t * 2 * d, 2 * m * d * t, 0
     if name == "k_key_partials":       # read K, V; MMAs K W^T and phi'(K)^T [V | 1]
         return t * 4 * d, 2 * m * d * t + 2 * m * (d + 1) * t, 0
-    if name == "k_state_image":        # read the per-run partial states, write the fp16 images
+    if name == "k_state_image":        # read the per-run partial states and stabilisers, write the fp16 images
         runs = n_sms + BH - 1
-        return runs * (d + 1) * m * 4 + BH * (d // 64) * (m // 128) * 20480, 0, 0
+        return runs * (d + 2) * m * 4 + BH * (d // 64) * (m // 128) * 20480, 0, 0
     if name == "k_query_out":          # read Q; write fp32 out; MMAs Q W^T and phi(Q) [S | z]
         return t * (2 * d + 4 * d), 2 * m * d * t + 2 * m * (d + 1) * t, 0
     if name == "k_key_logit_max":      # read K; write -|k|^2/2

@@ -102,23 +102,24 @@ Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_
 // Bidirectional bf16 forward: per-run key maxima, per-run partial states [S | z] (feature-major
 // columns), their largest magnitudes, and the per-head fp16 state images (unless a ctx holds them).
 struct BidirLayout {
-    Flat f_max, f;  // 128-token tiles of k_key_max, 64-token tiles of k_key_partials
+    Flat f;  // 64-token key tiles of k_key_partials
     int BH;
-    size_t off_run_max, off_part, off_amax, off_state, total;
+    size_t off_part, off_D, off_amax, off_Dmax, off_state, total;
 };
 
 BidirLayout bidir_layout(const favor_shape *s, bool state_in_ws) {
     BidirLayout l{};
     l.BH = s->B * s->H;
-    l.f_max = make_flat(l.BH, s->L, num_sms(), kTile);
     l.f = make_flat(l.BH, s->L, num_sms(), kKeyTile);
     const size_t slots = (size_t)flat_slots(l.f, l.BH);
     size_t off = 0;
-    l.off_run_max = off;
-    off += align256((size_t)flat_slots(l.f_max, l.BH) * 8 * 4);
     l.off_part = off;
     off += align256(slots * (s->d + 1) * s->m * 4);
+    l.off_D = off;
+    off += align256(slots * s->m * 4);
     l.off_amax = off;
+    off += align256(slots * 8 * 4);
+    l.off_Dmax = off;
     off += align256(slots * 8 * 4);
     l.off_state = off;
     if (state_in_ws) off += align256((size_t)l.BH * state_floats(s->m, s->d) * 4);
@@ -210,36 +211,32 @@ favor_status fwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, 
                             float *out, void *ctx, uint8_t *ws, size_t ws_bytes, const favor_opts *o, cudaStream_t st) {
     const BidirLayout l = bidir_layout(s, ctx == nullptr);
     if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
-    CUtensorMap mQ, mK, mK64, mV64, mW, mO;
-    if (!make_token_map(&mQ, Q, l.BH, s->L, s->d) || !make_token_map(&mK, K, l.BH, s->L, s->d) ||
-        !make_token_map(&mK64, K, l.BH, s->L, s->d, kKeyTile) || !make_token_map(&mV64, V, l.BH, s->L, s->d, kKeyTile) ||
-        !make_w_map(&mW, W, s->m, s->d) || !make_out_map(&mO, out, l.BH, s->L, s->d))
+    CUtensorMap mQ, mK64, mV64, mW, mO;
+    if (!make_token_map(&mQ, Q, l.BH, s->L, s->d) || !make_token_map(&mK64, K, l.BH, s->L, s->d, kKeyTile) ||
+        !make_token_map(&mV64, V, l.BH, s->L, s->d, kKeyTile) || !make_w_map(&mW, W, s->m, s->d) ||
+        !make_out_map(&mO, out, l.BH, s->L, s->d))
         return FAVOR_ERR_CUDA;
-    float *run_max = (float *)(ws + l.off_run_max);
     float *part = (float *)(ws + l.off_part);
+    float *partD = (float *)(ws + l.off_D);
     float *amax = (float *)(ws + l.off_amax);
+    float *Dmax = (float *)(ws + l.off_Dmax);
     uint8_t *state = ctx ? (uint8_t *)ctx : ws + l.off_state;
     const size_t stride = state_floats(s->m, s->d) * 4;
 
-    KeyMaxParams2 km{s->L, s->m, l.f_max, run_max};
+    KeyStateParams2 ks{s->L, s->m, l.f, part, partD, amax, Dmax};
     record_stage(o, 0, st);
-    cudaError_t e = launch_key_max(mK, mW, km, s->d, st);
+    cudaError_t e = launch_key_partials(mK64, mV64, mW, ks, s->d, opt_poly_pct(o), st);
     record_stage(o, 1, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-    KeyStateParams2 ks{s->L, s->m, l.f, l.f_max, run_max, part, amax};
+    ImageParams ip{s->m, s->d, l.f, part, partD, amax, Dmax, state, stride};
     record_stage(o, 2, st);
-    e = launch_key_partials(mK64, mV64, mW, ks, s->d, opt_poly_pct(o), st);
+    e = launch_state_image(ip, l.BH, st);
     record_stage(o, 3, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-    ImageParams ip{s->m, s->d, l.f, part, amax, state, stride};
-    record_stage(o, 4, st);
-    e = launch_state_image(ip, l.BH, st);
-    record_stage(o, 5, st);
-    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     QueryParams qp{s->L, s->d, s->m, l.BH, 0, state, stride};
-    record_stage(o, 6, st);
+    record_stage(o, 4, st);
     e = launch_query_out(mQ, mW, mO, qp, opt_poly_pct(o), st);
-    record_stage(o, 7, st);
+    record_stage(o, 5, st);
     return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 

@@ -1,13 +1,14 @@
 // Key side of the bidirectional bf16 tensor-core path ("Fast Attention Via Positive Orthogonal
 // Random Features", codewithpapers.app/method/favor: the FA-part needs (K')^T V and (K')^T 1_L).
 //
-//   k_key_max      : the per-(batch, head) key stabiliser C = max_{j,r} u_r(k_j), with
-//                    u_r(k) = w_r.k - |k|^2/2, as one maximum per (CTA, head) run.
 //   k_key_partials : per run, the partial state [S | z] = sum_j phi'(k_j) [v_j | 1] with
-//                    phi'(k) = 2^8 exp(u(k) - C). Both the 2^8 and C cancel in D^-1.
+//                    phi'_r(k) = 2^(A - D_r) exp(u_r(k)), u_r(k) = w_r.k - |k|^2/2, where D_r is a
+//                    per-feature stabiliser kept by the run (log2 units) and A = 4. The image
+//                    kernel brings every run and feature to one per-(batch, head) reference
+//                    before the state is used, so the stabilisers cancel in D^-1.
 //
-// Work split: the BH * ceil(L/TILE) key tiles (TILE = 128 tokens for k_key_max, 64 for
-// k_key_partials), head-major, are cut into contiguous ranges of T tiles, one per persistent CTA.
+// Work split: the BH * ceil(L/64) key tiles, head-major, are cut into contiguous ranges of T
+// tiles, one per persistent CTA.
 // A run is the part of one head inside one CTA's range; run
 // (CTA c, head bh) owns slot c + bh of the per-run outputs (runs are ordered by both c and bh, so
 // c + bh is distinct for distinct runs). A head's runs are the CTAs first_cta(bh)..last_cta(bh).
@@ -58,186 +59,24 @@ __device__ __forceinline__ float key_sq_norm(const uint8_t *tile, int row) {
     return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
-// The per-(batch, head) key maximum from the maxima of the head's runs.
-__device__ __forceinline__ float head_key_max(const float *run_max, const Flat &f, int bh) {
-    float c = -INFINITY;
-    for (int cta = flat_first_cta(f, bh); cta <= flat_last_cta(f, bh); ++cta)
-        for (int w = 0; w < 8; ++w) c = fmaxf(c, run_max[(size_t)(cta + bh) * 8 + w]);
-    return c;
-}
-
-// ============================================================================ k_key_max
-//
-// D[token, r] = K_tile W^T (bf16, M = 128 tokens, N = m, K = d) into one of two TMEM buffers;
-// epilogue warpgroup e takes the tiles of parity e: each token row's max over r minus |k|^2/2,
-// kept as a running max per run and written as one value per warp into the run's slot (every
-// warp writes every run of its CTA, -inf where it saw none of the run's tiles).
-
-struct KeyMaxParams2 {
-    int L, m;
-    Flat f;          // 128-token tiles
-    float *run_max;  // [slots][8]
-};
-
-template <int D>
-__global__ void __launch_bounds__(384, 1)
-k_key_max(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapW, KeyMaxParams2 p) {
-    constexpr int KB = D / 64, STAGES = 4;
-    constexpr uint32_t TILE = KB * kTile * 128;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *sW = smem;
-    uint8_t *sK = sW + (size_t)KB * p.m * 128;
-    uint64_t *bars = (uint64_t *)(sK + (size_t)STAGES * TILE);
-    uint64_t *full = bars, *empty = bars + STAGES, *w_full = empty + STAGES;
-    uint64_t *p_full = w_full + 1, *p_empty = p_full + 2, *drain = p_empty + 2;
-    uint32_t *tmem_slot = (uint32_t *)(drain + 1);
-    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int f0 = blockIdx.x * p.f.T, f1 = min(f0 + p.f.T, p.f.total);
-    const int n = max(f1 - f0, 0);
-    const uint32_t tmem_cols = p.m * 2 <= 256 ? 256u : 512u;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + 128);
-        }
-        mbar_init(w_full, 1);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&p_full[b], 1);
-            mbar_init(&p_empty[b], 128);
-        }
-        mbar_init(drain, 1);
-        *abort_flag = 0;
-        fence_barrier_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, tmem_cols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        if (n > 0) {
-            if (elect_one()) {
-                prefetch_tensormap(&mapK);
-                prefetch_tensormap(&mapW);
-                mbar_arrive_expect_tx(w_full, KB * p.m * 128);
-                for (int kb = 0; kb < KB; ++kb) tma_load_2d(sW + (size_t)kb * p.m * 128, &mapW, w_full, kb * 64, 0);
-            }
-            __syncwarp();
-            int issued = 0;
-            for (int g = 0; g < n; ++g) {
-                const int s = g % STAGES, fl = f0 + g;
-                if (!mbar_wait_all(&empty[s], ((g / STAGES) & 1) ^ 1, abort_flag)) break;
-                if (elect_one()) {
-                    mbar_arrive_expect_tx(&full[s], TILE);
-                    for (int kb = 0; kb < KB; ++kb)
-                        tma_load_3d(sK + (size_t)s * TILE + kb * kTile * 128, &mapK, &full[s], kb * 64,
-                                    (fl % p.f.nt) * kTile, fl / p.f.nt);
-                }
-                __syncwarp();
-                ++issued;
-            }
-            volatile int no_abort = 0;
-            for (int i = max(issued - STAGES, 0); i < issued; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, &no_abort);
-            mbar_wait(w_full, 0, &no_abort);
-        }
-    } else if (warp == 1) {
-        if (n > 0) {
-            const uint32_t idesc = make_idesc(kTile, p.m, kFmtBF16, 0, 0);
-            const uint64_t dK = make_sdesc(smem_u32(sK), 16, 1024), dW = make_sdesc(smem_u32(sW), 16, 1024);
-            bool ok = mbar_wait_all(w_full, 0, abort_flag);
-            for (int g = 0; ok && g < n; ++g) {
-                const int s = g % STAGES, b = g & 1;
-                if (!mbar_wait_all(&full[s], (g / STAGES) & 1, abort_flag)) break;
-                if (!mbar_wait_all(&p_empty[b], ((g >> 1) & 1) ^ 1, abort_flag)) break;
-                tc_fence_after();
-                const uint64_t a = dK + (uint32_t)s * (TILE / 16);
-                if (elect_one()) {
-                    mma_ss_x4(tmem + b * p.m, a, dW, idesc, 0u, 2, 2);
-                    if (KB == 2)
-                        mma_ss_x4(tmem + b * p.m, a + kTile * 128 / 16, dW + (uint32_t)p.m * 8, idesc, 1u, 2, 2);
-                    mma_commit(&p_full[b]);
-                    mma_commit(&empty[s]);
-                }
-                __syncwarp();
-            }
-            if (elect_one()) mma_commit(drain);
-            __syncwarp();
-            volatile int no_abort = 0;
-            mbar_wait(drain, 0, &no_abort);
-        }
-    } else if (warp >= 4) {
-        const int e = (warp - 4) >> 2;  // this warpgroup takes the tiles g with g % 2 == e
-        const int row = (warp & 3) * 32 + lane;
-        const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
-        const size_t wslot = (size_t)e * 4 + (warp & 3);
-        int cur = -1;
-        float run = -INFINITY;
-        for (int g = 0; g < n; ++g) {
-            const int s = g % STAGES, fl = f0 + g, bh = fl / p.f.nt, t = fl % p.f.nt;
-            if (bh != cur) {
-                if (cur >= 0) {
-                    for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
-                    if (lane == 0) p.run_max[(size_t)(blockIdx.x + cur) * 8 + wslot] = run;
-                }
-                cur = bh;
-                run = -INFINITY;
-            }
-            if ((g & 1) != e) continue;
-            if (!mbar_wait_all(&p_full[e], (g >> 1) & 1, abort_flag)) break;
-            tc_fence_after();
-            float a = -INFINITY, b = -INFINITY, c2 = -INFINITY, d2 = -INFINITY;
-            for (int c = 0; c < p.m; c += 64) {
-                float v[64];
-                tmem_ld64_nowait(tmem + lane_off + e * p.m + c, v);
-                asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&v[0])), FAVOR_RW32((&v[32]))::"memory");
-#pragma unroll
-                for (int i = 0; i < 64; i += 8) {
-                    a = fmax3(a, v[i], v[i + 1]);
-                    b = fmax3(b, v[i + 2], v[i + 3]);
-                    c2 = fmax3(c2, v[i + 4], v[i + 5]);
-                    d2 = fmax3(d2, v[i + 6], v[i + 7]);
-                }
-            }
-            const float rmax = fmaxf(fmaxf(a, b), fmaxf(c2, d2));
-            tc_fence_before();
-            mbar_arrive(&p_empty[e]);
-            const float k2 = key_sq_norm<KB, kTile>(sK + (size_t)s * TILE, row);
-            mbar_arrive(&empty[s]);
-            if (t * kTile + row < p.L) run = fmaxf(run, rmax - 0.5f * k2);
-        }
-        if (cur >= 0) {
-            for (int o = 16; o > 0; o >>= 1) run = fmaxf(run, __shfl_xor_sync(0xffffffffu, run, o));
-            if (lane == 0) p.run_max[(size_t)(blockIdx.x + cur) * 8 + wslot] = run;
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, tmem_cols);
-}
-
 // ============================================================================ k_key_partials
 //
 // Per key tile of 64 tokens, with the m features as 128-feature halves h, one per exponent
 // warpgroup, each with its own TMEM buffers (the halves never wait on each other):
-//   P_h^T = W_h K_tile^T (bf16 MMA; TMEM lanes are features, columns are tokens)
-//   -> warpgroup h: phi'_h = 2^(P_h^T log2e + B_j) with the per-token bias
-//      B_j = -(|k_j|^2/2 + C) log2e + 8 + b_t, rounded to fp16 into TMEM
+//   P_h^T = W_h K_tile^T - D_r ln2 (bf16 MMA accumulating onto a per-row value the warpgroup
+//           stored beforehand; TMEM lanes are features, columns are tokens)
+//   -> warpgroup h: t = P_h^T log2e + B_j with B_j = -|k_j|^2/2 log2e + A + b_t, i.e.
+//      t = u_r(k_j) log2e - D_r + A + b_t; phi' = 2^t rounded to fp16 into TMEM
 //   -> [S_h | z_h] += phi'_h [V'_t | 2^-b_t] (fp16 MMA, A from TMEM, B the converted V tile read
 //      MN-major plus one column holding 2^-b_t), accumulated in TMEM over the run.
+// Stabiliser D_r (integer): set on a run's first tile so that the row's largest t is in (A+b-1, A+b];
+// raised whenever a later tile's largest t would exceed 15 (fp16 holds 2^t only up to t < 16),
+// the row's accumulated [S | z] being scaled by 2^-delta in TMEM. Typical inputs raise it rarely.
 // V'_t = V_t 2^-b_t with b_t = clamp(e_t - 7, -8, 7) and e_t the exponent of the tile's largest
 // |v|: V_t is converted bf16 -> fp16 in place, and the factor 2^b_t moved into phi' keeps every
-// product phi' v' equal to 2^8 phi v. Tokens past L get phi' = 0 and a zero ones entry.
-// At the end of a run warpgroup h writes its 128 feature rows of [S_h | z_h] (fp32) and the
-// rows' largest magnitude to the run's slot.
+// product phi' v' equal to 2^(A - D_r) phi v. Tokens past L get phi' = 0 and a zero ones entry.
+// At the end of a run warpgroup h writes its 128 feature rows of [S_h | z_h] (fp32), D_r, and the
+// rows' largest magnitude and largest D_r to the run's slot.
 // Warp roles (16 warps): 0-3 convert V, write the ones column and the biases B_j; 4-7 / 8-11
 // exponentials of feature half 0 / 1 and the run-end write; 12 TMA; 13 MMA issue; 14 the tile's
 // largest |v|; 15 idle.
@@ -245,16 +84,17 @@ k_key_max(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUte
 
 struct KeyStateParams2 {
     int L, m;
-    Flat f;                // 64-token tiles of this kernel
-    Flat f_max;            // 128-token tiles of k_key_max (its run slots)
-    const float *run_max;  // [slots of f_max][8] (k_key_max)
-    float *part;           // [slots of f][d+1][m]: column c of [S | z] for features 0..m-1
-    float *part_amax;      // [slots of f][8]: per (half, warp) largest |entry| of the run's rows
+    Flat f;            // 64-token tiles
+    float *part;       // [slots][d+1][m]: column c of [S | z] for features 0..m-1
+    float *part_D;     // [slots][m]: the run's stabiliser D_r per feature
+    float *part_amax;  // [slots][8]: per (half, warp) largest |entry| of the run's rows
+    float *part_Dmax;  // [slots][8]: per (half, warp) largest D_r
 };
 
 constexpr int kKeyThreads = 512;
-constexpr int kKeyTile = 64;             // tokens per key tile of k_key_partials
-constexpr float kKeyFeatureShift = 8.f;  // phi' = 2^8 phi
+constexpr int kKeyTile = 64;            // tokens per key tile of k_key_partials
+constexpr float kKeyFeatureShift = 4.f;  // A: the run's largest phi' is about 2^(A + b_t)
+constexpr float kLn2 = 0.6931471805599453f;
 
 template <int D>
 struct KeyCfg {
@@ -267,18 +107,28 @@ struct KeyCfg {
     static constexpr uint32_t T_PHI = 128, T_S = 192;
 };
 
+// t = v log2e + B_j for a row of 64 logits (in place); returns the row's largest t.
+__device__ __forceinline__ float key_logits(float (&v)[64], const float *bias) {
+    float a = -INFINITY, b = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 64; e += 4) {
+        const float4 b4 = *(const float4 *)(bias + e);
+        v[e] = fmaf(v[e], kLog2e, b4.x);
+        v[e + 1] = fmaf(v[e + 1], kLog2e, b4.y);
+        v[e + 2] = fmaf(v[e + 2], kLog2e, b4.z);
+        v[e + 3] = fmaf(v[e + 3], kLog2e, b4.w);
+        a = fmax3(a, v[e], v[e + 1]);
+        b = fmax3(b, v[e + 2], v[e + 3]);
+    }
+    return fmaxf(a, b);
+}
+
+// phi' = 2^t (in place), rounded to fp16 pairs. Per 32 columns the first 32 - POLY exponentials
+// go to MUFU ex2, the last POLY to the FMA-pipe polynomial.
 template <int POLY>
-__device__ __forceinline__ void key_features(float (&v)[64], const float *bias, uint32_t (&hv)[32]) {
+__device__ __forceinline__ void key_features(float (&v)[64], uint32_t (&hv)[32]) {
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-#pragma unroll
-        for (int e = c * 32; e < c * 32 + 32; e += 4) {
-            const float4 b4 = *(const float4 *)(bias + e);
-            v[e] = fmaf(v[e], kLog2e, b4.x);
-            v[e + 1] = fmaf(v[e + 1], kLog2e, b4.y);
-            v[e + 2] = fmaf(v[e + 2], kLog2e, b4.z);
-            v[e + 3] = fmaf(v[e + 3], kLog2e, b4.w);
-        }
 #pragma unroll
         for (int e = c * 32; e < c * 32 + 32 - POLY; ++e) v[e] = ex2_approx(v[e]);
 #pragma unroll
@@ -295,6 +145,44 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&h)[3
         "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
         FAVOR_U16(h, 0), FAVOR_U16(h, 16)
         : "memory");
+}
+
+// Fills 64 consecutive columns of this thread's TMEM lane with x (warp-collective; not waited).
+__device__ __forceinline__ void tmem_fill64(uint32_t taddr, float x) {
+    const uint32_t u = __float_as_uint(x);
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+        "r"(u)
+        : "memory");
+}
+
+// Scales columns [0, n) of this thread's TMEM lane by s (warp-collective; n a multiple of 16;
+// waited). Touches no column at or past n.
+__device__ __forceinline__ void tmem_scale_row(uint32_t taddr, int n, float s) {
+    for (int c0 = 0; c0 < n; c0 += 16) {
+        float w[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15}, [%16];"
+            : "=f"(w[0]), "=f"(w[1]), "=f"(w[2]), "=f"(w[3]), "=f"(w[4]), "=f"(w[5]), "=f"(w[6]), "=f"(w[7]),
+              "=f"(w[8]), "=f"(w[9]), "=f"(w[10]), "=f"(w[11]), "=f"(w[12]), "=f"(w[13]), "=f"(w[14]), "=f"(w[15])
+            : "r"(taddr + c0));
+        asm volatile("tcgen05.wait::ld.sync.aligned;"
+                     : "+f"(w[0]), "+f"(w[1]), "+f"(w[2]), "+f"(w[3]), "+f"(w[4]), "+f"(w[5]), "+f"(w[6]), "+f"(w[7]),
+                       "+f"(w[8]), "+f"(w[9]), "+f"(w[10]), "+f"(w[11]), "+f"(w[12]), "+f"(w[13]), "+f"(w[14]),
+                       "+f"(w[15])::"memory");
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] *= s;
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15, %16};" ::"r"(taddr + c0),
+            "f"(w[0]), "f"(w[1]), "f"(w[2]), "f"(w[3]), "f"(w[4]), "f"(w[5]), "f"(w[6]), "f"(w[7]), "f"(w[8]),
+            "f"(w[9]), "f"(w[10]), "f"(w[11]), "f"(w[12]), "f"(w[13]), "f"(w[14]), "f"(w[15])
+            : "memory");
+    }
+    tmem_wait_st();
 }
 
 template <int D, int POLY>
@@ -417,7 +305,8 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
             }
         } else if (warp == 13 && n > 0) {
             // MMA issue in a fixed order: the projections of tile g+1 as soon as each half's P has
-            // been read, then the state MMAs of tile g once its V tile is converted and phi' is in TMEM.
+            // been read (and refilled with -D_r ln2), then the state MMAs of tile g once its V tile
+            // is converted and phi' is in TMEM.
             const uint32_t idesc1 = make_idesc(128, kKeyTile, kFmtBF16, 0, 0);
             const uint32_t idesc2 = make_idesc(128, ON, kFmtF16, 0, 1);
             const uint64_t dW = make_sdesc(smem_u32(sW), 16, 1024), dS = make_sdesc(smem_u32(sStage), 16, 1024);
@@ -426,7 +315,8 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 const uint64_t a = dW + (uint32_t)h * (128 * 128 / 16);
                 const uint64_t b = dS + (uint32_t)(g % STAGES) * (C::STAGE / 16);
                 if (elect_one()) {
-                    mma_ss_x4(tmem + h * 64, a, b, idesc1, 0u, 2, 2);
+                    // the first projection has no stored -D_r ln2 to accumulate onto (D_r = 0)
+                    mma_ss_x4(tmem + h * 64, a, b, idesc1, g > 0 ? 1u : 0u, 2, 2);
                     if (KB == 2)
                         mma_ss_x4(tmem + h * 64, a + (uint32_t)p.m * 8, b + kKeyTile * 128 / 16, idesc1, 1u, 2, 2);
                     mma_commit(&p_full[h]);
@@ -482,37 +372,56 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
         const int h = (warp - 4) >> 2, row = (warp & 3) * 32 + lane;
         if (h < halves) {
             const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
+            const uint32_t tP = tmem + lane_off + h * 64, tS = tmem + lane_off + C::T_S + h * ON;
             int runs = 0;
+            float Dr = 0.f;  // this feature's stabiliser D_r in the current run
             for (int g = 0; g < n; ++g) {
                 const int s = g % STAGES;
                 if (!mbar_wait_all(&p_full[h], g & 1, abort_flag)) break;
                 if (!mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag)) break;
                 tc_fence_after();
                 float v[64];
-                tmem_ld64_nowait(tmem + lane_off + h * 64, v);
+                tmem_ld64_nowait(tP, v);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&v[0])), FAVOR_RW32((&v[32]))::"memory");
+                const float tmax = key_logits(v, sBias + s * kKeyTile);
+                const float lim = kKeyFeatureShift + (float)sShift[s];  // target for the row's largest t
+                const bool first = first_of_run(g), last = last_of_run(g);
+                // new stabiliser: on a run's first tile always, later only when 2^t would overflow fp16
+                const float delta = (first || tmax > 15.f) ? ceilf(tmax - lim) : 0.f;
+                const bool any_shift = __any_sync(0xffffffffu, delta != 0.f);
+                if (any_shift) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) v[e] -= delta;
+                    Dr += delta;
+                }
+                // the next tile's projection accumulates onto -D_r ln2 (0 when it starts a new run)
+                tmem_fill64(tP, last ? 0.f : -Dr * kLn2);
+                tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&p_free[h]);
                 uint32_t hv[32];
-                key_features<POLY>(v, sBias + s * kKeyTile, hv);
+                key_features<POLY>(v, hv);
                 if (g > 0 && !mbar_wait_all(&phi_free[h], (g - 1) & 1, abort_flag)) break;
                 tc_fence_after();
+                // a raised stabiliser rescales the row's accumulated [S | z] (the previous tile's
+                // state MMA has completed: phi_free)
+                if (!first && __any_sync(0xffffffffu, delta > 0.f))
+                    tmem_scale_row(tS, ON, __uint_as_float((uint32_t)(127 - (int)delta) << 23));
                 tmem_st32u(tmem + lane_off + C::T_PHI + h * 32, hv);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&phi_full[h]);
-                if (last_of_run(g)) {
+                if (last) {
                     if (!mbar_wait_all(&acc_full[h], runs & 1, abort_flag)) break;
                     tc_fence_after();
                     const int bh = (f0 + g) / nt;
                     const size_t rs = (size_t)blockIdx.x + bh;
                     float *dst = p.part + rs * (D + 1) * p.m + h * 128 + row;
                     float amax = 0.f;
-                    const uint32_t sa = tmem + lane_off + C::T_S + h * ON;
 #pragma unroll
                     for (int c0 = 0; c0 < D; c0 += 64) {
                         float w[64];
-                        tmem_ld64_nowait(sa + c0, w);
+                        tmem_ld64_nowait(tS + c0, w);
                         asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&w[0])), FAVOR_RW32((&w[32]))::"memory");
 #pragma unroll
                         for (int c = 0; c < 64; ++c) {
@@ -520,13 +429,22 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                             amax = fmaxf(amax, fabsf(w[c]));
                         }
                     }
-                    const float z = tmem_ld1(sa + D);
+                    const float z = tmem_ld1(tS + D);
                     dst[(size_t)D * p.m] = z;
                     amax = fmaxf(amax, z);
+                    p.part_D[rs * p.m + h * 128 + row] = Dr;
                     tc_fence_before();
                     mbar_arrive(&acc_empty[h]);
-                    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                    if (lane == 0) p.part_amax[rs * 8 + h * 4 + (warp & 3)] = amax;
+                    float dmax = Dr;
+                    for (int o = 16; o > 0; o >>= 1) {
+                        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                        dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+                    }
+                    if (lane == 0) {
+                        p.part_amax[rs * 8 + h * 4 + (warp & 3)] = amax;
+                        p.part_Dmax[rs * 8 + h * 4 + (warp & 3)] = dmax;
+                    }
+                    Dr = 0.f;
                     ++runs;
                 }
             }
@@ -536,14 +454,8 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
         // Converter warpgroup: thread j < 64 handles token j of each tile (its |k_j|^2, bias and
         // ones entry); all 128 threads convert 4 * KB of the tile's 16-byte V chunks each.
         const int j = threadIdx.x;
-        int cur = -1;
-        float chead = 0.f;
         for (int g = 0; g < n; ++g) {
-            const int s = g % STAGES, fl = f0 + g, bh = fl / nt, t = fl % nt;
-            if (bh != cur) {
-                chead = head_key_max(p.run_max, p.f_max, bh);
-                cur = bh;
-            }
+            const int s = g % STAGES, fl = f0 + g, t = fl % nt;
             if (!mbar_wait_all(&vmax_full[s], (g / STAGES) & 1, abort_flag)) break;
             uint8_t *st = sStage + (size_t)s * C::STAGE;
             const int b = sShift[s];
@@ -563,8 +475,7 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 const uint32_t ones = pack_f16x2(valid ? scale : 0.f, 0.f) & 0xFFFFu;
                 *(uint16_t *)(st + 2 * C::TILE + j * 128 + ((j & 7) << 4)) = (uint16_t)ones;
                 const float k2 = key_sq_norm<KB, kKeyTile>(st, j);
-                sBias[s * kKeyTile + j] =
-                    valid ? fmaf(-(0.5f * k2 + chead), kLog2e, kKeyFeatureShift + (float)b) : -INFINITY;
+                sBias[s * kKeyTile + j] = valid ? fmaf(-0.5f * k2, kLog2e, kKeyFeatureShift + (float)b) : -INFINITY;
             }
             fence_async_smem();
             mbar_arrive(&conv_full[s]);
@@ -579,29 +490,9 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
 // ============================================================================ host launchers
 
 template <int D>
-static size_t key_max_smem(int m) {
-    return 1024 + (size_t)(D / 64) * m * 128 + 4 * (size_t)(D / 64) * kTile * 128 + 256;
-}
-
-template <int D>
 static size_t key_partials_smem(int m) {
     using C = KeyCfg<D>;
     return 1024 + (size_t)C::KB * m * 128 + (size_t)C::STAGES * C::STAGE + C::STAGES * kKeyTile * 4 + 64 + 512;
-}
-
-cudaError_t launch_key_max(const CUtensorMap &mK, const CUtensorMap &mW, const KeyMaxParams2 &p, int d,
-                           cudaStream_t st) {
-    const dim3 grid(p.f.n_cta);
-    if (d == 64) {
-        const size_t sm = key_max_smem<64>(p.m);
-        cudaFuncSetAttribute(k_key_max<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        k_key_max<64><<<grid, 384, sm, st>>>(mK, mW, p);
-    } else {
-        const size_t sm = key_max_smem<128>(p.m);
-        cudaFuncSetAttribute(k_key_max<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        k_key_max<128><<<grid, 384, sm, st>>>(mK, mW, p);
-    }
-    return cudaGetLastError();
 }
 
 // The register split of k_key_partials (80 + 2 x 184 + 56 per warpgroup lane) fits the 128 per

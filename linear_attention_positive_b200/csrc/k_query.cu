@@ -1,7 +1,8 @@
 // Bidirectional state image and query-side output of the bf16 tensor-core path.
 //
 //   k_state_image : sums the per-run partial states in run order into the per-head state
-//                   [S | z] = (K')^T [V | 1_L], scales it by a power of two so that its largest
+//                   [S | z] = (K')^T [V | 1_L] (each run's per-feature stabilisers brought to one
+//                   per-head reference), scales it by a power of two so that its largest
 //                   magnitude lies in [2^14, 2^15), and writes it as fp16 in the layout the output
 //                   MMA reads (the scale cancels between numerator and denominator).
 //   k_query_out   : out = D^-1 (Q' S), D = diag(Q' z) ("Fast Attention Via Positive Orthogonal
@@ -41,24 +42,42 @@ struct ImageParams {
     int m, d;
     Flat f;                  // partition of the key tiles (runs and their slots)
     const float *part;       // [slots][d+1][m]
+    const float *part_D;     // [slots][m] per-run, per-feature stabilisers (log2 units)
     const float *part_amax;  // [slots][8]
+    const float *part_Dmax;  // [slots][8]
     uint8_t *image;          // per head at image + bh * image_stride
     size_t image_stride;     // bytes
 };
 
 constexpr int kImageThreads = 128;
 
-// One thread per 16-byte image chunk (8 features of one row): the head's runs summed in CTA
-// order, times 2^(15 - e) where 2^e exceeds (number of runs) x (largest run magnitude), which
-// bounds the sums, rounded to fp16. Grid: (chunks / 128, heads).
+// 2^e for an integer-valued e (0 below 2^-126).
+__device__ __forceinline__ float pow2i(float e) {
+    const int i = (int)e;
+    return i < -126 ? 0.f : __uint_as_float((uint32_t)(127 + i) << 23);
+}
+
+// One thread per 16-byte image chunk (8 features of one row). The head's runs are brought to one
+// reference stabiliser C (the largest D over its runs and features): each run's feature row r is
+// weighted by 2^(D_r - C), exactly, and summed in CTA order. The sums are scaled by 2^(15 - e),
+// 2^e exceeding the bound sum_runs max_warp amax 2^(Dmax - C) on their magnitude, and rounded to
+// fp16. Grid: (chunks / 128, heads).
 __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
     const int bh = blockIdx.y;
     const int c_first = flat_first_cta(p.f, bh), c_last = flat_last_cta(p.f, bh);
     const int halves = p.m / 128, nhs = p.d / 64;
-    float amax = 0.f;
+    float C = -INFINITY;
     for (int c = c_first; c <= c_last; ++c)
-        for (int w = 0; w < 4 * halves; ++w) amax = fmaxf(amax, p.part_amax[(size_t)(c + bh) * 8 + w]);
-    const float bound = amax * (float)(c_last - c_first + 1);
+        for (int w = 0; w < 4 * halves; ++w) C = fmaxf(C, p.part_Dmax[(size_t)(c + bh) * 8 + w]);
+    float bound = 0.f;
+    for (int c = c_first; c <= c_last; ++c) {
+        float b = 0.f;
+        for (int w = 0; w < 4 * halves; ++w) {
+            const size_t i = (size_t)(c + bh) * 8 + w;
+            b = fmaxf(b, p.part_amax[i] * pow2i(p.part_Dmax[i] - C));
+        }
+        bound += b;
+    }
     int ex = 0;
     frexpf(bound, &ex);  // bound < 2^ex
     const float scale = bound > 0.f ? ldexpf(1.f, 15 - ex) : 1.f;
@@ -73,16 +92,18 @@ __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
         const int col = row < 64 ? nh * 64 + row : p.d;
         const int r0 = h * 128 + kb * 64 + 8 * (pch ^ (row & 7));
         for (int c = c_first; c <= c_last; ++c) {
-            const float4 *src = (const float4 *)(p.part + ((size_t)(c + bh) * (p.d + 1) + col) * p.m + r0);
-            const float4 a = src[0], b = src[1];
-            v[0] += a.x;
-            v[1] += a.y;
-            v[2] += a.z;
-            v[3] += a.w;
-            v[4] += b.x;
-            v[5] += b.y;
-            v[6] += b.z;
-            v[7] += b.w;
+            const size_t slot = (size_t)(c + bh);
+            const float4 *src = (const float4 *)(p.part + (slot * (p.d + 1) + col) * p.m + r0);
+            const float4 *dd = (const float4 *)(p.part_D + slot * p.m + r0);
+            const float4 a = src[0], b = src[1], da = dd[0], db = dd[1];
+            v[0] = fmaf(a.x, pow2i(da.x - C), v[0]);
+            v[1] = fmaf(a.y, pow2i(da.y - C), v[1]);
+            v[2] = fmaf(a.z, pow2i(da.z - C), v[2]);
+            v[3] = fmaf(a.w, pow2i(da.w - C), v[3]);
+            v[4] = fmaf(b.x, pow2i(db.x - C), v[4]);
+            v[5] = fmaf(b.y, pow2i(db.y - C), v[5]);
+            v[6] = fmaf(b.z, pow2i(db.z - C), v[6]);
+            v[7] = fmaf(b.w, pow2i(db.w - C), v[7]);
         }
     }
     uint4 u;

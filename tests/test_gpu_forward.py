@@ -91,6 +91,29 @@ def test_bf16_many_short_heads(cuda_device):
     assert rel_max_err(out, oracle_fwd(x, W64, False)) <= TOL["bf16"]
 
 
+def test_bf16_key_stabiliser_raised_within_a_range(cuda_device):
+    # 300 key tiles of 64 tokens over at most 148 persistent CTAs (3 consecutive tiles each). Keys
+    # k_j = a w_0 + noise with a = 0.2, 0.6, 1.0 on tiles 0, 1, 2 (mod 3): u_0 climbs by ~15 nats
+    # inside every CTA's range, so the per-feature stabiliser set on a range's first tile is raised
+    # on the next ones and the accumulated state rescaled. Queries lean towards w_0 as well, so
+    # the feature that dominates the keys is not one the queries discount.
+    w = Workload("t", 1, 1, 64 * 300, 64, 256, False, "bf16", False, 2, 58)
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    w0 = W64[0].astype(np.float32)[None, :]
+    a = np.array([0.2, 0.6, 1.0], dtype=np.float32)[(np.arange(w.L) // 64) % 3][:, None]
+    x["K"][0, 0] = a * w0 + 0.3 * x["K"][0, 0]
+    x["Q"][0, 0] = 0.1 * w0 + x["Q"][0, 0]
+    x["K"] = round_to_bf16(x["K"])
+    x["Q"] = round_to_bf16(x["Q"])
+    K64 = x["K"][0, 0].astype(np.float64)
+    u0 = K64 @ W64[0] - 0.5 * (K64 ** 2).sum(1)
+    assert u0[128:192].max() - u0[:64].max() > 12.0  # nats: more than the 2^15 headroom of fp16
+    out = run_fwd(w, x, Wr, cuda_device, causal=False)
+    assert np.isfinite(out).all()
+    assert rel_max_err(out, oracle_fwd(x, W64, False)) <= TOL["bf16"]
+
+
 def test_bf16_value_tiles_of_very_different_magnitude(cuda_device):
     # One key tile's values near 3e4 and another's near 1e-5: the per-tile power-of-two scaling
     # of V keeps both inside fp16's normal range.
