@@ -92,6 +92,35 @@ __device__ __forceinline__ bool mbar_wait_all(uint64_t *bar, uint32_t parity, vo
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
 
+// mbar_wait for a warp whose wait is off the critical path (producers that run ahead): lane 0
+// polls, sleeping between polls so that the shared-memory pipe stays free for the consumers.
+__device__ __forceinline__ bool mbar_wait_lazy(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    int ok = 1;
+    if ((threadIdx.x & 31u) == 0) {
+        const uint32_t a = smem_u32(bar);
+        if (!mbar_try_wait(a, parity)) {
+            const unsigned long long t0 = globaltimer_ns();
+            for (uint32_t it = 1;; ++it) {
+                __nanosleep(64);
+                if (mbar_try_wait(a, parity)) break;
+                if ((it & 15u) == 0) {
+                    if (*abort) { ok = 0; break; }
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        record_status(FAVOR_ERR_TIMEOUT);
+                        *abort = 1;
+                        ok = 0;
+                        break;
+                    }
+                }
+            }
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    // the other lanes observe the completed phase too (acquire for their own later accesses)
+    if (ok && (threadIdx.x & 31u) != 0) ok = mbar_try_wait(smem_u32(bar), parity) ? 1 : 0;
+    return __all_sync(0xffffffffu, ok != 0);
+}
+
 // -------------------------------------------------------------------------------- TMA / bulk copy
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {

@@ -80,7 +80,12 @@ __device__ __forceinline__ float key_sq_norm(const uint8_t *tile, int row) {
 // Warp roles (16 warps): 0-3 convert V, write the ones column and the biases B_j; 4-7 / 8-11
 // exponentials of feature half 0 / 1 and the run-end write; 12 TMA; 13 MMA issue; 14 the tile's
 // largest |v|; 15 idle.
-// TMEM columns: P_h^T [64h, +64), phi'_h [128 + 32h, +32) (fp16 pairs), [S_h | z_h] [192 + h*ON, +ON).
+// P_h^T is double-buffered where TMEM allows (d = 64): the projection of tile g+2 runs while tile g+1
+// is loaded and tile g's exponentials are computed. The -D_r ln2 it accumulates onto is written
+// when the buffer is released, two tiles ahead; the exponent warpgroup corrects by the difference
+// to the current D_r (zero unless D_r changed in between: a raise, or a run boundary).
+// TMEM columns: P_h^T [64 (NPB h + b), +64), phi'_h [T_PHI + 32h, +32) (fp16 pairs),
+// [S_h | z_h] [T_PHI + 64 + h*ON, +ON).
 
 struct KeyStateParams2 {
     int L, m;
@@ -104,7 +109,8 @@ struct KeyCfg {
     static constexpr uint32_t TILE = KB * kKeyTile * 128;  // K or V tile
     static constexpr uint32_t ONES = kKeyTile * 128;
     static constexpr uint32_t STAGE = 2 * TILE + ONES;     // K tile | V tile | ones block
-    static constexpr uint32_t T_PHI = 128, T_S = 192;
+    static constexpr int NPB = D == 64 ? 2 : 1;              // P buffers per half (TMEM allowing)
+    static constexpr uint32_t T_PHI = 128 * NPB, T_S = T_PHI + 64;
 };
 
 // t = v log2e + B_j for a row of 64 logits (in place); returns the row's largest t.
@@ -200,8 +206,9 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
     int *sShift = (int *)(sBias + STAGES * kKeyTile);               // [STAGES] (16-int slot)
     uint64_t *bars = (uint64_t *)(sShift + 16);
     uint64_t *full = bars, *empty = full + STAGES, *vmax_full = empty + STAGES, *conv_full = vmax_full + STAGES;
-    uint64_t *w_full = conv_full + STAGES, *p_full = w_full + 1, *p_free = p_full + 2;
-    uint64_t *phi_full = p_free + 2, *phi_free = phi_full + 2, *acc_full = phi_free + 2, *acc_empty = acc_full + 2;
+    // p_full / p_free: one barrier per (half, P buffer), so no waiter can fall two phases behind
+    uint64_t *w_full = conv_full + STAGES, *p_full = w_full + 1, *p_free = p_full + 4;
+    uint64_t *phi_full = p_free + 4, *phi_free = phi_full + 2, *acc_full = phi_free + 2, *acc_empty = acc_full + 2;
     uint64_t *drain = acc_empty + 2;
     uint32_t *tmem_slot = (uint32_t *)(drain + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
@@ -225,9 +232,11 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
             mbar_init(&conv_full[s], 128);
         }
         mbar_init(w_full, 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&p_full[i], 1);
+            mbar_init(&p_free[i], 128);
+        }
         for (int h = 0; h < 2; ++h) {
-            mbar_init(&p_full[h], 1);
-            mbar_init(&p_free[h], 128);
             mbar_init(&phi_full[h], 128);
             mbar_init(&phi_free[h], 1);
             mbar_init(&acc_full[h], 1);
@@ -263,7 +272,7 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
             int issued = 0;
             for (int g = 0; g < n; ++g) {
                 const int s = g % STAGES, fl = f0 + g;
-                if (!mbar_wait_all(&empty[s], ((g / STAGES) & 1) ^ 1, abort_flag)) break;
+                if (!mbar_wait_lazy(&empty[s], ((g / STAGES) & 1) ^ 1, abort_flag)) break;
                 if (elect_one()) {
                     mbar_arrive_expect_tx(&full[s], 2 * C::TILE);
                     uint8_t *st = sStage + (size_t)s * C::STAGE;
@@ -283,7 +292,7 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
             // Largest |v| of each V tile (bf16 magnitudes compared as integers) -> b_t.
             for (int g = 0; g < n; ++g) {
                 const int s = g % STAGES;
-                if (!mbar_wait_all(&full[s], (g / STAGES) & 1, abort_flag)) break;
+                if (!mbar_wait_lazy(&full[s], (g / STAGES) & 1, abort_flag)) break;
                 const uint8_t *vt = sStage + (size_t)s * C::STAGE + C::TILE;
                 uint32_t mx = 0;
 #pragma unroll 4
@@ -311,35 +320,40 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
             const uint32_t idesc2 = make_idesc(128, ON, kFmtF16, 0, 1);
             const uint64_t dW = make_sdesc(smem_u32(sW), 16, 1024), dS = make_sdesc(smem_u32(sStage), 16, 1024);
             const uint64_t dV = make_sdesc(smem_u32(sStage) + C::TILE, kKeyTile * 128, 1024);
+            constexpr int NPB = C::NPB;
             auto project = [&](int g, int h) {
                 const uint64_t a = dW + (uint32_t)h * (128 * 128 / 16);
                 const uint64_t b = dS + (uint32_t)(g % STAGES) * (C::STAGE / 16);
+                const uint32_t d = tmem + (uint32_t)(h * NPB + g % NPB) * 64;
                 if (elect_one()) {
-                    // the first projection has no stored -D_r ln2 to accumulate onto (D_r = 0)
-                    mma_ss_x4(tmem + h * 64, a, b, idesc1, g > 0 ? 1u : 0u, 2, 2);
-                    if (KB == 2)
-                        mma_ss_x4(tmem + h * 64, a + (uint32_t)p.m * 8, b + kKeyTile * 128 / 16, idesc1, 1u, 2, 2);
-                    mma_commit(&p_full[h]);
+                    // the first NPB projections have no stored -D_r ln2 to accumulate onto
+                    mma_ss_x4(d, a, b, idesc1, g >= NPB ? 1u : 0u, 2, 2);
+                    if (KB == 2) mma_ss_x4(d, a + (uint32_t)p.m * 8, b + kKeyTile * 128 / 16, idesc1, 1u, 2, 2);
+                    mma_commit(&p_full[h * 2 + g % NPB]);
                 }
                 __syncwarp();
             };
             int runs[2] = {0, 0};
-            bool ok = mbar_wait_all(w_full, 0, abort_flag) && mbar_wait_all(&full[0], 0, abort_flag);
-            if (ok) {
+            bool ok = mbar_wait_all(w_full, 0, abort_flag);
+            for (int g = 0; ok && g < min(NPB, n); ++g) {
+                if (!mbar_wait_all(&full[g % STAGES], (g / STAGES) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                for (int h = 0; h < halves; ++h) project(0, h);
+                for (int h = 0; h < halves; ++h) project(g, h);
             }
+            // the projection of tile g2 into the buffer tile g2 - NPB used, once that is released
+            auto project_next = [&](int g2, int g) {
+                if (!mbar_wait_all(&full[g2 % STAGES], (g2 / STAGES) & 1, abort_flag)) return false;
+                for (int h = 0; h < halves; ++h) {
+                    if (!mbar_wait_all(&p_free[h * 2 + g % NPB], (g / NPB) & 1, abort_flag)) return false;
+                    tc_fence_after();
+                    project(g2, h);
+                }
+                return true;
+            };
             for (int g = 0; ok && g < n; ++g) {
                 const int s = g % STAGES;
-                if (g + 1 < n) {
-                    if (!mbar_wait_all(&full[(g + 1) % STAGES], ((g + 1) / STAGES) & 1, abort_flag)) break;
-                    for (int h = 0; ok && h < halves; ++h) {
-                        if (!mbar_wait_all(&p_free[h], g & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
-                        project(g + 1, h);
-                    }
-                    if (!ok) break;
-                }
+                // single-buffered P: the next projection goes ahead of this tile's state MMAs
+                if (NPB == 1 && g + 1 < n && !project_next(g + 1, g)) break;
                 if (!mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag)) break;
                 const bool first = first_of_run(g), last = last_of_run(g);
                 const uint64_t vd = dV + (uint32_t)s * (C::STAGE / 16);
@@ -361,6 +375,8 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 if (!ok) break;
                 if (elect_one()) mma_commit(&empty[s]);
                 __syncwarp();
+                // double-buffered P: the projection two tiles ahead, into the buffer this tile used
+                if (NPB == 2 && g + 2 < n && !project_next(g + 2, g)) break;
             }
             if (elect_one()) mma_commit(drain);
             __syncwarp();
@@ -371,36 +387,56 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
         regs_inc<184>();
         const int h = (warp - 4) >> 2, row = (warp & 3) * 32 + lane;
         if (h < halves) {
+            constexpr int NPB = C::NPB;
             const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
-            const uint32_t tP = tmem + lane_off + h * 64, tS = tmem + lane_off + C::T_S + h * ON;
+            const uint32_t tP = tmem + lane_off + h * NPB * 64, tS = tmem + lane_off + C::T_S + h * ON;
             int runs = 0;
-            float Dr = 0.f;  // this feature's stabiliser D_r in the current run
-            for (int g = 0; g < n; ++g) {
-                const int s = g % STAGES;
-                if (!mbar_wait_all(&p_full[h], g & 1, abort_flag)) break;
-                if (!mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag)) break;
+            float Dr = 0.f;                        // this feature's stabiliser D_r in the current run
+            float fillD[2] = {0.f, 0.f};           // D_r the buffer's stored -D_r ln2 stands for
+            float v[64];
+            if (n > 0 && mbar_wait_all(&p_full[h * 2], 0, abort_flag)) {
                 tc_fence_after();
-                float v[64];
                 tmem_ld64_nowait(tP, v);
+            }
+            for (int g = 0; g < n; ++g) {
+                const int s = g % STAGES, b = g % NPB;
+                if (!mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag)) break;
                 asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&v[0])), FAVOR_RW32((&v[32]))::"memory");
-                const float tmax = key_logits(v, sBias + s * kKeyTile);
-                const float lim = kKeyFeatureShift + (float)sShift[s];  // target for the row's largest t
                 const bool first = first_of_run(g), last = last_of_run(g);
+                const float Dbase = first ? 0.f : Dr;
+                // the buffer's projection accumulated onto -fillD ln2; bring it to Dbase
+                const float corr = Dbase - fillD[b];
+                float tmax = key_logits(v, sBias + s * kKeyTile);
+                if (__any_sync(0xffffffffu, corr != 0.f)) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) v[e] -= corr;
+                    tmax -= corr;
+                }
+                const float lim = kKeyFeatureShift + (float)sShift[s];  // target for the row's largest t
                 // new stabiliser: on a run's first tile always, later only when 2^t would overflow fp16
                 const float delta = (first || tmax > 15.f) ? ceilf(tmax - lim) : 0.f;
-                const bool any_shift = __any_sync(0xffffffffu, delta != 0.f);
-                if (any_shift) {
+                if (__any_sync(0xffffffffu, delta != 0.f)) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e) v[e] -= delta;
-                    Dr += delta;
                 }
-                // the next tile's projection accumulates onto -D_r ln2 (0 when it starts a new run)
-                tmem_fill64(tP, last ? 0.f : -Dr * kLn2);
-                tmem_wait_st();
+                Dr = Dbase + delta;
+                // release this buffer for tile g + NPB, with -D_r ln2 as the value it accumulates onto
+                // (0 if that tile starts a new run)
+                if (g + NPB < n) {
+                    fillD[b] = first_of_run(g + NPB) ? 0.f : Dr;
+                    tmem_fill64(tP + b * 64, -fillD[b] * kLn2);
+                    tmem_wait_st();
+                }
                 tc_fence_before();
-                mbar_arrive(&p_free[h]);
+                mbar_arrive(&p_free[h * 2 + b]);
                 uint32_t hv[32];
                 key_features<POLY>(v, hv);
+                // prefetch the next tile's logits (its projection ran meanwhile)
+                if (g + 1 < n) {
+                    if (!mbar_wait_all(&p_full[h * 2 + (g + 1) % NPB], ((g + 1) / NPB) & 1, abort_flag)) break;
+                    tc_fence_after();
+                    tmem_ld64_nowait(tP + ((g + 1) % NPB) * 64, v);
+                }
                 if (g > 0 && !mbar_wait_all(&phi_free[h], (g - 1) & 1, abort_flag)) break;
                 tc_fence_after();
                 // a raised stabiliser rescales the row's accumulated [S | z] (the previous tile's
@@ -422,14 +458,17 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                     for (int c0 = 0; c0 < D; c0 += 64) {
                         float w[64];
                         tmem_ld64_nowait(tS + c0, w);
-                        asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&w[0])), FAVOR_RW32((&w[32]))::"memory");
+                        asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&w[0])), FAVOR_RW32((&w[32])),
+                                     FAVOR_RW32((&v[0])), FAVOR_RW32((&v[32]))::"memory");
 #pragma unroll
                         for (int c = 0; c < 64; ++c) {
                             dst[(size_t)(c0 + c) * p.m] = w[c];
                             amax = fmaxf(amax, fabsf(w[c]));
                         }
                     }
-                    const float z = tmem_ld1(tS + D);
+                    float z;
+                    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=f"(z) : "r"(tS + D));
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+f"(z), FAVOR_RW32((&v[0])), FAVOR_RW32((&v[32]))::"memory");
                     dst[(size_t)D * p.m] = z;
                     amax = fmaxf(amax, z);
                     p.part_D[rs * p.m + h * 128 + row] = Dr;
@@ -444,7 +483,6 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                         p.part_amax[rs * 8 + h * 4 + (warp & 3)] = amax;
                         p.part_Dmax[rs * 8 + h * 4 + (warp & 3)] = dmax;
                     }
-                    Dr = 0.f;
                     ++runs;
                 }
             }
@@ -456,7 +494,7 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
         const int j = threadIdx.x;
         for (int g = 0; g < n; ++g) {
             const int s = g % STAGES, fl = f0 + g, t = fl % nt;
-            if (!mbar_wait_all(&vmax_full[s], (g / STAGES) & 1, abort_flag)) break;
+            if (!mbar_wait_lazy(&vmax_full[s], (g / STAGES) & 1, abort_flag)) break;
             uint8_t *st = sStage + (size_t)s * C::STAGE;
             const int b = sShift[s];
             const float scale = __uint_as_float((uint32_t)(127 - b) << 23);  // 2^-b
@@ -492,7 +530,7 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
 template <int D>
 static size_t key_partials_smem(int m) {
     using C = KeyCfg<D>;
-    return 1024 + (size_t)C::KB * m * 128 + (size_t)C::STAGES * C::STAGE + C::STAGES * kKeyTile * 4 + 64 + 512;
+    return 1024 + (size_t)C::KB * m * 128 + (size_t)C::STAGES * C::STAGE + C::STAGES * kKeyTile * 4 + 64 + 640;
 }
 
 // The register split of k_key_partials (80 + 2 x 184 + 56 per warpgroup lane) fits the 128 per

@@ -63,24 +63,53 @@ __device__ __forceinline__ float pow2i(float e) {
 // 2^e exceeding the bound sum_runs max_warp amax 2^(Dmax - C) on their magnitude, and rounded to
 // fp16. Grid: (chunks / 128, heads).
 __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
+    __shared__ float sC, sScale, sStat[kImageThreads];
     const int bh = blockIdx.y;
     const int c_first = flat_first_cta(p.f, bh), c_last = flat_last_cta(p.f, bh);
     const int halves = p.m / 128, nhs = p.d / 64;
-    float C = -INFINITY;
-    for (int c = c_first; c <= c_last; ++c)
-        for (int w = 0; w < 4 * halves; ++w) C = fmaxf(C, p.part_Dmax[(size_t)(c + bh) * 8 + w]);
-    float bound = 0.f;
-    for (int c = c_first; c <= c_last; ++c) {
-        float b = 0.f;
-        for (int w = 0; w < 4 * halves; ++w) {
-            const size_t i = (size_t)(c + bh) * 8 + w;
-            b = fmaxf(b, p.part_amax[i] * pow2i(p.part_Dmax[i] - C));
+    // per-(run, warp) statistics, one per thread (a head spans at most a few runs)
+    const int nstat = (c_last - c_first + 1) * 8;
+    float dm = -INFINITY, am = 0.f;
+    for (int i = threadIdx.x; i < nstat; i += kImageThreads) {
+        if ((i & 7) < 4 * halves) {
+            const size_t k = (size_t)(c_first + (i >> 3) + bh) * 8 + (i & 7);
+            dm = fmaxf(dm, p.part_Dmax[k]);
         }
-        bound += b;
     }
-    int ex = 0;
-    frexpf(bound, &ex);  // bound < 2^ex
-    const float scale = bound > 0.f ? ldexpf(1.f, 15 - ex) : 1.f;
+    sStat[threadIdx.x] = dm;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float C = -INFINITY;
+        for (int i = 0; i < kImageThreads; ++i) C = fmaxf(C, sStat[i]);
+        sC = C;
+    }
+    __syncthreads();
+    const float C = sC;
+    for (int i = threadIdx.x; i < nstat; i += kImageThreads)
+        if ((i & 7) < 4 * halves) {
+            const size_t k = (size_t)(c_first + (i >> 3) + bh) * 8 + (i & 7);
+            am = fmaxf(am, p.part_amax[k] * pow2i(p.part_Dmax[k] - C));  // per run the max over warps...
+        }
+    // ... summed over runs: every run's warps are taken by consecutive threads (8 per run), so the
+    // bound is the sum over runs of the max over that run's 8 threads' values
+    sStat[threadIdx.x] = am;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float bound = 0.f;
+        for (int r = 0; r < min(nstat, kImageThreads) / 8; ++r) {
+            float b = 0.f;
+            for (int w = 0; w < 8; ++w) b = fmaxf(b, sStat[r * 8 + w]);
+            bound += b;
+        }
+        // runs beyond the first kImageThreads / 8 (very short heads over many CTAs) were folded by
+        // the strided loop into those threads' maxima: adding them per run keeps the bound valid
+        if (nstat > kImageThreads) bound *= (float)((nstat + kImageThreads - 1) / kImageThreads);
+        int ex = 0;
+        frexpf(bound, &ex);  // bound < 2^ex
+        sScale = bound > 0.f ? ldexpf(1.f, 15 - ex) : 1.f;
+    }
+    __syncthreads();
+    const float scale = sScale;
 
     const int chunks = nhs * halves * 2 * kImgRows * 8;
     const int q = blockIdx.x * kImageThreads + threadIdx.x;
@@ -282,7 +311,7 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             for (int g = 0; g < n_items; ++g) {
                 const ItemInfo it = item_info<NH>(g, f0, f1, nt);
                 const int s = g % STAGES;
-                if (!mbar_wait_all(&empty[s], ((g / STAGES) & 1) ^ 1, abort_flag)) break;
+                if (!mbar_wait_lazy(&empty[s], ((g / STAGES) & 1) ^ 1, abort_flag)) break;
                 if (elect_one()) {
                     mbar_arrive_expect_tx(&full[s], C::Q_TILE);
                     for (int kb = 0; kb < KB; ++kb)
@@ -302,7 +331,7 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             for (int g = 0; g < n_items; ++g) {
                 const ItemInfo it = item_info<NH>(g, f0, f1, nt);
                 if (!it.first_of_group) continue;
-                if (!mbar_wait_all(img_empty, (it.group & 1) ^ 1, abort_flag)) break;
+                if (!mbar_wait_lazy(img_empty, (it.group & 1) ^ 1, abort_flag)) break;
                 if (elect_one()) {
                     mbar_arrive_expect_tx(img_full, img_bytes);
                     const uint8_t *src = p.image + (size_t)it.bh * p.image_stride + (size_t)it.nh * img_bytes;
