@@ -29,28 +29,45 @@ struct ScanParams {
     float *seg_state;       // [BH, n_split, state_floats]: exclusive prefix per segment
 };
 
-// One thread per state element, walking the segments in order (grid: element blocks x heads).
+// One thread per position of the state image (so the image writes are coalesced), walking the
+// segments in order with the loads of four segments in flight (grid: element blocks x heads).
 __global__ void __launch_bounds__(256) k_state_scan(ScanParams p) {
     const int bh = blockIdx.y;
     const size_t md = (size_t)p.m * p.d, sf = state_floats(p.m, p.d);
     float *base = p.seg_state + (size_t)bh * p.n_split * sf;
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < md) {
-        const int r = (int)(i / p.d), c = (int)(i % p.d);
-        const uint32_t off = state_image_offset(r, c, p.m);
-        const float *src = p.part_S + (size_t)bh * p.n_split * md + i;
+        // image byte offset 4i -> (r, c), the inverse of state_image_offset
+        const uint32_t B = (uint32_t)i * 4u, half = (uint32_t)p.m * 256u;
+        const uint32_t nh = B / half, rem = B % half, kb = rem / 8192u, rem2 = rem % 8192u;
+        const uint32_t cc = rem2 / 128u, phys = (rem2 % 128u) / 16u, pos = (rem2 % 16u) / 4u;
+        const int r = (int)(kb * 32u + ((phys ^ (cc & 7u)) * 4u) + pos), c = (int)(nh * 64u + cc);
+        const float *src = p.part_S + (size_t)bh * p.n_split * md + (size_t)r * p.d + c;
         float run = 0.f;
-        for (int s = 0; s < p.n_split; ++s) {
-            *(float *)((uint8_t *)(base + (size_t)s * sf) + off) = tf32_store(run);
-            run += src[(size_t)s * md];
+        int sg = 0;
+        for (; sg + 4 <= p.n_split; sg += 4) {
+            const float a0 = src[(size_t)sg * md], a1 = src[(size_t)(sg + 1) * md];
+            const float a2 = src[(size_t)(sg + 2) * md], a3 = src[(size_t)(sg + 3) * md];
+            base[(size_t)sg * sf + i] = tf32_store(run);
+            run += a0;
+            base[(size_t)(sg + 1) * sf + i] = tf32_store(run);
+            run += a1;
+            base[(size_t)(sg + 2) * sf + i] = tf32_store(run);
+            run += a2;
+            base[(size_t)(sg + 3) * sf + i] = tf32_store(run);
+            run += a3;
+        }
+        for (; sg < p.n_split; ++sg) {
+            base[(size_t)sg * sf + i] = tf32_store(run);
+            run += src[(size_t)sg * md];
         }
     } else if (i < md + p.m) {
         const int r = (int)(i - md);
         const float *src = p.part_z + (size_t)bh * p.n_split * p.m + r;
         float run = 0.f;
-        for (int s = 0; s < p.n_split; ++s) {
-            base[(size_t)s * sf + md + r] = run;
-            run += src[(size_t)s * p.m];
+        for (int sg = 0; sg < p.n_split; ++sg) {
+            base[(size_t)sg * sf + md + r] = run;
+            run += src[(size_t)sg * p.m];
         }
     } else if (i < md + p.m + p.n_split) {
         float *t = base + (i - md - p.m) * sf + md + p.m;
@@ -58,8 +75,6 @@ __global__ void __launch_bounds__(256) k_state_scan(ScanParams p) {
         t[1] = t[2] = t[3] = 0.f;
     }
 }
-
-// ============================================================================ exact prefix
 
 struct PrefixParams {
     int L, d, m, P;              // P = tokens per head recomputed exactly
@@ -73,89 +88,134 @@ struct PrefixParams {
 
 __device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
-// Warp per token: phi(q) = exp(w.q - max_r w.q), phi(k) = exp(w.k - |k|^2/2 - C), fp32.
+// phi(q) = exp(w.q - max_r w.q) and phi(k) = exp(w.k - |k|^2/2 - C) in fp32 for the first P tokens
+// of each head. CTA per (32 tokens, head); thread r computes feature r (its W row in registers)
+// for all 32 tokens; the per-token max over features goes through shared memory.
 __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) {
-    __shared__ float xs[8][2][128];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.y, j = blockIdx.x * 8 + warp;
-    if (j >= p.P) return;
-    const size_t row = ((size_t)bh * p.L + j) * p.d;
-    for (int e = lane; e < p.d; e += 32) {
-        xs[warp][0][e] = bf16_to_f(p.Q[row + e]);
-        xs[warp][1][e] = bf16_to_f(p.K[row + e]);
+    __shared__ uint16_t xq[32][64], xk[32][64];
+    __shared__ float su[32][256], smax[32];
+    const int bh = blockIdx.y, j0 = blockIdx.x * 32, t = threadIdx.x;
+    for (int idx = t; idx < 32 * 64; idx += 256) {
+        const int a = idx >> 6, e = idx & 63;
+        const int j = j0 + a;
+        const size_t row = ((size_t)bh * p.L + j) * p.d;
+        xq[a][e] = (j < p.P && e < p.d) ? p.Q[row + e] : (uint16_t)0;
+        xk[a][e] = (j < p.P && e < p.d) ? p.K[row + e] : (uint16_t)0;
     }
-    __syncwarp();
-    const float C = p.head_max[bh], bj = p.bias[(size_t)bh * p.L + j];
-    float uq[16];
-    float qmax = -INFINITY;
-    for (int k = 0; k < p.m / 32; ++k) {
-        const int r = lane + 32 * k;
-        float sq = 0.f, sk = 0.f;
-        for (int e = 0; e < p.d; ++e) {
-            const float w = bf16_to_f(p.W[(size_t)r * p.d + e]);
-            sq = fmaf(w, xs[warp][0][e], sq);
-            sk = fmaf(w, xs[warp][1][e], sk);
+    __syncthreads();
+    const float C = p.head_max[bh];
+    if (t < p.m) {
+        float w[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) w[e] = e < p.d ? bf16_to_f(p.W[(size_t)t * p.d + e]) : 0.f;
+        for (int a = 0; a < 32; ++a) {
+            float sq0 = 0.f, sq1 = 0.f, sk0 = 0.f, sk1 = 0.f;
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+                sq0 = fmaf(w[e], bf16_to_f(xq[a][e]), sq0);
+                sq1 = fmaf(w[e + 1], bf16_to_f(xq[a][e + 1]), sq1);
+                sk0 = fmaf(w[e], bf16_to_f(xk[a][e]), sk0);
+                sk1 = fmaf(w[e + 1], bf16_to_f(xk[a][e + 1]), sk1);
+            }
+            su[a][t] = sq0 + sq1;
+            const int j = j0 + a;
+            if (j < p.P) p.phiK[((size_t)bh * p.P + j) * p.m + t] = expf(sk0 + sk1 + p.bias[(size_t)bh * p.L + j] - C);
         }
-        uq[k] = sq;
-        qmax = fmaxf(qmax, sq);
-        p.phiK[((size_t)bh * p.P + j) * p.m + r] = expf(sk + bj - C);
     }
-    for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
-    for (int k = 0; k < p.m / 32; ++k)
-        p.phiQ[((size_t)bh * p.P + j) * p.m + lane + 32 * k] = expf(uq[k] - qmax);
+    __syncthreads();
+    {
+        const int warp = t >> 5, lane = t & 31;
+        for (int a = warp * 4; a < warp * 4 + 4; ++a) {
+            float mx = -INFINITY;
+            for (int r = lane; r < p.m; r += 32) mx = fmaxf(mx, su[a][r]);
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) smax[a] = mx;
+        }
+    }
+    __syncthreads();
+    if (t < p.m)
+        for (int a = 0; a < 32; ++a) {
+            const int j = j0 + a;
+            if (j < p.P) p.phiQ[((size_t)bh * p.P + j) * p.m + t] = expf(su[a][t] - smax[a]);
+        }
 }
 
-// 32 queries per CTA; key tiles of 32 up to the diagonal; scores and sums in fp32.
+// Masked attention over the first P tokens in fp32: CTA per (64 queries, head), 256 threads.
+// Per 64-key block up to the diagonal: scores S = phi(Q) phi(K)^T (4 x 4 per thread, features in
+// 32-wide slices through shared memory), the mask j <= i, then num += S V and den += rowsum(S)
+// (4 queries x 4 value columns per thread).
 __global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
-    extern __shared__ float sh[];
-    const int m = p.m, d = p.d;
-    float *sq = sh;                   // 32 x (m+1)
-    float *sk = sq + 32 * (m + 1);    // 32 x (m+1)
-    float *sv = sk + 32 * (m + 1);    // 32 x d
-    float *sa = sv + 32 * d;          // 32 x 33 scores
-    const int bh = blockIdx.y, i0 = blockIdx.x * 32, t = threadIdx.x;
-    const int qi = t >> 3, cg = t & 7;           // this thread: query qi, columns cg*(d/8)..
-    const int cols = d / 8;
-    for (int idx = t; idx < 32 * m; idx += 256) {
-        const int a = idx / m, r = idx % m;
-        sq[a * (m + 1) + r] = (i0 + a < p.P) ? p.phiQ[((size_t)bh * p.P + i0 + a) * m + r] : 0.f;
+    // the feature slices (score phase) and the masked scores (output phase) share one buffer
+    __shared__ __align__(16) float buf[64 * 65];
+    __shared__ __align__(16) float sv[64][64];  // V block
+    float(*aq)[64] = (float(*)[64])buf;         // [32 features][64 queries]
+    float(*ak)[64] = (float(*)[64])(buf + 32 * 64);
+    float(*ss)[65] = (float(*)[65])buf;         // [64 queries][64 keys + pad]
+    const int bh = blockIdx.y, i0 = blockIdx.x * 64, t = threadIdx.x;
+    const int ti = (t >> 4) * 4, tj = (t & 15) * 4;  // this thread's 4 x 4 score block / 4 x 4 output block
+    float num[4][4], den[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        den[a] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) num[a][c] = 0.f;
     }
-    float num[16];
-    for (int c = 0; c < 16; ++c) num[c] = 0.f;
-    float den = 0.f;
-    for (int j0 = 0; j0 <= i0 && j0 < p.P; j0 += 32) {
-        __syncthreads();
-        for (int idx = t; idx < 32 * m; idx += 256) {
-            const int a = idx / m, r = idx % m;
-            sk[a * (m + 1) + r] = (j0 + a < p.P) ? p.phiK[((size_t)bh * p.P + j0 + a) * m + r] : 0.f;
+    const float *phq = p.phiQ + (size_t)bh * p.P * p.m;
+    const float *phk = p.phiK + (size_t)bh * p.P * p.m;
+    for (int j0 = 0; j0 <= i0 && j0 < p.P; j0 += 64) {
+        float sc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) sc[a][b] = 0.f;
+        for (int f0 = 0; f0 < p.m; f0 += 32) {
+            __syncthreads();
+            for (int idx = t; idx < 64 * 32; idx += 256) {
+                const int a = idx >> 5, f = idx & 31;
+                aq[f][a] = (i0 + a < p.P) ? phq[(size_t)(i0 + a) * p.m + f0 + f] : 0.f;
+                ak[f][a] = (j0 + a < p.P) ? phk[(size_t)(j0 + a) * p.m + f0 + f] : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 8
+            for (int f = 0; f < 32; ++f) {
+                const float4 q4 = *(const float4 *)&aq[f][ti], k4 = *(const float4 *)&ak[f][tj];
+                const float qv[4] = {q4.x, q4.y, q4.z, q4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) sc[a][b] = fmaf(qv[a], kv[b], sc[a][b]);
+            }
         }
-        for (int idx = t; idx < 32 * d; idx += 256) {
-            const int a = idx / d, e = idx % d;
-            sv[a * d + e] = (j0 + a < p.P) ? bf16_to_f(p.V[((size_t)bh * p.L + j0 + a) * d + e]) : 0.f;
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) ss[ti + a][tj + b] = (j0 + tj + b <= i0 + ti + a) ? sc[a][b] : 0.f;
+        for (int idx = t; idx < 64 * 64; idx += 256) {
+            const int a = idx >> 6, e = idx & 63;
+            sv[a][e] = (j0 + a < p.P && e < p.d) ? bf16_to_f(p.V[((size_t)bh * p.L + j0 + a) * p.d + e]) : 0.f;
         }
         __syncthreads();
-        for (int idx = t; idx < 32 * 32; idx += 256) {
-            const int a = idx >> 5, b = idx & 31;
-            float s = 0.f;
-            for (int r = 0; r < m; ++r) s = fmaf(sq[a * (m + 1) + r], sk[b * (m + 1) + r], s);
-            sa[a * 33 + b] = (j0 + b <= i0 + a) ? s : 0.f;
-        }
-        __syncthreads();
-        for (int b = 0; b < 32; ++b) {
-            const float a = sa[qi * 33 + b];
-            if (cg == 0) den += a;
-            for (int c = 0; c < cols; ++c) num[c] = fmaf(a, sv[b * d + cg * cols + c], num[c]);
+        for (int j = 0; j < 64; ++j) {
+            const float4 v4 = *(const float4 *)&sv[j][tj];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const float sa = ss[ti + a][j];
+                num[a][0] = fmaf(sa, v4.x, num[a][0]);
+                num[a][1] = fmaf(sa, v4.y, num[a][1]);
+                num[a][2] = fmaf(sa, v4.z, num[a][2]);
+                num[a][3] = fmaf(sa, v4.w, num[a][3]);
+                den[a] += sa;
+            }
         }
     }
-    // den lives in the cg == 0 thread of each query; share it through the score buffer.
-    __syncthreads();
-    if (cg == 0) sa[qi * 33 + 32] = den;
-    __syncthreads();
-    den = sa[qi * 33 + 32];
-    const int i = i0 + qi;
-    if (i < p.P && i < p.L) {
-        float *o = p.out + ((size_t)bh * p.L + i) * d + cg * cols;
-        for (int c = 0; c < cols; ++c) o[c] = num[c] / den;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int i = i0 + ti + a;
+        if (i < p.P && i < p.L && tj < p.d) {
+            float *o = p.out + ((size_t)bh * p.L + i) * p.d + tj;
+            *(float4 *)o = make_float4(num[a][0] / den[a], num[a][1] / den[a], num[a][2] / den[a], num[a][3] / den[a]);
+        }
     }
 }
 
@@ -539,12 +599,10 @@ cudaError_t launch_state_scan(const ScanParams &p, int BH, cudaStream_t st) {
 
 cudaError_t launch_causal_prefix(const PrefixParams &p, int BH, cudaStream_t st) {
     if (p.P <= 0) return cudaSuccess;
-    k_causal_prefix_features<<<dim3((p.P + 7) / 8, BH), 256, 0, st>>>(p);
+    k_causal_prefix_features<<<dim3((p.P + 31) / 32, BH), 256, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t sm = (size_t)(2 * 32 * (p.m + 1) + 32 * p.d + 32 * 33) * sizeof(float);
-    cudaFuncSetAttribute(k_causal_prefix_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_causal_prefix_attn<<<dim3((p.P + 31) / 32, BH), 256, sm, st>>>(p);
+    k_causal_prefix_attn<<<dim3((p.P + 63) / 64, BH), 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
