@@ -65,10 +65,13 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Tokens per head that the causal path recomputes exactly in fp32 (see k_causal.cu).
 constexpr int kCausalExactPrefix = 512;
+// Row stride of the feature-major fp32 scratch of those tokens.
+int prefix_stride(int P) { return (P + 31) & ~31; }
 
 struct Bf16Layout {
     int BH, n_tiles, tiles_per_split, n_split, P_exact;
-    size_t off_bias, off_split_max, off_head_max, off_part_S, off_part_z, off_state, off_seg, off_phi, total;
+    size_t off_bias, off_split_max, off_head_max, off_part_S, off_part_z, off_state, off_seg_S, off_seg_z, off_phi,
+        total;
 };
 
 Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_ws, int causal = 0) {
@@ -91,10 +94,12 @@ Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_
     l.off_state = off;
     if (state_in_ws) off += align256((size_t)l.BH * state_floats(s->m, s->d) * 4);
     l.P_exact = causal ? std::min(s->L, kCausalExactPrefix) : 0;
-    l.off_seg = off;
-    if (causal) off += align256((size_t)l.BH * l.n_split * state_floats(s->m, s->d) * 4);
+    l.off_seg_S = off;
+    if (causal) off += align256((size_t)l.BH * l.n_split * s->m * s->d * 4);
+    l.off_seg_z = off;
+    if (causal) off += align256((size_t)l.BH * l.n_split * s->m * 4);
     l.off_phi = off;
-    if (causal) off += align256((size_t)2 * l.BH * l.P_exact * s->m * 4);
+    if (causal) off += align256((size_t)2 * l.BH * prefix_stride(l.P_exact) * s->m * 4);
     l.total = off;
     return l;
 }
@@ -170,13 +175,13 @@ bool make_token_map(CUtensorMap *map, const void *base, int BH, int L, int d, in
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [m, d] bf16 W as a 2-D map (d, m) with 64 x m boxes, 128-byte swizzle.
-bool make_w_map(CUtensorMap *map, const void *base, int m, int d) {
+// [m, d] bf16 W as a 2-D map (d, m) with 64 x rows boxes (rows = m by default), 128-byte swizzle.
+bool make_w_map(CUtensorMap *map, const void *base, int m, int d, int rows = 0) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)m};
     const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)m};
+    const cuuint32_t box[2] = {64, (cuuint32_t)(rows > 0 ? rows : m)};
     const cuuint32_t estr[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -245,9 +250,10 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     if (!causal) return fwd_bf16_bidir(s, Q, K, V, W, out, ctx, ws, ws_bytes, o, st);
     const Bf16Layout l = bf16_layout(s, o, ctx == nullptr, causal);
     if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
-    CUtensorMap mQ, mK, mW;
+    CUtensorMap mQ, mK, mV, mW, mW128;
     if (!make_token_map(&mQ, Q, l.BH, s->L, s->d) || !make_token_map(&mK, K, l.BH, s->L, s->d) ||
-        !make_w_map(&mW, W, s->m, s->d))
+        !make_token_map(&mV, V, l.BH, s->L, s->d) || !make_w_map(&mW, W, s->m, s->d) ||
+        !make_w_map(&mW128, W, s->m, s->d, 128))
         return FAVOR_ERR_CUDA;
     // Per-key -|k|^2/2 goes straight into the context (after the state blocks) when one is kept.
     float *bias = ctx ? (float *)((uint8_t *)ctx + align256((size_t)l.BH * state_floats(s->m, s->d) * 4))
@@ -256,7 +262,8 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     float *head_max = (float *)(ws + l.off_head_max);
     float *part_S = (float *)(ws + l.off_part_S);
     float *part_z = (float *)(ws + l.off_part_z);
-    float *state = ctx ? (float *)ctx : (float *)(ws + l.off_state);
+    float *seg_S = (float *)(ws + l.off_seg_S);
+    float *seg_z = (float *)(ws + l.off_seg_z);
 
     KeyMaxParams km{s->L, s->d, s->m, l.n_split, l.tiles_per_split, bias, split_max};
     record_stage(o, 0, st);
@@ -269,27 +276,26 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     e = launch_key_state(mK, mW, ks, l.BH, st);
     record_stage(o, 3, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-    if (causal) {
-        ScanParams sp{s->m, s->d, l.n_split, part_S, part_z, head_max, (float *)(ws + l.off_seg)};
-        record_stage(o, 4, st);
-        e = launch_state_scan(sp, l.BH, st);
-        record_stage(o, 5, st);
-        if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-        CausalParams cp{s->L, s->d, s->m, l.tiles_per_split, l.P_exact, (const uint16_t *)V, bias,
-                        (const float *)(ws + l.off_seg), l.n_split, out};
-        record_stage(o, 6, st);
-        e = launch_causal_out(mQ, mK, mW, cp, l.BH, st);
-        record_stage(o, 7, st);
-        if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-        float *phi = (float *)(ws + l.off_phi);
-        PrefixParams pp{s->L, s->d, s->m, l.P_exact, (const uint16_t *)Q, (const uint16_t *)K, (const uint16_t *)V,
-                        (const uint16_t *)W, bias, head_max, phi, phi + (size_t)l.BH * l.P_exact * s->m, out};
-        record_stage(o, 8, st);
-        e = launch_causal_prefix(pp, l.BH, st);
-        record_stage(o, 9, st);
-        return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
-    }
-    return FAVOR_ERR_INVALID_ARG;
+    ScanParams sp{s->m, s->d, l.n_split, 1.f * (1 << (int)kChunkKeyShift), part_S, part_z, seg_S, seg_z};
+    record_stage(o, 4, st);
+    e = launch_state_scan(sp, l.BH, st);
+    record_stage(o, 5, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    ChunkParams cp{s->L, s->m, l.n_split, l.tiles_per_split, l.P_exact, l.BH * l.n_split, bias, head_max,
+                   seg_S, seg_z, out};
+    record_stage(o, 6, st);
+    e = launch_causal_chunk(mQ, mK, mV, mW128, cp, opt_poly_pct(o), st);
+    record_stage(o, 7, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    float *phi = (float *)(ws + l.off_phi);
+    const int Ps = prefix_stride(l.P_exact);
+    PrefixParams pp{s->L, s->d, s->m, l.P_exact, Ps, (const uint16_t *)Q, (const uint16_t *)K,
+                    (const uint16_t *)V, (const uint16_t *)W, bias, head_max, phi,
+                    phi + (size_t)l.BH * Ps * s->m, out};
+    record_stage(o, 8, st);
+    e = launch_causal_prefix(pp, l.BH, st);
+    record_stage(o, 9, st);
+    return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 
 }  // namespace

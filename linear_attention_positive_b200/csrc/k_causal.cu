@@ -6,14 +6,13 @@
 //   out_i = phi(q_i)^T S_i / phi(q_i)^T z_i,   S_i = sum_{j<=i} phi(k_j) v_j^T,  z_i = sum_{j<=i} phi(k_j).
 //
 // Sequence parallelism: the sequence of each head is cut into segments (runs of 128-token
-// tiles). k_key_state (shared with the bidirectional path) gives each segment's aggregate
-// [S | z]; k_state_scan turns them into exclusive prefixes; k_causal_out walks each segment's
-// tiles in order from that prefix:
+// tiles). k_key_state gives each segment's aggregate [S | z]; k_state_scan turns them into
+// exclusive prefixes; k_causal_chunk walks each segment's tiles in order from that prefix:
 //   out_tile = ( phi(Q_t) S_<t + mask(phi(Q_t) phi(K_t)^T) V_t ) / ( phi(Q_t) z_<t + rowsum(mask(...)) ),
 //   S_<t+1 = S_<t + phi(K_t)^T V_t.
 // k_causal_prefix_* recompute the first tokens of every head in fp32 on CUDA cores: there the
 // output is a weighted mean of few values, its magnitude is far above the RMS of a long output,
-// and the 11-bit tf32 operands alone would use up the error budget.
+// and the 11-bit fp16 operands alone would use up the error budget.
 
 #include "common.cuh"
 
@@ -23,66 +22,60 @@ namespace favor {
 
 struct ScanParams {
     int m, d, n_split;
+    float scale;            // factor on the prefixes (the key shift 2^A of k_causal_chunk)
     const float *part_S;    // [BH, n_split, m, d]
     const float *part_z;    // [BH, n_split, m]
-    const float *head_max;  // [BH]
-    float *seg_state;       // [BH, n_split, state_floats]: exclusive prefix per segment
+    float *seg_S;           // [BH, n_split, m, d]: exclusive prefix of S per segment, times scale
+    float *seg_z;           // [BH, n_split, m]
 };
 
-// One thread per position of the state image (so the image writes are coalesced), walking the
-// segments in order with the loads of four segments in flight (grid: element blocks x heads).
+// One thread per element of [S | z] (coalesced across the segment records), walking the segments
+// in order with the loads of eight segments in flight (grid: element blocks x heads).
 __global__ void __launch_bounds__(256) k_state_scan(ScanParams p) {
     const int bh = blockIdx.y;
-    const size_t md = (size_t)p.m * p.d, sf = state_floats(p.m, p.d);
-    float *base = p.seg_state + (size_t)bh * p.n_split * sf;
+    const size_t md = (size_t)p.m * p.d;
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const float *src;
+    float *dst;
+    size_t stride;
     if (i < md) {
-        // image byte offset 4i -> (r, c), the inverse of state_image_offset
-        const uint32_t B = (uint32_t)i * 4u, half = (uint32_t)p.m * 256u;
-        const uint32_t nh = B / half, rem = B % half, kb = rem / 8192u, rem2 = rem % 8192u;
-        const uint32_t cc = rem2 / 128u, phys = (rem2 % 128u) / 16u, pos = (rem2 % 16u) / 4u;
-        const int r = (int)(kb * 32u + ((phys ^ (cc & 7u)) * 4u) + pos), c = (int)(nh * 64u + cc);
-        const float *src = p.part_S + (size_t)bh * p.n_split * md + (size_t)r * p.d + c;
-        float run = 0.f;
-        int sg = 0;
-        for (; sg + 4 <= p.n_split; sg += 4) {
-            const float a0 = src[(size_t)sg * md], a1 = src[(size_t)(sg + 1) * md];
-            const float a2 = src[(size_t)(sg + 2) * md], a3 = src[(size_t)(sg + 3) * md];
-            base[(size_t)sg * sf + i] = tf32_store(run);
-            run += a0;
-            base[(size_t)(sg + 1) * sf + i] = tf32_store(run);
-            run += a1;
-            base[(size_t)(sg + 2) * sf + i] = tf32_store(run);
-            run += a2;
-            base[(size_t)(sg + 3) * sf + i] = tf32_store(run);
-            run += a3;
-        }
-        for (; sg < p.n_split; ++sg) {
-            base[(size_t)sg * sf + i] = tf32_store(run);
-            run += src[(size_t)sg * md];
-        }
+        src = p.part_S + (size_t)bh * p.n_split * md + i;
+        dst = p.seg_S + (size_t)bh * p.n_split * md + i;
+        stride = md;
     } else if (i < md + p.m) {
-        const int r = (int)(i - md);
-        const float *src = p.part_z + (size_t)bh * p.n_split * p.m + r;
-        float run = 0.f;
-        for (int sg = 0; sg < p.n_split; ++sg) {
-            base[(size_t)sg * sf + md + r] = run;
-            run += src[(size_t)sg * p.m];
+        src = p.part_z + (size_t)bh * p.n_split * p.m + (i - md);
+        dst = p.seg_z + (size_t)bh * p.n_split * p.m + (i - md);
+        stride = p.m;
+    } else {
+        return;
+    }
+    float run = 0.f;
+    int sg = 0;
+    for (; sg + 8 <= p.n_split; sg += 8) {
+        float a[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a[k] = src[(size_t)(sg + k) * stride];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            dst[(size_t)(sg + k) * stride] = run * p.scale;
+            run += a[k];
         }
-    } else if (i < md + p.m + p.n_split) {
-        float *t = base + (i - md - p.m) * sf + md + p.m;
-        t[0] = p.head_max[bh];
-        t[1] = t[2] = t[3] = 0.f;
+    }
+    for (; sg < p.n_split; ++sg) {
+        const float a = src[(size_t)sg * stride];
+        dst[(size_t)sg * stride] = run * p.scale;
+        run += a;
     }
 }
 
 struct PrefixParams {
     int L, d, m, P;              // P = tokens per head recomputed exactly
+    int Ps;                      // row stride of the feature scratch: P rounded up to 32
     const uint16_t *Q, *K, *V;   // bf16 [BH, L, d]
     const uint16_t *W;           // bf16 [m, d]
     const float *bias;           // [BH, L]  -|k|^2/2
     const float *head_max;       // [BH]
-    float *phiQ, *phiK;          // [BH, P, m] fp32 scratch
+    float *phiQ, *phiK;          // [BH, m, Ps] fp32 scratch, feature-major
     float *out;                  // fp32 [BH, L, d]
 };
 
@@ -90,10 +83,12 @@ __device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float(
 
 // phi(q) = exp(w.q - max_r w.q) and phi(k) = exp(w.k - |k|^2/2 - C) in fp32 for the first P tokens
 // of each head. CTA per (32 tokens, head); thread r computes feature r (its W row in registers)
-// for all 32 tokens; the per-token max over features goes through shared memory.
+// for all 32 tokens and stores them as one contiguous run of its feature row; the per-token max
+// over features goes through shared memory.
 __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) {
     __shared__ uint16_t xq[32][64], xk[32][64];
-    __shared__ float su[32][256], smax[32];
+    __shared__ float su[32][257], smax[32];
+    __shared__ float sbias[32];
     const int bh = blockIdx.y, j0 = blockIdx.x * 32, t = threadIdx.x;
     for (int idx = t; idx < 32 * 64; idx += 256) {
         const int a = idx >> 6, e = idx & 63;
@@ -102,12 +97,14 @@ __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) 
         xq[a][e] = (j < p.P && e < p.d) ? p.Q[row + e] : (uint16_t)0;
         xk[a][e] = (j < p.P && e < p.d) ? p.K[row + e] : (uint16_t)0;
     }
+    if (t < 32) sbias[t] = j0 + t < p.P ? p.bias[(size_t)bh * p.L + j0 + t] - p.head_max[bh] : -INFINITY;
     __syncthreads();
-    const float C = p.head_max[bh];
+    float w[64];
     if (t < p.m) {
-        float w[64];
 #pragma unroll
         for (int e = 0; e < 64; ++e) w[e] = e < p.d ? bf16_to_f(p.W[(size_t)t * p.d + e]) : 0.f;
+        float ok[32];
+#pragma unroll
         for (int a = 0; a < 32; ++a) {
             float sq0 = 0.f, sq1 = 0.f, sk0 = 0.f, sk1 = 0.f;
 #pragma unroll
@@ -118,9 +115,11 @@ __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) 
                 sk1 = fmaf(w[e + 1], bf16_to_f(xk[a][e + 1]), sk1);
             }
             su[a][t] = sq0 + sq1;
-            const int j = j0 + a;
-            if (j < p.P) p.phiK[((size_t)bh * p.P + j) * p.m + t] = expf(sk0 + sk1 + p.bias[(size_t)bh * p.L + j] - C);
+            ok[a] = expf(sk0 + sk1 + sbias[a]);
         }
+        float4 *dst = (float4 *)(p.phiK + ((size_t)bh * p.m + t) * p.Ps + j0);
+#pragma unroll
+        for (int a = 0; a < 32; a += 4) dst[a / 4] = make_float4(ok[a], ok[a + 1], ok[a + 2], ok[a + 3]);
     }
     __syncthreads();
     {
@@ -133,16 +132,20 @@ __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) 
         }
     }
     __syncthreads();
-    if (t < p.m)
-        for (int a = 0; a < 32; ++a) {
-            const int j = j0 + a;
-            if (j < p.P) p.phiQ[((size_t)bh * p.P + j) * p.m + t] = expf(su[a][t] - smax[a]);
-        }
+    if (t < p.m) {
+        float oq[32];
+#pragma unroll
+        for (int a = 0; a < 32; ++a) oq[a] = j0 + a < p.P ? expf(su[a][t] - smax[a]) : 0.f;
+        float4 *dst = (float4 *)(p.phiQ + ((size_t)bh * p.m + t) * p.Ps + j0);
+#pragma unroll
+        for (int a = 0; a < 32; a += 4) dst[a / 4] = make_float4(oq[a], oq[a + 1], oq[a + 2], oq[a + 3]);
+    }
 }
 
-// Masked attention over the first P tokens in fp32: CTA per (64 queries, head), 256 threads.
-// Per 64-key block up to the diagonal: scores S = phi(Q) phi(K)^T (4 x 4 per thread, features in
-// 32-wide slices through shared memory), the mask j <= i, then num += S V and den += rowsum(S)
+// Masked attention over the first P tokens in fp32: CTA per (64 queries, head), 256 threads, the
+// CTAs with the most key blocks first. Per 64-key block up to the diagonal: scores
+// S = phi(Q) phi(K)^T (4 x 4 per thread, features in 32-wide slices through shared memory, read
+// as rows of the feature-major scratch), the mask j <= i, then num += S V and den += rowsum(S)
 // (4 queries x 4 value columns per thread).
 __global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
     // the feature slices (score phase) and the masked scores (output phase) share one buffer
@@ -151,7 +154,7 @@ __global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
     float(*aq)[64] = (float(*)[64])buf;         // [32 features][64 queries]
     float(*ak)[64] = (float(*)[64])(buf + 32 * 64);
     float(*ss)[65] = (float(*)[65])buf;         // [64 queries][64 keys + pad]
-    const int bh = blockIdx.y, i0 = blockIdx.x * 64, t = threadIdx.x;
+    const int bh = blockIdx.y, i0 = (gridDim.x - 1 - blockIdx.x) * 64, t = threadIdx.x;
     const int ti = (t >> 4) * 4, tj = (t & 15) * 4;  // this thread's 4 x 4 score block / 4 x 4 output block
     float num[4][4], den[4];
 #pragma unroll
@@ -160,8 +163,8 @@ __global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) num[a][c] = 0.f;
     }
-    const float *phq = p.phiQ + (size_t)bh * p.P * p.m;
-    const float *phk = p.phiK + (size_t)bh * p.P * p.m;
+    const float *phq = p.phiQ + (size_t)bh * p.m * p.Ps;
+    const float *phk = p.phiK + (size_t)bh * p.m * p.Ps;
     for (int j0 = 0; j0 <= i0 && j0 < p.P; j0 += 64) {
         float sc[4][4];
 #pragma unroll
@@ -171,9 +174,9 @@ __global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
         for (int f0 = 0; f0 < p.m; f0 += 32) {
             __syncthreads();
             for (int idx = t; idx < 64 * 32; idx += 256) {
-                const int a = idx >> 5, f = idx & 31;
-                aq[f][a] = (i0 + a < p.P) ? phq[(size_t)(i0 + a) * p.m + f0 + f] : 0.f;
-                ak[f][a] = (j0 + a < p.P) ? phk[(size_t)(j0 + a) * p.m + f0 + f] : 0.f;
+                const int f = idx >> 6, a = idx & 63;
+                aq[f][a] = (i0 + a < p.P) ? phq[(size_t)(f0 + f) * p.Ps + i0 + a] : 0.f;
+                ak[f][a] = (j0 + a < p.P) ? phk[(size_t)(f0 + f) * p.Ps + j0 + a] : 0.f;
             }
             __syncthreads();
 #pragma unroll 8
@@ -219,380 +222,828 @@ __global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
     }
 }
 
-// ============================================================================ k_causal_out
+// ============================================================================ k_causal_chunk
 //
-// One CTA per (batch-head, segment), 256 threads (two warpgroups), phases in sequence per tile.
-// TMEM (512 columns):  R0 [0,128)   phi(Q) half h (fp32/tf32), later the state update dS_h
-//                      R1 [128,256) phi(K)^T half h (features on lanes, tokens on columns)
-//                      R2 [256,384) intra-tile scores A (q rows, k columns)
-//                      R3 [384,448) output accumulator (d = 64)
-// The full query projection for the per-row max uses R0..R1 before the halves.
-// Shared: W (bf16), the running state S as the tf32 K-major operand image and z (fp32), the Q/K
-// tiles (bf16, TMA), V^T (tf32 K-major), two 32-feature slots of phi(K) as the K-major B operand
-// of the score MMA.
+// The chunked scan over 128-token tiles, on fp16 operands with fp32 accumulation. The m features
+// are split over a cluster of m/128 CTAs (one SM each): CTA rank r owns features
+// [128 r, 128 r + 128), its own fp32 running state S_r (features x 64 values, in TMEM) and z_r,
+// and produces a partial output per query row; the partials are combined through distributed
+// shared memory. Per tile t of a segment (tokens j0 .. j0 + 127), in CTA rank r:
+//   P    = Q_t W_r^T                       (bf16 MMA; queries on TMEM lanes)
+//   phiq = 2^(P log2e - c_i), c_i its row maximum over the CTA's features, fp16 into TMEM;
+//          den_q = phiq . z_<t on CUDA cores
+//   P^T  = W_r K_t^T                       (bf16 MMA; features on TMEM lanes)
+//   phik = 2^(P^T log2e + beta_j), beta_j = (-|k_j|^2/2 - C) log2e + A + b_t, fp16 into shared
+//          memory as [feature][token] rows; z_<t+1 = z_<t + 2^-b_t sum_j phik
+//   Simg = fp16(S_<t 2^-sigma_t)           (converted from TMEM; S_<t of a segment's first tile
+//          is the prefix the scan wrote)
+//   O    = phiq Simg                       (fp16 MMA, A from TMEM)
+//   A    = phiq phik^T                     (fp16 MMA) -> masked (key > query -> 0), row sums
+//          den_a = 2^-b_t sum_j A_ij in fp32, fp16(A 2^-sigma_t) in place
+//   S   += phik^T V'_t                     (fp16 MMA, V'_t = V_t 2^-b_t converted in place)
+//   O   += A V'_t
+//   partial numerator O 2^sigma_t, partial denominator den_q + den_a, both relative to 2^c_i.
+// C is the per-(batch, head) key maximum, so phik <= 2^(A + b_t) with A = 8 (fp16 headroom for keys
+// far below the maximum); b_t = clamp(e_t - 13, 0, 7) with e_t the exponent of the tile's largest
+// |v| keeps V'_t in fp16 range; every product phik v' carries the same 2^A, which cancels in the
+// ratio. sigma_t >= b_t keeps the scaled S and A below 2^15.
+// Warp roles (16 warps): 0-3 query exponentials; 4-7 key exponentials and the state image; 8-11
+// masking and the output epilogue (one tile behind); 12 TMA; 13 MMA issue; 14-15 V conversion and
+// the key terms beta_j.
+// TMEM columns: P [0,128), phiq [128,192), A [192,320) (fp16 in [192,256)), S [320,384),
+// O [384 + 64 b, +64) for b = tile parity.
 
-struct CausalParams {
-    int L, d, m, tiles_per_split, P_exact;
-    const uint16_t *V;        // bf16 [BH, L, d]
-    const float *bias;        // [BH, L]
-    const float *seg_state;   // [BH, n_split, state_floats]
-    int n_split;
-    float *out;               // fp32 [BH, L, d]
+struct ChunkParams {
+    int L, m, n_split, tiles_per_split, P_exact;
+    int n_seg;                 // BH * n_split
+    const float *bias;         // [BH, L]: -|k_j|^2/2
+    const float *head_max;     // [BH]: C
+    const float *seg_S;        // [BH, n_split, m, 64]: exclusive prefix of S per segment, times 2^A
+    const float *seg_z;        // [BH, n_split, m]: the same for z
+    float *out;                // fp32 [BH, L, 64]
 };
 
-constexpr int kCausalThreads = 256;
+constexpr int kChunkThreads = 512;
+constexpr float kChunkKeyShift = 8.f;
 
-template <int D>
-struct CausalSmem {
-    static constexpr uint32_t W_BYTES = (D / 64) * 256 * 128;   // m <= 256
-    static constexpr uint32_t S_BYTES = 256 * D * 4;
-    static constexpr uint32_t QK_BYTES = (D / 64) * kTile * 128;
-    static constexpr uint32_t VT_BYTES = kTile * D * 4;
-    static constexpr uint32_t KB_SLOT = kTile * 128;            // 128 tokens x 32 fp32
+namespace chunk {
+constexpr uint32_t TILE = 16384;                                // 128 rows x 128 bytes
+constexpr int STAGES = 2;
+constexpr uint32_t OFF_W = 0;                                   // W rows of the CTA's features
+constexpr uint32_t OFF_QK = TILE;                               // stage s: Q | K
+constexpr uint32_t OFF_V = OFF_QK + STAGES * 2 * TILE;          // stage s: V (fp16 after conversion)
+constexpr uint32_t OFF_PHIK = OFF_V + STAGES * TILE;            // [token block][feature][64 tokens]
+constexpr uint32_t OFF_SIMG = OFF_PHIK + 2 * TILE;              // [feature][64 values]
+constexpr int RECV_ROW = 68;                                    // floats: numerator, den, c, pad
+constexpr uint32_t RECV_SLOT = 64 * RECV_ROW * 4;               // 64 rows (two warps' bulk copies)
+constexpr uint32_t OFF_RECV = OFF_SIMG + TILE;                  // [2 slots][64 rows]
+constexpr uint32_t OFF_SEND = OFF_RECV + 2 * RECV_SLOT;         // staging of the rows sent
+constexpr uint32_t OFF_F = OFF_SEND + RECV_SLOT;                // float arrays (indices below)
+constexpr int F_ZSNAP = 0, F_BETA = 256, F_DENQ = 512, F_DENA = 768, F_CQ = 1024;  // [2][128] each
+constexpr int F_SIGMA = 1280, F_SIGE = 1282, F_AMAX = 1288, F_END = 1296;
+constexpr uint32_t OFF_BAR = OFF_F + F_END * 4;
+enum {
+    B_FULL_QK = 0, B_EMPTY_QK = 2, B_FULL_V = 4, B_EMPTY_V = 6, B_CONV = 8, B_BETA_FULL = 10, B_BETA_FREE = 12,
+    B_W = 14, B_PQ_FULL, B_PK_FULL, B_PQ_FREE, B_PK_FREE, B_Z_FULL,
+    B_PHIQ_FULL = B_Z_FULL + 2, B_PHIQ_FREE, B_PHIK_FULL, B_PHIK_FREE, B_S_READY, B_S_DONE, B_SIG_FULL,
+    B_SC_FULL = B_SIG_FULL + 2, B_MASK_DONE, B_O_FULL, B_O_EMPTY = B_O_FULL + 2, B_DEN_FULL = B_O_EMPTY + 2,
+    B_RECV_FULL = B_DEN_FULL + 2, B_RECV_FREE = B_RECV_FULL + 2, B_AMAX = B_RECV_FREE + 2, B_DRAIN = B_AMAX + 2,
+    N_BAR = B_DRAIN + 2
+};
+constexpr uint32_t BYTES = OFF_BAR + N_BAR * 8 + 16;
+constexpr uint32_t T_P = 0, T_PHIQ = 128, T_A = 192, T_S = 320, T_O = 384;
+}  // namespace chunk
+
+// The tiles one cluster walks: segments cid, cid + n_cl, ..., each its run of 128-token tiles.
+struct ChunkSteps {
+    int seg, tile, t1, bh, n_cl, nt;
+    bool ok, first;
+    __device__ void enter(const ChunkParams &p) {
+        for (; seg < p.n_seg; seg += n_cl) {
+            bh = seg / p.n_split;
+            tile = (seg % p.n_split) * p.tiles_per_split;
+            t1 = min(tile + p.tiles_per_split, nt);
+            if (tile < t1) { ok = first = true; return; }
+        }
+        ok = false;
+    }
+    __device__ ChunkSteps(const ChunkParams &p, int cid, int n_cl_) : seg(cid), n_cl(n_cl_) {
+        nt = (p.L + kTile - 1) / kTile;
+        enter(p);
+    }
+    __device__ void next(const ChunkParams &p) {
+        first = false;
+        if (++tile == t1) {
+            seg += n_cl;
+            enter(p);
+        }
+    }
 };
 
-template <int D>
-__global__ void __launch_bounds__(kCausalThreads, 1)
-k_causal_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-             const __grid_constant__ CUtensorMap mapW, CausalParams p) {
-    using SM = CausalSmem<D>;
-    constexpr int KB = D / 64;
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+// Arrive (release, cluster scope) on an mbarrier in another CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// mbar_wait_all for a barrier that another CTA of the cluster arrives on (acquire at cluster
+// scope, so that the other CTA's stores before its arrive are visible).
+__device__ __forceinline__ bool mbar_wait_cluster_all(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    const uint32_t a = smem_u32(bar);
+    bool ok = mbar_try_wait_cluster(a, parity);
+    if (!ok) {
+        const unsigned long long t0 = globaltimer_ns();
+        for (uint32_t it = 1;; ++it) {
+            if (mbar_try_wait_cluster(a, parity)) { ok = true; break; }
+            if ((it & 63u) == 0) {
+                if (*abort) break;
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    record_status(FAVOR_ERR_TIMEOUT);
+                    *abort = 1;
+                    break;
+                }
+            }
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Stores 16 consecutive 32-bit columns of this thread's TMEM lane (warp-collective; not waited).
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&h)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        FAVOR_U16(h, 0)
+        : "memory");
+}
+
+// Bulk copy of `bytes` from this CTA's shared memory into another CTA of the cluster (destination
+// and its mbarrier as cluster addresses); completes as transaction bytes on that mbarrier.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "r"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+
+// phiq = 2^(v log2e - cl) over a row of 128 logits, in place. Per 32 columns the first 32 - POLY
+// exponentials go to MUFU ex2, the rest to the FMA-pipe polynomial.
+template <int POLY>
+__device__ __forceinline__ void chunk_query_exps(float (&v)[128], float cl) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int e = c * 32; e < c * 32 + 32; ++e) v[e] = fmaf(v[e], kLog2e, -cl);
+#pragma unroll
+        for (int e = c * 32; e < c * 32 + 32 - POLY; ++e) v[e] = ex2_approx(v[e]);
+#pragma unroll
+        for (int e = c * 32 + 32 - POLY; e < c * 32 + 32; e += 2) exp2_poly_pair(v[e], v[e + 1], v[e], v[e + 1]);
+    }
+}
+
+// phik = 2^(v log2e + beta_j) over a row of 128 tokens, rounded to fp16 pairs; returns the row's
+// sum (fp32, before rounding).
+template <int POLY>
+__device__ __forceinline__ float chunk_key_features(float (&v)[128], const float *beta, uint32_t (&hv)[64]) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int e = c * 32; e < c * 32 + 32; e += 4) {
+            const float4 b4 = *(const float4 *)(beta + e);
+            v[e] = fmaf(v[e], kLog2e, b4.x);
+            v[e + 1] = fmaf(v[e + 1], kLog2e, b4.y);
+            v[e + 2] = fmaf(v[e + 2], kLog2e, b4.z);
+            v[e + 3] = fmaf(v[e + 3], kLog2e, b4.w);
+        }
+#pragma unroll
+        for (int e = c * 32; e < c * 32 + 32 - POLY; ++e) v[e] = ex2_approx(v[e]);
+#pragma unroll
+        for (int e = c * 32 + 32 - POLY; e < c * 32 + 32; e += 2) exp2_poly_pair(v[e], v[e + 1], v[e], v[e + 1]);
+#pragma unroll
+        for (int e = c * 32; e < c * 32 + 32; e += 2) {
+            s0 += v[e];
+            s1 += v[e + 1];
+            hv[e >> 1] = pack_f16x2(v[e], v[e + 1]);
+        }
+    }
+    return s0 + s1;
+}
+
+// Shared-memory descriptors as their low 32 bits (start address and LBO fields; the high word, SBO
+// = 1024 with the sm_100 version and 128-byte swizzle, is the same for every operand here), so the
+// issuing warp keeps one register per operand.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t desc_lo(uint32_t smem_addr, uint32_t lbo_bytes) {
+    return ((smem_addr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+// D (+)= sum over 4 K-steps of A_k B_k, A and B in shared memory (low descriptor words advancing by
+// a_step / b_step 16-byte units per step).
+__device__ __forceinline__ void mma_ss4(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, uint32_t acc,
+                                        uint32_t a_step, uint32_t b_step) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t.reg .b32 al, bl;\n\t.reg .b64 ad, bd;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+        "mov.b64 ad, {%1, %7};\n\tmov.b64 bd, {%2, %7};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t"
+        "add.u32 al, %1, %5;\n\tadd.u32 bl, %2, %6;\n\tmov.b64 ad, {al, %7};\n\tmov.b64 bd, {bl, %7};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, t;\n\t"
+        "add.u32 al, al, %5;\n\tadd.u32 bl, bl, %6;\n\tmov.b64 ad, {al, %7};\n\tmov.b64 bd, {bl, %7};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, t;\n\t"
+        "add.u32 al, al, %5;\n\tadd.u32 bl, bl, %6;\n\tmov.b64 ad, {al, %7};\n\tmov.b64 bd, {bl, %7};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, t;\n\t}" ::"r"(d),
+        "r"(a), "r"(b), "r"(idesc), "r"(acc), "r"(a_step), "r"(b_step), "r"(kDescHi)
+        : "memory");
+}
+// The same with A in TMEM (8 columns per K-step).
+__device__ __forceinline__ void mma_ts4(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t idesc, uint32_t acc,
+                                        uint32_t b_step) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t.reg .b32 al, bl;\n\t.reg .b64 bd;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+        "mov.b64 bd, {%2, %6};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %3, p;\n\t"
+        "add.u32 al, %1, 8;\n\tadd.u32 bl, %2, %5;\n\tmov.b64 bd, {bl, %6};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [al], bd, %3, t;\n\t"
+        "add.u32 al, al, 8;\n\tadd.u32 bl, bl, %5;\n\tmov.b64 bd, {bl, %6};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [al], bd, %3, t;\n\t"
+        "add.u32 al, al, 8;\n\tadd.u32 bl, bl, %5;\n\tmov.b64 bd, {bl, %6};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [al], bd, %3, t;\n\t}" ::"r"(d),
+        "r"(a_tmem), "r"(b), "r"(idesc), "r"(acc), "r"(b_step), "r"(kDescHi)
+        : "memory");
+}
+
+// 1/x to about one ulp (MUFU; no slow-path subroutine around the epilogue's registers).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
+
+template <int CL, int POLY>
+__global__ void __launch_bounds__(kChunkThreads, 1)
+k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+               const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapW, ChunkParams p) {
+    using namespace chunk;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *sW = smem;
-    uint8_t *sS = sW + SM::W_BYTES;                 // state image (m x D fp32, K-major tf32)
-    uint8_t *sQ = sS + SM::S_BYTES;
-    uint8_t *sK = sQ + SM::QK_BYTES;
-    uint8_t *sVt = sK + SM::QK_BYTES;               // [4 blocks of 32 tokens][D rows][32 fp32]
-    uint8_t *sKB = sVt + SM::VT_BYTES;              // 2 slots x [128 tokens][32 fp32]
-    float *sZ = (float *)(sKB + 2 * SM::KB_SLOT);   // m
-    float *sRow = sZ + 256;                          // 2 x 128: per-row partials (max / sums)
-    float *sC = sRow + 256;                          // 128: query row max
-    float *sDen = sC + 128;                          // 128: phi(q).z_<t
-    float *sBB = sDen + 128;                         // 128: (-|k|^2/2 - C) log2e
-    float *sZp = sBB + 128;                          // 2 x 256: z partials of this tile
-    uint64_t *bars = (uint64_t *)(sZp + 512);
-    uint64_t *tma_bar = bars, *mma_bar = bars + 1;
-    uint32_t *tmem_slot = (uint32_t *)(bars + 2);
+    float *sf = (float *)(smem + OFF_F);
+    uint64_t *bar = (uint64_t *)(smem + OFF_BAR);
+    uint32_t *tmem_slot = (uint32_t *)(bar + N_BAR);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
-
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wg = warp >> 2;                        // warpgroup: column half of every epilogue
-    const int row = (warp & 3) * 32 + lane;          // TMEM lane owned by this thread
-    const int split = blockIdx.x, bh = blockIdx.y;
-    const int n_tiles_total = (p.L + kTile - 1) / kTile;
-    const int t0 = split * p.tiles_per_split;
-    const int n_tiles = max(min(t0 + p.tiles_per_split, n_tiles_total) - t0, 0);
-    const int m = p.m, halves = m / 128;
-    const uint32_t R0 = 0, R1 = 128, R2 = 256, R3 = 384;
-    const float *seg = p.seg_state + ((size_t)bh * p.n_split + split) * state_floats(m, D);
-    uint32_t tma_phase = 0, mma_phase = 0;
-    bool ok = true;
+    const uint32_t rank = CL > 1 ? cluster_rank() : 0u;
+    const int cid = blockIdx.x / CL, n_cl = gridDim.x / CL;
 
     if (tid == 0) {
-        mbar_init(tma_bar, 1);
-        mbar_init(mma_bar, 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&bar[B_FULL_QK + s], 1);
+            mbar_init(&bar[B_EMPTY_QK + s], 1);
+            mbar_init(&bar[B_FULL_V + s], 1);
+            mbar_init(&bar[B_EMPTY_V + s], 1);
+            mbar_init(&bar[B_CONV + s], 32);
+        }
+        mbar_init(&bar[B_W], 1);
+        mbar_init(&bar[B_PQ_FULL], 1);
+        mbar_init(&bar[B_PK_FULL], 1);
+        mbar_init(&bar[B_PQ_FREE], 128);
+        mbar_init(&bar[B_PK_FREE], 128);
+        mbar_init(&bar[B_PHIQ_FULL], 128);
+        mbar_init(&bar[B_PHIQ_FREE], 1);
+        mbar_init(&bar[B_PHIK_FULL], 128);
+        mbar_init(&bar[B_PHIK_FREE], 1);
+        mbar_init(&bar[B_S_READY], 128);
+        mbar_init(&bar[B_S_DONE], 1);
+        mbar_init(&bar[B_SC_FULL], 1);
+        mbar_init(&bar[B_MASK_DONE], 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar[B_BETA_FULL + b], 32);
+            mbar_init(&bar[B_BETA_FREE + b], 128);
+            mbar_init(&bar[B_Z_FULL + b], 128);
+            mbar_init(&bar[B_SIG_FULL + b], 128);
+            mbar_init(&bar[B_O_FULL + b], 1);
+            mbar_init(&bar[B_O_EMPTY + b], 128);
+            mbar_init(&bar[B_DEN_FULL + b], 256);
+            mbar_init(&bar[B_RECV_FULL + b], 1);
+            mbar_init(&bar[B_RECV_FREE + b], 64);
+            mbar_init(&bar[B_AMAX + b], 4);
+        }
+        mbar_init(&bar[B_DRAIN], 1);
+        mbar_init(&bar[B_DRAIN + 1], 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0) {
+    if (warp == 13) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (CL > 1) cluster_sync_all();  // the partner's barriers exist before any remote arrive or copy
     const uint32_t tmem = *tmem_slot;
-    const float Clog2 = seg[(size_t)m * D + m] * kLog2e;
+    const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
+    const int row = (warp & 3) * 32 + lane;  // TMEM lane of this thread (query row or feature)
 
-    // Segment start: W, the state prefix image and z.
-    if (tid == 0) {
-        prefetch_tensormap(&mapQ);
-        prefetch_tensormap(&mapK);
-        mbar_arrive_expect_tx(tma_bar, SM::W_BYTES / 256 * m + (uint32_t)m * D * 4 + m * 4);
-        for (int kb = 0; kb < KB; ++kb) tma_load_2d(sW + (size_t)kb * m * 128, &mapW, tma_bar, kb * 64, 0);
-        for (uint32_t off = 0; off < (uint32_t)m * D * 4; off += 32768)
-            bulk_load(sS + off, (const uint8_t *)seg + off, min(32768u, (uint32_t)m * D * 4 - off), tma_bar);
-        bulk_load(sZ, seg + (size_t)m * D, m * 4, tma_bar);
-    }
-    ok = mbar_wait(tma_bar, tma_phase, abort_flag);
-    tma_phase ^= 1;
-
-    auto mma_sync = [&]() -> bool {  // all threads: wait for the MMAs committed by thread 0
-        const bool r = mbar_wait(mma_bar, mma_phase, abort_flag);
-        mma_phase ^= 1;
-        tc_fence_after();
-        return r;
-    };
-    auto to_mma = [&]() {  // epilogue writes (TMEM and shared) before MMAs issued by thread 0
-        tmem_wait_st();
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-    };
-
-    for (int it = 0; ok && it < n_tiles; ++it) {
-        const int tile = t0 + it, j0 = tile * kTile;
-        // ---- loads: Q, K tiles by TMA; V^T (tf32) and the key biases by the threads
-        if (tid == 0) {
-            mbar_arrive_expect_tx(tma_bar, 2 * SM::QK_BYTES);
-            for (int kb = 0; kb < KB; ++kb) {
-                tma_load_3d(sQ + kb * kTile * 128, &mapQ, tma_bar, kb * 64, j0, bh);
-                tma_load_3d(sK + kb * kTile * 128, &mapK, tma_bar, kb * 64, j0, bh);
+    if (warp >= 12) {
+        regs_dec<64>();
+        if (warp == 12) {
+            // ---- TMA: W once; Q, K of tile g and V of tile g - 1 per step (V is needed later and
+            // its stage is held until the tile's last MMA); the key terms
+            // beta_j = (-|k_j|^2/2 - C) log2e + A of tile g (4 tokens per lane)
+            if (elect_one()) {
+                prefetch_tensormap(&mapQ);
+                prefetch_tensormap(&mapK);
+                prefetch_tensormap(&mapV);
+                prefetch_tensormap(&mapW);
+                mbar_arrive_expect_tx(&bar[B_W], TILE);
+                tma_load_2d(smem + OFF_W, &mapW, &bar[B_W], 0, 128 * (int)rank);
             }
-        }
-        {
-            const int tok = tid & 127, vh = tid >> 7;  // value half
-            const int j = j0 + tok;
-            const int kb = tok >> 5, ch = (tok & 31) >> 2, pos = tok & 3;
-            uint8_t *dst = sVt + kb * (D * 128) + pos * 4;
-            const uint4 *src = (const uint4 *)(p.V + ((size_t)bh * p.L + j) * D);
-            for (int e0 = vh * (D / 2); e0 < (vh + 1) * (D / 2); e0 += 8) {
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (j < p.L) v = __ldg(src + e0 / 8);
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    *(float *)(dst + sw128_offset(e0 + 2 * e, ch)) = __uint_as_float(w4[e] << 16);
-                    *(float *)(dst + sw128_offset(e0 + 2 * e + 1, ch)) = __uint_as_float(w4[e] & 0xFFFF0000u);
-                }
-            }
-            if (vh == 0) sBB[tok] = j < p.L ? p.bias[(size_t)bh * p.L + j] * kLog2e - Clog2 : -INFINITY;
-        }
-        if (!(ok = mbar_wait(tma_bar, tma_phase, abort_flag))) break;
-        tma_phase ^= 1;
-        to_mma();
-
-        // ---- 1. full query projection (per-row max)
-        if (tid == 0) {
-            const uint32_t idesc = make_idesc(kTile, m, kFmtBF16, 0, 0);
-            for (int k = 0; k < D / 16; ++k)
-                mma_f16_ss(tmem + R0, make_sdesc(smem_u32(sQ) + (k >> 2) * kTile * 128 + (k & 3) * 32, 16, 1024),
-                           make_sdesc(smem_u32(sW) + (k >> 2) * m * 128 + (k & 3) * 32, 16, 1024), idesc, k > 0);
-            mma_commit(mma_bar);
-        }
-        if (!(ok = mma_sync())) break;
-        {
-            float rmax = -INFINITY;
-            for (int c0 = wg * (m / 2); c0 < (wg + 1) * (m / 2); c0 += 32) {
-                float v[32];
-                tmem_ld32(tmem_lane_addr(tmem + R0, warp, c0), v);
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) rmax = fmax3(rmax, v[e], v[e + 1]);
-            }
-            sRow[wg * 128 + row] = rmax;
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-            if (wg == 0) {
-                sC[row] = fmaxf(sRow[row], sRow[128 + row]) * kLog2e;
-                sDen[row] = 0.f;
-            }
-            __syncthreads();
-        }
-
-        for (int h = 0; h < halves; ++h) {
-            // ---- 2a. projections of feature half h: phi(Q)_h (tokens x 128) and phi(K)_h^T
-            if (tid == 0) {
-                const uint32_t id_q = make_idesc(kTile, 128, kFmtBF16, 0, 0);
-                for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t kq = (k >> 2) * kTile * 128 + (k & 3) * 32;
-                    const uint32_t kw = (k >> 2) * m * 128 + h * 128 * 128 + (k & 3) * 32;
-                    mma_f16_ss(tmem + R0, make_sdesc(smem_u32(sQ) + kq, 16, 1024),
-                               make_sdesc(smem_u32(sW) + kw, 16, 1024), id_q, k > 0);
-                    mma_f16_ss(tmem + R1, make_sdesc(smem_u32(sW) + kw, 16, 1024),
-                               make_sdesc(smem_u32(sK) + kq, 16, 1024), id_q, k > 0);
-                }
-                mma_commit(mma_bar);
-            }
-            if (!(ok = mma_sync())) break;
-            // ---- 2b. exponentials in place (tf32 operands), phi(q).z_<t, z partials, phi(K) B slots
-            {
-                const float cl = sC[row];
-                float den = 0.f;
-                for (int c0 = wg * 64; c0 < wg * 64 + 64; c0 += 32) {
-                    const uint32_t ta = tmem_lane_addr(tmem + R0, warp, c0);
-                    float v[32];
-                    tmem_ld32(ta, v);
-                    const float *z = sZ + h * 128 + c0;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        float used;
-                        v[e] = tf32_round_store(ex2_approx(fmaf(v[e], kLog2e, -cl)), used);
-                        den = fmaf(used, z[e], den);
+            __syncwarp();
+            int g = 0, pbh = 0, ptile = 0;
+            bool ok = true;
+            for (ChunkSteps it(p, cid, n_cl);; ++g) {
+                const bool have = it.ok;
+                if (have) {
+                    const int s = g % STAGES, b = g & 1;
+                    if (!(ok = mbar_wait_lazy(&bar[B_EMPTY_QK + s], ((g / STAGES) & 1) ^ 1, abort_flag))) break;
+                    if (elect_one()) {
+                        uint8_t *st = smem + OFF_QK + s * 2 * TILE;
+                        mbar_arrive_expect_tx(&bar[B_FULL_QK + s], 2 * TILE);
+                        tma_load_3d(st, &mapQ, &bar[B_FULL_QK + s], 0, it.tile * kTile, it.bh);
+                        tma_load_3d(st + TILE, &mapK, &bar[B_FULL_QK + s], 0, it.tile * kTile, it.bh);
                     }
-                    tmem_st32(ta, v);
-                }
-                atomicAdd(&sDen[row], den);
-            }
-            {
-                // thread <-> feature f = 128 h + row; columns = tokens [64 wg, 64 wg + 64)
-                float zs = 0.f;
-                for (int c0 = wg * 64; c0 < wg * 64 + 64; c0 += 32) {
-                    const uint32_t ta = tmem_lane_addr(tmem + R1, warp, c0);
-                    float v[32];
-                    tmem_ld32(ta, v);
+                    __syncwarp();
+                    if (g >= 2 && !(ok = mbar_wait_all(&bar[B_BETA_FREE + b], ((g >> 1) - 1) & 1, abort_flag))) break;
+                    const float cb = kChunkKeyShift - p.head_max[it.bh] * kLog2e;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        float used;
-                        v[e] = tf32_round_store(ex2_approx(fmaf(v[e], kLog2e, sBB[c0 + e])), used);
-                        zs += used;
+                    for (int k = 0; k < 4; ++k) {
+                        const int jt = lane * 4 + k, j = it.tile * kTile + jt;
+                        sf[F_BETA + b * 128 + jt] =
+                            j < p.L ? fmaf(p.bias[(size_t)it.bh * p.L + j], kLog2e, cb) : -INFINITY;
                     }
-                    tmem_st32(ta, v);
+                    mbar_arrive(&bar[B_BETA_FULL + b]);
                 }
-                sZp[wg * 256 + h * 128 + row] = zs;
-            }
-            // ---- 2c. state term O (+)= phi(Q)_h S_<t[half h] (reads the state image before it changes)
-            to_mma();
-            if (tid == 0) {
-                const uint32_t id_o = make_idesc(kTile, D, kFmtTF32, 0, 0);
-                for (int k8 = 0; k8 < 16; ++k8) {
-                    const int f0 = h * 128 + k8 * 8;
-                    const uint32_t b = smem_u32(sS) + (f0 >> 5) * (D * 128) + (k8 & 3) * 32;
-                    mma_tf32_ts(tmem + R3, tmem + R0 + k8 * 8, make_sdesc(b, 16, 1024), id_o, (h > 0 || k8 > 0) ? 1u : 0u);
+                if (g > 0) {
+                    const int e = g - 1, s = e % STAGES;
+                    if (!(ok = mbar_wait_lazy(&bar[B_EMPTY_V + s], ((e / STAGES) & 1) ^ 1, abort_flag))) break;
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&bar[B_FULL_V + s], TILE);
+                        tma_load_3d(smem + OFF_V + s * TILE, &mapV, &bar[B_FULL_V + s], 0, ptile * kTile, pbh);
+                    }
+                    __syncwarp();
                 }
-                mma_commit(mma_bar);
+                if (!have) break;
+                pbh = it.bh;
+                ptile = it.tile;
+                it.next(p);
             }
-            // ---- 2d. intra scores A (+)= phi(Q)_h phi(K)_h^T, 32 features per slot, two slots
-            for (int cp = 0; cp < 2; ++cp) {
-                if (!(ok = mma_sync())) break;  // previous MMAs done: slots and state image free
-                // phi(K) chunks 2cp, 2cp+1 of half h -> slots: row = token, 32 features
-                {
-                    const int f = row;                       // feature within the half
-                    const int chunk = f >> 5;
-                    if ((chunk >> 1) == cp) {
-                        uint8_t *slot = sKB + (chunk & 1) * SM::KB_SLOT;
-                        const int fc = f & 31, ch = fc >> 2, pos = fc & 3;
-                        for (int c0 = wg * 64; c0 < wg * 64 + 64; c0 += 32) {
-                            float v[32];
-                            tmem_ld32(tmem_lane_addr(tmem + R1, warp, c0), v);
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                *(float *)(slot + sw128_offset(c0 + e, ch) + pos * 4) = v[e];
+            // wait for the copies in flight (bounded) before the CTA may exit
+            volatile int no_abort = 0;
+            const int nq = ok ? g : g + 1;  // Q/K copies issued
+            for (int i = max(nq - STAGES, 0); i < nq; ++i)
+                mbar_wait(&bar[B_FULL_QK + i % STAGES], (i / STAGES) & 1, &no_abort);
+            const int nv = ok ? g : max(g - 1, 0);
+            for (int i = max(nv - STAGES, 0); i < nv; ++i)
+                mbar_wait(&bar[B_FULL_V + i % STAGES], (i / STAGES) & 1, &no_abort);
+            mbar_wait(&bar[B_W], 0, &no_abort);
+        } else if (warp == 13 || warp == 14) {
+            // ---- MMA issue in two independent streams (each thread's commits track its own MMAs):
+            // warp 13 the projections into P (Q W^T, W K^T), warp 14 everything that produces the
+            // output and the state (scores, state term, state update, masked A V')
+            const uint32_t id_proj = make_idesc(128, 128, kFmtBF16, 0, 0);
+            const uint32_t id_64 = make_idesc(128, 64, kFmtF16, 0, 1);
+            const uint32_t id_sc = make_idesc(128, 128, kFmtF16, 0, 1);
+            const uint32_t base = smem_u32(smem);
+            constexpr uint32_t kTileU = TILE / 16, kRow16 = 2048 / 16, kHalfU = 8192 / 16;
+            int n = 0;
+            for (ChunkSteps it(p, cid, n_cl); it.ok; it.next(p)) ++n;
+            bool ok = true;
+            if (warp == 13) {
+                // K-major operands (LBO unused)
+                const uint32_t dW = desc_lo(base + OFF_W, 16);
+                const uint32_t dQK = desc_lo(base + OFF_QK, 16);
+                ok = mbar_wait_all(&bar[B_W], 0, abort_flag);
+                if (ok && n > 0) {
+                    ok = mbar_wait_all(&bar[B_FULL_QK], 0, abort_flag);
+                    tc_fence_after();
+                    if (ok && elect_one()) {
+                        mma_ss4(tmem + T_P, dQK, dW, id_proj, 0u, 2, 2);
+                        mma_commit(&bar[B_PQ_FULL]);
+                    }
+                    __syncwarp();
+                }
+                for (int g = 0; ok && g < n; ++g) {
+                    const int s = g % STAGES;
+                    const uint32_t ph = g & 1;
+                    // K projection of tile g, once the query warps have read P; frees the Q/K stage
+                    if (!(ok = mbar_wait_all(&bar[B_PQ_FREE], ph, abort_flag))) break;
+                    tc_fence_after();
+                    if (elect_one()) {
+                        mma_ss4(tmem + T_P, dW, dQK + (2 * s + 1) * kTileU, id_proj, 0u, 2, 2);
+                        mma_commit(&bar[B_PK_FULL]);
+                        mma_commit(&bar[B_EMPTY_QK + s]);
+                    }
+                    __syncwarp();
+                    // Q projection of tile g + 1, once the key warps have read P
+                    if (g + 1 < n) {
+                        const int s1 = (g + 1) % STAGES;
+                        if (!(ok = mbar_wait_all(&bar[B_FULL_QK + s1], ((g + 1) / STAGES) & 1, abort_flag))) break;
+                        if (!(ok = mbar_wait_all(&bar[B_PK_FREE], ph, abort_flag))) break;
+                        tc_fence_after();
+                        if (elect_one()) {
+                            mma_ss4(tmem + T_P, dQK + 2 * s1 * kTileU, dW, id_proj, 0u, 2, 2);
+                            mma_commit(&bar[B_PQ_FULL]);
                         }
+                        __syncwarp();
                     }
                 }
-                to_mma();
-                if (tid == 0) {
-                    const uint32_t id_a = make_idesc(kTile, kTile, kFmtTF32, 0, 0);
-                    for (int s = 0; s < 2; ++s) {
-                        const int chunk = 2 * cp + s;
-                        for (int k8 = 0; k8 < 4; ++k8)
-                            mma_tf32_ts(tmem + R2, tmem + R0 + chunk * 32 + k8 * 8,
-                                        make_sdesc(smem_u32(sKB) + s * SM::KB_SLOT + k8 * 32, 16, 1024), id_a,
-                                        (h > 0 || chunk > 0 || k8 > 0) ? 1u : 0u);
+            } else {
+                // MN-major operands (LBO = 16 KB between 64-wide blocks) and phik^T as K-major A
+                const uint32_t dV0 = desc_lo(base + OFF_V, TILE);
+                const uint32_t dKB = desc_lo(base + OFF_PHIK, TILE);
+                const uint32_t dKA = desc_lo(base + OFF_PHIK, 16);
+                const uint32_t dSimg = desc_lo(base + OFF_SIMG, TILE);
+                // O += mask(A) V' of tile e
+                auto issue_av = [&](int e) -> bool {
+                    if (!mbar_wait_all(&bar[B_MASK_DONE], e & 1, abort_flag)) return false;
+                    tc_fence_after();
+                    if (elect_one()) {
+                        const uint32_t tO = tmem + T_O + 64 * (e & 1), dV = dV0 + (e % STAGES) * kTileU;
+                        mma_ts4(tO, tmem + T_A, dV, id_64, 1u, kRow16);
+                        mma_ts4(tO, tmem + T_A + 32, dV + kHalfU, id_64, 1u, kRow16);
+                        mma_commit(&bar[B_O_FULL + (e & 1)]);
+                        mma_commit(&bar[B_EMPTY_V + e % STAGES]);
                     }
-                    mma_commit(mma_bar);
+                    __syncwarp();
+                    return true;
+                };
+                int g = 0;
+                for (; ok && g < n; ++g) {
+                    const int s = g % STAGES, b = g & 1;
+                    const uint32_t ph = g & 1;
+                    // the previous tile's O += mask(A) V' (before this tile's scores overwrite A)
+                    if (g > 0 && !(ok = issue_av(g - 1))) break;
+                    // A = phiq phik^T
+                    if (!(ok = mbar_wait_all(&bar[B_PHIQ_FULL], ph, abort_flag))) break;
+                    if (!(ok = mbar_wait_all(&bar[B_PHIK_FULL], ph, abort_flag))) break;
+                    tc_fence_after();
+                    if (elect_one()) {
+                        mma_ts4(tmem + T_A, tmem + T_PHIQ, dKB, id_sc, 0u, kRow16);
+                        mma_ts4(tmem + T_A, tmem + T_PHIQ + 32, dKB + kHalfU, id_sc, 1u, kRow16);
+                        mma_commit(&bar[B_SC_FULL]);
+                    }
+                    __syncwarp();
+                    // O = phiq Simg
+                    if (!(ok = mbar_wait_all(&bar[B_S_READY], ph, abort_flag))) break;
+                    if (g >= 2 && !(ok = mbar_wait_all(&bar[B_O_EMPTY + b], ((g >> 1) - 1) & 1, abort_flag))) break;
+                    tc_fence_after();
+                    if (elect_one()) {
+                        const uint32_t tO = tmem + T_O + 64 * b;
+                        mma_ts4(tO, tmem + T_PHIQ, dSimg, id_64, 0u, kRow16);
+                        mma_ts4(tO, tmem + T_PHIQ + 32, dSimg + kHalfU, id_64, 1u, kRow16);
+                        mma_commit(&bar[B_PHIQ_FREE]);
+                    }
+                    __syncwarp();
+                    // S += phik^T V'
+                    if (!(ok = mbar_wait_all(&bar[B_CONV + s], (g / STAGES) & 1, abort_flag))) break;
+                    tc_fence_after();
+                    if (elect_one()) {
+                        const uint32_t dV = dV0 + s * kTileU;
+                        mma_ss4(tmem + T_S, dKA, dV, id_64, 1u, 2, kRow16);
+                        mma_ss4(tmem + T_S, dKA + kTileU, dV + kHalfU, id_64, 1u, 2, kRow16);
+                        mma_commit(&bar[B_PHIK_FREE]);
+                        mma_commit(&bar[B_S_DONE]);
+                    }
+                    __syncwarp();
                 }
+                if (ok && n > 0) issue_av(n - 1);
             }
-            if (!ok) break;
-            if (!(ok = mma_sync())) break;
-            // ---- 2e. state update of half h: dS_h = phi(K)_h^T V^T into R0 (phi(Q)_h consumed)
-            if (tid == 0) {
-                const uint32_t id_s = make_idesc(128, D, kFmtTF32, 0, 0);
-                for (int k8 = 0; k8 < 16; ++k8) {
-                    const uint32_t b = smem_u32(sVt) + (k8 >> 2) * (D * 128) + (k8 & 3) * 32;
-                    mma_tf32_ts(tmem + R0, tmem + R1 + k8 * 8, make_sdesc(b, 16, 1024), id_s, k8 > 0);
-                }
-                mma_commit(mma_bar);
-            }
-            if (!(ok = mma_sync())) break;
-            // S image[half h] += dS_h (thread <-> feature, value columns split by warpgroup)
-            {
-                const int f = h * 128 + row;
-                const int kb = f >> 5, ch = (f & 31) >> 2, pos = f & 3;
-                for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
-                    float v[32];
-                    tmem_ld32(tmem_lane_addr(tmem + R0, warp, c0), v);
+            if (elect_one()) mma_commit(&bar[B_DRAIN + (warp - 13)]);
+            __syncwarp();
+            volatile int no_abort = 0;
+            mbar_wait(&bar[B_DRAIN + (warp - 13)], 0, &no_abort);
+        } else {
+            // ---- V tiles bf16 -> fp16 in place (entries beyond the fp16 range are reported)
+            int g = 0;
+            for (ChunkSteps it(p, cid, n_cl); it.ok; it.next(p), ++g) {
+                const int s = g % STAGES;
+                if (!mbar_wait_lazy(&bar[B_FULL_V + s], (g / STAGES) & 1, abort_flag)) break;
+                uint8_t *vt = smem + OFF_V + s * TILE;
+                uint32_t mx = 0;
+#pragma unroll 4
+                for (int q = lane; q < (int)(TILE / 16); q += 32) {
+                    uint4 *pq = (uint4 *)(vt + q * 16);
+                    const uint4 w = *pq;
+                    mx = __vmaxu2(mx, w.x & 0x7FFF7FFFu);
+                    mx = __vmaxu2(mx, w.y & 0x7FFF7FFFu);
+                    mx = __vmaxu2(mx, w.z & 0x7FFF7FFFu);
+                    mx = __vmaxu2(mx, w.w & 0x7FFF7FFFu);
+                    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+                    uint32_t h[4];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        float *s = (float *)(sS + kb * (D * 128) + sw128_offset(c0 + e, ch) + pos * 4);
-                        *s = tf32_store(tf32_load(*s) + v[e]);
-                    }
+                    for (int k = 0; k < 4; ++k)
+                        h[k] = pack_f16x2(__uint_as_float(u[k] << 16), __uint_as_float(u[k] & 0xFFFF0000u));
+                    *pq = make_uint4(h[0], h[1], h[2], h[3]);
                 }
+                // bf16 magnitudes from 2^16 up (and inf / nan) do not fit fp16
+                if (max(mx & 0xFFFFu, mx >> 16) >= 0x4780u) record_status(FAVOR_ERR_UNSUPPORTED);
+                fence_async_smem();
+                mbar_arrive(&bar[B_CONV + s]);
             }
-            tc_fence_before();
-            __syncthreads();
+        }
+    } else if (warp < 4) {
+        // ---- query exponentials: thread = query row
+        regs_inc<176>();
+        int g = 0;
+        for (ChunkSteps it(p, cid, n_cl); it.ok; it.next(p), ++g) {
+            const int b = g & 1;
+            float v[128];
+            if (!mbar_wait_all(&bar[B_PQ_FULL], g & 1, abort_flag)) break;
             tc_fence_after();
-        }
-        if (!ok) break;
-        // z += this tile's key sums (after every phi(q).z_<t of the tile used the old z)
-        for (int f = tid; f < m; f += kCausalThreads) sZ[f] += sZp[f] + sZp[256 + f];
-        // ---- 3. mask the scores (k > q or k past L -> 0), row sums, tf32 A operand in place
-        {
-            const int qi = row;
-            float rs = 0.f;
-            for (int c0 = wg * 64; c0 < wg * 64 + 64; c0 += 32) {
-                const uint32_t ta = tmem_lane_addr(tmem + R2, warp, c0);
-                float v[32];
-                tmem_ld32(ta, v);
+            tmem_ld128(tmem + lane_off + T_P, v);
+            tc_fence_before();
+            mbar_arrive(&bar[B_PQ_FREE]);
+            const float cl = row_max128(v) * kLog2e;
+            chunk_query_exps<POLY>(v, cl);
+            // den_q = phiq . z_<t (z_<t is published before the state term of tile g - 1 frees phiq)
+            if (!mbar_wait_all(&bar[B_Z_FULL + b], (g >> 1) & 1, abort_flag)) break;
+            const float *z = sf + F_ZSNAP + b * 128;
+            float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int kj = c0 + e;
-                    float used;
-                    v[e] = tf32_round_store((kj <= qi && j0 + kj < p.L) ? v[e] : 0.f, used);
-                    rs += used;
-                }
-                tmem_st32(ta, v);
+            for (int e = 0; e < 128; e += 4) {
+                const float4 z4 = *(const float4 *)(z + e);
+                d0 = fmaf(v[e], z4.x, d0);
+                d1 = fmaf(v[e + 1], z4.y, d1);
+                d0 = fmaf(v[e + 2], z4.z, d0);
+                d1 = fmaf(v[e + 3], z4.w, d1);
             }
-            sRow[wg * 128 + row] = rs;
-        }
-        to_mma();
-        // ---- 4. O += A V
-        if (tid == 0) {
-            const uint32_t id_o = make_idesc(kTile, D, kFmtTF32, 0, 0);
-            for (int k8 = 0; k8 < 16; ++k8) {
-                const uint32_t b = smem_u32(sVt) + (k8 >> 2) * (D * 128) + (k8 & 3) * 32;
-                mma_tf32_ts(tmem + R3, tmem + R2 + k8 * 8, make_sdesc(b, 16, 1024), id_o, 1u);
-            }
-            mma_commit(mma_bar);
-        }
-        if (!(ok = mma_sync())) break;
-        // ---- 5. out = O / (phi(q).z_<t + rowsum(A)); rows before P_exact come from the exact pass
-        {
-            const int i = j0 + row;
-            const float den = sDen[row] + sRow[row] + sRow[128 + row];
-            const float inv = 1.0f / den;
-            for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
-                float v[32];
-                tmem_ld32(tmem_lane_addr(tmem + R3, warp, c0), v);
-                if (i < p.L && i >= p.P_exact) {
-                    float *o = p.out + ((size_t)bh * p.L + i) * D + c0;
+            if (g > 0 && !mbar_wait_all(&bar[B_PHIQ_FREE], (g - 1) & 1, abort_flag)) break;
+            tc_fence_after();
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *(float4 *)(o + e) = make_float4(v[e] * inv, v[e + 1] * inv, v[e + 2] * inv, v[e + 3] * inv);
+            for (int h = 0; h < 4; ++h) {
+                uint32_t hv[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) hv[e] = pack_f16x2(v[32 * h + 2 * e], v[32 * h + 2 * e + 1]);
+                tmem_st16u(tmem + lane_off + T_PHIQ + 16 * h, hv);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bar[B_PHIQ_FULL]);
+            if (g >= 2 && !mbar_wait_all(&bar[B_O_EMPTY + b], ((g >> 1) - 1) & 1, abort_flag)) break;
+            sf[F_DENQ + b * 128 + row] = d0 + d1;
+            sf[F_CQ + b * 128 + row] = cl;
+            mbar_arrive(&bar[B_DEN_FULL + b]);
+        }
+    } else if (warp < 8) {
+        // ---- key exponentials, z, and the fp16 state image: thread = feature
+        regs_inc<176>();
+        const int f = row;
+        const int fg = 128 * (int)rank + f;  // feature index within m
+        float z = 0.f;
+        int g = 0;
+        for (ChunkSteps it(p, cid, n_cl); it.ok; it.next(p), ++g) {
+            const int s = g % STAGES, b = g & 1;
+            const size_t srow = (size_t)it.seg * p.m + fg;
+            if (it.first) {
+                // a segment starts from the scan's prefix: S master <- seg_S once the last state
+                // MMA of the previous segment has completed; z_<t published for the query warps
+                z = p.seg_z[srow];
+                sf[F_ZSNAP + b * 128 + f] = z;
+                mbar_arrive(&bar[B_Z_FULL + b]);
+                if (g > 0 && !mbar_wait_all(&bar[B_S_DONE], (g - 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                const float4 *src = (const float4 *)(p.seg_S + srow * 64);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float w[32];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 a = __ldg(src + 8 * h + c);
+                        w[4 * c] = a.x;
+                        w[4 * c + 1] = a.y;
+                        w[4 * c + 2] = a.z;
+                        w[4 * c + 3] = a.w;
+                    }
+                    tmem_st32(tmem + lane_off + T_S + 32 * h, w);
+                }
+                tmem_wait_st();
+            }
+            float v[128];
+            if (!mbar_wait_all(&bar[B_PK_FULL], g & 1, abort_flag)) break;
+            tc_fence_after();
+            tmem_ld128(tmem + lane_off + T_P, v);
+            tc_fence_before();
+            mbar_arrive(&bar[B_PK_FREE]);
+            if (!mbar_wait_all(&bar[B_BETA_FULL + b], (g >> 1) & 1, abort_flag)) break;
+            uint32_t hv[64];
+            z += chunk_key_features<POLY>(v, sf + F_BETA + b * 128, hv);
+            mbar_arrive(&bar[B_BETA_FREE + b]);
+            {
+                // z_<t+1 for the next tile, unless that tile starts a segment (its z is the prefix)
+                ChunkSteps nx = it;
+                nx.next(p);
+                if (nx.ok && !nx.first) {
+                    sf[F_ZSNAP + (b ^ 1) * 128 + f] = z;
+                    mbar_arrive(&bar[B_Z_FULL + (b ^ 1)]);
                 }
             }
+            // phik of tile g into shared memory ([token block][feature][64 tokens])
+            if (g > 0 && !mbar_wait_all(&bar[B_PHIK_FREE], (g - 1) & 1, abort_flag)) break;
+            uint8_t *pk = smem + OFF_PHIK + f * 128;
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *(uint4 *)(pk + blk * TILE + ((c ^ (f & 7)) << 4)) =
+                        make_uint4(hv[32 * blk + 4 * c], hv[32 * blk + 4 * c + 1], hv[32 * blk + 4 * c + 2],
+                                   hv[32 * blk + 4 * c + 3]);
+            fence_async_smem();
+            mbar_arrive(&bar[B_PHIK_FULL]);
+            // state image of tile g from S_<g (the state MMA of tile g - 1 has completed)
+            if (g > 0 && !it.first && !mbar_wait_all(&bar[B_S_DONE], (g - 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            float w[64];
+            tmem_ld64_nowait(tmem + lane_off + T_S, w);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&w[0])), FAVOR_RW32((&w[32]))::"memory");
+            float amax = 0.f;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) amax = fmaxf(amax, fabsf(w[c]));
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            if (lane == 0) {
+                sf[F_AMAX + b * 4 + (warp & 3)] = amax;
+                mbar_arrive(&bar[B_AMAX + b]);
+            }
+            if (!mbar_wait_all(&bar[B_AMAX + b], (g >> 1) & 1, abort_flag)) break;
+            amax = fmaxf(fmaxf(sf[F_AMAX + b * 4], sf[F_AMAX + b * 4 + 1]),
+                         fmaxf(sf[F_AMAX + b * 4 + 2], sf[F_AMAX + b * 4 + 3]));
+            // sigma: amax 2^-sigma < 2^15
+            const int ea = (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127;
+            const int sig = max(ea - 14, 0);
+            const float sc = pow2i(-sig);
+            uint8_t *simg = smem + OFF_SIMG + f * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint4 u;
+                u.x = pack_f16x2(w[8 * c] * sc, w[8 * c + 1] * sc);
+                u.y = pack_f16x2(w[8 * c + 2] * sc, w[8 * c + 3] * sc);
+                u.z = pack_f16x2(w[8 * c + 4] * sc, w[8 * c + 5] * sc);
+                u.w = pack_f16x2(w[8 * c + 6] * sc, w[8 * c + 7] * sc);
+                *(uint4 *)(simg + ((c ^ (f & 7)) << 4)) = u;
+            }
+            if (f == 0) sf[F_SIGMA + b] = (float)sig;
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bar[B_S_READY]);
+            mbar_arrive(&bar[B_SIG_FULL + b]);
         }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-    }
-    // Drain outstanding copies and MMAs before the CTA exits and TMEM is released (bounded).
-    if (tid == 0) {
-        volatile int no_abort = 0;
-        if (!ok) mbar_wait(tma_bar, tma_phase, &no_abort);  // a copy may still be in flight
-        mma_commit(mma_bar);
-        mbar_wait(mma_bar, mma_phase, &no_abort);
+    } else {
+        // ---- masking (tile g) and the output epilogue (tile g - 1): thread = query row
+        regs_dec<96>();
+        const int q = warp & 3;
+        ChunkSteps it(p, cid, n_cl);
+        int pbh = 0, pj0 = 0;
+        for (int g = 0;; ++g) {
+            const bool have = it.ok;
+            if (have) {
+                // masking of tile g
+                const int b = g & 1;
+                if (!mbar_wait_all(&bar[B_SC_FULL], g & 1, abort_flag)) break;
+                if (!mbar_wait_all(&bar[B_SIG_FULL + b], (g >> 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                const int sig = (int)sf[F_SIGMA + b];
+                const float sc = pow2i(-sig);
+                float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    uint32_t h[16];
+                    if (k <= q) {
+                        float a[32];
+                        tmem_ld32(tmem + lane_off + T_A + 32 * k, a);
+                        if (k == q) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) a[e] = e <= lane ? a[e] : 0.f;
+                        }
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            rs0 += a[e];
+                            rs1 += a[e + 1];
+                            h[e >> 1] = pack_f16x2(a[e] * sc, a[e + 1] * sc);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) h[e] = 0u;
+                    }
+                    tmem_st16u(tmem + lane_off + T_A + 16 * k, h);
+                }
+                if (g >= 2 && !mbar_wait_all(&bar[B_O_EMPTY + b], ((g >> 1) - 1) & 1, abort_flag)) break;
+                sf[F_DENA + b * 128 + row] = rs0 + rs1;
+                if (row == 0) sf[F_SIGE + b] = (float)sig;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bar[B_MASK_DONE]);
+                mbar_arrive(&bar[B_DEN_FULL + b]);
+            }
+            if (g > 0) {
+                // output epilogue of tile e = g - 1
+                const int e = g - 1, b = e & 1;
+                if (!mbar_wait_all(&bar[B_O_FULL + b], (e >> 1) & 1, abort_flag)) break;
+                if (!mbar_wait_all(&bar[B_DEN_FULL + b], (e >> 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                float o[64];
+                tmem_ld64_nowait(tmem + lane_off + T_O + 64 * b, o);
+                asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&o[0])), FAVOR_RW32((&o[32]))::"memory");
+                const float den = sf[F_DENQ + b * 128 + row] + sf[F_DENA + b * 128 + row];
+                const float cq = sf[F_CQ + b * 128 + row];
+                const float up = pow2i((int)sf[F_SIGE + b]);
+                tc_fence_before();
+                mbar_arrive(&bar[B_O_EMPTY + b]);
+                const int i = pj0 + row;
+                float *dst = p.out + ((size_t)pbh * p.L + i) * 64;
+                const bool store = i < p.L && i >= p.P_exact;
+                if (CL == 1) {
+                    const float inv = up * rcp_approx(den);
+                    if (store)
+#pragma unroll
+                        for (int c = 0; c < 64; c += 4)
+                            *(float4 *)(dst + c) =
+                                make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+                } else {
+                    const uint32_t partner = rank ^ 1u;
+                    if ((uint32_t)(row >> 6) != rank) {
+                        // rows the partner finishes: stage them, one bulk copy per warp
+                        if (e >= 2 && !mbar_wait_cluster_all(&bar[B_RECV_FREE + b], ((e >> 1) - 1) & 1, abort_flag))
+                            break;
+                        if (lane == 0) bulk_wait_group_read<0>();  // the previous copy has read the staging rows
+                        __syncwarp();
+                        float *srow = (float *)(smem + OFF_SEND) + (row & 63) * RECV_ROW;
+#pragma unroll
+                        for (int c = 0; c < 64; c += 4)
+                            *(float4 *)(srow + c) = make_float4(o[c] * up, o[c + 1] * up, o[c + 2] * up, o[c + 3] * up);
+                        *(float4 *)(srow + 64) = make_float4(den, cq, 0.f, 0.f);
+                        fence_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            const uint32_t off = (uint32_t)((row & 63) * RECV_ROW * 4);  // this warp's first row
+                            bulk_copy_to_peer(cluster_map(smem_u32(smem + OFF_RECV + b * RECV_SLOT) + off, partner),
+                                              smem_u32(smem + OFF_SEND) + off, 32 * RECV_ROW * 4,
+                                              cluster_map(smem_u32(&bar[B_RECV_FULL + b]), partner));
+                            bulk_commit_group();
+                        }
+                        __syncwarp();
+                    } else {
+                        // rows this CTA finishes: the partner's half arrives by bulk copy
+                        if (row == 64 * (int)rank) mbar_arrive_expect_tx(&bar[B_RECV_FULL + b], 64 * RECV_ROW * 4);
+                        if (!mbar_wait_cluster_all(&bar[B_RECV_FULL + b], (e >> 1) & 1, abort_flag)) break;
+                        const float *slot = (const float *)(smem + OFF_RECV + b * RECV_SLOT) + (row & 63) * RECV_ROW;
+                        const float4 dc = *(const float4 *)(slot + 64);
+                        const float m2 = fmaxf(cq, dc.y);
+                        const float wa = ex2_approx(cq - m2), wb = ex2_approx(dc.y - m2);
+                        const float inv = rcp_approx(den * wa + dc.x * wb);
+                        const float sa = up * wa * inv, sb = wb * inv;
+#pragma unroll
+                        for (int c = 0; c < 64; c += 4) {
+                            const float4 r4 = *(const float4 *)(slot + c);
+                            o[c] = fmaf(o[c], sa, r4.x * sb);
+                            o[c + 1] = fmaf(o[c + 1], sa, r4.y * sb);
+                            o[c + 2] = fmaf(o[c + 2], sa, r4.z * sb);
+                            o[c + 3] = fmaf(o[c + 3], sa, r4.w * sb);
+                        }
+                        mbar_arrive_remote(cluster_map(smem_u32(&bar[B_RECV_FREE + b]), partner));
+                        if (store)
+#pragma unroll
+                            for (int c = 0; c < 64; c += 4)
+                                *(float4 *)(dst + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+                    }
+                }
+            }
+            if (!have) break;
+            pbh = it.bh;
+            pj0 = it.tile * kTile;
+            it.next(p);
+        }
+        // the last bulk copies have read their staging rows before the CTA may exit
+        if (CL > 1 && lane == 0) bulk_wait_group_all();
     }
     tc_fence_before();
     __syncthreads();
+    if (CL > 1) cluster_sync_all();  // no CTA leaves while its partner may still access its memory
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 13) tmem_dealloc(tmem, 512);
 }
 
 // ============================================================================ host launchers
 
-template <int D>
-static size_t causal_smem() {
-    using SM = CausalSmem<D>;
-    return 1024 + SM::W_BYTES + SM::S_BYTES + 2 * SM::QK_BYTES + SM::VT_BYTES + 2 * SM::KB_SLOT +
-           (256 + 256 + 128 * 3 + 512) * 4 + 256;
-}
-
 cudaError_t launch_state_scan(const ScanParams &p, int BH, cudaStream_t st) {
-    const size_t n = (size_t)p.m * p.d + p.m + p.n_split;
+    const size_t n = (size_t)p.m * p.d + p.m;
     k_state_scan<<<dim3((unsigned)((n + 255) / 256), BH), 256, 0, st>>>(p);
     return cudaGetLastError();
 }
@@ -606,14 +1057,71 @@ cudaError_t launch_causal_prefix(const PrefixParams &p, int BH, cudaStream_t st)
     return cudaGetLastError();
 }
 
-cudaError_t launch_causal_out(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mW,
-                              const CausalParams &p, int BH, cudaStream_t st) {
-    const dim3 grid(p.n_split, BH);
-    if (p.d != 64) return cudaErrorInvalidValue;
-    const size_t sm = causal_smem<64>();
-    cudaFuncSetAttribute(k_causal_out<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_causal_out<64><<<grid, kCausalThreads, sm, st>>>(mQ, mK, mW, p);
-    return cudaGetLastError();
+// The register split of k_causal_chunk (176 + 176 + 96 + 64 per warpgroup lane) fits the 128 per
+// thread it is launched with; the launch is refused unless the kernel carries exactly 128.
+template <int CL, int POLY>
+static cudaError_t launch_causal_chunk_t(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mV,
+                                         const CUtensorMap &mW, const ChunkParams &p, cudaStream_t st) {
+    static int checked = 0;
+    static int n_cl = 0;
+    const size_t sm = 1024 + chunk::BYTES;
+    if (checked == 0) {
+        cudaFuncAttributes a{};
+        checked = (cudaFuncGetAttributes(&a, k_causal_chunk<CL, POLY>) == cudaSuccess && a.numRegs == 128) ? 1 : -1;
+        if (checked > 0 &&
+            cudaFuncSetAttribute(k_causal_chunk<CL, POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+                cudaSuccess)
+            checked = -1;
+        if (checked > 0) {
+            cudaLaunchConfig_t cfg{};
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = CL;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(CL * 1024);
+            cfg.blockDim = dim3(kChunkThreads);
+            cfg.dynamicSmemBytes = sm;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n_cl, k_causal_chunk<CL, POLY>, &cfg) != cudaSuccess || n_cl < 1)
+                checked = -1;
+        }
+    }
+    if (checked < 0) return cudaErrorInvalidConfiguration;
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(CL * std::min(n_cl, p.n_seg)));
+    cfg.blockDim = dim3(kChunkThreads);
+    cfg.dynamicSmemBytes = sm;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_causal_chunk<CL, POLY>, mQ, mK, mV, mW, p);
+}
+
+cudaError_t launch_causal_chunk(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mV,
+                                const CUtensorMap &mW, const ChunkParams &p, int poly_pct, cudaStream_t st) {
+    const int poly = poly_pct < 13 ? 0 : poly_pct < 31 ? 8 : poly_pct < 44 ? 12 : 16;
+    if (p.m == 128) {
+        switch (poly) {
+            case 0: return launch_causal_chunk_t<1, 0>(mQ, mK, mV, mW, p, st);
+            case 8: return launch_causal_chunk_t<1, 8>(mQ, mK, mV, mW, p, st);
+            case 12: return launch_causal_chunk_t<1, 12>(mQ, mK, mV, mW, p, st);
+            default: return launch_causal_chunk_t<1, 16>(mQ, mK, mV, mW, p, st);
+        }
+    }
+    if (p.m != 256) return cudaErrorInvalidValue;
+    switch (poly) {
+        case 0: return launch_causal_chunk_t<2, 0>(mQ, mK, mV, mW, p, st);
+        case 8: return launch_causal_chunk_t<2, 8>(mQ, mK, mV, mW, p, st);
+        case 12: return launch_causal_chunk_t<2, 12>(mQ, mK, mV, mW, p, st);
+        default: return launch_causal_chunk_t<2, 16>(mQ, mK, mV, mW, p, st);
+    }
 }
 
 }  // namespace favor
