@@ -36,7 +36,7 @@ L2_FLUSH_BYTES = 256 << 20
 
 # Kernels favor_fwd launches for the bf16 path, in launch order (stage k <-> events 2k, 2k+1).
 FWD_STAGES = ["k_key_partials", "k_state_image", "k_query_out"]
-CAUSAL_STAGES = ["k_key_logit_max", "k_key_state", "k_state_scan", "k_causal_out", "k_causal_prefix"]
+CAUSAL_STAGES = ["k_key_logit_max", "k_key_state", "k_state_scan", "k_causal_chunk", "k_causal_prefix"]
 
 
 def load_peaks():
@@ -65,8 +65,10 @@ def stage_work(name, w, n_sms=148):
         return t * (2 * d + 4), 2 * m * d * t, 0
     if name == "k_key_state":          # read K, V, -|k|^2/2
         return t * (4 * d + 4), 2 * m * d * t, 2 * m * d * t
-    if name == "k_causal_out":         # read Q, K, V, -|k|^2/2; write fp32 out
-        return t * (10 * d + 4), 6 * m * d * t, (4 * m * d + 2 * 128 * m + 2 * 128 * d) * t
+    if name == "k_causal_chunk":       # read Q, K, V, -|k|^2/2; write fp32 out; fp16 MMAs per token:
+        # Q W^T and K W^T (2 x 2md), state term and state update (2 x 2md), scores and masked A V
+        # over the 128-token tile (2 * 128 * m + 2 * 128 * d)
+        return t * (10 * d + 4), (8 * m * d + 2 * 128 * m + 2 * 128 * d) * t, 0
     return 0, 0, 0
 
 

@@ -284,7 +284,8 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     ChunkParams cp{s->L, s->m, l.n_split, l.tiles_per_split, l.P_exact, l.BH * l.n_split, bias, head_max,
                    seg_S, seg_z, out};
     record_stage(o, 6, st);
-    e = launch_causal_chunk(mQ, mK, mV, mW128, cp, opt_poly_pct(o), st);
+    // all exponentials on MUFU unless a share is asked for: the chunk kernel is not MUFU-bound
+    e = launch_causal_chunk(mQ, mK, mV, mW128, cp, o ? o->exp_poly_pct : 0, st);
     record_stage(o, 7, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     float *phi = (float *)(ws + l.off_phi);

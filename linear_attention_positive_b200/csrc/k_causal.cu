@@ -82,44 +82,57 @@ struct PrefixParams {
 __device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
 // phi(q) = exp(w.q - max_r w.q) and phi(k) = exp(w.k - |k|^2/2 - C) in fp32 for the first P tokens
-// of each head. CTA per (32 tokens, head); thread r computes feature r (its W row in registers)
-// for all 32 tokens and stores them as one contiguous run of its feature row; the per-token max
-// over features goes through shared memory.
+// of each head. CTA per (32 tokens, head); the tokens' q and k rows are widened to fp32 in shared
+// memory once; thread r computes feature r (its W row in registers) token by token and stores its
+// 32 values as one contiguous run of its feature row; the per-token max over features goes through
+// shared memory.
 __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) {
-    __shared__ uint16_t xq[32][64], xk[32][64];
-    __shared__ float su[32][257], smax[32];
-    __shared__ float sbias[32];
+    extern __shared__ __align__(16) float fsm[];  // xq [32][64], xk [32][64], su [32][256], smax, sbias
+    float(*xq)[64] = (float(*)[64])fsm;
+    float(*xk)[64] = (float(*)[64])(fsm + 32 * 64);
+    float(*su)[256] = (float(*)[256])(fsm + 2 * 32 * 64);
+    float *smax = fsm + 2 * 32 * 64 + 32 * 256, *sbias = smax + 32;
     const int bh = blockIdx.y, j0 = blockIdx.x * 32, t = threadIdx.x;
-    for (int idx = t; idx < 32 * 64; idx += 256) {
-        const int a = idx >> 6, e = idx & 63;
-        const int j = j0 + a;
-        const size_t row = ((size_t)bh * p.L + j) * p.d;
-        xq[a][e] = (j < p.P && e < p.d) ? p.Q[row + e] : (uint16_t)0;
-        xk[a][e] = (j < p.P && e < p.d) ? p.K[row + e] : (uint16_t)0;
+    {
+        // 32 token rows of q and k (64 bf16 each) as 16-byte loads, widened to fp32
+        const int a = t >> 3, e8 = (t & 7) * 8, j = j0 + a;
+        const size_t row = ((size_t)bh * p.L + j) * p.d + e8;
+        const uint4 rq = j < p.P ? *(const uint4 *)(p.Q + row) : make_uint4(0, 0, 0, 0);
+        const uint4 rk = j < p.P ? *(const uint4 *)(p.K + row) : make_uint4(0, 0, 0, 0);
+        const uint32_t wq[4] = {rq.x, rq.y, rq.z, rq.w}, wk[4] = {rk.x, rk.y, rk.z, rk.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            xq[a][e8 + 2 * h] = __uint_as_float(wq[h] << 16);
+            xq[a][e8 + 2 * h + 1] = __uint_as_float(wq[h] & 0xFFFF0000u);
+            xk[a][e8 + 2 * h] = __uint_as_float(wk[h] << 16);
+            xk[a][e8 + 2 * h + 1] = __uint_as_float(wk[h] & 0xFFFF0000u);
+        }
     }
     if (t < 32) sbias[t] = j0 + t < p.P ? p.bias[(size_t)bh * p.L + j0 + t] - p.head_max[bh] : -INFINITY;
     __syncthreads();
-    float w[64];
     if (t < p.m) {
+        float w[64];
 #pragma unroll
         for (int e = 0; e < 64; ++e) w[e] = e < p.d ? bf16_to_f(p.W[(size_t)t * p.d + e]) : 0.f;
-        float ok[32];
-#pragma unroll
+        float *dk = p.phiK + ((size_t)bh * p.m + t) * p.Ps + j0;
+#pragma unroll 1
         for (int a = 0; a < 32; ++a) {
-            float sq0 = 0.f, sq1 = 0.f, sk0 = 0.f, sk1 = 0.f;
+            float q0 = 0.f, q1 = 0.f, k0 = 0.f, k1 = 0.f;
 #pragma unroll
-            for (int e = 0; e < 64; e += 2) {
-                sq0 = fmaf(w[e], bf16_to_f(xq[a][e]), sq0);
-                sq1 = fmaf(w[e + 1], bf16_to_f(xq[a][e + 1]), sq1);
-                sk0 = fmaf(w[e], bf16_to_f(xk[a][e]), sk0);
-                sk1 = fmaf(w[e + 1], bf16_to_f(xk[a][e + 1]), sk1);
+            for (int e = 0; e < 64; e += 4) {
+                const float4 x4 = *(const float4 *)&xq[a][e], y4 = *(const float4 *)&xk[a][e];
+                q0 = fmaf(w[e], x4.x, q0);
+                q1 = fmaf(w[e + 1], x4.y, q1);
+                q0 = fmaf(w[e + 2], x4.z, q0);
+                q1 = fmaf(w[e + 3], x4.w, q1);
+                k0 = fmaf(w[e], y4.x, k0);
+                k1 = fmaf(w[e + 1], y4.y, k1);
+                k0 = fmaf(w[e + 2], y4.z, k0);
+                k1 = fmaf(w[e + 3], y4.w, k1);
             }
-            su[a][t] = sq0 + sq1;
-            ok[a] = expf(sk0 + sk1 + sbias[a]);
+            su[a][t] = q0 + q1;
+            dk[a] = expf(k0 + k1 + sbias[a]);
         }
-        float4 *dst = (float4 *)(p.phiK + ((size_t)bh * p.m + t) * p.Ps + j0);
-#pragma unroll
-        for (int a = 0; a < 32; a += 4) dst[a / 4] = make_float4(ok[a], ok[a + 1], ok[a + 2], ok[a + 3]);
     }
     __syncthreads();
     {
@@ -133,94 +146,139 @@ __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) 
     }
     __syncthreads();
     if (t < p.m) {
-        float oq[32];
-#pragma unroll
-        for (int a = 0; a < 32; ++a) oq[a] = j0 + a < p.P ? expf(su[a][t] - smax[a]) : 0.f;
-        float4 *dst = (float4 *)(p.phiQ + ((size_t)bh * p.m + t) * p.Ps + j0);
-#pragma unroll
-        for (int a = 0; a < 32; a += 4) dst[a / 4] = make_float4(oq[a], oq[a + 1], oq[a + 2], oq[a + 3]);
+        float *dq = p.phiQ + ((size_t)bh * p.m + t) * p.Ps + j0;
+#pragma unroll 4
+        for (int a = 0; a < 32; ++a) dq[a] = j0 + a < p.P ? expf(su[a][t] - smax[a]) : 0.f;
     }
 }
 
-// Masked attention over the first P tokens in fp32: CTA per (64 queries, head), 256 threads, the
-// CTAs with the most key blocks first. Per 64-key block up to the diagonal: scores
-// S = phi(Q) phi(K)^T (4 x 4 per thread, features in 32-wide slices through shared memory, read
-// as rows of the feature-major scratch), the mask j <= i, then num += S V and den += rowsum(S)
-// (4 queries x 4 value columns per thread).
+// Masked attention over the first P tokens in fp32: CTA per (32 queries, head), 256 threads. The
+// queries' phi (all m features) stays in shared memory; per 64-key block up to the diagonal the
+// keys' phi is brought in 128-feature halves. Scores S = phi(Q) phi(K)^T (2 queries x 4 keys per
+// thread), the mask j <= i, then num += S V and den += rowsum(S) (2 queries x 4 values per
+// thread). Dynamic shared memory: qT [m][32], kT [128][64], V block [64][64], S [32][68].
+constexpr int kPrefixQ = 32;
 __global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
-    // the feature slices (score phase) and the masked scores (output phase) share one buffer
-    __shared__ __align__(16) float buf[64 * 65];
-    __shared__ __align__(16) float sv[64][64];  // V block
-    float(*aq)[64] = (float(*)[64])buf;         // [32 features][64 queries]
-    float(*ak)[64] = (float(*)[64])(buf + 32 * 64);
-    float(*ss)[65] = (float(*)[65])buf;         // [64 queries][64 keys + pad]
-    const int bh = blockIdx.y, i0 = (gridDim.x - 1 - blockIdx.x) * 64, t = threadIdx.x;
-    const int ti = (t >> 4) * 4, tj = (t & 15) * 4;  // this thread's 4 x 4 score block / 4 x 4 output block
-    float num[4][4], den[4];
+    extern __shared__ __align__(16) float psm[];
+    float *qT = psm;                         // [m][32]
+    float *kT = qT + (size_t)p.m * kPrefixQ;  // [128][64]
+    float *sv = kT + 128 * 64;               // [64][64]
+    float *ss = sv + 64 * 64;                // [32][68]
+    const int bh = blockIdx.y, i0 = (gridDim.x - 1 - blockIdx.x) * kPrefixQ, t = threadIdx.x;
+    const float *phq = p.phiQ + (size_t)bh * p.m * p.Ps;
+    const float *phk = p.phiK + (size_t)bh * p.m * p.Ps;
+    // qT: m rows of 32 queries (i0 + 31 < Ps: rows of the scratch are padded to multiples of 32)
+    for (int idx = t; idx < p.m * (kPrefixQ / 4); idx += 256 * 4) {
+        float4 r[4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
+        for (int u = 0; u < 4; ++u) {
+            const int k = idx + 256 * u, f = k >> 3, a4 = (k & 7) * 4;
+            r[u] = k < p.m * (kPrefixQ / 4) ? *(const float4 *)(phq + (size_t)f * p.Ps + i0 + a4) : make_float4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int k = idx + 256 * u;
+            if (k < p.m * (kPrefixQ / 4)) *(float4 *)(qT + 4 * k) = r[u];
+        }
+    }
+    const int tq = (t >> 4) * 2, tk = (t & 15) * 4;  // scores: 2 queries x 4 keys
+    float num[2][4], den[2];
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
         den[a] = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) num[a][c] = 0.f;
     }
-    const float *phq = p.phiQ + (size_t)bh * p.m * p.Ps;
-    const float *phk = p.phiK + (size_t)bh * p.m * p.Ps;
-    for (int j0 = 0; j0 <= i0 && j0 < p.P; j0 += 64) {
-        float sc[4][4];
+    for (int j0 = 0; j0 < i0 + kPrefixQ && j0 < p.P; j0 += 64) {
+        float sc[2][4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
             for (int b = 0; b < 4; ++b) sc[a][b] = 0.f;
-        for (int f0 = 0; f0 < p.m; f0 += 32) {
-            __syncthreads();
-            for (int idx = t; idx < 64 * 32; idx += 256) {
-                const int f = idx >> 6, a = idx & 63;
-                aq[f][a] = (i0 + a < p.P) ? phq[(size_t)(f0 + f) * p.Ps + i0 + a] : 0.f;
-                ak[f][a] = (j0 + a < p.P) ? phk[(size_t)(f0 + f) * p.Ps + j0 + a] : 0.f;
+        for (int f0 = 0; f0 < p.m; f0 += 128) {
+            __syncthreads();  // previous readers of kT / sv / ss are done
+            {
+                // kT: 128 feature rows of 64 keys as float4 (a float4 never crosses the padded row end;
+                // entries past P are zero in the scratch)
+                float4 r[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int k = t + 256 * u, f = k >> 4, a4 = (k & 15) * 4;
+                    r[u] = j0 + a4 < p.Ps ? *(const float4 *)(phk + (size_t)(f0 + f) * p.Ps + j0 + a4)
+                                          : make_float4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) *(float4 *)(kT + 4 * (t + 256 * u)) = r[u];
+            }
+            if (f0 == 0) {
+                // V block: 64 keys x 64 values (bf16, 8 per 16-byte load), zero past P
+                uint4 r[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int k = t + 256 * u, a = k >> 3, e8 = (k & 7) * 8;
+                    r[u] = j0 + a < p.P ? *(const uint4 *)(p.V + ((size_t)bh * p.L + j0 + a) * p.d + e8)
+                                        : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int k = t + 256 * u;
+                    const uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+                    float *dst = sv + 8 * k;
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        dst[2 * h] = __uint_as_float(w[h] << 16);
+                        dst[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+                    }
+                }
             }
             __syncthreads();
-#pragma unroll 8
-            for (int f = 0; f < 32; ++f) {
-                const float4 q4 = *(const float4 *)&aq[f][ti], k4 = *(const float4 *)&ak[f][tj];
-                const float qv[4] = {q4.x, q4.y, q4.z, q4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-                for (int a = 0; a < 4; ++a)
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) sc[a][b] = fmaf(qv[a], kv[b], sc[a][b]);
+#pragma unroll 4
+            for (int f = 0; f < 128; ++f) {
+                const float2 q2 = *(const float2 *)&qT[(f0 + f) * kPrefixQ + tq];
+                const float4 k4 = *(const float4 *)&kT[f * 64 + tk];
+                sc[0][0] = fmaf(q2.x, k4.x, sc[0][0]);
+                sc[0][1] = fmaf(q2.x, k4.y, sc[0][1]);
+                sc[0][2] = fmaf(q2.x, k4.z, sc[0][2]);
+                sc[0][3] = fmaf(q2.x, k4.w, sc[0][3]);
+                sc[1][0] = fmaf(q2.y, k4.x, sc[1][0]);
+                sc[1][1] = fmaf(q2.y, k4.y, sc[1][1]);
+                sc[1][2] = fmaf(q2.y, k4.z, sc[1][2]);
+                sc[1][3] = fmaf(q2.y, k4.w, sc[1][3]);
             }
         }
-        __syncthreads();
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int b = 0; b < 4; ++b) ss[ti + a][tj + b] = (j0 + tj + b <= i0 + ti + a) ? sc[a][b] : 0.f;
-        for (int idx = t; idx < 64 * 64; idx += 256) {
-            const int a = idx >> 6, e = idx & 63;
-            sv[a][e] = (j0 + a < p.P && e < p.d) ? bf16_to_f(p.V[((size_t)bh * p.L + j0 + a) * p.d + e]) : 0.f;
-        }
+            for (int b = 0; b < 4; ++b) ss[(tq + a) * 68 + tk + b] = (j0 + tk + b <= i0 + tq + a) ? sc[a][b] : 0.f;
         __syncthreads();
+        // num[2 queries][4 values] += S V over the block's 64 keys
+#pragma unroll 4
         for (int j = 0; j < 64; ++j) {
-            const float4 v4 = *(const float4 *)&sv[j][tj];
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                const float sa = ss[ti + a][j];
-                num[a][0] = fmaf(sa, v4.x, num[a][0]);
-                num[a][1] = fmaf(sa, v4.y, num[a][1]);
-                num[a][2] = fmaf(sa, v4.z, num[a][2]);
-                num[a][3] = fmaf(sa, v4.w, num[a][3]);
-                den[a] += sa;
-            }
+            const float4 v4 = *(const float4 *)&sv[j * 64 + tk];
+            const float s0 = ss[tq * 68 + j], s1 = ss[(tq + 1) * 68 + j];
+            num[0][0] = fmaf(s0, v4.x, num[0][0]);
+            num[0][1] = fmaf(s0, v4.y, num[0][1]);
+            num[0][2] = fmaf(s0, v4.z, num[0][2]);
+            num[0][3] = fmaf(s0, v4.w, num[0][3]);
+            num[1][0] = fmaf(s1, v4.x, num[1][0]);
+            num[1][1] = fmaf(s1, v4.y, num[1][1]);
+            num[1][2] = fmaf(s1, v4.z, num[1][2]);
+            num[1][3] = fmaf(s1, v4.w, num[1][3]);
+            den[0] += s0;
+            den[1] += s1;
         }
     }
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        const int i = i0 + ti + a;
-        if (i < p.P && i < p.L && tj < p.d) {
-            float *o = p.out + ((size_t)bh * p.L + i) * p.d + tj;
+    for (int a = 0; a < 2; ++a) {
+        const int i = i0 + tq + a;
+        if (i < p.P && i < p.L && tk < p.d) {
+            float *o = p.out + ((size_t)bh * p.L + i) * p.d + tk;
             *(float4 *)o = make_float4(num[a][0] / den[a], num[a][1] / den[a], num[a][2] / den[a], num[a][3] / den[a]);
         }
     }
 }
+
+static size_t prefix_attn_smem(int m) { return ((size_t)m * kPrefixQ + 128 * 64 + 64 * 64 + 32 * 68) * 4; }
 
 // ============================================================================ k_causal_chunk
 //
@@ -392,21 +450,6 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, ui
                  : "memory");
 }
 
-// phiq = 2^(v log2e - cl) over a row of 128 logits, in place. Per 32 columns the first 32 - POLY
-// exponentials go to MUFU ex2, the rest to the FMA-pipe polynomial.
-template <int POLY>
-__device__ __forceinline__ void chunk_query_exps(float (&v)[128], float cl) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int e = c * 32; e < c * 32 + 32; ++e) v[e] = fmaf(v[e], kLog2e, -cl);
-#pragma unroll
-        for (int e = c * 32; e < c * 32 + 32 - POLY; ++e) v[e] = ex2_approx(v[e]);
-#pragma unroll
-        for (int e = c * 32 + 32 - POLY; e < c * 32 + 32; e += 2) exp2_poly_pair(v[e], v[e + 1], v[e], v[e + 1]);
-    }
-}
-
 // phik = 2^(v log2e + beta_j) over a row of 128 tokens, rounded to fp16 pairs; returns the row's
 // sum (fp32, before rounding).
 template <int POLY>
@@ -554,7 +597,7 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
     const int row = (warp & 3) * 32 + lane;  // TMEM lane of this thread (query row or feature)
 
     if (warp >= 12) {
-        regs_dec<64>();
+        regs_dec<72>();
         if (warp == 12) {
             // ---- TMA: W once; Q, K of tile g and V of tile g - 1 per step (V is needed later and
             // its stage is held until the tile's last MMA); the key terms
@@ -761,8 +804,9 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
             }
         }
     } else if (warp < 4) {
-        // ---- query exponentials: thread = query row
-        regs_inc<176>();
+        // ---- query exponentials: thread = query row (the row of logits in registers, so P is
+        // released at once)
+        regs_inc<208>();
         int g = 0;
         for (ChunkSteps it(p, cid, n_cl); it.ok; it.next(p), ++g) {
             const int b = g & 1;
@@ -773,7 +817,15 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
             tc_fence_before();
             mbar_arrive(&bar[B_PQ_FREE]);
             const float cl = row_max128(v) * kLog2e;
-            chunk_query_exps<POLY>(v, cl);
+#pragma unroll
+            for (int e = 0; e < 128; ++e) v[e] = fmaf(v[e], kLog2e, -cl);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int e = 32 * c; e < 32 * c + 32 - POLY; ++e) v[e] = ex2_approx(v[e]);
+#pragma unroll
+                for (int e = 32 * c + 32 - POLY; e < 32 * c + 32; e += 2) exp2_poly_pair(v[e], v[e + 1], v[e], v[e + 1]);
+            }
             // den_q = phiq . z_<t (z_<t is published before the state term of tile g - 1 frees phiq)
             if (!mbar_wait_all(&bar[B_Z_FULL + b], (g >> 1) & 1, abort_flag)) break;
             const float *z = sf + F_ZSNAP + b * 128;
@@ -805,7 +857,7 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
         }
     } else if (warp < 8) {
         // ---- key exponentials, z, and the fp16 state image: thread = feature
-        regs_inc<176>();
+        regs_dec<104>();
         const int f = row;
         const int fg = 128 * (int)rank + f;  // feature index within m
         float z = 0.f;
@@ -837,16 +889,59 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                 }
                 tmem_wait_st();
             }
-            float v[128];
+            // phik = 2^(P^T log2e + beta_j) per 32-token chunk straight from TMEM (the next chunk's load
+            // in flight), each chunk stored to shared memory as fp16 ([token block][feature][64 tokens])
+            // once the previous tile's MMAs have read phik; P is held until the last chunk is read
             if (!mbar_wait_all(&bar[B_PK_FULL], g & 1, abort_flag)) break;
+            if (!mbar_wait_all(&bar[B_BETA_FULL + b], (g >> 1) & 1, abort_flag)) break;
+            if (g > 0 && !mbar_wait_all(&bar[B_PHIK_FREE], (g - 1) & 1, abort_flag)) break;
             tc_fence_after();
-            tmem_ld128(tmem + lane_off + T_P, v);
+            const float *beta = sf + F_BETA + b * 128;
+            uint8_t *pk = smem + OFF_PHIK + f * 128;
+            float zs0 = 0.f, zs1 = 0.f;
+            float va[32], vb[32];
+            tmem_ld32(tmem + lane_off + T_P, va);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float(&v)[32] = (c & 1) ? vb : va;
+                float(&vn)[32] = (c & 1) ? va : vb;
+                if (c < 3)
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+                        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+                        "%30, %31}, [%32];"
+                        : FAVOR_REG32(vn)
+                        : "r"(tmem + lane_off + T_P + 32 * (c + 1)));
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 b4 = *(const float4 *)(beta + 32 * c + e);
+                    v[e] = fmaf(v[e], kLog2e, b4.x);
+                    v[e + 1] = fmaf(v[e + 1], kLog2e, b4.y);
+                    v[e + 2] = fmaf(v[e + 2], kLog2e, b4.z);
+                    v[e + 3] = fmaf(v[e + 3], kLog2e, b4.w);
+                }
+#pragma unroll
+                for (int e = 0; e < 32 - POLY; ++e) v[e] = ex2_approx(v[e]);
+#pragma unroll
+                for (int e = 32 - POLY; e < 32; e += 2) exp2_poly_pair(v[e], v[e + 1], v[e], v[e + 1]);
+                uint32_t hv[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    zs0 += v[e];
+                    zs1 += v[e + 1];
+                    hv[e >> 1] = pack_f16x2(v[e], v[e + 1]);
+                }
+                // tokens 32c .. 32c + 31: block c >> 1, 16-byte chunks 4 (c & 1) .. + 3
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    *(uint4 *)(pk + (c >> 1) * TILE + (((4 * (c & 1) + u) ^ (f & 7)) << 4)) =
+                        make_uint4(hv[4 * u], hv[4 * u + 1], hv[4 * u + 2], hv[4 * u + 3]);
+                if (c < 3) asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32(vn)::"memory");
+            }
             tc_fence_before();
             mbar_arrive(&bar[B_PK_FREE]);
-            if (!mbar_wait_all(&bar[B_BETA_FULL + b], (g >> 1) & 1, abort_flag)) break;
-            uint32_t hv[64];
-            z += chunk_key_features<POLY>(v, sf + F_BETA + b * 128, hv);
             mbar_arrive(&bar[B_BETA_FREE + b]);
+            z += zs0 + zs1;
             {
                 // z_<t+1 for the next tile, unless that tile starts a segment (its z is the prefix)
                 ChunkSteps nx = it;
@@ -856,27 +951,19 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                     mbar_arrive(&bar[B_Z_FULL + (b ^ 1)]);
                 }
             }
-            // phik of tile g into shared memory ([token block][feature][64 tokens])
-            if (g > 0 && !mbar_wait_all(&bar[B_PHIK_FREE], (g - 1) & 1, abort_flag)) break;
-            uint8_t *pk = smem + OFF_PHIK + f * 128;
-#pragma unroll
-            for (int blk = 0; blk < 2; ++blk)
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *(uint4 *)(pk + blk * TILE + ((c ^ (f & 7)) << 4)) =
-                        make_uint4(hv[32 * blk + 4 * c], hv[32 * blk + 4 * c + 1], hv[32 * blk + 4 * c + 2],
-                                   hv[32 * blk + 4 * c + 3]);
             fence_async_smem();
             mbar_arrive(&bar[B_PHIK_FULL]);
             // state image of tile g from S_<g (the state MMA of tile g - 1 has completed)
             if (g > 0 && !it.first && !mbar_wait_all(&bar[B_S_DONE], (g - 1) & 1, abort_flag)) break;
             tc_fence_after();
-            float w[64];
-            tmem_ld64_nowait(tmem + lane_off + T_S, w);
-            asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&w[0])), FAVOR_RW32((&w[32]))::"memory");
             float amax = 0.f;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                float w[32];
+                tmem_ld32(tmem + lane_off + T_S + 32 * h, w);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) amax = fmaxf(amax, fabsf(w[c]));
+                for (int c = 0; c < 32; ++c) amax = fmaxf(amax, fabsf(w[c]));
+            }
             for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             if (lane == 0) {
                 sf[F_AMAX + b * 4 + (warp & 3)] = amax;
@@ -890,14 +977,19 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
             const int sig = max(ea - 14, 0);
             const float sc = pow2i(-sig);
             uint8_t *simg = smem + OFF_SIMG + f * 128;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                float w[32];
+                tmem_ld32(tmem + lane_off + T_S + 32 * h, w);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 u;
-                u.x = pack_f16x2(w[8 * c] * sc, w[8 * c + 1] * sc);
-                u.y = pack_f16x2(w[8 * c + 2] * sc, w[8 * c + 3] * sc);
-                u.z = pack_f16x2(w[8 * c + 4] * sc, w[8 * c + 5] * sc);
-                u.w = pack_f16x2(w[8 * c + 6] * sc, w[8 * c + 7] * sc);
-                *(uint4 *)(simg + ((c ^ (f & 7)) << 4)) = u;
+                for (int c = 0; c < 4; ++c) {
+                    uint4 u;
+                    u.x = pack_f16x2(w[8 * c] * sc, w[8 * c + 1] * sc);
+                    u.y = pack_f16x2(w[8 * c + 2] * sc, w[8 * c + 3] * sc);
+                    u.z = pack_f16x2(w[8 * c + 4] * sc, w[8 * c + 5] * sc);
+                    u.w = pack_f16x2(w[8 * c + 6] * sc, w[8 * c + 7] * sc);
+                    *(uint4 *)(simg + (((4 * h + c) ^ (f & 7)) << 4)) = u;
+                }
             }
             if (f == 0) sf[F_SIGMA + b] = (float)sig;
             fence_async_smem();
@@ -906,15 +998,59 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
             mbar_arrive(&bar[B_SIG_FULL + b]);
         }
     } else {
-        // ---- masking (tile g) and the output epilogue (tile g - 1): thread = query row
-        regs_dec<96>();
+        // ---- masking (tile g) and the output epilogue (tile e = g - 1): thread = query row. Per
+        // step: the partial output of tile e is read from TMEM (rows the partner finishes are
+        // staged and sent at once), tile g is masked, then this CTA's rows of tile e are finished
+        // with the partner's half, which has arrived meanwhile.
         const int q = warp & 3;
+        const bool keep = CL == 1 || (uint32_t)(row >> 6) == rank;  // warp-uniform
+        const uint32_t partner = rank ^ 1u;
         ChunkSteps it(p, cid, n_cl);
         int pbh = 0, pj0 = 0;
         for (int g = 0;; ++g) {
             const bool have = it.ok;
+            const int e = g - 1, eb = e & 1;
+            float o[64], den = 0.f, cq = 0.f, up = 1.f;
+            if (g > 0) {
+                // A. tile e: partial output and denominators
+                if (!mbar_wait_all(&bar[B_O_FULL + eb], (e >> 1) & 1, abort_flag)) break;
+                if (!mbar_wait_all(&bar[B_DEN_FULL + eb], (e >> 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                tmem_ld64_nowait(tmem + lane_off + T_O + 64 * eb, o);
+                asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&o[0])), FAVOR_RW32((&o[32]))::"memory");
+                den = sf[F_DENQ + eb * 128 + row] + sf[F_DENA + eb * 128 + row];
+                cq = sf[F_CQ + eb * 128 + row];
+                up = pow2i((int)sf[F_SIGE + eb]);
+                tc_fence_before();
+                mbar_arrive(&bar[B_O_EMPTY + eb]);
+                if (!keep) {
+                    // rows the partner finishes: stage them, one bulk copy per warp
+                    if (e >= 2 && !mbar_wait_cluster_all(&bar[B_RECV_FREE + eb], ((e >> 1) - 1) & 1, abort_flag))
+                        break;
+                    if (lane == 0) bulk_wait_group_read<0>();  // the previous copy has read the staging rows
+                    __syncwarp();
+                    float *srow = (float *)(smem + OFF_SEND) + (row & 63) * RECV_ROW;
+#pragma unroll
+                    for (int c = 0; c < 64; c += 4)
+                        *(float4 *)(srow + c) = make_float4(o[c] * up, o[c + 1] * up, o[c + 2] * up, o[c + 3] * up);
+                    *(float4 *)(srow + 64) = make_float4(den, cq, 0.f, 0.f);
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const uint32_t off = (uint32_t)((row & 63) * RECV_ROW * 4);  // this warp's first row
+                        bulk_copy_to_peer(cluster_map(smem_u32(smem + OFF_RECV + eb * RECV_SLOT) + off, partner),
+                                          smem_u32(smem + OFF_SEND) + off, 32 * RECV_ROW * 4,
+                                          cluster_map(smem_u32(&bar[B_RECV_FULL + eb]), partner));
+                        bulk_commit_group();
+                    }
+                    __syncwarp();
+                } else if (CL > 1 && row == 64 * (int)rank) {
+                    // arm for the partner's two bulk copies of tile e
+                    mbar_arrive_expect_tx(&bar[B_RECV_FULL + eb], 64 * RECV_ROW * 4);
+                }
+            }
             if (have) {
-                // masking of tile g
+                // B. masking of tile g
                 const int b = g & 1;
                 if (!mbar_wait_all(&bar[B_SC_FULL], g & 1, abort_flag)) break;
                 if (!mbar_wait_all(&bar[B_SIG_FULL + b], (g >> 1) & 1, abort_flag)) break;
@@ -922,7 +1058,7 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                 const int sig = (int)sf[F_SIGMA + b];
                 const float sc = pow2i(-sig);
                 float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
+#pragma unroll 1
                 for (int k = 0; k < 4; ++k) {
                     uint32_t h[16];
                     if (k <= q) {
@@ -930,17 +1066,17 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                         tmem_ld32(tmem + lane_off + T_A + 32 * k, a);
                         if (k == q) {
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) a[e] = e <= lane ? a[e] : 0.f;
+                            for (int c = 0; c < 32; ++c) a[c] = c <= lane ? a[c] : 0.f;
                         }
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            rs0 += a[e];
-                            rs1 += a[e + 1];
-                            h[e >> 1] = pack_f16x2(a[e] * sc, a[e + 1] * sc);
+                        for (int c = 0; c < 32; c += 2) {
+                            rs0 += a[c];
+                            rs1 += a[c + 1];
+                            h[c >> 1] = pack_f16x2(a[c] * sc, a[c + 1] * sc);
                         }
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) h[e] = 0u;
+                        for (int c = 0; c < 16; ++c) h[c] = 0u;
                     }
                     tmem_st16u(tmem + lane_off + T_A + 16 * k, h);
                 }
@@ -952,20 +1088,8 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                 mbar_arrive(&bar[B_MASK_DONE]);
                 mbar_arrive(&bar[B_DEN_FULL + b]);
             }
-            if (g > 0) {
-                // output epilogue of tile e = g - 1
-                const int e = g - 1, b = e & 1;
-                if (!mbar_wait_all(&bar[B_O_FULL + b], (e >> 1) & 1, abort_flag)) break;
-                if (!mbar_wait_all(&bar[B_DEN_FULL + b], (e >> 1) & 1, abort_flag)) break;
-                tc_fence_after();
-                float o[64];
-                tmem_ld64_nowait(tmem + lane_off + T_O + 64 * b, o);
-                asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&o[0])), FAVOR_RW32((&o[32]))::"memory");
-                const float den = sf[F_DENQ + b * 128 + row] + sf[F_DENA + b * 128 + row];
-                const float cq = sf[F_CQ + b * 128 + row];
-                const float up = pow2i((int)sf[F_SIGE + b]);
-                tc_fence_before();
-                mbar_arrive(&bar[B_O_EMPTY + b]);
+            if (g > 0 && keep) {
+                // C. this CTA's rows of tile e
                 const int i = pj0 + row;
                 float *dst = p.out + ((size_t)pbh * p.L + i) * 64;
                 const bool store = i < p.L && i >= p.P_exact;
@@ -974,55 +1098,27 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                     if (store)
 #pragma unroll
                         for (int c = 0; c < 64; c += 4)
-                            *(float4 *)(dst + c) =
-                                make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+                            *(float4 *)(dst + c) = make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
                 } else {
-                    const uint32_t partner = rank ^ 1u;
-                    if ((uint32_t)(row >> 6) != rank) {
-                        // rows the partner finishes: stage them, one bulk copy per warp
-                        if (e >= 2 && !mbar_wait_cluster_all(&bar[B_RECV_FREE + b], ((e >> 1) - 1) & 1, abort_flag))
-                            break;
-                        if (lane == 0) bulk_wait_group_read<0>();  // the previous copy has read the staging rows
-                        __syncwarp();
-                        float *srow = (float *)(smem + OFF_SEND) + (row & 63) * RECV_ROW;
+                    if (!mbar_wait_cluster_all(&bar[B_RECV_FULL + eb], (e >> 1) & 1, abort_flag)) break;
+                    const float *slot = (const float *)(smem + OFF_RECV + eb * RECV_SLOT) + (row & 63) * RECV_ROW;
+                    const float4 dc = *(const float4 *)(slot + 64);
+                    const float m2 = fmaxf(cq, dc.y);
+                    const float wa = ex2_approx(cq - m2), wb = ex2_approx(dc.y - m2);
+                    const float inv = rcp_approx(den * wa + dc.x * wb);
+                    const float sa = up * wa * inv, sb = wb * inv;
 #pragma unroll
-                        for (int c = 0; c < 64; c += 4)
-                            *(float4 *)(srow + c) = make_float4(o[c] * up, o[c + 1] * up, o[c + 2] * up, o[c + 3] * up);
-                        *(float4 *)(srow + 64) = make_float4(den, cq, 0.f, 0.f);
-                        fence_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            const uint32_t off = (uint32_t)((row & 63) * RECV_ROW * 4);  // this warp's first row
-                            bulk_copy_to_peer(cluster_map(smem_u32(smem + OFF_RECV + b * RECV_SLOT) + off, partner),
-                                              smem_u32(smem + OFF_SEND) + off, 32 * RECV_ROW * 4,
-                                              cluster_map(smem_u32(&bar[B_RECV_FULL + b]), partner));
-                            bulk_commit_group();
-                        }
-                        __syncwarp();
-                    } else {
-                        // rows this CTA finishes: the partner's half arrives by bulk copy
-                        if (row == 64 * (int)rank) mbar_arrive_expect_tx(&bar[B_RECV_FULL + b], 64 * RECV_ROW * 4);
-                        if (!mbar_wait_cluster_all(&bar[B_RECV_FULL + b], (e >> 1) & 1, abort_flag)) break;
-                        const float *slot = (const float *)(smem + OFF_RECV + b * RECV_SLOT) + (row & 63) * RECV_ROW;
-                        const float4 dc = *(const float4 *)(slot + 64);
-                        const float m2 = fmaxf(cq, dc.y);
-                        const float wa = ex2_approx(cq - m2), wb = ex2_approx(dc.y - m2);
-                        const float inv = rcp_approx(den * wa + dc.x * wb);
-                        const float sa = up * wa * inv, sb = wb * inv;
-#pragma unroll
-                        for (int c = 0; c < 64; c += 4) {
-                            const float4 r4 = *(const float4 *)(slot + c);
-                            o[c] = fmaf(o[c], sa, r4.x * sb);
-                            o[c + 1] = fmaf(o[c + 1], sa, r4.y * sb);
-                            o[c + 2] = fmaf(o[c + 2], sa, r4.z * sb);
-                            o[c + 3] = fmaf(o[c + 3], sa, r4.w * sb);
-                        }
-                        mbar_arrive_remote(cluster_map(smem_u32(&bar[B_RECV_FREE + b]), partner));
-                        if (store)
-#pragma unroll
-                            for (int c = 0; c < 64; c += 4)
-                                *(float4 *)(dst + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+                    for (int c = 0; c < 64; c += 4) {
+                        const float4 r4 = *(const float4 *)(slot + c);
+                        o[c] = fmaf(o[c], sa, r4.x * sb);
+                        o[c + 1] = fmaf(o[c + 1], sa, r4.y * sb);
+                        o[c + 2] = fmaf(o[c + 2], sa, r4.z * sb);
+                        o[c + 3] = fmaf(o[c + 3], sa, r4.w * sb);
                     }
+                    mbar_arrive_remote(cluster_map(smem_u32(&bar[B_RECV_FREE + eb]), partner));
+                    if (store)
+#pragma unroll
+                        for (int c = 0; c < 64; c += 4) *(float4 *)(dst + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
                 }
             }
             if (!have) break;
@@ -1050,14 +1146,18 @@ cudaError_t launch_state_scan(const ScanParams &p, int BH, cudaStream_t st) {
 
 cudaError_t launch_causal_prefix(const PrefixParams &p, int BH, cudaStream_t st) {
     if (p.P <= 0) return cudaSuccess;
-    k_causal_prefix_features<<<dim3((p.P + 31) / 32, BH), 256, 0, st>>>(p);
+    const size_t fsm = (2 * 32 * 64 + 32 * 256 + 64) * 4;
+    cudaFuncSetAttribute(k_causal_prefix_features, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
+    k_causal_prefix_features<<<dim3((p.P + 31) / 32, BH), 256, fsm, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    k_causal_prefix_attn<<<dim3((p.P + 63) / 64, BH), 256, 0, st>>>(p);
+    const size_t sm = prefix_attn_smem(p.m);
+    cudaFuncSetAttribute(k_causal_prefix_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_causal_prefix_attn<<<dim3((p.P + kPrefixQ - 1) / kPrefixQ, BH), 256, sm, st>>>(p);
     return cudaGetLastError();
 }
 
-// The register split of k_causal_chunk (176 + 176 + 96 + 64 per warpgroup lane) fits the 128 per
+// The register split of k_causal_chunk (208 + 104 + 128 + 72 per warpgroup lane) fits the 128 per
 // thread it is launched with; the launch is refused unless the kernel carries exactly 128.
 template <int CL, int POLY>
 static cudaError_t launch_causal_chunk_t(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mV,

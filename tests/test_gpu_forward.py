@@ -252,3 +252,23 @@ def test_bf16_causal_config4_full_size_all_rows(cuda_device):
         sq += float(np.sum(ref * ref))
     rms = np.sqrt(sq / (w.H * w.L * w.d))
     assert max(errs) / rms <= TOL["bf16"]
+
+
+def test_bf16_causal_values_beyond_fp16_range_are_reported(cuda_device):
+    """The causal bf16 path feeds V to fp16 tensor-core operands: a value entry of magnitude 2^16 or
+    more cannot be represented there, and the call reports FAVOR_ERR_UNSUPPORTED through the device
+    status word instead of returning a silently wrong output. Entries just below the limit pass."""
+    w = Workload("t", 1, 1, 700, 64, 256, True, "bf16", False, 3, 41)
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    Q, K = (to_torch(x[k], w.dtype, cuda_device) for k in "QK")
+    Wt = to_torch(Wr, w.dtype, cuda_device)
+    V = x["V"].copy()
+    V[0, 0, 600, 5] = 60000.0      # bf16 rounds it to 59904: inside the fp16 range
+    out = api.fwd(Q, K, to_torch(V, w.dtype, cuda_device), Wt, causal=True)
+    assert api.sync_status() == api.FAVOR_OK
+    assert np.isfinite(out.cpu().numpy()).all()
+    V[0, 0, 600, 5] = 70000.0      # beyond it
+    api.fwd(Q, K, to_torch(V, w.dtype, cuda_device), Wt, causal=True)
+    assert api.sync_status() == api.FAVOR_ERR_UNSUPPORTED
+    assert api.sync_status() == api.FAVOR_OK  # the status word is cleared by the read
