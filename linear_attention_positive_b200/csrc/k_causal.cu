@@ -87,11 +87,14 @@ __device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float(
 // 32 values as one contiguous run of its feature row; the per-token max over features goes through
 // shared memory.
 __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) {
-    extern __shared__ __align__(16) float fsm[];  // xq [32][64], xk [32][64], su [32][256], smax, sbias
+    // xq, xk [32][64] token rows; su [32][257] query logits then phi(q); sk [32][257] phi(k);
+    // smax, sbias [32]
+    extern __shared__ __align__(16) float fsm[];
     float(*xq)[64] = (float(*)[64])fsm;
     float(*xk)[64] = (float(*)[64])(fsm + 32 * 64);
-    float(*su)[256] = (float(*)[256])(fsm + 2 * 32 * 64);
-    float *smax = fsm + 2 * 32 * 64 + 32 * 256, *sbias = smax + 32;
+    float(*su)[257] = (float(*)[257])(fsm + 2 * 32 * 64);  // rows padded: token-wise reads stay conflict-free
+    float(*sk)[257] = (float(*)[257])(fsm + 2 * 32 * 64 + 32 * 257);
+    float *smax = fsm + 2 * 32 * 64 + 2 * 32 * 257, *sbias = smax + 32;
     const int bh = blockIdx.y, j0 = blockIdx.x * 32, t = threadIdx.x;
     {
         // 32 token rows of q and k (64 bf16 each) as 16-byte loads, widened to fp32
@@ -112,9 +115,17 @@ __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) 
     __syncthreads();
     if (t < p.m) {
         float w[64];
+        const uint4 *wr = (const uint4 *)(p.W + (size_t)t * p.d);
 #pragma unroll
-        for (int e = 0; e < 64; ++e) w[e] = e < p.d ? bf16_to_f(p.W[(size_t)t * p.d + e]) : 0.f;
-        float *dk = p.phiK + ((size_t)bh * p.m + t) * p.Ps + j0;
+        for (int e = 0; e < 64; e += 8) {
+            const uint4 u = __ldg(wr + e / 8);
+            const uint32_t h4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                w[e + 2 * h] = __uint_as_float(h4[h] << 16);
+                w[e + 2 * h + 1] = __uint_as_float(h4[h] & 0xFFFF0000u);
+            }
+        }
 #pragma unroll 1
         for (int a = 0; a < 32; ++a) {
             float q0 = 0.f, q1 = 0.f, k0 = 0.f, k1 = 0.f;
@@ -131,7 +142,7 @@ __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) 
                 k1 = fmaf(w[e + 3], y4.w, k1);
             }
             su[a][t] = q0 + q1;
-            dk[a] = expf(k0 + k1 + sbias[a]);
+            sk[a][t] = expf(k0 + k1 + sbias[a]);
         }
     }
     __syncthreads();
@@ -145,10 +156,18 @@ __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) 
         }
     }
     __syncthreads();
-    if (t < p.m) {
-        float *dq = p.phiQ + ((size_t)bh * p.m + t) * p.Ps + j0;
+    if (t < p.m)
 #pragma unroll 4
-        for (int a = 0; a < 32; ++a) dq[a] = j0 + a < p.P ? expf(su[a][t] - smax[a]) : 0.f;
+        for (int a = 0; a < 32; ++a) su[a][t] = j0 + a < p.P ? expf(su[a][t] - smax[a]) : 0.f;
+    __syncthreads();
+    {
+        // feature rows out: warp w writes rows f = w, w + 8, ...; lane = token (128-byte rows)
+        const int warp = t >> 5, lane = t & 31;
+        for (int f = warp; f < p.m; f += 8) {
+            const size_t o = ((size_t)bh * p.m + f) * p.Ps + j0 + lane;
+            p.phiK[o] = sk[lane][f];
+            p.phiQ[o] = su[lane][f];
+        }
     }
 }
 
@@ -901,7 +920,7 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
             float zs0 = 0.f, zs1 = 0.f;
             float va[32], vb[32];
             tmem_ld32(tmem + lane_off + T_P, va);
-#pragma unroll
+#pragma unroll 2
             for (int c = 0; c < 4; ++c) {
                 float(&v)[32] = (c & 1) ? vb : va;
                 float(&vn)[32] = (c & 1) ? va : vb;
@@ -1146,7 +1165,7 @@ cudaError_t launch_state_scan(const ScanParams &p, int BH, cudaStream_t st) {
 
 cudaError_t launch_causal_prefix(const PrefixParams &p, int BH, cudaStream_t st) {
     if (p.P <= 0) return cudaSuccess;
-    const size_t fsm = (2 * 32 * 64 + 32 * 256 + 64) * 4;
+    const size_t fsm = (2 * 32 * 64 + 2 * 32 * 257 + 64) * 4;
     cudaFuncSetAttribute(k_causal_prefix_features, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
     k_causal_prefix_features<<<dim3((p.P + 31) / 32, BH), 256, fsm, st>>>(p);
     cudaError_t e = cudaGetLastError();
