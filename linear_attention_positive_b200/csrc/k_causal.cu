@@ -171,19 +171,20 @@ __global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) 
     }
 }
 
-// Masked attention over the first P tokens in fp32: CTA per (32 queries, head), 256 threads. The
+// Masked attention over the first P tokens in fp32: 32-query blocks, two per CTA (below), 256 threads. The
 // queries' phi (all m features) stays in shared memory; per 64-key block up to the diagonal the
 // keys' phi is brought in 128-feature halves. Scores S = phi(Q) phi(K)^T (2 queries x 4 keys per
 // thread), the mask j <= i, then num += S V and den += rowsum(S) (2 queries x 4 values per
 // thread). Dynamic shared memory: qT [m][32], kT [128][64], V block [64][64], S [32][68].
 constexpr int kPrefixQ = 32;
-__global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
+__device__ __forceinline__ void prefix_attn_block(const PrefixParams &p, int i0) {
     extern __shared__ __align__(16) float psm[];
     float *qT = psm;                         // [m][32]
     float *kT = qT + (size_t)p.m * kPrefixQ;  // [128][64]
     float *sv = kT + 128 * 64;               // [64][64]
     float *ss = sv + 64 * 64;                // [32][68]
-    const int bh = blockIdx.y, i0 = (gridDim.x - 1 - blockIdx.x) * kPrefixQ, t = threadIdx.x;
+    const int bh = blockIdx.y, t = threadIdx.x;
+    __syncthreads();  // the previous block's readers of the shared buffers are done
     const float *phq = p.phiQ + (size_t)bh * p.m * p.Ps;
     const float *phk = p.phiK + (size_t)bh * p.m * p.Ps;
     // qT: m rows of 32 queries (i0 + 31 < Ps: rows of the scratch are padded to multiples of 32)
@@ -295,6 +296,13 @@ __global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
             *(float4 *)o = make_float4(num[a][0] / den[a], num[a][1] / den[a], num[a][2] / den[a], num[a][3] / den[a]);
         }
     }
+}
+
+// Query blocks i and n - 1 - i share a CTA, so every CTA does about the same number of key blocks.
+__global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
+    const int nq = (p.P + kPrefixQ - 1) / kPrefixQ, qa = blockIdx.x, qb = nq - 1 - blockIdx.x;
+    prefix_attn_block(p, qb * kPrefixQ);
+    if (qa < qb) prefix_attn_block(p, qa * kPrefixQ);
 }
 
 static size_t prefix_attn_smem(int m) { return ((size_t)m * kPrefixQ + 128 * 64 + 64 * 64 + 32 * 68) * 4; }
@@ -1172,7 +1180,8 @@ cudaError_t launch_causal_prefix(const PrefixParams &p, int BH, cudaStream_t st)
     if (e != cudaSuccess) return e;
     const size_t sm = prefix_attn_smem(p.m);
     cudaFuncSetAttribute(k_causal_prefix_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_causal_prefix_attn<<<dim3((p.P + kPrefixQ - 1) / kPrefixQ, BH), 256, sm, st>>>(p);
+    const int nq = (p.P + kPrefixQ - 1) / kPrefixQ;
+    k_causal_prefix_attn<<<dim3((nq + 1) / 2, BH), 256, sm, st>>>(p);
     return cudaGetLastError();
 }
 
