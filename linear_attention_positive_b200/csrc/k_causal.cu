@@ -318,23 +318,24 @@ static size_t prefix_attn_smem(int m) { return ((size_t)m * kPrefixQ + 128 * 64 
 //   phiq = 2^(P log2e - c_i), c_i its row maximum over the CTA's features, fp16 into TMEM;
 //          den_q = phiq . z_<t on CUDA cores
 //   P^T  = W_r K_t^T                       (bf16 MMA; features on TMEM lanes)
-//   phik = 2^(P^T log2e + beta_j), beta_j = (-|k_j|^2/2 - C) log2e + A + b_t, fp16 into shared
-//          memory as [feature][token] rows; z_<t+1 = z_<t + 2^-b_t sum_j phik
+//   phik = 2^(P^T log2e + beta_j), beta_j = (-|k_j|^2/2 - C) log2e + A, fp16 into shared memory
+//          as [feature][token] rows; z_<t+1 = z_<t + sum_j phik
 //   Simg = fp16(S_<t 2^-sigma_t)           (converted from TMEM; S_<t of a segment's first tile
 //          is the prefix the scan wrote)
 //   O    = phiq Simg                       (fp16 MMA, A from TMEM)
 //   A    = phiq phik^T                     (fp16 MMA) -> masked (key > query -> 0), row sums
-//          den_a = 2^-b_t sum_j A_ij in fp32, fp16(A 2^-sigma_t) in place
-//   S   += phik^T V'_t                     (fp16 MMA, V'_t = V_t 2^-b_t converted in place)
-//   O   += A V'_t
+//          den_a = sum_j A_ij in fp32, fp16(A 2^-sigma_t) in place
+//   S   += phik^T V_t                      (fp16 MMA, V_t converted bf16 -> fp16 in place)
+//   O   += A V_t
 //   partial numerator O 2^sigma_t, partial denominator den_q + den_a, both relative to 2^c_i.
-// C is the per-(batch, head) key maximum, so phik <= 2^(A + b_t) with A = 8 (fp16 headroom for keys
-// far below the maximum); b_t = clamp(e_t - 13, 0, 7) with e_t the exponent of the tile's largest
-// |v| keeps V'_t in fp16 range; every product phik v' carries the same 2^A, which cancels in the
-// ratio. sigma_t >= b_t keeps the scaled S and A below 2^15.
-// Warp roles (16 warps): 0-3 query exponentials; 4-7 key exponentials and the state image; 8-11
-// masking and the output epilogue (one tile behind); 12 TMA; 13 MMA issue; 14-15 V conversion and
-// the key terms beta_j.
+// C is the per-(batch, head) key maximum, so phik <= 2^A with A = 8 (fp16 headroom for keys far
+// below the maximum); every product phik v carries the same 2^A, which cancels in the ratio.
+// sigma_t keeps the scaled S below 2^15, and with phik <= 2^8 over 128 features the scaled scores
+// stay below 2^15 too. V entries must fit fp16 (magnitude below 2^16): larger or non-finite
+// entries are reported as FAVOR_ERR_UNSUPPORTED through the device status word.
+// Warp roles (16 warps): 0-3 query exponentials and den_q; 4-7 key exponentials, z and the state
+// image; 8-11 masking and the output epilogue (one tile behind); 12 TMA and the key terms beta_j;
+// 13 projection MMAs; 14 scores, state term, state update and masked A V MMAs; 15 V conversion.
 // TMEM columns: P [0,128), phiq [128,192), A [192,320) (fp16 in [192,256)), S [320,384),
 // O [384 + 64 b, +64) for b = tile parity.
 
@@ -419,10 +420,6 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t smem_addr, uint32_t ran
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
     return r;
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
-}
 // Arrive (release, cluster scope) on an mbarrier in another CTA of the cluster.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
@@ -475,35 +472,6 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, ui
     asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "r"(src), "r"(bytes), "r"(mbar)
                  : "memory");
-}
-
-// phik = 2^(v log2e + beta_j) over a row of 128 tokens, rounded to fp16 pairs; returns the row's
-// sum (fp32, before rounding).
-template <int POLY>
-__device__ __forceinline__ float chunk_key_features(float (&v)[128], const float *beta, uint32_t (&hv)[64]) {
-    float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int e = c * 32; e < c * 32 + 32; e += 4) {
-            const float4 b4 = *(const float4 *)(beta + e);
-            v[e] = fmaf(v[e], kLog2e, b4.x);
-            v[e + 1] = fmaf(v[e + 1], kLog2e, b4.y);
-            v[e + 2] = fmaf(v[e + 2], kLog2e, b4.z);
-            v[e + 3] = fmaf(v[e + 3], kLog2e, b4.w);
-        }
-#pragma unroll
-        for (int e = c * 32; e < c * 32 + 32 - POLY; ++e) v[e] = ex2_approx(v[e]);
-#pragma unroll
-        for (int e = c * 32 + 32 - POLY; e < c * 32 + 32; e += 2) exp2_poly_pair(v[e], v[e + 1], v[e], v[e + 1]);
-#pragma unroll
-        for (int e = c * 32; e < c * 32 + 32; e += 2) {
-            s0 += v[e];
-            s1 += v[e + 1];
-            hv[e >> 1] = pack_f16x2(v[e], v[e + 1]);
-        }
-    }
-    return s0 + s1;
 }
 
 // Shared-memory descriptors as their low 32 bits (start address and LBO fields; the high word, SBO
