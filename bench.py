@@ -370,9 +370,23 @@ def run_ours(args, w):
             line["roofline"] = {"kernel": dom, "bound": "hbm", "achieved": nbytes / sec / 1e9, "peak": hbm_peak,
                                 "unit": "GB/s", "frac": (nbytes / sec / 1e9) / hbm_peak,
                                 "traffic": measured_traffic(dom, w.name), "note": f"peak {peak_src} copy bandwidth"}
+        # Path-level fractions (work of the definition, not of the kernels): Q, K, V, O bytes at the
+        # measured copy bandwidth; 6 L m d FLOPs per head at the measured bf16 rate; 2 m exponentials
+        # per token at 16 MUFU ex2 per clock per SM, at the SM clock sampled during the timed steps.
         path_bytes = w.tokens * (6 * w.d + 4 * w.d)
+        step_s = ms_per_step * 1e-3
+        path_flops = 6 * w.tokens * w.m * w.d
+        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+        sm_hz = (clk["sm_mhz"] if clk and clk.get("sm_mhz") else 1965.0) * 1e6
+        path_exps = 2 * w.m * w.tokens
         line["path_roofline"] = {"hbm_bytes_per_step": path_bytes,
-                                 "hbm_frac": path_bytes / (ms_per_step * 1e-3) / (hbm_peak * 1e9)}
+                                 "hbm_frac": path_bytes / step_s / (hbm_peak * 1e9),
+                                 "tensor_flops_per_step": path_flops,
+                                 "tensor_frac": path_flops / step_s / (tc_peak * 1e12),
+                                 "exps_per_step": path_exps,
+                                 "mufu_frac": path_exps / step_s / (16 * n_sm * sm_hz),
+                                 "note": "hbm: Q, K, V bf16 + O fp32; tensor: 6 L m d per head at the measured "
+                                         "bf16 peak; mufu: 2 m ex2 per token at 16 per clock per SM"}
     if clk is not None:
         line["clocks"] = clk
     if world == 1 and not args.no_cpu_baseline:
