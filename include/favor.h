@@ -72,7 +72,8 @@ typedef struct {
 /* Tuning knobs; pass NULL for defaults. Zero fields take their defaults too.
  *   split_tiles : 128-token tiles per CTA for the key-side reduction (and per causal segment)
  *   exp_poly_pct: percent (0..100) of feature exponentials evaluated by the FMA-pipe
- *                 polynomial instead of the MUFU ex2 unit (bf16 path)
+ *                 polynomial instead of the MUFU ex2 unit (bf16 path); 0 (the default) puts
+ *                 all of them on MUFU
  *   stage_events: NULL, or 2 * FAVOR_MAX_STAGES caller-created cudaEvent_t handles (as void*);
  *                 the call records events[2k] before and events[2k+1] after its k-th kernel
  *                 launch on the call's stream (NULL entries are skipped). For timing. */

@@ -48,10 +48,11 @@ favor_status shape_supported(const favor_shape *s, int causal, int backward) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Share of feature exponentials on the FMA-pipe polynomial (percent); 0 takes the default.
+// Share of feature exponentials on the FMA-pipe polynomial (percent); 0 takes the default, all on
+// MUFU (measured fastest on B200 for every kernel: the kernels are latency-bound, not MUFU-bound).
 int opt_poly_pct(const favor_opts *o) {
     const int v = o ? o->exp_poly_pct : 0;
-    return v > 0 ? std::min(v, 100) : 37;
+    return v > 0 ? std::min(v, 100) : 0;
 }
 
 int opt_split_tiles(const favor_opts *o) {
@@ -284,8 +285,7 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     ChunkParams cp{s->L, s->m, l.n_split, l.tiles_per_split, l.P_exact, l.BH * l.n_split, bias, head_max,
                    seg_S, seg_z, out};
     record_stage(o, 6, st);
-    // all exponentials on MUFU unless a share is asked for: the chunk kernel is not MUFU-bound
-    e = launch_causal_chunk(mQ, mK, mV, mW128, cp, o ? o->exp_poly_pct : 0, st);
+    e = launch_causal_chunk(mQ, mK, mV, mW128, cp, opt_poly_pct(o), st);
     record_stage(o, 7, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     float *phi = (float *)(ws + l.off_phi);
