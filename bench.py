@@ -227,6 +227,28 @@ def workload_config(w, n):
             "l2": "flushed between steps (256 MB write, outside the timed events)"}
 
 
+# ------------------------------------------------------------------------------------ ranks
+
+def max_over_ranks(values, world, device=None):
+    """Element-wise maximum of a list of floats over all ranks (one all-reduce MAX; the job takes as
+    long as its slowest rank). At world size 1 the values come back unchanged."""
+    if world == 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_rate(tokens_per_rank, world, job_ms, steps):
+    """(ms per step, whole-job tokens/s) for `steps` steps that took job_ms on the slowest rank, each
+    rank processing tokens_per_rank per step (weak scaling: the per-rank work is fixed)."""
+    ms_per_step = job_ms / steps
+    return ms_per_step, tokens_per_rank * world / (ms_per_step * 1e-3)
+
+
 # ------------------------------------------------------------------------------------ GPU arm
 
 def run_ours(args, w):
@@ -301,13 +323,8 @@ def run_ours(args, w):
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     stage_ms = [[stage_ev[k][2 * i].elapsed_time(stage_ev[k][2 * i + 1]) for k in range(args.steps)]
                 for i in range(n_stage)]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    job_ms = float(t.item())
-    ms_per_step = job_ms / args.steps
-    value = w.tokens * world / (ms_per_step * 1e-3)
+    job_ms = max_over_ranks([sum(step_ms)], world, dev)[0]
+    ms_per_step, value = job_rate(w.tokens, world, job_ms, args.steps)
 
     # End to end through the public API: pinned host inputs in, fp32 output back, every step.
     pin = {k: torch.from_numpy(x[k]).to(tdt).pin_memory() for k in x}
@@ -328,9 +345,8 @@ def run_ours(args, w):
         out_h.copy_(out, non_blocking=True)
         e2e_ev[k][1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps], dtype=torch.float64, device=dev)
+    e2e_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps], world, dev)[0]
     if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
@@ -344,7 +360,7 @@ def run_ours(args, w):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": workload_config(w, world),
-        "e2e": {"value": w.tokens * world / (float(e2e_ms.item()) * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_rate(w.tokens, world, e2e_ms, 1)[1], "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": (n_stage + (1 if w.causal else 0)) * args.steps if w.dtype == "bf16" else args.steps,
         "device_status": api.status_string(status),
