@@ -70,7 +70,9 @@ typedef struct {
 #define FAVOR_MAX_STAGES 8
 
 /* Tuning knobs; pass NULL for defaults. Zero fields take their defaults too.
- *   split_tiles : 128-token tiles per CTA for the key-side reduction (and per causal segment)
+ *   split_tiles : 128-token tiles per causal segment (the unit of the causal key-side reduction
+ *                 and of the chunked scan; default 8); the bidirectional path spreads its key
+ *                 tiles over the SMs by itself
  *   exp_poly_pct: percent (0..100) of feature exponentials evaluated by the FMA-pipe
  *                 polynomial instead of the MUFU ex2 unit (bf16 path); 0 (the default) puts
  *                 all of them on MUFU
