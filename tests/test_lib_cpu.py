@@ -88,3 +88,27 @@ def test_status_strings(favor_lib):
     for code in range(6):
         assert api.status_string(code).startswith("FAVOR_")
     assert "unknown" in api.status_string(99)
+
+
+def test_causal_bf16_workspace_covers_its_parts(favor_lib):
+    """The causal bf16 forward keeps, in the caller's workspace, the per-key -|k|^2/2 terms, the
+    per-segment partial states and their exclusive prefixes ([m, d] + [m] fp32 per segment each)
+    and the fp32 features of the exactly recomputed first tokens; shorter segments mean more of
+    them. d = 128 has no causal bf16 forward (sized zero, refused before any launch)."""
+    B, H, L, d = 1, 16, 65536, 64
+    for m in (128, 256):
+        sh = api.make_shape(B, H, L, d, m, api.FAVOR_BF16)
+        n_seg = B * H * (((L + 127) // 128 + 7) // 8)        # default: 8 tiles of 128 per segment
+        parts = (B * H * L * 4                                 # -|k|^2/2
+                 + 2 * n_seg * m * (d + 1) * 4                 # partial states and prefixes
+                 + 2 * B * H * m * 512 * 4)                    # exact-prefix features
+        ws = api.workspace_size(sh, causal=True)
+        assert ws >= parts and ws % 256 == 0
+        short = api.workspace_size(sh, causal=True, opts=api.make_opts(split_tiles=2))
+        assert short > ws
+    tall = api.make_shape(1, 1, 1024, 128, 256, api.FAVOR_BF16)
+    assert api.workspace_size(tall, causal=True) == 0
+    assert api.workspace_size(tall, causal=False) > 0
+    p = ctypes.c_void_p(256)
+    assert favor_lib.favor_fwd(ctypes.byref(tall), p, p, p, p, 1, p, None, p, 1 << 30, None, None) == \
+        api.FAVOR_ERR_UNSUPPORTED
