@@ -125,6 +125,20 @@ def test_error_vs_softmax_falls_as_m_grows():
     assert all(a > b for a, b in zip(errs, errs[1:])), errs
 
 
+def test_softmax_reference_matches_library_softmax():
+    # The exact-softmax reference used above, against scipy's softmax row by row (causal rows
+    # see keys 0..i only).
+    from scipy.special import softmax
+
+    rng = np.random.default_rng(5)
+    L, d = 12, 6
+    Q, K, V = (rng.standard_normal((L, d)) for _ in range(3))
+    ref_b = softmax(Q @ K.T, axis=1) @ V
+    ref_c = np.stack([softmax(K[: i + 1] @ Q[i]) @ V[: i + 1] for i in range(L)])
+    assert np.allclose(favor.softmax_attention(Q, K, V), ref_b, rtol=1e-12, atol=1e-14)
+    assert np.allclose(favor.softmax_attention(Q, K, V, causal=True), ref_c, rtol=1e-12, atol=1e-14)
+
+
 # ------------------------------------------------------------------ invariants I1-I8
 
 def _small(seed=0, L=40, d=8, m=24, scale=0.7):

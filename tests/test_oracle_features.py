@@ -119,3 +119,24 @@ def test_golden_W_regression():
 def test_draw_rejects_bad_sizes():
     with pytest.raises(ValueError):
         features.draw_W(1, 0, 64)
+
+
+def test_blocks_are_independent():
+    # Separate d-row blocks come from separate Gaussian streams. For independent Haar-distributed
+    # orthonormal blocks U0, U1 the product U0 U1^T is Haar on O(d), whose trace has mean 0 and
+    # variance 1; blocks that shared their directions would give trace d. The chi norms of row i
+    # in block 0 and row i in block 1 are independent draws (Pearson correlation ~ 0).
+    d, n = 16, 300
+    tr = np.empty(n)
+    n0, n1 = [], []
+    for s in range(n):
+        W = features.draw_W(500 + s, 2 * d, d)
+        U0, U1 = features.block_directions(W, d)
+        tr[s] = np.trace(U0 @ U1.T)
+        n0.append(np.linalg.norm(W[:d], axis=1))
+        n1.append(np.linalg.norm(W[d:], axis=1))
+    assert abs(tr.mean()) < 4.0 / math.sqrt(n)
+    t2 = tr * tr
+    assert abs(t2.mean() - 1.0) < 4.0 * t2.std(ddof=1) / math.sqrt(n)
+    n0, n1 = np.concatenate(n0), np.concatenate(n1)
+    assert abs(np.corrcoef(n0, n1)[0, 1]) < 4.0 / math.sqrt(n0.size)
