@@ -112,3 +112,23 @@ def test_causal_bf16_workspace_covers_its_parts(favor_lib):
     p = ctypes.c_void_p(256)
     assert favor_lib.favor_fwd(ctypes.byref(tall), p, p, p, p, 1, p, None, p, 1 << 30, None, None) == \
         api.FAVOR_ERR_UNSUPPORTED
+
+
+def test_empty_inputs_are_refused_before_launch(favor_lib):
+    """Empty tensors (B, H or L zero) are an argument error on every entry point, answered on the
+    host before any CUDA call (the library documents L >= 1); their workspace and ctx sizes are 0."""
+    p = ctypes.c_void_p(256)
+    null = None
+    for dims in ((1, 1, 0), (0, 1, 256), (1, 0, 256)):
+        for dt in (api.FAVOR_F32, api.FAVOR_BF16):
+            sh = api.make_shape(*dims, 64, 128, dt)
+            assert api.workspace_size(sh) == 0 and api.workspace_size(sh, True, True) == 0
+            assert favor_lib.favor_ctx_size(ctypes.byref(sh), 0) == 0
+            for causal in (0, 1):
+                assert favor_lib.favor_fwd(ctypes.byref(sh), p, p, p, p, causal, p, null, p, 1 << 20, null,
+                                           null) == api.FAVOR_ERR_INVALID_ARG
+                assert favor_lib.favor_bwd(ctypes.byref(sh), p, p, p, p, p, p, null, causal, p, p, p, p, 1 << 20,
+                                           null, null) == api.FAVOR_ERR_INVALID_ARG
+            if dt == api.FAVOR_BF16:
+                assert favor_lib.favor_fwd_static_scratch(ctypes.byref(sh), p, p, p, p, p,
+                                                          null) == api.FAVOR_ERR_INVALID_ARG
