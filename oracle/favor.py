@@ -191,6 +191,22 @@ def bwd(Q, K, V, W, dO, causal=False):
 
 
 # --------------------------------------------------------------------------------------------
+# Recurrent single-token step (causal decoding)
+# --------------------------------------------------------------------------------------------
+
+def decode_step(S, z, q, k, v, W):
+    """One step of the masked FA-part's prefix-sum recurrence for a new token t with query q,
+    key k and value v (one head): S_t = S_{t-1} + phi(k) v^T, z_t = z_{t-1} + phi(k),
+    out_t = phi(q)^T S_t / phi(q)^T z_t. The empty state is S = 0 (m x d), z = 0 (m).
+    Returns (out_t, S_t, z_t); the inputs are not modified."""
+    pk = phi(k[None, :], W)[0]
+    pq = phi(q[None, :], W)[0]
+    S = S + np.outer(pk, v)
+    z = z + pk
+    return (pq @ S) / (pq @ z), S, z
+
+
+# --------------------------------------------------------------------------------------------
 # Row-sampled evaluation for full-size parity checks
 # --------------------------------------------------------------------------------------------
 

@@ -258,3 +258,24 @@ def test_batched_wrappers_match_per_head():
         assert np.array_equal(out[1, 0], f(x["Q"][1, 0], x["K"][1, 0], x["V"][1, 0], W))
         ref = g(x["Q"][0, 1], x["K"][0, 1], x["V"][0, 1], W, x["dO"][0, 1])
         assert np.array_equal(dK[0, 1], ref[1])
+
+
+# ------------------------------------------------------------------ recurrent single-token step
+
+def test_decode_steps_reproduce_brute_force_causal_rows():
+    """Running the single-token step from the empty state over a sequence gives, at every step,
+    the row of the explicit masked L x L attention; the carried state equals the explicit sums
+    (K')^T V and (K')^T 1 over the tokens seen so far."""
+    w = WORKLOADS[1].with_(L=48, d=16, m=32)
+    x = _head(w)
+    W = features.draw_W(3, w.m, w.d)
+    ref, _ = favor.attention_brute(x["Q"], x["K"], x["V"], W, causal=True)
+    S, z = np.zeros((w.m, w.d)), np.zeros(w.m)
+    for t in range(w.L):
+        o, S2, z2 = favor.decode_step(S, z, x["Q"][t], x["K"][t], x["V"][t], W)
+        assert not np.shares_memory(S2, S)
+        S, z = S2, z2
+        assert np.abs(o - ref[t]).max() <= 1e-12 * np.abs(ref).max()
+    Kp = favor.phi(x["K"], W)
+    assert np.allclose(S, Kp.T @ x["V"], rtol=1e-12, atol=0)
+    assert np.allclose(z, Kp.sum(axis=0), rtol=1e-12, atol=0)

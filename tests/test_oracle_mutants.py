@@ -79,6 +79,7 @@ def _favor_pins():
         ("error falls with m", PF.test_error_vs_softmax_falls_as_m_grows, ()),
         ("MC mean orthogonal", PF.test_mc_mean_matches_softmax_kernel_4sigma_orthogonal, ()),
         ("orthogonal variance", PF.test_orthogonal_variance_not_above_iid, ()),
+        ("decode steps vs brute force", PF.test_decode_steps_reproduce_brute_force_causal_rows, ()),
     ]
 
 
@@ -167,6 +168,10 @@ FAVOR_MUTANTS = {
     "causal rows: read one key early": ("while nxt < len(rows) and rows[nxt] == i:",
                                         "while nxt < len(rows) and rows[nxt] == i + 1:"),
     "bidir rows: first rows for requested": ("Qp = phi(Q[rows], W)\n    return", "Qp = phi(Q[:len(rows)], W)\n    return"),
+    "decode: output before the state update": ("S = S + np.outer(pk, v)\n    z = z + pk\n    return (pq @ S) / (pq @ z), S, z",
+                                               "out = (pq @ S) / (pq @ z)\n    S = S + np.outer(pk, v)\n    z = z + pk\n    return out, S, z"),
+    "decode: key features for the query": ("pq = phi(q[None, :], W)[0]", "pq = phi(k[None, :], W)[0]"),
+    "decode: normaliser left unchanged": ("    z = z + pk\n    return (pq @ S)", "    return (pq @ S)"),
 }
 
 FEATURE_MUTANTS = {
