@@ -37,6 +37,10 @@ L2_FLUSH_BYTES = 256 << 20
 # Kernels favor_fwd launches for the bf16 path, in launch order (stage k <-> events 2k, 2k+1).
 FWD_STAGES = ["k_key_partials", "k_state_image", "k_query_out"]
 CAUSAL_STAGES = ["k_key_logit_max", "k_key_state", "k_state_scan", "k_causal_chunk", "k_causal_prefix"]
+# Kernels favor_bwd launches (bf16 bidirectional: split-precision GEMM passes and two reductions).
+BWD_STAGES = ["gemm_phi_k", "gemm_state_partial", "reduce_state", "gemm_phi_q", "gemm_gs", "gemm_t_q", "gemm_dq",
+              "gemm_G_partial", "reduce_G", "gemm_dv", "gemm_t_k", "gemm_dk"]
+BWD_CAUSAL_STAGES = ["k_widen_q", "k_widen_k", "k_widen_v", "k_widen_do", "k_widen_w", "k_f32_head_bwd"]
 
 
 def load_peaks():
@@ -65,6 +69,28 @@ def stage_work(name, w, n_sms=148):
         return t * (2 * d + 4), 2 * m * d * t, 0
     if name == "k_key_state":          # read K, V, -|k|^2/2
         return t * (4 * d + 4), 2 * m * d * t, 2 * m * d * t
+    # Backward passes: the bytes each launch must move given the materialised hi/lo bf16
+    # intermediates (4 B per element: phi(K), phi(Q), t are m wide, [g | s] is d + 64 wide) and the
+    # tensor FLOPs of its split products (3 MMAs when both operands are split, 2 when one is exact).
+    Np = d + 64
+    if name in ("gemm_phi_k", "gemm_phi_q"):   # read K (or Q); write phi hi/lo
+        return t * (2 * d + 4 * m), 2 * m * d * t, 0
+    if name == "gemm_state_partial":           # read phi(K) hi/lo and V
+        return t * (4 * m + 2 * d), 2 * 2 * m * (d + 1) * t, 0
+    if name == "gemm_G_partial":               # read phi(Q) hi/lo and [g | s] hi/lo
+        return t * (4 * m + 4 * Np), 3 * 2 * m * (d + 1) * t, 0
+    if name in ("reduce_state", "reduce_G"):   # read the partial states, write the hi/lo images
+        return 0, 0, 0
+    if name == "gemm_gs":                      # read phi(Q) hi/lo and dO; write [g | s] hi/lo
+        return t * (4 * m + 2 * d + 4 * Np), 3 * 2 * m * (d + 1) * t, 0
+    if name == "gemm_t_q":                     # read [g | s] and phi(Q) hi/lo; write t hi/lo and sum t
+        return t * (4 * Np + 8 * m + 4), 3 * 2 * m * (d + 1) * t, 0
+    if name in ("gemm_dq", "gemm_dk"):         # read t hi/lo, x and sum t; write dx fp32
+        return t * (4 * m + 2 * d + 4 + 4 * d), 2 * 2 * m * d * t, 0
+    if name == "gemm_dv":                      # read phi(K) hi/lo; write dV fp32
+        return t * (4 * m + 4 * d), 3 * 2 * m * d * t, 0
+    if name == "gemm_t_k":                     # read V and phi(K) hi/lo; write t hi/lo and sum t
+        return t * (2 * d + 8 * m + 4), 2 * 2 * m * (d + 1) * t, 0
     if name == "k_causal_chunk":       # read Q, K, V, -|k|^2/2; write fp32 out; fp16 MMAs per token:
         # Q W^T and K W^T (2 x 2md), state term and state update (2 x 2md), scores and masked A V
         # over the 128-token tile (2 * 128 * m + 2 * 128 * d)
@@ -185,8 +211,7 @@ def run_reference(args, w):
     if rank != 0:
         return
     x = make_inputs(w)
-    W64 = round_to_bf16(api_draw(w).astype(np.float32)).astype(np.float64) if w.dtype == "bf16" else \
-        api_draw(w).astype(np.float32).astype(np.float64)
+    W64 = oracle_W(w)
     n_heads = pick_sample(w, x, W64, budget_s=max(1.0, 60.0 / max(args.steps + args.warmup, 1)))
     heads = [(i // w.H, i % w.H) for i in range(n_heads)]
     for _ in range(args.warmup):
@@ -214,6 +239,15 @@ def api_draw(w):
     from linear_attention_positive_b200 import api
 
     return api.draw_features(w.w_seed, w.m, w.d)
+
+
+def oracle_W(w):
+    """W as the oracle consumes it: the oracle's own draw, rounded to the workload's dtype (the
+    same values the kernels read; the library's draw is pinned bit-identical to it)."""
+    from oracle import features
+
+    W = features.draw_W(w.w_seed, w.m, w.d).astype(np.float32)
+    return (round_to_bf16(W) if w.dtype == "bf16" else W).astype(np.float64)
 
 
 def metric_name(w):
@@ -251,6 +285,181 @@ def job_rate(tokens_per_rank, world, job_ms, steps):
 
 # ------------------------------------------------------------------------------------ GPU arm
 
+def stage_names(w):
+    """Kernel launches of one step, in launch order (stage k <-> stage events 2k, 2k+1); the
+    backward's launches follow the forward's."""
+    if w.dtype != "bf16":
+        return ["k_f32_head"] + (["k_f32_head_bwd"] if w.backward else [])
+    names = list(CAUSAL_STAGES if w.causal else FWD_STAGES)
+    if w.backward:
+        names += BWD_CAUSAL_STAGES if w.causal else BWD_STAGES
+    return names
+
+
+def stage_roofline(name, w, ms, peaks, peak_src, n_sms, traffic_key=None):
+    nbytes, f_bf16, f_tf32 = stage_work(name, w, n_sms)
+    sec = ms * 1e-3
+    hbm_peak, tc_peak = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    t_hbm = nbytes / (hbm_peak * 1e9)
+    t_tc = f_bf16 / (tc_peak * 1e12) + f_tf32 / (tc_peak * TF32_PER_BF16 * 1e12)
+    traffic = measured_traffic(name, traffic_key or w.name)
+    if t_tc > t_hbm:
+        eq = f_bf16 + f_tf32 / TF32_PER_BF16
+        return {"kernel": name, "bound": "tensor", "achieved": eq / sec / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": (eq / sec / 1e12) / tc_peak, "traffic": traffic, "algorithmic_flops": eq,
+                "note": f"bf16-equivalent FLOPs per launch (tf32 at the nominal {TF32_PER_BF16:.3f}x rate); "
+                        f"peak {peak_src} burst bf16"}
+    return {"kernel": name, "bound": "hbm", "achieved": nbytes / sec / 1e9, "peak": hbm_peak, "unit": "GB/s",
+            "frac": (nbytes / sec / 1e9) / hbm_peak, "traffic": traffic, "algorithmic_bytes": nbytes,
+            "note": f"peak {peak_src} copy bandwidth"}
+
+
+def path_roofline(w, ms_per_step, peaks, clk, n_sm):
+    """Path-level fractions (work of the definition, not of the kernels): Q, K, V (and dO) bf16 read,
+    out (and dQ, dK, dV) fp32 written, at the measured copy bandwidth; 6 L m d FLOPs per head for the
+    forward (twice that again for the backward) at the measured bf16 rate; 2 m exponentials per
+    token per pass at 16 MUFU ex2 per clock per SM, at the SM clock sampled during the timed steps."""
+    bwd = 1 if w.backward else 0
+    path_bytes = w.tokens * ((6 * w.d + 4 * w.d) + bwd * (8 * w.d + 12 * w.d))
+    path_flops = (6 + 12 * bwd) * w.tokens * w.m * w.d
+    path_exps = (2 + 2 * bwd) * w.m * w.tokens
+    step_s = ms_per_step * 1e-3
+    sm_hz = (clk["sm_mhz"] if clk and clk.get("sm_mhz") else 1965.0) * 1e6
+    return {"hbm_bytes_per_step": path_bytes, "hbm_frac": path_bytes / step_s / (peaks["hbm_gbs"] * 1e9),
+            "tensor_flops_per_step": path_flops, "tensor_frac": path_flops / step_s / (peaks["bf16_tflops"] * 1e12),
+            "exps_per_step": path_exps, "mufu_frac": path_exps / step_s / (16 * n_sm * sm_hz),
+            "note": "hbm: bf16 inputs + fp32 outputs; tensor: 6 L m d per head forward, 12 L m d backward, "
+                    "at the measured bf16 peak; mufu: 2 m ex2 per token per pass at 16 per clock per SM"}
+
+
+class Runner:
+    """One workload resident on the device, timed step by step with CUDA events."""
+
+    def __init__(self, w, dev, api, torch, exp_poly_pct=0):
+        self.w, self.dev, self.api, self.torch = w, dev, api, torch
+        self.x = make_inputs(w)
+        Wf = api_draw(w).astype(np.float32)
+        self.tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.T = {k: torch.from_numpy(self.x[k]).to(self.tdt).to(dev) for k in self.x}
+        self.Wt = torch.from_numpy(round_to_bf16(Wf) if w.dtype == "bf16" else Wf).to(self.tdt).to(dev)
+        shape = api.make_shape(w.B, w.H, w.L, w.d, w.m, api.FAVOR_BF16 if w.dtype == "bf16" else api.FAVOR_F32)
+        self.ws = torch.empty(max(api.workspace_size(shape, w.causal, False), api.workspace_size(shape, w.causal, w.backward)),
+                              dtype=torch.uint8, device=dev)
+        self.ctx = torch.empty(api.ctx_size(shape, w.causal), dtype=torch.uint8, device=dev) if w.backward else None
+        self.out = torch.empty(self.T["Q"].shape, dtype=torch.float32, device=dev)
+        self.grads = [torch.empty(self.T["Q"].shape, dtype=torch.float32, device=dev) for _ in range(3)] \
+            if w.backward else None
+        self.stages = stage_names(w)
+        self.poly = exp_poly_pct
+        self.base_opts = api.make_opts(exp_poly_pct=exp_poly_pct)
+
+    def step(self, T=None, fwd_opts=None, bwd_opts=None):
+        api, w = self.api, self.w
+        T = T or self.T
+        api.fwd(T["Q"], T["K"], T["V"], self.Wt, causal=w.causal, out=self.out, ctx=self.ctx, workspace=self.ws,
+                opts=fwd_opts or self.base_opts)
+        if w.backward:
+            api.bwd_into(T["Q"], T["K"], T["V"], self.Wt, self.out, T["dO"], *self.grads, ctx=self.ctx,
+                         causal=w.causal, workspace=self.ws, opts=bwd_opts)
+
+    def n_fwd_stages(self):
+        return len(self.stages) - (len(BWD_CAUSAL_STAGES if self.w.causal else BWD_STAGES)
+                                   if self.w.backward and self.w.dtype == "bf16" else 0)
+
+    def time(self, steps, warmup, flush, world, dist):
+        torch, api = self.torch, self.api
+        stream = torch.cuda.current_stream()
+
+        def new_events(n):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+            for e in evs:
+                e.record()
+            return evs
+
+        for _ in range(warmup):
+            flush.zero_()
+            self.step()
+        torch.cuda.synchronize()
+        if api.sync_status() != api.FAVOR_OK:
+            raise RuntimeError(f"device status not OK after warm-up ({self.w.name})")
+        step_ev = [new_events(2) for _ in range(steps)]
+        fev = [new_events(2 * api.FAVOR_MAX_STAGES) for _ in range(steps)]
+        bev = [new_events(2 * api.FAVOR_MAX_STAGES) for _ in range(steps)]
+        fopts = [api.make_opts(exp_poly_pct=self.poly, stage_events=fev[k]) for k in range(steps)]
+        bopts = [api.make_opts(stage_events=bev[k]) for k in range(steps)]
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for k in range(steps):
+            flush.zero_()
+            step_ev[k][0].record(stream)
+            self.step(fwd_opts=fopts[k], bwd_opts=bopts[k])
+            step_ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        status = api.sync_status()
+        step_ms = [a.elapsed_time(b) for a, b in step_ev]
+        nf = self.n_fwd_stages()
+        stage_ms = {}
+        for i, name in enumerate(self.stages):
+            ev, j = (fev, i) if i < nf else (bev, i - nf)
+            key = name if name not in stage_ms else f"{name}#{i}"
+            stage_ms[key] = statistics.mean(ev[k][2 * j].elapsed_time(ev[k][2 * j + 1]) for k in range(steps))
+        return step_ms, stage_ms, status
+
+    def e2e(self, steps, flush, world, dist):
+        """Through the public API: pinned host inputs in, fp32 output (and gradients) back, every step."""
+        torch = self.torch
+        stream = torch.cuda.current_stream()
+        pin = {k: torch.from_numpy(self.x[k]).to(self.tdt).pin_memory() for k in self.x}
+        outs = [self.out] + (self.grads or [])
+        outs_h = [torch.empty(o.shape, dtype=torch.float32).pin_memory() for o in outs]
+        dT = {k: torch.empty_like(self.T[k]) for k in self.T}
+        evs = []
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        for _ in range(steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for name in dT:
+                dT[name].copy_(pin[name], non_blocking=True)
+            self.step(T=dT)
+            for o, oh in zip(outs, outs_h):
+                oh.copy_(o, non_blocking=True)
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        h2d = sum(pin[k].numel() * pin[k].element_size() for k in pin)
+        d2h = sum(oh.numel() * 4 for oh in outs_h)
+        return ms, h2d, d2h
+
+    def launches_per_step(self):
+        return len(self.stages)
+
+    def release(self):
+        for k in list(self.__dict__):
+            if k not in ("w", "stages", "api", "torch", "dev"):
+                setattr(self, k, None)
+        self.torch.cuda.empty_cache()
+
+
+def workload_summary(r, step_ms_list, stage_ms, peaks, peak_src, clk, n_sm, world):
+    w = r.w
+    ms_per_step, value = job_rate(w.tokens, world, sum(step_ms_list), len(step_ms_list))
+    rec = {"workload": w.name, "metric": metric_name(w), "ms_per_step": ms_per_step, "tokens_per_s": value,
+           "stage_ms": {k: round(v, 5) for k, v in stage_ms.items()}}
+    if w.dtype == "bf16":
+        dom = max(stage_ms, key=stage_ms.get)
+        rec["roofline"] = stage_roofline(dom.split("#")[0], w, stage_ms[dom], peaks, peak_src, n_sm)
+        rec["path_roofline"] = path_roofline(w, ms_per_step, peaks, clk, n_sm)
+    return rec
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -266,95 +475,47 @@ def run_ours(args, w):
         from datetime import timedelta
 
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-
-    x = make_inputs(w)
-    Wf = api_draw(w).astype(np.float32)
-    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    T = {k: torch.from_numpy(x[k]).to(tdt).to(dev) for k in x}
-    Wt = torch.from_numpy(round_to_bf16(Wf) if w.dtype == "bf16" else Wf).to(tdt).to(dev)
-    shape = api.make_shape(w.B, w.H, w.L, w.d, w.m, api.FAVOR_BF16 if w.dtype == "bf16" else api.FAVOR_F32)
-    stages = (CAUSAL_STAGES if w.causal else FWD_STAGES) if w.dtype == "bf16" else ["k_f32_head"]
-    n_stage = len(stages)
-    ws = torch.empty(max(api.workspace_size(shape, w.causal, False), api.workspace_size(shape, w.causal, w.backward)),
-                     dtype=torch.uint8, device=dev)
-    ctx = torch.empty(api.ctx_size(shape, w.causal), dtype=torch.uint8, device=dev) if w.backward else None
-    out = torch.empty(T["Q"].shape, dtype=torch.float32, device=dev)
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    peaks, peak_src = load_peaks()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
 
-    def new_events(n):
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        for e in evs:
-            e.record()
-        return evs
-
-    def step(opts=None):
-        api.fwd(T["Q"], T["K"], T["V"], Wt, causal=w.causal, out=out, ctx=ctx, workspace=ws, opts=opts)
-        if w.backward:
-            api.bwd(T["Q"], T["K"], T["V"], Wt, out, T["dO"], ctx=ctx, causal=w.causal, workspace=ws)
-
-    base_opts = api.make_opts(exp_poly_pct=args.exp_poly_pct)
-    for _ in range(args.warmup):
-        flush.zero_()
-        step(base_opts)
-    torch.cuda.synchronize()
-    if api.sync_status() != api.FAVOR_OK:
-        raise RuntimeError("device status not OK after warm-up")
-
-    step_ev = [new_events(2) for _ in range(args.steps)]
-    stage_ev = [new_events(2 * api.FAVOR_MAX_STAGES) for _ in range(args.steps)]
-    opts = [api.make_opts(exp_poly_pct=args.exp_poly_pct, stage_events=stage_ev[k]) for k in range(args.steps)]
-    torch.cuda.synchronize()
     clocks = ClockSampler(dev.index if dev.index is not None else local)
     clocks.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    for k in range(args.steps):
-        flush.zero_()
-        step_ev[k][0].record(stream)
-        step(opts[k])
-        step_ev[k][1].record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    status = api.sync_status()
-    step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    stage_ms = [[stage_ev[k][2 * i].elapsed_time(stage_ev[k][2 * i + 1]) for k in range(args.steps)]
-                for i in range(n_stage)]
+    r = Runner(w, dev, api, torch, args.exp_poly_pct)
+    step_ms, stage_ms, status = r.time(args.steps, args.warmup, flush, world, dist)
     job_ms = max_over_ranks([sum(step_ms)], world, dev)[0]
     ms_per_step, value = job_rate(w.tokens, world, job_ms, args.steps)
+    e2e_ms, h2d, d2h = r.e2e(args.steps, flush, world, dist)
+    e2e_ms = max_over_ranks([e2e_ms], world, dev)[0]
+    headline_stage_ms = stage_ms
+    x_head, W_head = (r.x, None)
+    launches = r.launches_per_step() * args.steps
+    r.release()
 
-    # End to end through the public API: pinned host inputs in, fp32 output back, every step.
-    pin = {k: torch.from_numpy(x[k]).to(tdt).pin_memory() for k in x}
-    out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    dT = {k: torch.empty_like(T[k]) for k in T}
-    e2e_ev = [new_events(2) for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    for k in range(args.steps):
-        flush.zero_()
-        e2e_ev[k][0].record(stream)
-        for name in dT:
-            dT[name].copy_(pin[name], non_blocking=True)
-        api.fwd(dT["Q"], dT["K"], dT["V"], Wt, causal=w.causal, out=out, ctx=ctx, workspace=ws, opts=base_opts)
-        if w.backward:
-            dq, dk, dv = api.bwd(dT["Q"], dT["K"], dT["V"], Wt, out, dT["dO"], ctx=ctx, causal=w.causal, workspace=ws)
-        out_h.copy_(out, non_blocking=True)
-        e2e_ev[k][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps], world, dev)[0]
+    # The other workloads of the method, each from its own event-timed loop (same steps / warm-up).
+    others = {}
+    if not args.headline_only:
+        for k in args.also:
+            if k == args.workload:
+                continue
+            wk = WORKLOADS[k]
+            rk = Runner(wk, dev, api, torch, args.exp_poly_pct)
+            sm, stg, st_k = rk.time(args.steps, args.warmup, flush, world, dist)
+            sm_job = max_over_ranks([sum(sm)], world, dev)[0]
+            rec = workload_summary(rk, [sm_job / args.steps] * args.steps, stg, peaks, peak_src, None, n_sm, world)
+            rec["device_status"] = api.status_string(st_k)
+            others[str(k)] = rec
+            rk.release()
+    clk = clocks.stop()
+    for k, rec in others.items():  # MUFU fractions at the clock sampled over all timed loops
+        if "path_roofline" in rec:
+            rec["path_roofline"] = path_roofline(WORKLOADS[int(k)], rec["ms_per_step"], peaks, clk, n_sm)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
-    h2d = sum(pin[k].numel() * pin[k].element_size() for k in pin)
-    d2h = out_h.numel() * 4
 
-    peaks, peak_src = load_peaks()
     line = {
         "metric": metric_name(w), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -362,55 +523,24 @@ def run_ours(args, w):
         "config": workload_config(w, world),
         "e2e": {"value": job_rate(w.tokens, world, e2e_ms, 1)[1], "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (n_stage + (1 if w.causal else 0)) * args.steps if w.dtype == "bf16" else args.steps,
+        "gpu_launches": launches,
         "device_status": api.status_string(status),
     }
-    if w.dtype == "bf16" and not w.backward:
-        avg = {stages[i]: statistics.mean(stage_ms[i]) for i in range(n_stage)}
-        line["stage_ms"] = {k: round(v, 5) for k, v in avg.items()}
-        dom = max(avg, key=avg.get)
-        nbytes, f_bf16, f_tf32 = stage_work(dom, w, torch.cuda.get_device_properties(dev).multi_processor_count)
-        sec = avg[dom] * 1e-3
-        hbm_peak = peaks["hbm_gbs"]
-        tc_peak = peaks["bf16_tflops"]
-        t_hbm = nbytes / (hbm_peak * 1e9)
-        t_tc = f_bf16 / (tc_peak * 1e12) + f_tf32 / (tc_peak * TF32_PER_BF16 * 1e12)
-        if t_tc > t_hbm:
-            eq = f_bf16 + f_tf32 / TF32_PER_BF16
-            line["roofline"] = {"kernel": dom, "bound": "tensor", "achieved": eq / sec / 1e12, "peak": tc_peak,
-                                "unit": "TFLOP/s", "frac": (eq / sec / 1e12) / tc_peak,
-                                "traffic": measured_traffic(dom, w.name),
-                                "note": f"bf16-equivalent FLOPs (tf32 counted at the nominal {TF32_PER_BF16:.3f}x rate); "
-                                        f"peak {peak_src} burst bf16"}
-        else:
-            line["roofline"] = {"kernel": dom, "bound": "hbm", "achieved": nbytes / sec / 1e9, "peak": hbm_peak,
-                                "unit": "GB/s", "frac": (nbytes / sec / 1e9) / hbm_peak,
-                                "traffic": measured_traffic(dom, w.name), "note": f"peak {peak_src} copy bandwidth"}
-        # Path-level fractions (work of the definition, not of the kernels): Q, K, V, O bytes at the
-        # measured copy bandwidth; 6 L m d FLOPs per head at the measured bf16 rate; 2 m exponentials
-        # per token at 16 MUFU ex2 per clock per SM, at the SM clock sampled during the timed steps.
-        path_bytes = w.tokens * (6 * w.d + 4 * w.d)
-        step_s = ms_per_step * 1e-3
-        path_flops = 6 * w.tokens * w.m * w.d
-        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
-        sm_hz = (clk["sm_mhz"] if clk and clk.get("sm_mhz") else 1965.0) * 1e6
-        path_exps = 2 * w.m * w.tokens
-        line["path_roofline"] = {"hbm_bytes_per_step": path_bytes,
-                                 "hbm_frac": path_bytes / step_s / (hbm_peak * 1e9),
-                                 "tensor_flops_per_step": path_flops,
-                                 "tensor_frac": path_flops / step_s / (tc_peak * 1e12),
-                                 "exps_per_step": path_exps,
-                                 "mufu_frac": path_exps / step_s / (16 * n_sm * sm_hz),
-                                 "note": "hbm: Q, K, V bf16 + O fp32; tensor: 6 L m d per head at the measured "
-                                         "bf16 peak; mufu: 2 m ex2 per token at 16 per clock per SM"}
+    if w.dtype == "bf16":
+        line["stage_ms"] = {k: round(v, 5) for k, v in headline_stage_ms.items()}
+        dom = max(headline_stage_ms, key=headline_stage_ms.get)
+        line["roofline"] = stage_roofline(dom.split("#")[0], w, headline_stage_ms[dom], peaks, peak_src, n_sm)
+        line["path_roofline"] = path_roofline(w, ms_per_step, peaks, clk, n_sm)
     if clk is not None:
         line["clocks"] = clk
+    if others:
+        line["workloads"] = others
     if world == 1 and not args.no_cpu_baseline:
         try:
-            W64 = (round_to_bf16(Wf) if w.dtype == "bf16" else Wf).astype(np.float64)
-            n_heads = pick_sample(w, x, W64, budget_s=15.0)
+            W64 = oracle_W(w)
+            n_heads = pick_sample(w, x_head, W64, budget_s=15.0)
             t0 = time.perf_counter()
-            toks = oracle_sample(w, x, W64, [(i // w.H, i % w.H) for i in range(n_heads)])
+            toks = oracle_sample(w, x_head, W64, [(i // w.H, i % w.H) for i in range(n_heads)])
             sec = time.perf_counter() - t0
             line["cpu_baseline"] = {"value": toks / sec, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
                                     "sample": f"{n_heads} of {w.B * w.H} heads (L={w.L}), fp64 numpy oracle"}
@@ -430,9 +560,14 @@ def main():
                     help="percent of feature exponentials on the FMA-pipe polynomial (0: library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle sample after the timed region (for profiler runs)")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only --workload (not the other workloads reported under 'workloads')")
+    ap.add_argument("--also", default="3,4,5",
+                    help="comma-separated workloads timed after the headline and reported under 'workloads'")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    args.also = [int(v) for v in args.also.split(",") if v.strip()]
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)

@@ -26,7 +26,9 @@
  *     void*; NULL is the legacy default stream). Argument errors are reported before any launch.
  *     Device-side conditions (a bounded wait that ran out) are recorded in a device status word
  *     read by favor_sync_status().
- *   - No call allocates device memory: scratch comes from the caller's workspace.
+ *   - No call allocates device memory. favor_fwd and favor_bwd take their scratch from the
+ *     caller's workspace; favor_fwd_static_scratch takes it from the library's own fixed array
+ *     (FAVOR_STATIC_SCRATCH_BYTES, a __device__ variable every GPU that loads the library holds).
  *   - Nothing aborts, throws or prints; every call returns a favor_status.
  */
 #ifndef FAVOR_H
@@ -67,7 +69,7 @@ typedef struct {
 } favor_shape;
 
 /* Most kernel launches one call makes (the length of a stage_events array is 2x this). */
-#define FAVOR_MAX_STAGES 8
+#define FAVOR_MAX_STAGES 16
 
 /* Tuning knobs; pass NULL for defaults. Zero fields take their defaults too.
  *   split_tiles : 128-token tiles per causal segment (the unit of the causal key-side reduction
@@ -131,8 +133,11 @@ FAVOR_API size_t favor_ctx_size(const favor_shape *shape, int causal);
  *   ctx          : device, favor_ctx_size bytes, or NULL when no backward will follow
  *   workspace    : device, >= favor_workspace_size(shape, causal, 0, opts) bytes, 256-B aligned
  *   stream       : cudaStream_t as void*
- * Numerics: features are stabilised by a per-row max for queries and the per-(batch, head)
- * max over keys; both cancel exactly in D^-1. Inputs Q, K, V, W, out must be 16-byte aligned.
+ * Numerics: query features are stabilised by their row maximum. Key features, bidirectional: each
+ * persistent CTA keeps a per-feature stabiliser over its run of key tiles, and the runs are brought
+ * to one per-(batch, head) reference before the state is used; causal: the per-(batch, head)
+ * maximum key logit. All of them cancel exactly in D^-1. Inputs Q, K, V, W, out must be 16-byte
+ * aligned.
  */
 FAVOR_API favor_status favor_fwd(const favor_shape *shape, const void *Q, const void *K, const void *V,
                        const void *W, int causal, float *out, void *ctx, void *workspace,
@@ -164,8 +169,54 @@ FAVOR_API favor_status favor_bwd(const favor_shape *shape, const void *Q, const 
  */
 FAVOR_API favor_status favor_sync_status(void *stream);
 
+/*
+ * favor_decode_state_size -- bytes of the carried state of favor_decode_step for shape's B*H
+ * heads (shape->L is ignored here): per head (d*m + 2*m) fp32. Returns 0 for an unsupported shape
+ * (d in {64, 128}; m a multiple of 32, at most 256).
+ */
+FAVOR_API size_t favor_decode_state_size(const favor_shape *shape);
+
+/*
+ * favor_decode_step -- the masked FA-part advanced by one token per head: the prefix-sum
+ * recurrence S_t = S_{t-1} + phi(k_t) v_t^T, z_t = z_{t-1} + phi(k_t),
+ * out_t = phi(q_t)^T S_t / phi(q_t)^T z_t ("Random Features for Efficient Attention
+ * Approximation", abstract: masked self-attention; the causal form of the FA-part equations on
+ * "Fast Attention Via Positive Orthogonal Random Features", codewithpapers.app/method/favor).
+ * Feeding tokens 0..t one call at a time gives the rows of favor_fwd(..., causal = 1).
+ *
+ *   shape        : host pointer; L must be 1 (one token per head per call); B, H, d, m, dtype
+ *   q, k, v      : device, [B,H,d] in shape->dtype (this token's query, key and value)
+ *   W            : device, [m,d] in shape->dtype
+ *   state        : device, favor_decode_state_size(shape) bytes, read and updated in place. Per
+ *                  head (b*H + h): S'[c][r] (d x m), z'[r] (m), D[r] (m), fp32, with
+ *                  sum_j exp(u_r(k_j)) v_j[c] = exp(D[r]) S'[c][r] and
+ *                  sum_j exp(u_r(k_j)) = exp(D[r]) z'[r], u_r(x) = w_r.x - |x|^2/2. An all-zero
+ *                  buffer is the empty state (a feature with z'[r] = 0 holds no token).
+ *   out          : device, fp32 [B,H,d]; fully written
+ *   stream       : cudaStream_t as void*
+ * All pointers 16-byte aligned. Arithmetic is fp32 for either dtype. Returns FAVOR_ERR_INVALID_ARG
+ * (null or misaligned pointer, L != 1), FAVOR_ERR_UNSUPPORTED (d not 64/128, m not a multiple of
+ * 32 up to 256), FAVOR_ERR_CUDA (launch failure).
+ */
+FAVOR_API favor_status favor_decode_step(const favor_shape *shape, const void *q, const void *k, const void *v,
+                                         const void *W, float *state, float *out, void *stream);
+
 /* favor_status_string -- static, never-NULL description of a status code. */
 FAVOR_API const char *favor_status_string(favor_status status);
+
+/*
+ * favor_selftest_bounded_wait -- exercises the bounded device-side wait every kernel uses (the
+ * pages have no counterpart: this is a diagnostic of the library's failure reporting). One CTA
+ * waits on a shared-memory barrier that nothing arrives on, through the same bounded wait, with a
+ * limit of limit_us microseconds; the wait gives up, records FAVOR_ERR_TIMEOUT in the device status
+ * word, the CTA frees its tensor memory and returns. No copy or MMA is in flight, the context stays
+ * usable, and the next favor_sync_status(stream) returns FAVOR_ERR_TIMEOUT (and clears it).
+ *
+ *   limit_us : 1 .. 1000000
+ *   stream   : cudaStream_t as void*
+ * Returns FAVOR_ERR_INVALID_ARG for a limit outside that range, FAVOR_ERR_CUDA if the launch fails.
+ */
+FAVOR_API favor_status favor_selftest_bounded_wait(unsigned int limit_us, void *stream);
 
 /* Size of the library's own fixed scratch array used by favor_fwd_static_scratch (32 MiB). */
 #define FAVOR_STATIC_SCRATCH_BYTES (32u << 20)
@@ -192,7 +243,9 @@ FAVOR_API const char *favor_status_string(favor_status status);
  * with cudaGetSymbolAddress; make that first call before any stream capture. Every call on a
  * device shares the one array: calls that overlap on the GPU (different streams, no ordering
  * between them) race on it. No part of the array has to start at zero; each call overwrites
- * everything it reads. Calls no cudaMalloc, cudaFree or allocating library routine.
+ * everything it reads. Calls no cudaMalloc, cudaFree or allocating library routine. The device
+ * address is cached per device for the life of the process: a cudaDeviceReset between calls is not
+ * supported.
  */
 FAVOR_API favor_status favor_fwd_static_scratch(const favor_shape *shape, const void *Q, const void *K,
                                                 const void *V, const void *W, float *out, void *stream);

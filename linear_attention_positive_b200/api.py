@@ -31,6 +31,9 @@ EXPORTS = (
     "favor_bwd",
     "favor_sync_status",
     "favor_status_string",
+    "favor_decode_state_size",
+    "favor_decode_step",
+    "favor_selftest_bounded_wait",
     "favor_fwd_static_scratch",
 )
 
@@ -47,7 +50,7 @@ class Shape(ctypes.Structure):
                 ("m", ctypes.c_int), ("dtype", ctypes.c_int)]
 
 
-FAVOR_MAX_STAGES = 8
+FAVOR_MAX_STAGES = 16
 
 
 class Opts(ctypes.Structure):
@@ -82,6 +85,12 @@ def library():
     lib.favor_sync_status.restype = I
     lib.favor_status_string.argtypes = [I]
     lib.favor_status_string.restype = ctypes.c_char_p
+    lib.favor_decode_state_size.argtypes = [SP]
+    lib.favor_decode_state_size.restype = Z
+    lib.favor_decode_step.argtypes = [SP, P, P, P, P, P, P, P]
+    lib.favor_decode_step.restype = I
+    lib.favor_selftest_bounded_wait.argtypes = [ctypes.c_uint, P]
+    lib.favor_selftest_bounded_wait.restype = I
     lib.favor_fwd_static_scratch.argtypes = [SP, P, P, P, P, P, P]
     lib.favor_fwd_static_scratch.restype = I
     _LIB = lib
@@ -213,9 +222,57 @@ def bwd(Q, K, V, W, out, dout, ctx=None, causal=False, workspace=None, opts=None
     return dQ, dK, dV
 
 
+def bwd_into(Q, K, V, W, out, dout, dQ, dK, dV, ctx=None, causal=False, workspace=None, opts=None, stream=None):
+    """favor_bwd writing into caller-provided fp32 gradient tensors (no allocation when a workspace
+    is given)."""
+    _check_inputs((Q, K, V, W, dout), Q)
+    shape = _shape_of(Q, W)
+    if workspace is None:
+        ws_n = workspace_size(shape, causal, True, opts)
+        if ws_n == 0:
+            raise FavorError(FAVOR_ERR_UNSUPPORTED, "favor_workspace_size")
+        workspace = _alloc_bytes(ws_n, Q.device)
+    st = library().favor_bwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(W), _ptr(out), _ptr(dout),
+                             _ptr(ctx), int(causal), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(workspace),
+                             workspace.numel(), ctypes.byref(opts) if opts is not None else None,
+                             _stream_ptr(stream))
+    _check(st, "favor_bwd")
+    return dQ, dK, dV
+
+
 def sync_status(stream=None):
     """Synchronise the stream and return (and clear) the device status word."""
     return library().favor_sync_status(_stream_ptr(stream))
+
+
+def decode_state(B, H, d, m, device):
+    """A zero (empty) carried state for favor_decode_step."""
+    torch = _torch()
+    n = library().favor_decode_state_size(ctypes.byref(make_shape(B, H, 1, d, m, FAVOR_F32)))
+    if n == 0:
+        raise FavorError(FAVOR_ERR_UNSUPPORTED, "favor_decode_state_size")
+    return torch.zeros(n // 4, dtype=torch.float32, device=device)
+
+
+def decode_step(q, k, v, W, state, out=None, stream=None):
+    """One token per head through favor_decode_step. q, k, v: [B,H,d] (bf16 or fp32); state from
+    decode_state(), updated in place. Returns the fp32 output [B,H,d]."""
+    torch = _torch()
+    _check_inputs((q, k, v, W), q)
+    B, H, d = q.shape
+    shape = make_shape(B, H, 1, d, W.shape[0], _dtype_code(q))
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    st = library().favor_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(state),
+                                     _ptr(out), _stream_ptr(stream))
+    _check(st, "favor_decode_step")
+    return out
+
+
+def selftest_bounded_wait(limit_us, stream=None):
+    """Launches the library's bounded-wait self-test (a wait that nothing ends, given up after
+    limit_us); the next sync_status() reports FAVOR_ERR_TIMEOUT."""
+    _check(library().favor_selftest_bounded_wait(int(limit_us), _stream_ptr(stream)), "favor_selftest_bounded_wait")
 
 
 STATIC_SCRATCH_BYTES = 32 << 20

@@ -68,9 +68,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Returns false (after recording
-// FAVOR_ERR_TIMEOUT and raising *abort) if it does not complete within the limit, or at once if
+// FAVOR_ERR_TIMEOUT and raising *abort) if it does not complete within limit_ns, or at once if
 // *abort is already raised by another warp of the CTA.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                              unsigned long long limit_ns) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
@@ -78,13 +79,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (mbar_try_wait(a, parity)) return true;
         if ((it & 63u) == 0) {
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 record_status(FAVOR_ERR_TIMEOUT);
                 *abort = 1;
                 return false;
             }
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
 // mbar_wait for all lanes of a converged warp, with a warp-uniform result.

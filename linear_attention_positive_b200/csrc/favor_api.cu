@@ -18,6 +18,9 @@
 #include "k_keys_bidir.cu"
 #include "k_query.cu"
 #include "k_causal.cu"
+#include "k_gemm.cu"
+#include "k_selftest.cu"
+#include "k_decode.cu"
 
 namespace favor {
 namespace {
@@ -140,8 +143,61 @@ size_t bf16_bwd_bytes(const favor_shape *s) {
            align256(f32_workspace_floats(s->B * s->H, s->L, s->d, s->m) * 4);
 }
 
-size_t ctx_bytes(const favor_shape *s) {
-    return align256((size_t)s->B * s->H * state_floats(s->m, s->d) * 4) + align256((size_t)s->B * s->H * s->L * 4);
+// Forward-to-backward context: per-head state blocks (the bidirectional fp16 state image, or the
+// causal path's state), the causal per-key -|k|^2/2, and the per-head key reference C (log2
+// units) the bidirectional backward's key features are taken against.
+struct CtxLayout {
+    size_t off_state, off_bias, off_kref, total;
+};
+
+CtxLayout ctx_layout(const favor_shape *s) {
+    CtxLayout c{};
+    const size_t BH = (size_t)s->B * s->H;
+    c.off_state = 0;
+    c.off_bias = align256(BH * state_floats(s->m, s->d) * 4);
+    c.off_kref = c.off_bias + align256(BH * s->L * 4);
+    c.total = c.off_kref + align256(BH * 4);
+    return c;
+}
+
+size_t ctx_bytes(const favor_shape *s) { return ctx_layout(s).total; }
+
+// bf16 bidirectional backward: hi/lo bf16 intermediates of the split-precision GEMM passes.
+struct BwdLayout {
+    int BH, Np, n_split, kt_split;
+    size_t off_phk_hi, off_phk_lo, off_phq_hi, off_phq_lo, off_gs_hi, off_gs_lo, off_t_hi, off_t_lo, off_rowsum,
+        off_part, off_sz_hi, off_sz_lo, off_g_hi, off_g_lo, total;
+};
+
+BwdLayout bwd_layout(const favor_shape *s) {
+    BwdLayout l{};
+    l.BH = s->B * s->H;
+    l.Np = s->d + 64;
+    // split the token reduction of the state sums over enough CTAs to fill the GPU about twice
+    const int kt_total = (s->L + kGemmBK - 1) / kGemmBK;
+    const int tiles = l.BH * (s->m / 128);
+    int ns = std::max(1, std::min(kt_total, (2 * num_sms() + tiles - 1) / tiles));
+    l.kt_split = (kt_total + ns - 1) / ns;
+    l.n_split = (kt_total + l.kt_split - 1) / l.kt_split;
+    const size_t tok = (size_t)l.BH * s->L;
+    const size_t feat = align256(tok * s->m * 2), gsz = align256(tok * l.Np * 2), img = align256((size_t)l.BH * l.Np * s->m * 2);
+    size_t off = 0;
+    l.off_phk_hi = off; off += feat;
+    l.off_phk_lo = off; off += feat;
+    l.off_phq_hi = off; off += feat;
+    l.off_phq_lo = off; off += feat;
+    l.off_gs_hi = off; off += gsz;
+    l.off_gs_lo = off; off += gsz;
+    l.off_t_hi = off; off += feat;
+    l.off_t_lo = off; off += feat;
+    l.off_rowsum = off; off += align256(tok * 4);
+    l.off_part = off; off += align256((size_t)l.BH * l.n_split * s->m * l.Np * 4);
+    l.off_sz_hi = off; off += img;
+    l.off_sz_lo = off; off += img;
+    l.off_g_hi = off; off += img;
+    l.off_g_lo = off; off += img;
+    l.total = off;
+    return l;
 }
 
 // ------------------------------------------------------------------------------ tensor maps
@@ -203,6 +259,20 @@ bool make_out_map(CUtensorMap *map, void *base, int BH, int L, int d) {
            CUDA_SUCCESS;
 }
 
+// bf16 [batch][outer][inner] tensor as a 3-D map (inner, outer, batch) with 64 x box_outer x 1
+// boxes, 128-byte swizzle; coordinates past the tensor read as zeros.
+bool make_map3(CUtensorMap *map, const void *base, int inner, int outer, int batch, int box_outer) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)outer, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * outer * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_outer, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 favor_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA; }
 
 // Records the caller's timing event (2k before / 2k+1 after launch k), if one was supplied.
@@ -227,6 +297,7 @@ favor_status fwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, 
     float *amax = (float *)(ws + l.off_amax);
     float *Dmax = (float *)(ws + l.off_Dmax);
     uint8_t *state = ctx ? (uint8_t *)ctx : ws + l.off_state;
+    float *kref = ctx ? (float *)((uint8_t *)ctx + ctx_layout(s).off_kref) : nullptr;
     const size_t stride = state_floats(s->m, s->d) * 4;
 
     KeyStateParams2 ks{s->L, s->m, l.f, part, partD, amax, Dmax};
@@ -234,7 +305,7 @@ favor_status fwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, 
     cudaError_t e = launch_key_partials(mK64, mV64, mW, ks, s->d, opt_poly_pct(o), st);
     record_stage(o, 1, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-    ImageParams ip{s->m, s->d, l.f, part, partD, amax, Dmax, state, stride};
+    ImageParams ip{s->m, s->d, l.f, part, partD, amax, Dmax, state, stride, kref};
     record_stage(o, 2, st);
     e = launch_state_image(ip, l.BH, st);
     record_stage(o, 3, st);
@@ -257,8 +328,7 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
         !make_w_map(&mW128, W, s->m, s->d, 128))
         return FAVOR_ERR_CUDA;
     // Per-key -|k|^2/2 goes straight into the context (after the state blocks) when one is kept.
-    float *bias = ctx ? (float *)((uint8_t *)ctx + align256((size_t)l.BH * state_floats(s->m, s->d) * 4))
-                      : (float *)(ws + l.off_bias);
+    float *bias = ctx ? (float *)((uint8_t *)ctx + ctx_layout(s).off_bias) : (float *)(ws + l.off_bias);
     float *split_max = (float *)(ws + l.off_split_max);
     float *head_max = (float *)(ws + l.off_head_max);
     float *part_S = (float *)(ws + l.off_part_S);
@@ -271,8 +341,9 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     cudaError_t e = launch_key_logit_max(mK, mW, km, l.BH, st);
     record_stage(o, 1, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    float *kref = ctx ? (float *)((uint8_t *)ctx + ctx_layout(s).off_kref) : nullptr;
     KeyStateParams ks{s->L, s->d, s->m, l.n_split, l.tiles_per_split, (const uint16_t *)V, bias, split_max,
-                      part_S, part_z, head_max};
+                      part_S, part_z, head_max, kref};
     record_stage(o, 2, st);
     e = launch_key_state(mK, mW, ks, l.BH, st);
     record_stage(o, 3, st);
@@ -299,6 +370,157 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------- bf16 backward
+
+// Bidirectional bf16 backward (W fixed) as split-precision GEMM passes. With
+// phi(k) = 2^(u(k) log2e - C) (C: the head's key reference from the forward's context) and
+// phi(q) = exp(W q - rowmax) (a per-row constant that cancels):
+//   [S | z] = phi(K)^T [V | 1]                      (state, reduced over tokens)
+//   [num | den] = phi(Q) [S | z] -> g = dO/den, s = -(dO . num/den)/den
+//   dphi(Q) = [g | s] [S | z]^T, t = phi(Q) * dphi(Q), dQ = t W - Q rowsum(t)
+//   [G | h] = phi(Q)^T [g | s]                      (reduced over tokens)
+//   dV = phi(K) G,  dphi(K) = [V | 1] [G | h]^T, t = phi(K) * dphi(K), dK = t W - K rowsum(t)
+// Every constant factor cancels (C between [S | z] and [G | h], the row maxima between [num | den]
+// and [g | s]), so no rescaling is needed.
+favor_status bwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W,
+                            const void *dout, const void *ctx, float *dQ, float *dK, float *dV, uint8_t *ws,
+                            size_t ws_bytes, const favor_opts *o, cudaStream_t st) {
+    const BwdLayout l = bwd_layout(s);
+    if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
+    const int BH = l.BH, L = s->L, d = s->d, m = s->m, Np = l.Np;
+    auto at = [&](size_t off) { return (uint16_t *)(ws + off); };
+    uint16_t *phk_hi = at(l.off_phk_hi), *phk_lo = at(l.off_phk_lo), *phq_hi = at(l.off_phq_hi),
+             *phq_lo = at(l.off_phq_lo), *gs_hi = at(l.off_gs_hi), *gs_lo = at(l.off_gs_lo), *t_hi = at(l.off_t_hi),
+             *t_lo = at(l.off_t_lo), *sz_hi = at(l.off_sz_hi), *sz_lo = at(l.off_sz_lo), *g_hi = at(l.off_g_hi),
+             *g_lo = at(l.off_g_lo);
+    float *rowsum = (float *)(ws + l.off_rowsum), *part = (float *)(ws + l.off_part);
+    const float *kref = (const float *)((const uint8_t *)ctx + ctx_layout(s).off_kref);
+
+    // token-major operands (box rows 128 for K-major A, 64 for the other reads)
+    CUtensorMap mK, mQ, mV, mW_k, mW_n, mPhk[2], mPhkT[2], mPhq[2], mPhqT[2], mGs[2], mGsT[2], mT[2], mSzK[2],
+        mSzN[2], mGK[2], mGN[2];
+    bool ok = make_map3(&mK, K, d, L, BH, 128) && make_map3(&mQ, Q, d, L, BH, 128) && make_map3(&mV, V, d, L, BH, 128) &&
+              make_map3(&mW_k, W, d, m, 1, m) && make_map3(&mW_n, W, d, m, 1, 64);
+    uint16_t *phk[2] = {phk_hi, phk_lo}, *phq[2] = {phq_hi, phq_lo}, *gs[2] = {gs_hi, gs_lo}, *tt[2] = {t_hi, t_lo},
+             *sz[2] = {sz_hi, sz_lo}, *gi[2] = {g_hi, g_lo};
+    CUtensorMap mVn;
+    ok = ok && make_map3(&mVn, V, d, L, BH, 64);
+    for (int i = 0; ok && i < 2; ++i)
+        ok = make_map3(&mPhk[i], phk[i], m, L, BH, 128) && make_map3(&mPhkT[i], phk[i], m, L, BH, 64) &&
+             make_map3(&mPhq[i], phq[i], m, L, BH, 128) && make_map3(&mPhqT[i], phq[i], m, L, BH, 64) &&
+             make_map3(&mGs[i], gs[i], Np, L, BH, 128) && make_map3(&mGsT[i], gs[i], Np, L, BH, 64) &&
+             make_map3(&mT[i], tt[i], m, L, BH, 128) && make_map3(&mSzK[i], sz[i], m, Np, BH, Np) &&
+             make_map3(&mSzN[i], sz[i], m, Np, BH, 64) && make_map3(&mGK[i], gi[i], m, Np, BH, d) &&
+             make_map3(&mGN[i], gi[i], m, Np, BH, 64);
+    if (!ok) return FAVOR_ERR_CUDA;
+
+    int stage = 0;
+    cudaError_t e = cudaSuccess;
+    auto run = [&](auto launch) {
+        if (e != cudaSuccess) return;
+        record_stage(o, 2 * stage, st);
+        e = launch();
+        record_stage(o, 2 * stage + 1, st);
+        ++stage;
+    };
+    auto args = [&](int M, int N, int Kd) {
+        GemmArgs a{};
+        a.M = M;
+        a.N = N;
+        a.K = Kd;
+        a.n_split = 1;
+        a.kt_split = (Kd + kGemmBK - 1) / kGemmBK;
+        a.a_batched = a.b_batched = 1;
+        return a;
+    };
+    // 1. phi(K)
+    GemmArgs a1 = args(L, m, d);
+    a1.b_batched = 0;
+    a1.ld_out = m;
+    a1.out_hi = phk_hi;
+    a1.out_lo = phk_lo;
+    a1.kc = kref;
+    run([&] { return launch_gemm_t<false, false, false, false, kEpiPhiKey>(mK, mK, mW_k, mW_k, a1, m, BH, st); });
+    // 2. [S | z] partial sums over token splits, 3. reduced to the hi/lo image [Np][m]
+    GemmArgs a2 = args(m, Np, L);
+    a2.n_split = l.n_split;
+    a2.kt_split = l.kt_split;
+    a2.b_ones = 1;
+    a2.ld_out = Np;
+    a2.out_f32 = part;
+    run([&] { return launch_gemm_t<true, true, true, false, kEpiPartial>(mPhkT[0], mPhkT[1], mVn, mVn, a2, Np, BH, st); });
+    run([&] { return launch_reduce_image(part, l.n_split, m, Np, sz_hi, sz_lo, BH, st); });
+    // 4. phi(Q)
+    GemmArgs a4 = args(L, m, d);
+    a4.b_batched = 0;
+    a4.ld_out = m;
+    a4.out_hi = phq_hi;
+    a4.out_lo = phq_lo;
+    run([&] { return launch_gemm_t<false, false, false, false, kEpiPhiQuery>(mQ, mQ, mW_k, mW_k, a4, m, BH, st); });
+    // 5. [num | den] -> [g | s]
+    GemmArgs a5 = args(L, Np, m);
+    a5.ld_out = Np;
+    a5.out_hi = gs_hi;
+    a5.out_lo = gs_lo;
+    a5.side_hi = (const uint16_t *)dout;
+    a5.ld_side = d;
+    a5.d = d;
+    run([&] { return launch_gemm_t<false, false, true, true, kEpiGS>(mPhq[0], mPhq[1], mSzK[0], mSzK[1], a5, Np, BH, st); });
+    // 6. dphi(Q) -> t = phi(Q) * dphi(Q) and its row sums
+    GemmArgs a6 = args(L, m, Np);
+    a6.ld_out = m;
+    a6.out_hi = t_hi;
+    a6.out_lo = t_lo;
+    a6.rowsum = rowsum;
+    a6.side_hi = phq_hi;
+    a6.side_lo = phq_lo;
+    a6.ld_side = m;
+    run([&] { return launch_gemm_t<false, true, true, true, kEpiT>(mGs[0], mGs[1], mSzN[0], mSzN[1], a6, m, BH, st); });
+    // 7. dQ = t W - Q rowsum(t)
+    GemmArgs a7 = args(L, d, m);
+    a7.b_batched = 0;
+    a7.ld_out = d;
+    a7.out_f32 = dQ;
+    a7.rowsum = rowsum;
+    a7.side_hi = (const uint16_t *)Q;
+    a7.ld_side = d;
+    run([&] { return launch_gemm_t<false, true, true, false, kEpiDX>(mT[0], mT[1], mW_n, mW_n, a7, d, BH, st); });
+    // 8. [G | h] partial sums over token splits, 9. reduced to the hi/lo image [Np][m]
+    GemmArgs a8 = args(m, Np, L);
+    a8.n_split = l.n_split;
+    a8.kt_split = l.kt_split;
+    a8.ld_out = Np;
+    a8.out_f32 = part;
+    run([&] { return launch_gemm_t<true, true, true, true, kEpiPartial>(mPhqT[0], mPhqT[1], mGsT[0], mGsT[1], a8, Np, BH, st); });
+    run([&] { return launch_reduce_image(part, l.n_split, m, Np, g_hi, g_lo, BH, st); });
+    // 10. dV = phi(K) G
+    GemmArgs a10 = args(L, d, m);
+    a10.ld_out = d;
+    a10.out_f32 = dV;
+    run([&] { return launch_gemm_t<false, false, true, true, kEpiF32>(mPhk[0], mPhk[1], mGK[0], mGK[1], a10, d, BH, st); });
+    // 11. dphi(K) = [V | 1] [G | h]^T -> t = phi(K) * dphi(K) and its row sums
+    GemmArgs a11 = args(L, m, Np);
+    a11.a_ones = 1;
+    a11.ld_out = m;
+    a11.out_hi = t_hi;
+    a11.out_lo = t_lo;
+    a11.rowsum = rowsum;
+    a11.side_hi = phk_hi;
+    a11.side_lo = phk_lo;
+    a11.ld_side = m;
+    run([&] { return launch_gemm_t<false, true, false, true, kEpiT>(mV, mV, mGN[0], mGN[1], a11, m, BH, st); });
+    // 12. dK = t W - K rowsum(t)
+    GemmArgs a12 = args(L, d, m);
+    a12.b_batched = 0;
+    a12.ld_out = d;
+    a12.out_f32 = dK;
+    a12.rowsum = rowsum;
+    a12.side_hi = (const uint16_t *)K;
+    a12.ld_side = d;
+    run([&] { return launch_gemm_t<false, true, true, false, kEpiDX>(mT[0], mT[1], mW_n, mW_n, a12, d, BH, st); });
+    return cuda_status(e);
+}
+
 }  // namespace
 }  // namespace favor
 
@@ -320,7 +542,7 @@ extern "C" size_t favor_workspace_size(const favor_shape *s, int causal, int bac
     if (!shape_ok(s) || (causal != 0 && causal != 1)) return 0;
     if (shape_supported(s, causal, backward) != FAVOR_OK) return 0;
     if (s->dtype == FAVOR_F32) return align256(f32_workspace_floats(s->B * s->H, s->L, s->d, s->m) * 4);
-    if (backward) return bf16_bwd_bytes(s);
+    if (backward) return causal ? bf16_bwd_bytes(s) : bwd_layout(s).total;
     if (!causal) return bidir_layout(s, true).total;
     return bf16_layout(s, o, true, causal).total;
 }
@@ -367,7 +589,11 @@ extern "C" favor_status favor_bwd(const favor_shape *s, const void *Q, const voi
     if (workspace == nullptr || ((uintptr_t)workspace & 255u) != 0) return FAVOR_ERR_WORKSPACE;
     if (ws_bytes < favor_workspace_size(s, causal, 1, o)) return FAVOR_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
-    (void)ctx;
+    if (s->dtype == FAVOR_BF16 && !causal) {
+        // the key reference of the forward's context keeps the backward's key features in range
+        if (ctx == nullptr || ((uintptr_t)ctx & 255u) != 0) return FAVOR_ERR_WORKSPACE;
+        return bwd_bf16_bidir(s, Q, K, V, W, dout, ctx, dQ, dK, dV, (uint8_t *)workspace, ws_bytes, o, st);
+    }
     if (s->dtype == FAVOR_BF16) {
         const size_t n = (size_t)s->B * s->H * s->L * s->d;
         uint8_t *ws = (uint8_t *)workspace;
@@ -402,6 +628,29 @@ extern "C" favor_status favor_sync_status(void *stream) {
         if (cudaMemcpyToSymbol(favor::g_status, &zero, sizeof(int)) != cudaSuccess) return FAVOR_ERR_CUDA;
     }
     return (favor_status)v;
+}
+
+extern "C" size_t favor_decode_state_size(const favor_shape *s) {
+    if (!shape_ok(s) || (s->d != 64 && s->d != 128) || s->m % 32 != 0 || s->m > 256) return 0;
+    return (size_t)s->B * s->H * ((size_t)s->d * s->m + 2 * (size_t)s->m) * 4;
+}
+
+extern "C" favor_status favor_decode_step(const favor_shape *s, const void *q, const void *k, const void *v,
+                                          const void *W, float *state, float *out, void *stream) {
+    if (!shape_ok(s) || s->L != 1 || q == nullptr || k == nullptr || v == nullptr || W == nullptr ||
+        state == nullptr || out == nullptr)
+        return FAVOR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(W) || !aligned16(state) || !aligned16(out))
+        return FAVOR_ERR_INVALID_ARG;
+    if ((s->d != 64 && s->d != 128) || s->m % 32 != 0 || s->m > 256 || (long long)s->B * s->H > (1ll << 31) - 1)
+        return FAVOR_ERR_UNSUPPORTED;
+    DecodeParams p{s->B * s->H, s->m, s->dtype == FAVOR_BF16 ? 1 : 0, q, k, v, W, state, out};
+    return cuda_status(launch_decode_step(p, s->d, (cudaStream_t)stream));
+}
+
+extern "C" favor_status favor_selftest_bounded_wait(unsigned int limit_us, void *stream) {
+    if (limit_us == 0 || limit_us > 1000000u) return FAVOR_ERR_INVALID_ARG;
+    return cuda_status(launch_wait_selftest(1000ull * limit_us, (cudaStream_t)stream));
 }
 
 // The no-allocation variant of the bidirectional forward (uses the definitions above).

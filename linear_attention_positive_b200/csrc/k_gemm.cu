@@ -1,0 +1,555 @@
+// Split-precision tcgen05 GEMM with fused FAVOR+ epilogues: the building block of the bf16
+// backward pass.
+//
+// The gradients of FAVOR+ are heavy-tailed (their largest entries are 50-90x their RMS), so a
+// single 16-bit rounding of any operand of the feature contractions (phi(Q), phi(K), the state
+// [S | z], the query-side sums [G | h], the products phi * dphi) already costs about 1e-2 x RMS
+// on its own. Every such operand is therefore carried as a pair of bf16 values x = hi + lo
+// (hi = bf16(x), lo = bf16(x - hi); 16 significant bits, fp32 range) and every product as
+// hi*hi + lo*hi + hi*lo: three kind::f16 MMAs with fp32 accumulation in TMEM (two when one side
+// is exact in bf16, as W, K, V and Q are). bf16 keeps fp32's exponent range, so no operand needs a
+// power-of-two range scale.
+//
+// C[M x N] = sum_k A[M x k] B[k x N] per batch (blockIdx.z = batch * n_split + split), one
+// 128 x BN output tile per CTA (BN <= 256 fp32 TMEM columns), K in 64-element tiles staged by TMA
+// (128-byte swizzle) through a ring of shared-memory stages:
+//   A K-major: [batch][M][K] rows of K (box 64 x 128); A M-major: [batch][K][M] (boxes 64 x 64)
+//   B K-major: [batch][N][K] (box 64 x BN);            B N-major: [batch][K][N] (boxes 64 x 64)
+// Optional constant blocks: a ones column appended to B (N-major, last 64 columns: column 0 = 1)
+// or to A (K-major, last 64 K columns: column 0 = 1), the [V | 1] operand of the state sums.
+// Warp roles (6 warps): 0 TMA, 1 MMA issue and TMEM allocation, 2-5 the epilogue (thread = row of
+// the tile; TMEM lane quarter = warp % 4), which for the key feature map also sums |k|^2 from the
+// A tiles while they stream through.
+
+#include "common.cuh"
+
+namespace favor {
+
+enum GemmEpi : int {
+    kEpiPhiQuery = 0,  // phi = exp(acc - rowmax) as hi/lo bf16 rows (N = m)
+    kEpiPhiKey = 1,    // phi = 2^(acc log2e - |x|^2/2 log2e - kc[batch]) as hi/lo bf16 rows (N = m)
+    kEpiGS = 2,        // [num | den | 0]: writes [g | s | 0] hi/lo, g = dO/den, s = -(dO . num/den)/den
+    kEpiT = 3,         // t = phi * acc (phi from hi/lo rows), hi/lo rows and the row sums of t
+    kEpiDX = 4,        // dx = acc - x * rowsum (x bf16 rows, rowsum fp32): fp32 rows
+    kEpiF32 = 5,       // acc as fp32 rows
+    kEpiPartial = 6,   // acc as fp32 rows of the split's partial tile [z][M][N]
+    kEpiMask = 7,      // causal mask inside the chunk (column j kept for j <= row i): hi/lo rows
+};
+
+struct GemmArgs {
+    int M, N, K;              // per batch
+    int n_split, kt_split;    // K split over CTAs: k-tiles per split
+    int a_batched, b_batched; // 0: the operand is shared by all batches (batch coordinate 0)
+    int a_ones, b_ones;       // constant ones block as the last K tile of A / last N block of B
+    // epilogue
+    int ld_out;               // row pitch (elements) of the epilogue's outputs
+    uint16_t *out_hi, *out_lo;
+    float *out_f32;
+    float *rowsum;            // [batch][M] (written by kEpiT, read by kEpiDX)
+    const uint16_t *side_hi, *side_lo;  // kEpiT: phi rows; kEpiGS / kEpiDX: dO / x rows (hi only)
+    int ld_side;
+    const float *kc;          // kEpiPhiKey: per-batch key reference (log2 units)
+    int d;                    // kEpiGS: number of value columns
+    // chunked (causal) use: the M tile is one 128-token chunk of batch blockIdx.z
+    int a_kofs;               // A's K coordinate starts at the tile's first row (A = a chunk's own rows)
+    int b_nofs, b_kofs;       // B's N (K-major) / K (N-major) coordinate starts at the tile's first row
+    int b_chunk, n_chunks;    // B's batch coordinate = batch * n_chunks + chunk (per-chunk images)
+    int b_ones_k;             // constant ones block as the last K tile of a K-major B
+    int a_mlocal;             // M-major A: M coordinate local to the chunk (0..127), not the token
+    const float *addend;      // NULL, or fp32 rows (pitch ld_add) added to the accumulator first
+    int ld_add;
+};
+
+constexpr int kGemmThreads = 192;
+constexpr int kGemmBK = 64;
+
+struct GemmSmem {
+    uint32_t a_bytes, b_bytes, stage_bytes;
+    int stages;
+};
+
+// Stage ring that fits next to the constant blocks (const_bytes) in about 196 KB.
+__host__ __device__ inline GemmSmem gemm_smem_plan(int BN, int a_parts, int b_parts, uint32_t const_bytes) {
+    GemmSmem g;
+    g.a_bytes = 128u * 128u;                      // 128 rows x 64 k x 2 B
+    g.b_bytes = (uint32_t)BN * 128u;              // BN x 64 k x 2 B
+    g.stage_bytes = a_parts * g.a_bytes + b_parts * g.b_bytes;
+    int s = (int)((196u * 1024u - const_bytes) / g.stage_bytes);
+    g.stages = s < 2 ? 2 : (s > 4 ? 4 : s);
+    return g;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float bf16_lo_f(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi_f(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// Splits 8 fp32 values into hi/lo bf16 (hi = rn(x), lo = rn(x - hi)) and stores 16 B of each.
+__device__ __forceinline__ void store_split8(uint16_t *hi, uint16_t *lo, const float *x) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        h[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+        l[i] = pack_bf16x2(x[2 * i] - bf16_lo_f(h[i]), x[2 * i + 1] - bf16_hi_f(h[i]));
+    }
+    *(uint4 *)hi = make_uint4(h[0], h[1], h[2], h[3]);
+    *(uint4 *)lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Loads 8 bf16 values (16 B) as fp32.
+__device__ __forceinline__ void load_bf16x8(const uint16_t *p, float *x) {
+    const uint4 w = *(const uint4 *)p;
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = bf16_lo_f(u[i]);
+        x[2 * i + 1] = bf16_hi_f(u[i]);
+    }
+}
+
+__host__ __device__ inline uint32_t gemm_const_bytes(const GemmArgs &p, int BN) {
+    return (p.a_ones ? 128u * 128u : 0u) + (p.b_ones_k ? (uint32_t)BN * 128u : 0u);
+}
+
+// Loads accumulator columns [c0, c0 + 32) of this thread's row and adds the addend row, if any.
+__device__ __forceinline__ void acc_row32(uint32_t t_row, int c0, const GemmArgs &p, size_t orow, int n0, bool valid,
+                                          float (&v)[32]) {
+    tmem_ld32(t_row + c0, v);
+    if (p.addend != nullptr && valid) {
+        const float4 *a = (const float4 *)(p.addend + orow * p.ld_add + n0 + c0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 x = a[j];
+            v[4 * j] += x.x;
+            v[4 * j + 1] += x.y;
+            v[4 * j + 2] += x.z;
+            v[4 * j + 3] += x.w;
+        }
+    }
+}
+
+template <bool A_MN, bool B_MN, bool A_SPLIT, bool B_SPLIT, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
+       const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mB2, GemmArgs p, int BN) {
+    constexpr int AP = A_SPLIT ? 2 : 1, BP = B_SPLIT ? 2 : 1;
+    constexpr bool NORM = EPI == kEpiPhiKey;
+    const GemmSmem plan = gemm_smem_plan(BN, AP, BP, gemm_const_bytes(p, BN));
+    const int STAGES = plan.stages;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sStage = smem;
+    uint8_t *sOnesA = sStage + (size_t)STAGES * plan.stage_bytes;  // 16 KB, used when a_ones
+    uint8_t *sOnesB = sOnesA + (p.a_ones ? 128 * 128 : 0);           // BN x 128 B, used when b_ones_k
+    uint64_t *bars = (uint64_t *)(sOnesB + (p.b_ones_k ? BN * 128 : 0));
+    uint64_t *full = bars, *empty = full + 4, *acc_full = empty + 4;
+    uint32_t *tmem_slot = (uint32_t *)(acc_full + 1);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * 128, n0 = blockIdx.y * BN;
+    const int batch = blockIdx.z / p.n_split, split = blockIdx.z % p.n_split;
+    const int kt_total = (p.K + kGemmBK - 1) / kGemmBK;
+    const int kt0 = split * p.kt_split, kt1 = min(kt0 + p.kt_split, kt_total);
+    const int nk = max(kt1 - kt0, 0);
+    const int ab = p.a_batched ? batch : 0;
+    const int bb = p.b_chunk ? batch * p.n_chunks + (int)blockIdx.x : (p.b_batched ? batch : 0);
+    const int a_k0 = p.a_kofs ? m0 : 0;           // offset of A's K coordinate
+    const int b_k0 = p.b_kofs ? m0 : 0, b_n0 = p.b_nofs ? m0 : n0;
+    const int nb_load = p.b_ones ? BN / 64 - 1 : BN / 64;  // N-major B blocks loaded by TMA
+    const int kt_ones = kt_total - 1;                      // the A ones block's K tile (a_ones)
+
+    // Constant blocks: the B ones block of every stage, the A ones block.
+    if (p.b_ones) {
+        for (int i = threadIdx.x; i < STAGES * BP * 64; i += kGemmThreads) {
+            const int s = i / (BP * 64), part = (i / 64) % BP, k = i % 64;
+            uint8_t *blk = sStage + (size_t)s * plan.stage_bytes + AP * plan.a_bytes + part * plan.b_bytes +
+                           (size_t)(BN / 64 - 1) * 8192;
+            uint4 *row = (uint4 *)(blk + k * 128);
+            for (int c = 0; c < 8; ++c) row[c] = make_uint4(0, 0, 0, 0);
+            // element (k, n = 0): chunk 0 ^ (k & 7); the lo part of a one is zero
+            if (part == 0) *(uint16_t *)(blk + k * 128 + ((k & 7) << 4)) = 0x3F80;
+        }
+    }
+    if (p.a_ones) {
+        for (int r = threadIdx.x; r < 128; r += kGemmThreads) {
+            uint4 *row = (uint4 *)(sOnesA + r * 128);
+            for (int c = 0; c < 8; ++c) row[c] = make_uint4(0, 0, 0, 0);
+            *(uint16_t *)(sOnesA + r * 128 + ((r & 7) << 4)) = 0x3F80;
+        }
+    }
+    if (p.b_ones_k) {
+        for (int r = threadIdx.x; r < BN; r += kGemmThreads) {
+            uint4 *row = (uint4 *)(sOnesB + r * 128);
+            for (int c = 0; c < 8; ++c) row[c] = make_uint4(0, 0, 0, 0);
+            *(uint16_t *)(sOnesB + r * 128 + ((r & 7) << 4)) = 0x3F80;
+        }
+    }
+    fence_async_smem();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NORM ? 5 : 1);
+        }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (elect_one()) {
+            prefetch_tensormap(&mA);
+            prefetch_tensormap(&mB);
+            if (A_SPLIT) prefetch_tensormap(&mA2);
+            if (B_SPLIT) prefetch_tensormap(&mB2);
+        }
+        __syncwarp();
+        int issued = 0;
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % STAGES, kt = kt0 + i, k0 = kt * kGemmBK;
+            if (!mbar_wait_lazy(&empty[s], ((i / STAGES) & 1) ^ 1, abort_flag)) break;
+            if (elect_one()) {
+                uint8_t *st = sStage + (size_t)s * plan.stage_bytes;
+                const bool a_const = p.a_ones && kt == kt_ones;
+                const bool b_const = p.b_ones_k && kt == kt_ones;
+                const uint32_t bytes = (a_const ? 0u : AP * plan.a_bytes) +
+                                       (b_const ? 0u : (B_MN ? BP * (uint32_t)nb_load * 8192u : BP * plan.b_bytes));
+                mbar_arrive_expect_tx(&full[s], bytes);
+                for (int part = 0; part < AP && !a_const; ++part) {
+                    const CUtensorMap *m = part ? &mA2 : &mA;
+                    uint8_t *dst = st + part * plan.a_bytes;
+                    if (A_MN) {
+                        const int am = p.a_mlocal ? 0 : m0;
+                        tma_load_3d(dst, m, &full[s], am, a_k0 + k0, ab);
+                        tma_load_3d(dst + 8192, m, &full[s], am + 64, a_k0 + k0, ab);
+                    } else {
+                        tma_load_3d(dst, m, &full[s], a_k0 + k0, m0, ab);
+                    }
+                }
+                for (int part = 0; part < BP && !b_const; ++part) {
+                    const CUtensorMap *m = part ? &mB2 : &mB;
+                    uint8_t *dst = st + AP * plan.a_bytes + part * plan.b_bytes;
+                    if (B_MN) {
+                        for (int j = 0; j < nb_load; ++j)
+                            tma_load_3d(dst + j * 8192, m, &full[s], b_n0 + 64 * j, b_k0 + k0, bb);
+                    } else {
+                        tma_load_3d(dst, m, &full[s], b_k0 + k0, b_n0, bb);
+                    }
+                }
+            }
+            __syncwarp();
+            ++issued;
+        }
+        volatile int no_abort = 0;
+        for (int i = max(issued - STAGES, 0); i < issued; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, &no_abort);
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issue
+        const uint32_t idesc = make_idesc(128, BN, kFmtBF16, A_MN ? 1u : 0u, B_MN ? 1u : 0u);
+        // K-step of 16: K-major operands advance 32 B, MN-major operands 16 rows of 128 B
+        constexpr uint32_t a_step = A_MN ? 2048 / 16 : 2, b_step = B_MN ? 2048 / 16 : 2;
+        const uint32_t a_lbo = A_MN ? 8192 : 16, b_lbo = B_MN ? 8192 : 16;
+        bool ok = true;
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % STAGES, kt = kt0 + i;
+            if (!mbar_wait_all(&full[s], (i / STAGES) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t st = smem_u32(sStage) + (uint32_t)s * plan.stage_bytes;
+            const bool a_const = p.a_ones && kt == kt_ones;
+            const bool b_const = p.b_ones_k && kt == kt_ones;
+            const uint32_t a_hi = a_const ? smem_u32(sOnesA) : st;
+            const uint32_t a_lo = st + plan.a_bytes;
+            const uint32_t b_hi = b_const ? smem_u32(sOnesB) : st + AP * plan.a_bytes, b_lo = b_hi + plan.b_bytes;
+            if (elect_one()) {
+                const uint32_t acc0 = i > 0 ? 1u : 0u;
+                mma_ss_x4(tmem, make_sdesc(a_hi, a_lbo, 1024), make_sdesc(b_hi, b_lbo, 1024), idesc, acc0, a_step, b_step);
+                if (A_SPLIT && !a_const)
+                    mma_ss_x4(tmem, make_sdesc(a_lo, a_lbo, 1024), make_sdesc(b_hi, b_lbo, 1024), idesc, 1u, a_step, b_step);
+                if (B_SPLIT && !b_const)
+                    mma_ss_x4(tmem, make_sdesc(a_hi, a_lbo, 1024), make_sdesc(b_lo, b_lbo, 1024), idesc, 1u, a_step, b_step);
+                mma_commit(&empty[s]);
+            }
+            __syncwarp();
+        }
+        if (elect_one()) mma_commit(acc_full);
+        __syncwarp();
+        (void)ok;
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int q = warp & 3;             // TMEM lane quarter
+        const int r = q * 32 + lane;        // row of the tile
+        const int row = m0 + r;             // row of the output
+        const bool valid = row < p.M;
+        const uint32_t t_row = tmem + (((uint32_t)q * 32u) << 16);
+        float sq = 0.f;                     // |x|^2 of this row (key feature map)
+        if (NORM) {
+            // A K-major: row r of each A tile, 8 chunks of 16 B; the whole K range is in this CTA
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % STAGES;
+                if (!mbar_wait_all(&full[s], (i / STAGES) & 1, abort_flag)) break;
+                const uint8_t *tile = sStage + (size_t)s * plan.stage_bytes;
+                float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    float x[8];
+                    load_bf16x8((const uint16_t *)(tile + sw128_offset(r, ch)), x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc4[e & 3] = fmaf(x[e], x[e], acc4[e & 3]);
+                }
+                sq += (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+            }
+        }
+        const bool have = nk > 0 && mbar_wait_all(acc_full, 0, abort_flag);
+        tc_fence_after();
+        const size_t orow = (size_t)batch * p.M + row;  // output row (batch-major)
+        if (have) {
+            if (EPI == kEpiPhiQuery || EPI == kEpiPhiKey) {
+                float shift;
+                if (EPI == kEpiPhiQuery) {
+                    float mx = -INFINITY;
+                    for (int c0 = 0; c0 < BN; c0 += 32) {
+                        float v[32];
+                        tmem_ld32(t_row + c0, v);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+                    }
+                    shift = mx * kLog2e;
+                } else {
+                    shift = 0.5f * sq * kLog2e + p.kc[batch];
+                }
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(t_row + c0, v);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = exp2f(fmaf(v[e], kLog2e, -shift));
+                    if (valid) {
+                        const size_t o = orow * p.ld_out + n0 + c0;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
+                    }
+                }
+            } else if (EPI == kEpiGS) {
+                // acc columns: num [0, d), den at d. Output [g | s | 0 ...] over BN columns.
+                float den = tmem_ld1(t_row + p.d);
+                if (p.addend != nullptr && valid) den += p.addend[orow * p.ld_add + p.d];
+                const float inv = 1.0f / den;
+                float dot = 0.f;
+                const uint16_t *dO = p.side_hi + orow * p.ld_side;
+                for (int c0 = 0; c0 < p.d; c0 += 32) {
+                    float v[32], g[32];
+                    acc_row32(t_row, c0, p, orow, 0, valid, v);
+                    if (valid) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) load_bf16x8(dO + c0 + 8 * j, &g[8 * j]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) g[e] = 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        dot = fmaf(g[e], v[e] * inv, dot);
+                        g[e] *= inv;
+                    }
+                    if (valid) {
+                        const size_t o = orow * p.ld_out + c0;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &g[8 * j]);
+                    }
+                }
+                if (valid) {
+                    const float s = -dot * inv;
+                    for (int c0 = p.d; c0 < BN; c0 += 8) {
+                        float z[8] = {c0 == p.d ? s : 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        store_split8(p.out_hi + orow * p.ld_out + c0, p.out_lo + orow * p.ld_out + c0, z);
+                    }
+                }
+            } else if (EPI == kEpiT) {
+                float tsum = 0.f;
+                const uint16_t *ph = p.side_hi + orow * p.ld_side + n0, *pl = p.side_lo + orow * p.ld_side + n0;
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    float v[32];
+                    acc_row32(t_row, c0, p, orow, n0, valid, v);
+                    if (valid) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            float h[8], l[8];
+                            load_bf16x8(ph + c0 + 8 * j, h);
+                            load_bf16x8(pl + c0 + 8 * j, l);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                v[8 * j + e] *= h[e] + l[e];
+                                tsum += v[8 * j + e];
+                            }
+                        }
+                        const size_t o = orow * p.ld_out + n0 + c0;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
+                    }
+                }
+                if (valid) p.rowsum[orow] = tsum;
+            } else if (EPI == kEpiDX) {
+                const float ts = valid ? p.rowsum[orow] : 0.f;
+                const uint16_t *x = p.side_hi + orow * p.ld_side + n0;
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    float v[32];
+                    acc_row32(t_row, c0, p, orow, n0, valid, v);
+                    if (valid) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            float xv[8];
+                            load_bf16x8(x + c0 + 8 * j, xv);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) v[8 * j + e] = fmaf(-xv[e], ts, v[8 * j + e]);
+                        }
+                        float4 *o = (float4 *)(p.out_f32 + orow * p.ld_out + n0 + c0);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    }
+                }
+            } else if (EPI == kEpiMask) {
+                // A chunk's 128 x 128 tile: row r is the chunk's query r, column j its key j
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(t_row + c0, v);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (c0 + e > r) v[e] = 0.f;
+                    if (valid) {
+                        const size_t o = orow * p.ld_out + c0;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
+                    }
+                }
+            } else {
+                // kEpiF32 (rows of batch) and kEpiPartial (rows of batch * n_split + split)
+                const size_t prow = EPI == kEpiPartial ? (size_t)blockIdx.z * p.M + row : orow;
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    float v[32];
+                    acc_row32(t_row, c0, p, orow, n0, valid, v);
+                    if (valid) {
+                        float4 *o = (float4 *)(p.out_f32 + prow * p.ld_out + n0 + c0);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    }
+                }
+            }
+        } else if (EPI == kEpiPartial && valid) {
+            // an empty split contributes zeros
+            for (int c0 = 0; c0 < BN; c0 += 4)
+                *(float4 *)(p.out_f32 + ((size_t)blockIdx.z * p.M + row) * p.ld_out + n0 + c0) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+// Sums the n_split partial tiles of each batch ([batch][split][M][Np] fp32, M = m features,
+// columns = values | z-or-h | zero padding) in split order and writes the hi/lo bf16 image
+// transposed: [batch][Np][m] (row n holds column n of every feature), the layout both the K-major
+// and the N-major reads of the image expect. Block (32, 8) per 64 features x 32 columns: partial
+// rows are read along n (coalesced), transposed through shared memory, written along the features.
+__global__ void __launch_bounds__(256) k_gemm_reduce_image(const float *__restrict__ part, int n_split, int m, int Np,
+                                                           uint16_t *img_hi, uint16_t *img_lo) {
+    __shared__ float tile[64][33];
+    const int batch = blockIdx.z, n_base = blockIdx.x * 32, r_base = blockIdx.y * 64;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int r = r_base + ty + 8 * j;
+        float acc = 0.f;
+        for (int s = 0; s < n_split; ++s) acc += part[(((size_t)batch * n_split + s) * m + r) * Np + n_base + tx];
+        tile[ty + 8 * j][tx] = acc;
+    }
+    __syncthreads();
+    // thread (tx, ty): columns n_base + ty + 8 i (i < 4), features r_base + 2 tx, + 1
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int nl = ty + 8 * i;
+        const float a = tile[2 * tx][nl], b = tile[2 * tx + 1][nl];
+        const uint32_t h = pack_bf16x2(a, b);
+        const uint32_t l = pack_bf16x2(a - bf16_lo_f(h), b - bf16_hi_f(h));
+        const size_t o = ((size_t)batch * Np + n_base + nl) * m + r_base + 2 * tx;
+        *(uint32_t *)(img_hi + o) = h;
+        *(uint32_t *)(img_lo + o) = l;
+    }
+}
+
+// Exclusive prefix (forward) or suffix (reverse) over the n_chunks per-chunk partial states of
+// each batch ([batch * n_chunks + c][m][Np] fp32), summed in chunk order, written as hi/lo bf16
+// images [batch * n_chunks + c][Np][m] (the layout of k_gemm_reduce_image). Block (32, 8) per
+// 64 features x 32 columns, walking the chunks.
+__global__ void __launch_bounds__(256) k_gemm_scan_image(const float *__restrict__ part, int n_chunks, int m, int Np,
+                                                         int reverse, uint16_t *img_hi, uint16_t *img_lo) {
+    __shared__ float tile[64][33];
+    const int batch = blockIdx.z, n_base = blockIdx.x * 32, r_base = blockIdx.y * 64;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < n_chunks; ++i) {
+        const int c = reverse ? n_chunks - 1 - i : i;
+        const size_t cb = (size_t)batch * n_chunks + c;
+        float val[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            tile[ty + 8 * j][tx] = acc[j];
+            val[j] = part[(cb * m + r_base + ty + 8 * j) * Np + n_base + tx];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int nl = ty + 8 * k;
+            const float a = tile[2 * tx][nl], b = tile[2 * tx + 1][nl];
+            const uint32_t h = pack_bf16x2(a, b);
+            const uint32_t l = pack_bf16x2(a - bf16_lo_f(h), b - bf16_hi_f(h));
+            const size_t o = (cb * Np + n_base + nl) * m + r_base + 2 * tx;
+            *(uint32_t *)(img_hi + o) = h;
+            *(uint32_t *)(img_lo + o) = l;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] += val[j];
+    }
+}
+
+// ------------------------------------------------------------------------------------ host side
+
+template <bool A_MN, bool B_MN, bool A_SPLIT, bool B_SPLIT, int EPI>
+static cudaError_t launch_gemm_t(const CUtensorMap &mA, const CUtensorMap &mA2, const CUtensorMap &mB,
+                                 const CUtensorMap &mB2, const GemmArgs &p, int BN, int batches, cudaStream_t st) {
+    const uint32_t cb = gemm_const_bytes(p, BN);
+    const GemmSmem plan = gemm_smem_plan(BN, A_SPLIT ? 2 : 1, B_SPLIT ? 2 : 1, cb);
+    const size_t smem = 1024 + (size_t)plan.stages * plan.stage_bytes + cb + 256;
+    auto kern = k_gemm<A_MN, B_MN, A_SPLIT, B_SPLIT, EPI>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const dim3 grid((p.M + 127) / 128, (p.N + BN - 1) / BN, batches * p.n_split);
+    kern<<<grid, kGemmThreads, smem, st>>>(mA, mA2, mB, mB2, p, BN);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan_image(const float *part, int n_chunks, int m, int Np, int reverse, uint16_t *hi, uint16_t *lo,
+                              int batches, cudaStream_t st) {
+    k_gemm_scan_image<<<dim3(Np / 32, m / 64, batches), dim3(32, 8), 0, st>>>(part, n_chunks, m, Np, reverse, hi, lo);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_image(const float *part, int n_split, int m, int Np, uint16_t *hi, uint16_t *lo, int batches,
+                                cudaStream_t st) {
+    k_gemm_reduce_image<<<dim3(Np / 32, m / 64, batches), dim3(32, 8), 0, st>>>(part, n_split, m, Np, hi, lo);
+    return cudaGetLastError();
+}
+
+}  // namespace favor

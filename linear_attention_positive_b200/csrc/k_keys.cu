@@ -197,6 +197,7 @@ struct KeyStateParams {
     float *part_S;           // [BH, n_split, m, d]
     float *part_z;           // [BH, n_split, m]
     float *head_max;         // [BH] (written by split 0)
+    float *key_ref;          // NULL, or [BH]: the same maximum in log2 units (the backward's reference)
 };
 
 template <int D>
@@ -260,6 +261,7 @@ k_key_state(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CU
         for (int s = 0; s < p.n_split; ++s) c = fmaxf(c, p.split_max[(size_t)bh * p.n_split + s]);
         *sC = c;
         if (split == 0) p.head_max[bh] = c;
+        if (split == 0 && p.key_ref != nullptr) p.key_ref[bh] = c * kLog2e;
         fence_barrier_init();
     }
     if (warp == 1) {

@@ -47,6 +47,7 @@ struct ImageParams {
     const float *part_Dmax;  // [slots][8]
     uint8_t *image;          // per head at image + bh * image_stride
     size_t image_stride;     // bytes
+    float *key_ref;          // NULL, or [BH]: the head's reference stabiliser C (log2 units)
 };
 
 constexpr int kImageThreads = 128;
@@ -63,10 +64,11 @@ __device__ __forceinline__ float pow2i(float e) {
 // 2^e exceeding the bound sum_runs max_warp amax 2^(Dmax - C) on their magnitude, and rounded to
 // fp16. Grid: (chunks / 128, heads).
 __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
-    __shared__ float sC, sScale, sStat[kImageThreads];
+    __shared__ float sC, sScale, sRed[kImageThreads / 32];
     const int bh = blockIdx.y;
     const int c_first = flat_first_cta(p.f, bh), c_last = flat_last_cta(p.f, bh);
     const int halves = p.m / 128, nhs = p.d / 64;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     // per-(run, warp) statistics, one per thread (a head spans at most a few runs)
     const int nstat = (c_last - c_first + 1) * 8;
     float dm = -INFINITY, am = 0.f;
@@ -76,12 +78,15 @@ __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
             dm = fmaxf(dm, p.part_Dmax[k]);
         }
     }
-    sStat[threadIdx.x] = dm;
+    for (int o = 16; o > 0; o >>= 1) dm = fmaxf(dm, __shfl_xor_sync(0xffffffffu, dm, o));
+    if (lane == 0) sRed[wid] = dm;
     __syncthreads();
     if (threadIdx.x == 0) {
-        float C = -INFINITY;
-        for (int i = 0; i < kImageThreads; ++i) C = fmaxf(C, sStat[i]);
+        float C = sRed[0];
+        for (int w = 1; w < kImageThreads / 32; ++w) C = fmaxf(C, sRed[w]);
         sC = C;
+        // the backward's key features 2^(u log2e - C) stay below 2^19 (every run's D_r <= C)
+        if (p.key_ref != nullptr && blockIdx.x == 0) p.key_ref[bh] = C;
     }
     __syncthreads();
     const float C = sC;
@@ -92,15 +97,15 @@ __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
         }
     // ... summed over runs: every run's warps are taken by consecutive threads (8 per run), so the
     // bound is the sum over runs of the max over that run's 8 threads' values
-    sStat[threadIdx.x] = am;
+    for (int o = 4; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    float bsum = (threadIdx.x & 7) == 0 ? am : 0.f;
+    for (int o = 16; o > 0; o >>= 1) bsum += __shfl_xor_sync(0xffffffffu, bsum, o);
+    __syncthreads();
+    if (lane == 0) sRed[wid] = bsum;
     __syncthreads();
     if (threadIdx.x == 0) {
         float bound = 0.f;
-        for (int r = 0; r < min(nstat, kImageThreads) / 8; ++r) {
-            float b = 0.f;
-            for (int w = 0; w < 8; ++w) b = fmaxf(b, sStat[r * 8 + w]);
-            bound += b;
-        }
+        for (int w = 0; w < kImageThreads / 32; ++w) bound += sRed[w];
         // runs beyond the first kImageThreads / 8 (very short heads over many CTAs) were folded by
         // the strided loop into those threads' maxima: adding them per run keeps the bound valid
         if (nstat > kImageThreads) bound *= (float)((nstat + kImageThreads - 1) / kImageThreads);
@@ -503,12 +508,17 @@ static size_t query_smem(int m) {
            (size_t)C::OUT_BUFS * C::OUT_BUF + 512 * 4 + 256;
 }
 
+// SM count of the current device (cached per device: the workspace layout and the persistent
+// grids depend on it).
 int num_sms() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
+    constexpr int kMaxDev = 64;
+    static int cached[kMaxDev] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) dev = 0;
+    int n = cached[dev];
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
     }
     return n;
 }

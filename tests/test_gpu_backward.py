@@ -1,6 +1,9 @@
 """GPU parity of the backward (dQ, dK, dV with W fixed) through the C ABI against the fp64
 oracle's chain-rule gradients (themselves pinned by finite differences). Tolerances as for the
-forward: 1e-4 * RMS on the fp32 path, 2e-2 * RMS with bf16 inputs, per gradient tensor."""
+forward: 1e-4 * RMS on the fp32 path, 2e-2 * RMS with bf16 inputs, per gradient tensor.
+
+The bf16 bidirectional backward runs the split-precision tensor-core passes and needs the
+context of a bf16 forward on the same inputs."""
 
 import numpy as np
 import pytest
@@ -54,6 +57,32 @@ def test_bf16_backward_small(cuda_device, causal):
         assert rel_max_err(g, r) <= TOL["bf16"]
 
 
+BIDIR_SHAPES = [
+    (1, 1, 1, 64, 256),      # a single token
+    (1, 1, 64, 128, 128),    # one 64-token tile, one feature tile
+    (2, 3, 1000, 64, 256),   # ragged tail, six heads
+    (1, 2, 777, 128, 256),   # d = 128, ragged
+    (2, 1, 4100, 64, 128),   # several token splits of the state sums
+    (1, 1, 300, 128, 128),
+]
+
+
+@pytest.mark.parametrize("B,H,L,d,m", BIDIR_SHAPES)
+def test_bf16_bidirectional_backward_shapes(cuda_device, B, H, L, d, m):
+    w = Workload("t", B, H, L, d, m, False, "bf16", True, 5, 30 + L)
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, m, d, "bf16")
+    _, grads = run_fwd_bwd(w, x, Wr, cuda_device, False)
+    for name, g, r in zip(("dQ", "dK", "dV"), grads, oracle_grads(x, W64, False)):
+        assert np.isfinite(g).all(), name
+        if L == 1 and name == "dQ":
+            # one key: the output is that key's value whatever the query, so dQ is exactly zero
+            # (the reference is rounding noise); bound the GPU's dQ against the upstream scale
+            assert np.abs(g).max() <= 1e-3 * np.sqrt(np.mean(x["dO"].astype(np.float64) ** 2)), name
+            continue
+        assert rel_max_err(g, r) <= TOL["bf16"], name
+
+
 def test_bf16_backward_config5_slice_L1024(cuda_device):
     """Workload 5's shape (B=2, H=8, d=128, m=256) on its first 1024 rows as a separate problem."""
     w = WORKLOADS[5]
@@ -65,3 +94,36 @@ def test_bf16_backward_config5_slice_L1024(cuda_device):
     assert rel_max_err(out, favor.fwd(X["Q"], X["K"], X["V"], W64)) <= TOL["bf16"]
     for g, r in zip(grads, oracle_grads(x, W64, False)):
         assert rel_max_err(g, r) <= TOL["bf16"]
+
+
+def test_bf16_backward_config5_full_length(cuda_device):
+    """Workload 5 at its full size (B=2, H=8, L=16384, d=128, m=256), in the launch configuration
+    the benchmark times: every gradient element of two heads against the fp64 oracle (run on those
+    heads alone: heads are independent), and all outputs finite."""
+    w = WORKLOADS[5]
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    _, grads = run_fwd_bwd(w, x, Wr, cuda_device, False)
+    for g in grads:
+        assert np.isfinite(g).all()
+    for b, h in ((0, 0), (1, 7)):
+        X = {k: x[k][b, h].astype(np.float64) for k in x}
+        ref = favor.bwd_bidirectional(X["Q"], X["K"], X["V"], W64, X["dO"])
+        for name, g, r in zip(("dQ", "dK", "dV"), grads, ref):
+            assert rel_max_err(g[b, h], r) <= TOL["bf16"], (name, b, h)
+
+
+def test_bf16_bidirectional_backward_needs_context(cuda_device):
+    import torch
+
+    w = Workload("t", 1, 1, 128, 64, 256, False, "bf16", True, 5, 3)
+    x = make_inputs(w)
+    Wr, _ = features_for(w.w_seed, w.m, w.d, "bf16")
+    T = {k: to_torch(x[k], "bf16", cuda_device) for k in x}
+    Wt = to_torch(Wr, "bf16", cuda_device)
+    out = api.fwd(T["Q"], T["K"], T["V"], Wt)
+    with pytest.raises(api.FavorError) as ei:
+        api.bwd(T["Q"], T["K"], T["V"], Wt, out, T["dO"], ctx=None)
+    assert ei.value.status == api.FAVOR_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert api.sync_status() == api.FAVOR_OK

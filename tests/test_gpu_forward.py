@@ -272,3 +272,16 @@ def test_bf16_causal_values_beyond_fp16_range_are_reported(cuda_device):
     api.fwd(Q, K, to_torch(V, w.dtype, cuda_device), Wt, causal=True)
     assert api.sync_status() == api.FAVOR_ERR_UNSUPPORTED
     assert api.sync_status() == api.FAVOR_OK  # the status word is cleared by the read
+
+
+@pytest.mark.parametrize("poly_pct", [25, 50, 100])
+@pytest.mark.parametrize("causal,d", [(False, 64), (False, 128), (True, 64)])
+def test_bf16_exponentials_on_the_fma_polynomial(cuda_device, poly_pct, causal, d):
+    """favor_opts.exp_poly_pct moves a share of the feature exponentials from MUFU ex2 to the
+    FMA-pipe polynomial (every kernel instantiates each share); outputs stay within tolerance."""
+    w = Workload("t", 1, 2, 1100, d, 256, causal, "bf16", False, 3 if causal else 2, 90 + poly_pct)
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    out = run_fwd(w, x, Wr, cuda_device, causal, opts=api.make_opts(exp_poly_pct=poly_pct))
+    assert np.isfinite(out).all()
+    assert rel_max_err(out, oracle_fwd(x, W64, causal)) <= TOL["bf16"]

@@ -132,3 +132,36 @@ def test_empty_inputs_are_refused_before_launch(favor_lib):
             if dt == api.FAVOR_BF16:
                 assert favor_lib.favor_fwd_static_scratch(ctypes.byref(sh), p, p, p, p, p,
                                                           null) == api.FAVOR_ERR_INVALID_ARG
+
+
+def test_decode_state_size_and_argument_errors(favor_lib):
+    """favor_decode_step answers argument errors on the host before any CUDA call."""
+    for d, m in ((64, 256), (128, 128), (64, 32)):
+        sh = api.make_shape(2, 3, 1, d, m, api.FAVOR_BF16)
+        assert favor_lib.favor_decode_state_size(ctypes.byref(sh)) == 2 * 3 * (d * m + 2 * m) * 4
+    for d, m in ((96, 256), (64, 48), (64, 512)):
+        sh = api.make_shape(1, 1, 1, d, m, api.FAVOR_BF16)
+        assert favor_lib.favor_decode_state_size(ctypes.byref(sh)) == 0
+    p, null = ctypes.c_void_p(256), None
+    ok = api.make_shape(1, 2, 1, 64, 256, api.FAVOR_BF16)
+    two = api.make_shape(1, 2, 2, 64, 256, api.FAVOR_BF16)
+    assert favor_lib.favor_decode_step(ctypes.byref(two), p, p, p, p, p, p, null) == api.FAVOR_ERR_INVALID_ARG
+    assert favor_lib.favor_decode_step(ctypes.byref(ok), null, p, p, p, p, p, null) == api.FAVOR_ERR_INVALID_ARG
+    assert favor_lib.favor_decode_step(ctypes.byref(ok), p, p, p, p, ctypes.c_void_p(260), p, null) == \
+        api.FAVOR_ERR_INVALID_ARG
+    odd = api.make_shape(1, 2, 1, 64, 48, api.FAVOR_BF16)
+    assert favor_lib.favor_decode_step(ctypes.byref(odd), p, p, p, p, p, p, null) == api.FAVOR_ERR_UNSUPPORTED
+
+
+def test_bounded_wait_selftest_rejects_limits_on_the_host(favor_lib):
+    assert favor_lib.favor_selftest_bounded_wait(0, None) == api.FAVOR_ERR_INVALID_ARG
+    assert favor_lib.favor_selftest_bounded_wait(1000001, None) == api.FAVOR_ERR_INVALID_ARG
+
+
+def test_bf16_bidirectional_backward_requires_the_forward_context(favor_lib):
+    sh = api.make_shape(1, 2, 300, 64, 256, api.FAVOR_BF16)
+    ws = api.workspace_size(sh, causal=False, backward=True)
+    assert ws > 0 and ws % 256 == 0
+    p = ctypes.c_void_p(256)
+    assert favor_lib.favor_bwd(ctypes.byref(sh), p, p, p, p, p, p, None, 0, p, p, p, p, ws, None, None) == \
+        api.FAVOR_ERR_WORKSPACE
