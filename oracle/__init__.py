@@ -25,11 +25,13 @@ Modules
 -------
 ``philox``   Philox4x64-10 counter-based generator (Salmon et al., SC'11).
 ``features`` Gaussian draws and the block-orthogonal random feature matrix W.
-``favor``    phi, bidirectional / causal forward, backward, brute-force definitions, softmax.
+``favor``    phi, bidirectional / causal forward, backward, the single-token causal step,
+             brute-force definitions, softmax.
+``kernels``  generalised attention (ReLU features) and the trigonometric softmax features.
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against something other than itself
 (a library routine, brute force on the explicit L x L matrix, closed forms, Monte-Carlo bounds,
 invariants, finite differences). No function is "parity unpinned".
 """
 
-from . import philox, features, favor  # noqa: F401
+from . import philox, features, favor, kernels  # noqa: F401
