@@ -36,11 +36,15 @@ L2_FLUSH_BYTES = 256 << 20
 
 # Kernels favor_fwd launches for the bf16 path, in launch order (stage k <-> events 2k, 2k+1).
 FWD_STAGES = ["k_key_partials", "k_state_image", "k_query_out"]
-CAUSAL_STAGES = ["k_key_logit_max", "k_key_state", "k_state_scan", "k_causal_chunk", "k_causal_prefix"]
+CAUSAL_STAGES = ["k_key_logit_max", "k_key_state", "k_state_scan", "k_causal_chunk", "gemm_causal_prefix"]
 # Kernels favor_bwd launches (bf16 bidirectional: split-precision GEMM passes and two reductions).
 BWD_STAGES = ["gemm_phi_k", "gemm_state_partial", "reduce_state", "gemm_phi_q", "gemm_gs", "gemm_t_q", "gemm_dq",
               "gemm_G_partial", "reduce_G", "gemm_dv", "gemm_t_k", "gemm_dk"]
-BWD_CAUSAL_STAGES = ["k_widen_q", "k_widen_k", "k_widen_v", "k_widen_do", "k_widen_w", "k_f32_head_bwd"]
+# (bf16 causal: the same passes split at 128-token chunks, with masked diagonal tiles and
+# per-chunk prefix / suffix state images)
+BWD_CAUSAL_STAGES = ["gemm_phi_k", "gemm_phi_q", "gemm_chunk_state", "scan_prefix", "gemm_mask_A", "gemm_nd_inter",
+                     "gemm_gs_intra", "gemm_mask_B", "gemm_dphiq_inter", "gemm_t_q_intra", "gemm_dq", "gemm_chunk_G",
+                     "scan_suffix", "gemm_dv_inter", "gemm_dv_intra", "gemm_dphik_inter", "gemm_t_k_intra", "gemm_dk"]
 
 
 def load_peaks():
@@ -73,10 +77,15 @@ def stage_work(name, w, n_sms=148):
     # intermediates (4 B per element: phi(K), phi(Q), t are m wide, [g | s] is d + 64 wide) and the
     # tensor FLOPs of its split products (3 MMAs when both operands are split, 2 when one is exact).
     Np = d + 64
+    mf = 2 * m if w.feature_map == "trig" else m   # features per token (sin and cos: 2m)
     if name in ("gemm_phi_k", "gemm_phi_q"):   # read K (or Q); write phi hi/lo
-        return t * (2 * d + 4 * m), 2 * m * d * t, 0
+        return t * (2 * d + 4 * mf), 2 * m * d * t, 0
     if name == "gemm_state_partial":           # read phi(K) hi/lo and V
-        return t * (4 * m + 2 * d), 2 * 2 * m * (d + 1) * t, 0
+        return t * (4 * mf + 2 * d), 2 * 2 * mf * (d + 1) * t, 0
+    if name == "sp_state+sp_output":           # both calls: read K, V, Q; phi hi/lo out and back; out
+        return t * (6 * d + 2 * 8 * m + 4 * d), (2 * 2 * m * d + 2 * 2 * m * (d + 1) + 3 * 2 * m * (d + 1)) * t, 0
+    if name == "gemm_out":                     # read phi(Q) hi/lo; write fp32 out
+        return t * (4 * mf + 4 * d), 3 * 2 * mf * (d + 1) * t, 0
     if name == "gemm_G_partial":               # read phi(Q) hi/lo and [g | s] hi/lo
         return t * (4 * m + 4 * Np), 3 * 2 * m * (d + 1) * t, 0
     if name in ("reduce_state", "reduce_G"):   # read the partial states, write the hi/lo images
@@ -91,6 +100,38 @@ def stage_work(name, w, n_sms=148):
         return t * (4 * m + 4 * d), 3 * 2 * m * d * t, 0
     if name == "gemm_t_k":                     # read V and phi(K) hi/lo; write t hi/lo and sum t
         return t * (2 * d + 8 * m + 4), 2 * 2 * m * (d + 1) * t, 0
+    C = 128  # causal backward chunk
+    if name == "gemm_chunk_state":             # read phi(K) hi/lo and V
+        return t * (4 * m + 2 * d), 2 * 2 * m * (d + 1) * t, 0
+    if name == "gemm_chunk_G":                 # read phi(Q) hi/lo and [g | s] hi/lo
+        return t * (4 * m + 4 * Np), 3 * 2 * m * (d + 1) * t, 0
+    if name in ("scan_prefix", "scan_suffix"):
+        return 0, 0, 0
+    if name == "gemm_mask_A":                  # read phi(Q), phi(K) hi/lo; write the masked tile hi/lo
+        return t * (8 * m + 4 * C), 3 * 2 * m * C * t, 0
+    if name == "gemm_nd_inter":                # read phi(Q) hi/lo; write fp32 [num | den] part
+        return t * (4 * m + 4 * Np), 3 * 2 * m * (d + 1) * t, 0
+    if name == "gemm_gs_intra":                # read A, V, the fp32 part and dO; write [g | s] hi/lo
+        return t * (4 * C + 4 * d + 8 * Np), 2 * 2 * C * (d + 1) * t, 0
+    if name == "gemm_mask_B":                  # read [g | s] hi/lo and V; write the masked tile hi/lo
+        return t * (4 * Np + 2 * d + 4 * C), 2 * 2 * C * (d + 1) * t, 0
+    if name == "gemm_dphiq_inter":             # read [g | s] hi/lo; write fp32 part
+        return t * (4 * Np + 4 * m), 3 * 2 * m * (d + 1) * t, 0
+    if name in ("gemm_t_q_intra", "gemm_t_k_intra"):  # read B, phi (two), the part; write t hi/lo
+        return t * (4 * C + 12 * m + 4 * m + 4), 3 * 2 * C * m * t, 0
+    if name == "gemm_dv_inter":                # read phi(K) hi/lo; write fp32 part
+        return t * (4 * m + 4 * d), 3 * 2 * m * d * t, 0
+    if name == "gemm_dv_intra":                # read A, g hi/lo and the part; write dV
+        return t * (4 * C + 4 * d + 8 * d), 3 * 2 * C * d * t, 0
+    if name == "gemm_dphik_inter":             # read V; write fp32 part
+        return t * (2 * d + 4 * m), 2 * 2 * m * (d + 1) * t, 0
+    if name == "gemm_causal_prefix":   # first 512 tokens per head at split precision (four GEMMs):
+        # read q, k, v; write and read phi hi/lo and the masked scores hi/lo; write out
+        P = min(w.L, 512)
+        Pp = (P + 127) // 128 * 128
+        nbytes = BH * P * (6 * d + 2 * 8 * m + 2 * 4 * Pp + 4 * d)
+        flops = BH * P * (2 * 2 * m * d + 3 * 2 * m * Pp + 2 * 2 * Pp * (d + 1))
+        return nbytes, flops, 0
     if name == "k_causal_chunk":       # read Q, K, V, -|k|^2/2; write fp32 out; fp16 MMAs per token:
         # Q W^T and K W^T (2 x 2md), state term and state update (2 x 2md), scores and masked A V
         # over the 128-token tile (2 * 128 * m + 2 * 128 * d)
@@ -252,6 +293,8 @@ def oracle_W(w):
 
 def metric_name(w):
     kind = "fwd+bwd" if w.backward else "fwd"
+    if w.feature_map != "positive":
+        return f"{w.feature_map}-feature attention {kind} tokens/s (B*H*L)"
     return f"FAVOR+ {kind} tokens/s (B*H*L)"
 
 
@@ -285,9 +328,19 @@ def job_rate(tokens_per_rank, world, job_ms, steps):
 
 # ------------------------------------------------------------------------------------ GPU arm
 
+MAP_STAGES = ["gemm_phi_k", "gemm_state_partial", "reduce_state", "gemm_phi_q", "gemm_out"]
+# the sequence-parallel calls, timed as one step (no per-launch events)
+SP_STAGES = ["sp_state", "sp_output"]
+MAP_CODES = {"positive": 0, "relu": 1, "trig": 2}
+
+
 def stage_names(w):
     """Kernel launches of one step, in launch order (stage k <-> stage events 2k, 2k+1); the
     backward's launches follow the forward's."""
+    if w.feature_map != "positive":
+        return list(MAP_STAGES)
+    if w.sequence_parallel:
+        return list(SP_STAGES)
     if w.dtype != "bf16":
         return ["k_f32_head"] + (["k_f32_head_bwd"] if w.backward else [])
     names = list(CAUSAL_STAGES if w.causal else FWD_STAGES)
@@ -322,7 +375,8 @@ def path_roofline(w, ms_per_step, peaks, clk, n_sm):
     bwd = 1 if w.backward else 0
     path_bytes = w.tokens * ((6 * w.d + 4 * w.d) + bwd * (8 * w.d + 12 * w.d))
     path_flops = (6 + 12 * bwd) * w.tokens * w.m * w.d
-    path_exps = (2 + 2 * bwd) * w.m * w.tokens
+    # transcendental evaluations: exp (positive map), sin and cos (trigonometric); none for ReLU
+    path_exps = 0 if w.feature_map == "relu" else (2 + 2 * bwd) * w.m * w.tokens
     step_s = ms_per_step * 1e-3
     sm_hz = (clk["sm_mhz"] if clk and clk.get("sm_mhz") else 1965.0) * 1e6
     return {"hbm_bytes_per_step": path_bytes, "hbm_frac": path_bytes / step_s / (peaks["hbm_gbs"] * 1e9),
@@ -343,19 +397,32 @@ class Runner:
         self.T = {k: torch.from_numpy(self.x[k]).to(self.tdt).to(dev) for k in self.x}
         self.Wt = torch.from_numpy(round_to_bf16(Wf) if w.dtype == "bf16" else Wf).to(self.tdt).to(dev)
         shape = api.make_shape(w.B, w.H, w.L, w.d, w.m, api.FAVOR_BF16 if w.dtype == "bf16" else api.FAVOR_F32)
-        self.ws = torch.empty(max(api.workspace_size(shape, w.causal, False), api.workspace_size(shape, w.causal, w.backward)),
+        mo = api.make_opts(feature_map=MAP_CODES[w.feature_map])
+        self.ws = torch.empty(max(api.workspace_size(shape, w.causal, False, mo),
+                                  api.workspace_size(shape, w.causal, w.backward, mo)),
                               dtype=torch.uint8, device=dev)
         self.ctx = torch.empty(api.ctx_size(shape, w.causal), dtype=torch.uint8, device=dev) if w.backward else None
         self.out = torch.empty(self.T["Q"].shape, dtype=torch.float32, device=dev)
         self.grads = [torch.empty(self.T["Q"].shape, dtype=torch.float32, device=dev) for _ in range(3)] \
             if w.backward else None
+        if w.sequence_parallel:
+            self.sp_state = torch.empty(api.library().favor_sp_state_size(api.ctypes.byref(shape)) // 4,
+                                        dtype=torch.float32, device=dev)
+            self.sp_ws = torch.empty(api.library().favor_sp_workspace_size(api.ctypes.byref(shape)),
+                                     dtype=torch.uint8, device=dev)
         self.stages = stage_names(w)
         self.poly = exp_poly_pct
-        self.base_opts = api.make_opts(exp_poly_pct=exp_poly_pct)
+        self.fmap = MAP_CODES[w.feature_map]
+        self.base_opts = api.make_opts(exp_poly_pct=exp_poly_pct, feature_map=self.fmap)
 
     def step(self, T=None, fwd_opts=None, bwd_opts=None):
         api, w = self.api, self.w
         T = T or self.T
+        if w.sequence_parallel:
+            # one rank's two calls; a multi-GPU run adds the all-reduce of the state in between
+            api.sp_state(T["K"], T["V"], self.Wt, state=self.sp_state, workspace=self.sp_ws)
+            api.sp_output(T["Q"], self.Wt, self.sp_state, out=self.out, workspace=self.sp_ws)
+            return
         api.fwd(T["Q"], T["K"], T["V"], self.Wt, causal=w.causal, out=self.out, ctx=self.ctx, workspace=self.ws,
                 opts=fwd_opts or self.base_opts)
         if w.backward:
@@ -382,11 +449,9 @@ class Runner:
         torch.cuda.synchronize()
         if api.sync_status() != api.FAVOR_OK:
             raise RuntimeError(f"device status not OK after warm-up ({self.w.name})")
+        # timed steps: events around each whole step only (an event recorded between two launches
+        # would keep the second from starting its prologue under the first's tail)
         step_ev = [new_events(2) for _ in range(steps)]
-        fev = [new_events(2 * api.FAVOR_MAX_STAGES) for _ in range(steps)]
-        bev = [new_events(2 * api.FAVOR_MAX_STAGES) for _ in range(steps)]
-        fopts = [api.make_opts(exp_poly_pct=self.poly, stage_events=fev[k]) for k in range(steps)]
-        bopts = [api.make_opts(stage_events=bev[k]) for k in range(steps)]
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -394,15 +459,28 @@ class Runner:
         for k in range(steps):
             flush.zero_()
             step_ev[k][0].record(stream)
-            self.step(fwd_opts=fopts[k], bwd_opts=bopts[k])
+            self.step()
             step_ev[k][1].record(stream)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         status = api.sync_status()
         step_ms = [a.elapsed_time(b) for a, b in step_ev]
+        # per-kernel breakdown from further steps with an event pair around every launch
+        fev = [new_events(2 * api.FAVOR_MAX_STAGES) for _ in range(steps)]
+        bev = [new_events(2 * api.FAVOR_MAX_STAGES) for _ in range(steps)]
+        fopts = [api.make_opts(exp_poly_pct=self.poly, stage_events=fev[k], feature_map=self.fmap)
+                 for k in range(steps)]
+        bopts = [api.make_opts(stage_events=bev[k]) for k in range(steps)]
+        torch.cuda.synchronize()
+        for k in range(steps):
+            flush.zero_()
+            self.step(fwd_opts=fopts[k], bwd_opts=bopts[k])
+        torch.cuda.synchronize()
         nf = self.n_fwd_stages()
         stage_ms = {}
+        if self.w.sequence_parallel:  # the two calls record no per-launch events
+            return step_ms, {"sp_state+sp_output": statistics.mean(step_ms)}, status
         for i, name in enumerate(self.stages):
             ev, j = (fev, i) if i < nf else (bev, i - nf)
             key = name if name not in stage_ms else f"{name}#{i}"
@@ -524,6 +602,7 @@ def run_ours(args, w):
         "e2e": {"value": job_rate(w.tokens, world, e2e_ms, 1)[1], "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
+        "stage_ms_note": "per-kernel times come from separate steps with an event pair around every launch",
         "device_status": api.status_string(status),
     }
     if w.dtype == "bf16":
@@ -562,7 +641,7 @@ def main():
                     help="skip the oracle sample after the timed region (for profiler runs)")
     ap.add_argument("--headline-only", action="store_true",
                     help="time only --workload (not the other workloads reported under 'workloads')")
-    ap.add_argument("--also", default="3,4,5",
+    ap.add_argument("--also", default="3,4,5,6,7,8",
                     help="comma-separated workloads timed after the headline and reported under 'workloads'")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -69,7 +69,7 @@ typedef struct {
 } favor_shape;
 
 /* Most kernel launches one call makes (the length of a stage_events array is 2x this). */
-#define FAVOR_MAX_STAGES 16
+#define FAVOR_MAX_STAGES 24
 
 /* Tuning knobs; pass NULL for defaults. Zero fields take their defaults too.
  *   split_tiles : 128-token tiles per causal segment (the unit of the causal key-side reduction
@@ -78,13 +78,28 @@ typedef struct {
  *   exp_poly_pct: percent (0..100) of feature exponentials evaluated by the FMA-pipe
  *                 polynomial instead of the MUFU ex2 unit (bf16 path); 0 (the default) puts
  *                 all of them on MUFU
+ *   feature_map : the random-feature map (bf16 bidirectional forward only; other calls refuse a
+ *                 non-default map with FAVOR_ERR_UNSUPPORTED):
+ *                 FAVOR_MAP_POSITIVE (0, default): phi(x) = exp(Wx - |x|^2/2)/sqrt(m), FAVOR+;
+ *                 FAVOR_MAP_RELU: phi(x) = max(Wx, 0)/sqrt(m), generalised (kernelizable)
+ *                 attention with the degree-1 arc-cosine kernel ("Rethinking Attention with
+ *                 Performers", abstract: attention mechanisms beyond softmax);
+ *                 FAVOR_MAP_TRIG: phi(x) = exp(|x|^2/2)/sqrt(m) [sin(Wx), cos(Wx)] (2m features),
+ *                 the trigonometric softmax features of FAVOR ("Random Features for Efficient
+ *                 Attention Approximation", thesis abstract: FAVOR to FAVOR+). Its normaliser can
+ *                 be negative or near zero on large-norm inputs; exp(|k|^2/2) must stay in fp32
+ *                 range (|k|^2 < 170).
  *   stage_events: NULL, or 2 * FAVOR_MAX_STAGES caller-created cudaEvent_t handles (as void*);
  *                 the call records events[2k] before and events[2k+1] after its k-th kernel
  *                 launch on the call's stream (NULL entries are skipped). For timing. */
+#define FAVOR_MAP_POSITIVE 0
+#define FAVOR_MAP_RELU 1
+#define FAVOR_MAP_TRIG 2
 typedef struct {
     int split_tiles;
     int exp_poly_pct;
-    int reserved[6];
+    int feature_map;
+    int reserved[5];
     void **stage_events;
 } favor_opts;
 
@@ -200,6 +215,43 @@ FAVOR_API size_t favor_decode_state_size(const favor_shape *shape);
  */
 FAVOR_API favor_status favor_decode_step(const favor_shape *shape, const void *q, const void *k, const void *v,
                                          const void *W, float *state, float *out, void *stream);
+
+/*
+ * Sequence-parallel bidirectional forward (bf16). The keys of one sequence may be spread over
+ * several calls -- one per rank, each holding a contiguous run of every head's tokens: the FA-part
+ * needs only the sums (K')^T V and (K')^T 1_L over all keys ("Fast Attention Via Positive
+ * Orthogonal Random Features", codewithpapers.app/method/favor, the FA-part equations), and sums
+ * over disjoint runs add. favor_sp_state writes a run's partial [S | z]; the caller adds the
+ * partial states of all runs (an all-reduce SUM across ranks); favor_sp_output then gives the
+ * outputs of any run of queries from the total.
+ *
+ * Every partial state is taken against the same per-feature offsets c_r = |w_r|^2/2 - 40 (natural
+ * log units), fixed by W alone: since u_r(k) = w_r.k - |k|^2/2 <= |w_r|^2/2 for every key, the key
+ * features exp(u_r(k) - c_r) never exceed e^40, and partial states from different calls add
+ * directly. Operands are carried as bf16 hi + lo pairs (fp32 accumulation), as in the backward.
+ *
+ * State layout (device, fp32, favor_sp_state_size bytes): [B*H][m][d + 64]; column c < d holds
+ * sum_j exp(u_r(k_j) - c_r) v_j[c], column d the same sum of 1, the other columns zero.
+ */
+FAVOR_API size_t favor_sp_state_size(const favor_shape *shape);
+/* favor_sp_workspace_size -- device workspace bytes of either call for this (local) shape; 0 if
+ * unsupported (bf16; d in {64, 128}; m in {128, 256}). */
+FAVOR_API size_t favor_sp_workspace_size(const favor_shape *shape);
+/*
+ * favor_sp_state -- partial state of the keys K, V (device, [B,H,L,d] bf16, L = this run's length)
+ * with W ([m,d] bf16): state (device, fp32, favor_sp_state_size bytes) is fully written.
+ * Returns FAVOR_ERR_INVALID_ARG (null or misaligned pointer, bad size), FAVOR_ERR_UNSUPPORTED,
+ * FAVOR_ERR_WORKSPACE, FAVOR_ERR_CUDA.
+ */
+FAVOR_API favor_status favor_sp_state(const favor_shape *shape, const void *K, const void *V, const void *W,
+                                      float *state, void *workspace, size_t ws_bytes, void *stream);
+/*
+ * favor_sp_output -- out_i = phi(q_i)^T S / phi(q_i)^T z for the queries Q (device, [B,H,L,d] bf16,
+ * L = this run's length) against state (device, fp32: the sum of the partial states of all key
+ * runs); out (device, fp32 [B,H,L,d]) is fully written. Errors as favor_sp_state.
+ */
+FAVOR_API favor_status favor_sp_output(const favor_shape *shape, const void *Q, const void *W, const float *state,
+                                       float *out, void *workspace, size_t ws_bytes, void *stream);
 
 /* favor_status_string -- static, never-NULL description of a status code. */
 FAVOR_API const char *favor_status_string(favor_status status);

@@ -31,6 +31,10 @@ EXPORTS = (
     "favor_bwd",
     "favor_sync_status",
     "favor_status_string",
+    "favor_sp_state_size",
+    "favor_sp_workspace_size",
+    "favor_sp_state",
+    "favor_sp_output",
     "favor_decode_state_size",
     "favor_decode_step",
     "favor_selftest_bounded_wait",
@@ -50,12 +54,17 @@ class Shape(ctypes.Structure):
                 ("m", ctypes.c_int), ("dtype", ctypes.c_int)]
 
 
-FAVOR_MAX_STAGES = 16
+FAVOR_MAX_STAGES = 24
+
+
+FAVOR_MAP_POSITIVE = 0
+FAVOR_MAP_RELU = 1
+FAVOR_MAP_TRIG = 2
 
 
 class Opts(ctypes.Structure):
-    _fields_ = [("split_tiles", ctypes.c_int), ("exp_poly_pct", ctypes.c_int), ("reserved", ctypes.c_int * 6),
-                ("stage_events", ctypes.POINTER(ctypes.c_void_p))]
+    _fields_ = [("split_tiles", ctypes.c_int), ("exp_poly_pct", ctypes.c_int), ("feature_map", ctypes.c_int),
+                ("reserved", ctypes.c_int * 5), ("stage_events", ctypes.POINTER(ctypes.c_void_p))]
 
 
 _LIB = None
@@ -85,6 +94,14 @@ def library():
     lib.favor_sync_status.restype = I
     lib.favor_status_string.argtypes = [I]
     lib.favor_status_string.restype = ctypes.c_char_p
+    lib.favor_sp_state_size.argtypes = [SP]
+    lib.favor_sp_state_size.restype = Z
+    lib.favor_sp_workspace_size.argtypes = [SP]
+    lib.favor_sp_workspace_size.restype = Z
+    lib.favor_sp_state.argtypes = [SP, P, P, P, P, P, Z, P]
+    lib.favor_sp_state.restype = I
+    lib.favor_sp_output.argtypes = [SP, P, P, P, P, P, Z, P]
+    lib.favor_sp_output.restype = I
     lib.favor_decode_state_size.argtypes = [SP]
     lib.favor_decode_state_size.restype = Z
     lib.favor_decode_step.argtypes = [SP, P, P, P, P, P, P, P]
@@ -110,10 +127,10 @@ def make_shape(B, H, L, d, m, dtype):
     return Shape(B, H, L, d, m, dtype)
 
 
-def make_opts(split_tiles=0, exp_poly_pct=0, stage_events=None):
+def make_opts(split_tiles=0, exp_poly_pct=0, stage_events=None, feature_map=FAVOR_MAP_POSITIVE):
     """Options struct. ``stage_events``: optional list of 2*FAVOR_MAX_STAGES torch.cuda.Event
     (enable_timing=True, already recorded once so their handles exist) or None entries."""
-    o = Opts(split_tiles, exp_poly_pct, (ctypes.c_int * 6)(), None)
+    o = Opts(split_tiles, exp_poly_pct, feature_map, (ctypes.c_int * 5)(), None)
     if stage_events is not None:
         arr = (ctypes.c_void_p * (2 * FAVOR_MAX_STAGES))()
         for i, ev in enumerate(stage_events[: 2 * FAVOR_MAX_STAGES]):
@@ -243,6 +260,51 @@ def bwd_into(Q, K, V, W, out, dout, dQ, dK, dV, ctx=None, causal=False, workspac
 def sync_status(stream=None):
     """Synchronise the stream and return (and clear) the device status word."""
     return library().favor_sync_status(_stream_ptr(stream))
+
+
+def sp_state(K, V, W, state=None, workspace=None, stream=None):
+    """Partial state [B*H, m, d+64] (fp32) of this run of keys through favor_sp_state."""
+    torch = _torch()
+    _check_inputs((K, V, W), K)
+    shape = _shape_of(K, W)
+    lib = library()
+    if state is None:
+        state = torch.empty(lib.favor_sp_state_size(ctypes.byref(shape)) // 4, dtype=torch.float32, device=K.device)
+    if workspace is None:
+        workspace = _alloc_bytes(lib.favor_sp_workspace_size(ctypes.byref(shape)), K.device)
+    st = lib.favor_sp_state(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(W), _ptr(state), _ptr(workspace),
+                            workspace.numel(), _stream_ptr(stream))
+    _check(st, "favor_sp_state")
+    return state
+
+
+def sp_output(Q, W, state, out=None, workspace=None, stream=None):
+    """Outputs of this run of queries against a total state, through favor_sp_output."""
+    torch = _torch()
+    _check_inputs((Q, W), Q)
+    shape = _shape_of(Q, W)
+    lib = library()
+    if out is None:
+        out = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = _alloc_bytes(lib.favor_sp_workspace_size(ctypes.byref(shape)), Q.device)
+    st = lib.favor_sp_output(ctypes.byref(shape), _ptr(Q), _ptr(W), _ptr(state), _ptr(out), _ptr(workspace),
+                             workspace.numel(), _stream_ptr(stream))
+    _check(st, "favor_sp_output")
+    return out
+
+
+def sp_forward(Q, K, V, W, group=None, state_fn=None, output_fn=None):
+    """Sequence-parallel bidirectional forward: this rank holds a contiguous run of every head's
+    tokens; its partial key state is summed over the ranks of ``group`` (one all-reduce) and its
+    queries are answered from the total. ``state_fn`` / ``output_fn`` default to sp_state /
+    sp_output (tests substitute host stand-ins to exercise the exchange without a GPU)."""
+    import torch.distributed as dist
+
+    state = (state_fn or sp_state)(K, V, W)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(state, op=dist.ReduceOp.SUM, group=group)
+    return (output_fn or sp_output)(Q, W, state)
 
 
 def decode_state(B, H, d, m, device):

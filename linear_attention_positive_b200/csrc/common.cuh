@@ -55,6 +55,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// (No explicit suspend-time hint: one of 100 us measured 5-7 % slower on the forward kernels, whose
+// consumer warps wake on the critical path.)
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -461,6 +463,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 __device__ __forceinline__ uint32_t elect_lane0() { return (threadIdx.x & 31u) == 0u; }
+
+// Programmatic dependent launch: let the next kernel on the stream (launched with the programmatic
+// serialization attribute) start its prologue once every CTA of this grid has reached this point,
+// and, in that next kernel, wait until this grid has completed and its writes are visible before
+// reading them.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // One lane of a converged warp (elect.sync): the warp runs a producer loop together, so its
 // descriptor arithmetic stays warp-uniform, and the elected lane issues the TMA / MMA instruction.

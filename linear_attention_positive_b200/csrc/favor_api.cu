@@ -44,8 +44,8 @@ favor_status shape_supported(const favor_shape *s, int causal, int backward) {
         return FAVOR_OK;
     }
     if (s->m != 128 && s->m != 256) return FAVOR_ERR_UNSUPPORTED;
-    if (causal && !backward && s->d != 64) return FAVOR_ERR_UNSUPPORTED;
-    if (backward && s->m > 512) return FAVOR_ERR_UNSUPPORTED;
+    // the causal path (forward, and the backward that reads its context) is built for d = 64
+    if (causal && s->d != 64) return FAVOR_ERR_UNSUPPORTED;
     return FAVOR_OK;
 }
 
@@ -58,6 +58,8 @@ int opt_poly_pct(const favor_opts *o) {
     return v > 0 ? std::min(v, 100) : 0;
 }
 
+int opt_feature_map(const favor_opts *o) { return o ? o->feature_map : FAVOR_MAP_POSITIVE; }
+
 int opt_split_tiles(const favor_opts *o) {
     const int v = o ? o->split_tiles : 0;
     return v > 0 ? std::min(v, 64) : 8;
@@ -67,15 +69,17 @@ int opt_split_tiles(const favor_opts *o) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Tokens per head that the causal path recomputes exactly in fp32 (see k_causal.cu).
+// Tokens per head whose causal outputs are recomputed at split precision (bf16 hi + lo operands,
+// fp32 accumulation): the first outputs of a head average few values and are far larger than the
+// head's RMS output, beyond what the fp16 chunk kernel resolves.
 constexpr int kCausalExactPrefix = 512;
-// Row stride of the feature-major fp32 scratch of those tokens.
-int prefix_stride(int P) { return (P + 31) & ~31; }
+// Key columns of the prefix's masked score matrix: P rounded up to the 128-wide GEMM tile.
+int prefix_cols(int P) { return (P + 127) & ~127; }
 
 struct Bf16Layout {
-    int BH, n_tiles, tiles_per_split, n_split, P_exact;
-    size_t off_bias, off_split_max, off_head_max, off_part_S, off_part_z, off_state, off_seg_S, off_seg_z, off_phi,
-        total;
+    int BH, n_tiles, tiles_per_split, n_split, P_exact, Ppad;
+    size_t off_bias, off_split_max, off_head_max, off_part_S, off_part_z, off_state, off_seg_S, off_seg_z,
+        off_kref, off_pq[2], off_pk[2], off_pa[2], total;
 };
 
 Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_ws, int causal = 0) {
@@ -102,8 +106,17 @@ Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_
     if (causal) off += align256((size_t)l.BH * l.n_split * s->m * s->d * 4);
     l.off_seg_z = off;
     if (causal) off += align256((size_t)l.BH * l.n_split * s->m * 4);
-    l.off_phi = off;
-    if (causal) off += align256((size_t)2 * l.BH * prefix_stride(l.P_exact) * s->m * 4);
+    l.Ppad = prefix_cols(l.P_exact);
+    l.off_kref = off;
+    if (causal) off += align256((size_t)l.BH * 4);
+    for (int i = 0; i < 2; ++i) {
+        l.off_pq[i] = off;
+        if (causal) off += align256((size_t)l.BH * l.P_exact * s->m * 2);
+        l.off_pk[i] = off;
+        if (causal) off += align256((size_t)l.BH * l.P_exact * s->m * 2);
+        l.off_pa[i] = off;
+        if (causal) off += align256((size_t)l.BH * l.P_exact * l.Ppad * 2);
+    }
     l.total = off;
     return l;
 }
@@ -136,12 +149,6 @@ BidirLayout bidir_layout(const favor_shape *s, bool state_in_ws) {
     return l;
 }
 
-// bf16 backward (current route): Q, K, V, dO and W widened to fp32, then the fp32 kernels.
-size_t bf16_bwd_bytes(const favor_shape *s) {
-    const size_t n = (size_t)s->B * s->H * s->L * s->d;
-    return 4 * align256(n * 4) + align256((size_t)s->m * s->d * 4) +
-           align256(f32_workspace_floats(s->B * s->H, s->L, s->d, s->m) * 4);
-}
 
 // Forward-to-backward context: per-head state blocks (the bidirectional fp16 state image, or the
 // causal path's state), the causal per-key -|k|^2/2, and the per-head key reference C (log2
@@ -161,6 +168,93 @@ CtxLayout ctx_layout(const favor_shape *s) {
 }
 
 size_t ctx_bytes(const favor_shape *s) { return ctx_layout(s).total; }
+
+// bf16 bidirectional forward with a feature map other than the positive one (generalised
+// attention, trigonometric features): phi(K), phi(Q) as hi/lo bf16 rows of mf features (m, or 2m
+// for sin and cos), the state's token-split partial sums, and its hi/lo image [d+64][mf].
+struct MapLayout {
+    int BH, Np, mf, n_split, kt_split;
+    size_t off_phk[2], off_phq[2], off_part, off_img[2], total;
+};
+
+MapLayout map_layout(const favor_shape *s, int map) {
+    MapLayout l{};
+    l.BH = s->B * s->H;
+    l.Np = s->d + 64;
+    l.mf = map == FAVOR_MAP_TRIG ? 2 * s->m : s->m;
+    const int kt_total = (s->L + kGemmBK - 1) / kGemmBK;
+    const int tiles = l.BH * (l.mf / 128);
+    const int ns = std::max(1, std::min(kt_total, (2 * num_sms() + tiles - 1) / tiles));
+    l.kt_split = (kt_total + ns - 1) / ns;
+    l.n_split = (kt_total + l.kt_split - 1) / l.kt_split;
+    const size_t tok = (size_t)l.BH * s->L;
+    const size_t feat = align256(tok * l.mf * 2), img = align256((size_t)l.BH * l.Np * l.mf * 2);
+    size_t off = 0;
+    for (int i = 0; i < 2; ++i) { l.off_phk[i] = off; off += feat; }
+    for (int i = 0; i < 2; ++i) { l.off_phq[i] = off; off += feat; }
+    l.off_part = off; off += align256((size_t)l.BH * l.n_split * l.mf * l.Np * 4);
+    for (int i = 0; i < 2; ++i) { l.off_img[i] = off; off += img; }
+    l.total = off;
+    return l;
+}
+
+// Sequence-parallel forward (bf16, bidirectional): per-feature offsets, phi(K) or phi(Q) hi/lo,
+// the token-split partial state, its hi/lo image.
+struct SpLayout {
+    int BH, Np, n_split, kt_split;
+    size_t off_c, off_phi[2], off_part, off_img[2], total;
+};
+
+SpLayout sp_layout(const favor_shape *s) {
+    SpLayout l{};
+    l.BH = s->B * s->H;
+    l.Np = s->d + 64;
+    const int kt_total = (s->L + kGemmBK - 1) / kGemmBK;
+    const int tiles = l.BH * (s->m / 128);
+    const int ns = std::max(1, std::min(kt_total, (2 * num_sms() + tiles - 1) / tiles));
+    l.kt_split = (kt_total + ns - 1) / ns;
+    l.n_split = (kt_total + l.kt_split - 1) / l.kt_split;
+    const size_t tok = (size_t)l.BH * s->L;
+    size_t off = 0;
+    l.off_c = off; off += align256((size_t)s->m * 4);
+    for (int i = 0; i < 2; ++i) { l.off_phi[i] = off; off += align256(tok * s->m * 2); }
+    l.off_part = off; off += align256((size_t)l.BH * l.n_split * s->m * l.Np * 4);
+    for (int i = 0; i < 2; ++i) { l.off_img[i] = off; off += align256((size_t)l.BH * l.Np * s->m * 2); }
+    l.total = off;
+    return l;
+}
+
+// bf16 causal backward: the same intermediates per token, the masked 128 x 128 diagonal tiles of
+// every chunk, an fp32 scratch for the between-chunk terms, and per-chunk state images.
+struct CausalBwdLayout {
+    int BH, Np, nc;
+    size_t off_phk[2], off_phq[2], off_gs[2], off_t[2], off_am[2], off_bm[2], off_x, off_rowsum, off_part, off_pimg[2],
+        off_rimg[2], total;
+};
+
+CausalBwdLayout causal_bwd_layout(const favor_shape *s) {
+    CausalBwdLayout l{};
+    l.BH = s->B * s->H;
+    l.Np = s->d + 64;
+    l.nc = (s->L + kTile - 1) / kTile;
+    const size_t tok = (size_t)l.BH * s->L;
+    const size_t feat = align256(tok * s->m * 2), gsz = align256(tok * l.Np * 2), msk = align256(tok * kTile * 2);
+    const size_t img = align256((size_t)l.BH * l.nc * l.Np * s->m * 2);
+    size_t off = 0;
+    for (int i = 0; i < 2; ++i) { l.off_phk[i] = off; off += feat; }
+    for (int i = 0; i < 2; ++i) { l.off_phq[i] = off; off += feat; }
+    for (int i = 0; i < 2; ++i) { l.off_gs[i] = off; off += gsz; }
+    for (int i = 0; i < 2; ++i) { l.off_t[i] = off; off += feat; }
+    for (int i = 0; i < 2; ++i) { l.off_am[i] = off; off += msk; }
+    for (int i = 0; i < 2; ++i) { l.off_bm[i] = off; off += msk; }
+    l.off_x = off; off += align256(tok * std::max(s->m, l.Np) * 4);
+    l.off_rowsum = off; off += align256(tok * 8);  // two partial row sums per token
+    l.off_part = off; off += align256((size_t)l.BH * l.nc * s->m * l.Np * 4);
+    for (int i = 0; i < 2; ++i) { l.off_pimg[i] = off; off += img; }
+    for (int i = 0; i < 2; ++i) { l.off_rimg[i] = off; off += img; }
+    l.total = off;
+    return l;
+}
 
 // bf16 bidirectional backward: hi/lo bf16 intermediates of the split-precision GEMM passes.
 struct BwdLayout {
@@ -190,7 +284,7 @@ BwdLayout bwd_layout(const favor_shape *s) {
     l.off_gs_lo = off; off += gsz;
     l.off_t_hi = off; off += feat;
     l.off_t_lo = off; off += feat;
-    l.off_rowsum = off; off += align256(tok * 4);
+    l.off_rowsum = off; off += align256(tok * 8);  // two partial row sums per token
     l.off_part = off; off += align256((size_t)l.BH * l.n_split * s->m * l.Np * 4);
     l.off_sz_hi = off; off += img;
     l.off_sz_lo = off; off += img;
@@ -283,6 +377,70 @@ void record_stage(const favor_opts *o, int slot, cudaStream_t st) {
 
 // ---------------------------------------------------------------------------- bf16 forward
 
+// Outputs of the first P = min(L, 512) tokens of every head at split precision, overwriting what the
+// chunk kernel left there: phi(K) = 2^(u(k) log2e - C), phi(Q) = exp(Wq - rowmax) as hi/lo bf16,
+// A = mask(phi(Q) phi(K)^T) (key j kept for j <= query i) as hi/lo, then out = num / den with
+// [num | den] = A [V | 1]: four launches of the split-precision GEMM (k_gemm.cu).
+favor_status causal_prefix(const favor_shape *s, const Bf16Layout &l, const void *Q, const void *K, const void *V,
+                           const void *W, const float *kref, float *out, uint8_t *ws, const favor_opts *o,
+                           cudaStream_t st) {
+    const int BH = l.BH, L = s->L, d = s->d, m = s->m, P = l.P_exact, Pp = l.Ppad, Np = d + 64;
+    uint16_t *pq[2], *pk[2], *pa[2];
+    for (int i = 0; i < 2; ++i) {
+        pq[i] = (uint16_t *)(ws + l.off_pq[i]);
+        pk[i] = (uint16_t *)(ws + l.off_pk[i]);
+        pa[i] = (uint16_t *)(ws + l.off_pa[i]);
+    }
+    CUtensorMap mK, mQ, mVn, mW, mPq[2], mPk[2], mPa[2];
+    bool ok = make_map3(&mK, K, d, L, BH, 128) && make_map3(&mQ, Q, d, L, BH, 128) && make_map3(&mVn, V, d, L, BH, 64) &&
+              make_map3(&mW, W, d, m, 1, m);
+    for (int i = 0; ok && i < 2; ++i)
+        ok = make_map3(&mPq[i], pq[i], m, P, BH, 128) && make_map3(&mPk[i], pk[i], m, P, BH, 128) &&
+             make_map3(&mPa[i], pa[i], Pp, P, BH, 128);
+    if (!ok) return FAVOR_ERR_CUDA;
+    auto args = [&](int M, int N, int Kd) {
+        GemmArgs a{};
+        a.M = M;
+        a.N = N;
+        a.K = Kd;
+        a.n_split = 1;
+        a.kt_split = (Kd + kGemmBK - 1) / kGemmBK;
+        a.a_batched = a.b_batched = 1;
+        return a;
+    };
+    GemmArgs ak = args(P, m, d);
+    ak.b_batched = 0;
+    ak.ld_out = m;
+    ak.out_hi = pk[0];
+    ak.out_lo = pk[1];
+    ak.kc = kref;
+    record_stage(o, 8, st);
+    cudaError_t e = launch_gemm_t<false, false, false, false, kEpiPhiKey>(mK, mK, mW, mW, ak, m, BH, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    GemmArgs aq = args(P, m, d);
+    aq.b_batched = 0;
+    aq.ld_out = m;
+    aq.out_hi = pq[0];
+    aq.out_lo = pq[1];
+    e = launch_gemm_t<false, false, false, false, kEpiPhiQuery>(mQ, mQ, mW, mW, aq, m, BH, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    GemmArgs aa = args(P, Pp, m);
+    aa.ld_out = Pp;
+    aa.out_hi = pa[0];
+    aa.out_lo = pa[1];
+    e = launch_gemm_t<false, false, true, true, kEpiMask>(mPq[0], mPq[1], mPk[0], mPk[1], aa, 128, BH, st);
+    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
+    GemmArgs ao = args(P, Np, Pp);
+    ao.b_ones = 1;
+    ao.ld_out = d;
+    ao.out_f32 = out;
+    ao.out_rows = L;
+    ao.d = d;
+    e = launch_gemm_t<false, true, true, false, kEpiOut>(mPa[0], mPa[1], mVn, mVn, ao, Np, BH, st);
+    record_stage(o, 9, st);
+    return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+}
+
 favor_status fwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W,
                             float *out, void *ctx, uint8_t *ws, size_t ws_bytes, const favor_opts *o, cudaStream_t st) {
     const BidirLayout l = bidir_layout(s, ctx == nullptr);
@@ -317,8 +475,87 @@ favor_status fwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, 
     return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 
+// Bidirectional forward with the ReLU or trigonometric feature map, as split-precision GEMM passes:
+// phi(K) (hi/lo), [S | z] = phi(K)^T [V | 1] over token splits and reduced to a hi/lo image,
+// phi(Q), then out = num / den from [num | den] = phi(Q) [S | z]. The 1/sqrt(m) of phi and, for the
+// trigonometric queries, exp(|q|^2/2) are per-row constants that cancel in D^-1.
+favor_status fwd_bf16_map(const favor_shape *s, int map, const void *Q, const void *K, const void *V, const void *W,
+                          float *out, uint8_t *ws, size_t ws_bytes, const favor_opts *o, cudaStream_t st) {
+    const MapLayout l = map_layout(s, map);
+    if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
+    const int BH = l.BH, L = s->L, d = s->d, m = s->m, mf = l.mf, Np = l.Np;
+    uint16_t *phk[2], *phq[2], *img[2];
+    for (int i = 0; i < 2; ++i) {
+        phk[i] = (uint16_t *)(ws + l.off_phk[i]);
+        phq[i] = (uint16_t *)(ws + l.off_phq[i]);
+        img[i] = (uint16_t *)(ws + l.off_img[i]);
+    }
+    float *part = (float *)(ws + l.off_part);
+    CUtensorMap mK, mQ, mVn, mW, mPhkT[2], mPhq[2], mImg[2];
+    bool ok = make_map3(&mK, K, d, L, BH, 128) && make_map3(&mQ, Q, d, L, BH, 128) && make_map3(&mVn, V, d, L, BH, 64) &&
+              make_map3(&mW, W, d, m, 1, m);
+    for (int i = 0; ok && i < 2; ++i)
+        ok = make_map3(&mPhkT[i], phk[i], mf, L, BH, 64) && make_map3(&mPhq[i], phq[i], mf, L, BH, 128) &&
+             make_map3(&mImg[i], img[i], mf, Np, BH, Np);
+    if (!ok) return FAVOR_ERR_CUDA;
+    auto args = [&](int M, int N, int Kd) {
+        GemmArgs a{};
+        a.M = M;
+        a.N = N;
+        a.K = Kd;
+        a.n_split = 1;
+        a.kt_split = (Kd + kGemmBK - 1) / kGemmBK;
+        a.a_batched = a.b_batched = 1;
+        return a;
+    };
+    int stage = 0;
+    cudaError_t e = cudaSuccess;
+    auto run = [&](auto launch) {
+        if (e != cudaSuccess) return;
+        record_stage(o, 2 * stage, st);
+        e = launch();
+        record_stage(o, 2 * stage + 1, st);
+        ++stage;
+    };
+    const bool trig = map == FAVOR_MAP_TRIG;
+    GemmArgs ak = args(L, m, d);
+    ak.b_batched = 0;
+    ak.ld_out = mf;
+    ak.out_hi = phk[0];
+    ak.out_lo = phk[1];
+    run([&] {
+        return trig ? launch_gemm_t<false, false, false, false, kEpiTrigK>(mK, mK, mW, mW, ak, m, BH, st)
+                    : launch_gemm_t<false, false, false, false, kEpiRelu>(mK, mK, mW, mW, ak, m, BH, st);
+    });
+    GemmArgs as = args(mf, Np, L);
+    as.n_split = l.n_split;
+    as.kt_split = l.kt_split;
+    as.b_ones = 1;
+    as.ld_out = Np;
+    as.out_f32 = part;
+    run([&] { return launch_gemm_t<true, true, true, false, kEpiPartial>(mPhkT[0], mPhkT[1], mVn, mVn, as, Np, BH, st); });
+    run([&] { return launch_reduce_image(part, l.n_split, mf, Np, img[0], img[1], BH, st); });
+    GemmArgs aq = args(L, m, d);
+    aq.b_batched = 0;
+    aq.ld_out = mf;
+    aq.out_hi = phq[0];
+    aq.out_lo = phq[1];
+    run([&] {
+        return trig ? launch_gemm_t<false, false, false, false, kEpiTrigQ>(mQ, mQ, mW, mW, aq, m, BH, st)
+                    : launch_gemm_t<false, false, false, false, kEpiRelu>(mQ, mQ, mW, mW, aq, m, BH, st);
+    });
+    GemmArgs ao = args(L, Np, mf);
+    ao.ld_out = d;
+    ao.out_f32 = out;
+    ao.d = d;
+    run([&] { return launch_gemm_t<false, false, true, true, kEpiOut>(mPhq[0], mPhq[1], mImg[0], mImg[1], ao, Np, BH, st); });
+    return cuda_status(e);
+}
+
 favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W, float *out,
                       void *ctx, uint8_t *ws, size_t ws_bytes, const favor_opts *o, cudaStream_t st, int causal) {
+    const int map = opt_feature_map(o);
+    if (map != FAVOR_MAP_POSITIVE) return fwd_bf16_map(s, map, Q, K, V, W, out, ws, ws_bytes, o, st);
     if (!causal) return fwd_bf16_bidir(s, Q, K, V, W, out, ctx, ws, ws_bytes, o, st);
     const Bf16Layout l = bf16_layout(s, o, ctx == nullptr, causal);
     if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
@@ -341,7 +578,8 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     cudaError_t e = launch_key_logit_max(mK, mW, km, l.BH, st);
     record_stage(o, 1, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-    float *kref = ctx ? (float *)((uint8_t *)ctx + ctx_layout(s).off_kref) : nullptr;
+    // the head's key reference in log2 units, for the exact prefix and (in the context) the backward
+    float *kref = ctx ? (float *)((uint8_t *)ctx + ctx_layout(s).off_kref) : (float *)(ws + l.off_kref);
     KeyStateParams ks{s->L, s->d, s->m, l.n_split, l.tiles_per_split, (const uint16_t *)V, bias, split_max,
                       part_S, part_z, head_max, kref};
     record_stage(o, 2, st);
@@ -359,15 +597,7 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     e = launch_causal_chunk(mQ, mK, mV, mW128, cp, opt_poly_pct(o), st);
     record_stage(o, 7, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-    float *phi = (float *)(ws + l.off_phi);
-    const int Ps = prefix_stride(l.P_exact);
-    PrefixParams pp{s->L, s->d, s->m, l.P_exact, Ps, (const uint16_t *)Q, (const uint16_t *)K,
-                    (const uint16_t *)V, (const uint16_t *)W, bias, head_max, phi,
-                    phi + (size_t)l.BH * Ps * s->m, out};
-    record_stage(o, 8, st);
-    e = launch_causal_prefix(pp, l.BH, st);
-    record_stage(o, 9, st);
-    return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
+    return causal_prefix(s, l, Q, K, V, W, kref, out, ws, o, st);
 }
 
 // ---------------------------------------------------------------------------- bf16 backward
@@ -521,6 +751,206 @@ favor_status bwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, 
     return cuda_status(e);
 }
 
+// Causal bf16 backward (W fixed) as split-precision GEMM passes over 128-token chunks c (one GEMM
+// M tile each). With P_c = sum_{j < 128c} phi(k_j) [v_j | 1]^T (exclusive prefix over chunks) and
+// R_c = sum_{i >= 128(c+1)} phi(q_i) [g_i | s_i]^T (exclusive suffix), and the chunk's masked tiles
+// A = mask(phi(Q_c) phi(K_c)^T), B = mask([g | s]_c [V | 1]_c^T) (column j kept for j <= row i):
+//   [num | den] = phi(Q_c) P_c + A [V | 1]_c             -> g, s
+//   dphi(Q)     = [g | s]_c P_c^T + B phi(K_c)           -> t, dQ = t W - Q rowsum(t)
+//   dV          = phi(K_c) R_c[:, :d] + A^T g_c
+//   dphi(K)     = [V | 1]_c R_c^T + B^T phi(Q_c)         -> t, dK = t W - K rowsum(t)
+// (the suffix sums G_j, h_j over i >= j of the masked recurrence, split at the chunk boundary).
+favor_status bwd_bf16_causal(const favor_shape *s, const void *Q, const void *K, const void *V, const void *W,
+                             const void *dout, const void *ctx, float *dQ, float *dK, float *dV, uint8_t *ws,
+                             size_t ws_bytes, const favor_opts *o, cudaStream_t st) {
+    const CausalBwdLayout l = causal_bwd_layout(s);
+    if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
+    const int BH = l.BH, L = s->L, d = s->d, m = s->m, Np = l.Np, nc = l.nc;
+    auto at = [&](size_t off) { return (uint16_t *)(ws + off); };
+    uint16_t *phk[2] = {at(l.off_phk[0]), at(l.off_phk[1])}, *phq[2] = {at(l.off_phq[0]), at(l.off_phq[1])},
+             *gs[2] = {at(l.off_gs[0]), at(l.off_gs[1])}, *tt[2] = {at(l.off_t[0]), at(l.off_t[1])},
+             *am[2] = {at(l.off_am[0]), at(l.off_am[1])}, *bm[2] = {at(l.off_bm[0]), at(l.off_bm[1])},
+             *pimg[2] = {at(l.off_pimg[0]), at(l.off_pimg[1])}, *rimg[2] = {at(l.off_rimg[0]), at(l.off_rimg[1])};
+    float *X = (float *)(ws + l.off_x), *rowsum = (float *)(ws + l.off_rowsum), *part = (float *)(ws + l.off_part);
+    const float *kref = (const float *)((const uint8_t *)ctx + ctx_layout(s).off_kref);
+
+    CUtensorMap mK, mQ, mV, mVn, mW_k, mW_n, mPhk[2], mPhkT[2], mPhq[2], mPhqT[2], mGs[2], mGsT[2], mT[2], mAm[2],
+        mAmT[2], mBm[2], mBmT[2], mPK[2], mPN[2], mRK[2], mRN[2];
+    bool ok = make_map3(&mK, K, d, L, BH, 128) && make_map3(&mQ, Q, d, L, BH, 128) && make_map3(&mV, V, d, L, BH, 128) &&
+              make_map3(&mVn, V, d, L, BH, 64) && make_map3(&mW_k, W, d, m, 1, m) && make_map3(&mW_n, W, d, m, 1, 64);
+    for (int i = 0; ok && i < 2; ++i)
+        ok = make_map3(&mPhk[i], phk[i], m, L, BH, 128) && make_map3(&mPhkT[i], phk[i], m, L, BH, 64) &&
+             make_map3(&mPhq[i], phq[i], m, L, BH, 128) && make_map3(&mPhqT[i], phq[i], m, L, BH, 64) &&
+             make_map3(&mGs[i], gs[i], Np, L, BH, 128) && make_map3(&mGsT[i], gs[i], Np, L, BH, 64) &&
+             make_map3(&mT[i], tt[i], m, L, BH, 128) && make_map3(&mAm[i], am[i], kTile, L, BH, 128) &&
+             make_map3(&mAmT[i], am[i], kTile, L, BH, 64) && make_map3(&mBm[i], bm[i], kTile, L, BH, 128) &&
+             make_map3(&mBmT[i], bm[i], kTile, L, BH, 64) && make_map3(&mPK[i], pimg[i], m, Np, BH * nc, Np) &&
+             make_map3(&mPN[i], pimg[i], m, Np, BH * nc, 64) && make_map3(&mRK[i], rimg[i], m, Np, BH * nc, d) &&
+             make_map3(&mRN[i], rimg[i], m, Np, BH * nc, 64);
+    if (!ok) return FAVOR_ERR_CUDA;
+
+    int stage = 0;
+    cudaError_t e = cudaSuccess;
+    auto run = [&](auto launch) {
+        if (e != cudaSuccess) return;
+        record_stage(o, 2 * stage, st);
+        e = launch();
+        record_stage(o, 2 * stage + 1, st);
+        ++stage;
+    };
+    auto args = [&](int M, int N, int Kd) {
+        GemmArgs a{};
+        a.M = M;
+        a.N = N;
+        a.K = Kd;
+        a.n_split = 1;
+        a.kt_split = (Kd + kGemmBK - 1) / kGemmBK;
+        a.a_batched = a.b_batched = 1;
+        return a;
+    };
+    // phi(K), phi(Q)
+    GemmArgs ak = args(L, m, d);
+    ak.b_batched = 0;
+    ak.ld_out = m;
+    ak.out_hi = phk[0];
+    ak.out_lo = phk[1];
+    ak.kc = kref;
+    run([&] { return launch_gemm_t<false, false, false, false, kEpiPhiKey>(mK, mK, mW_k, mW_k, ak, m, BH, st); });
+    GemmArgs aq = args(L, m, d);
+    aq.b_batched = 0;
+    aq.ld_out = m;
+    aq.out_hi = phq[0];
+    aq.out_lo = phq[1];
+    run([&] { return launch_gemm_t<false, false, false, false, kEpiPhiQuery>(mQ, mQ, mW_k, mW_k, aq, m, BH, st); });
+    // per-chunk key states phi(K_c)^T [V | 1]_c, exclusive prefix images P_c
+    GemmArgs as = args(m, Np, L);
+    as.n_split = nc;
+    as.kt_split = kTile / kGemmBK;
+    as.b_ones = 1;
+    as.ld_out = Np;
+    as.out_f32 = part;
+    run([&] { return launch_gemm_t<true, true, true, false, kEpiPartial>(mPhkT[0], mPhkT[1], mVn, mVn, as, Np, BH, st); });
+    run([&] { return launch_scan_image(part, nc, m, Np, 0, pimg[0], pimg[1], BH, st); });
+    // A = mask(phi(Q_c) phi(K_c)^T)
+    GemmArgs aa = args(L, kTile, m);
+    aa.b_nofs = 1;
+    aa.ld_out = kTile;
+    aa.out_hi = am[0];
+    aa.out_lo = am[1];
+    run([&] { return launch_gemm_t<false, false, true, true, kEpiMask>(mPhq[0], mPhq[1], mPhk[0], mPhk[1], aa, kTile, BH, st); });
+    // [num | den]: phi(Q_c) P_c into X, then A [V | 1]_c + X -> [g | s]
+    GemmArgs an = args(L, Np, m);
+    an.b_chunk = 1;
+    an.n_chunks = nc;
+    an.ld_out = Np;
+    an.out_f32 = X;
+    run([&] { return launch_gemm_t<false, false, true, true, kEpiF32>(mPhq[0], mPhq[1], mPK[0], mPK[1], an, Np, BH, st); });
+    GemmArgs ag = args(L, Np, kTile);
+    ag.b_kofs = 1;
+    ag.b_ones = 1;
+    ag.addend = X;
+    ag.ld_add = Np;
+    ag.ld_out = Np;
+    ag.out_hi = gs[0];
+    ag.out_lo = gs[1];
+    ag.side_hi = (const uint16_t *)dout;
+    ag.ld_side = d;
+    ag.d = d;
+    run([&] { return launch_gemm_t<false, true, true, false, kEpiGS>(mAm[0], mAm[1], mVn, mVn, ag, Np, BH, st); });
+    // B = mask([g | s]_c [V | 1]_c^T)
+    GemmArgs ab = args(L, kTile, Np);
+    ab.b_nofs = 1;
+    ab.b_ones_k = 1;
+    ab.ld_out = kTile;
+    ab.out_hi = bm[0];
+    ab.out_lo = bm[1];
+    run([&] { return launch_gemm_t<false, false, true, false, kEpiMask>(mGs[0], mGs[1], mV, mV, ab, kTile, BH, st); });
+    // dphi(Q): [g | s]_c P_c^T into X, then B phi(K_c) + X -> t, rowsum(t)
+    GemmArgs ad = args(L, m, Np);
+    ad.b_chunk = 1;
+    ad.n_chunks = nc;
+    ad.ld_out = m;
+    ad.out_f32 = X;
+    run([&] { return launch_gemm_t<false, true, true, true, kEpiF32>(mGs[0], mGs[1], mPN[0], mPN[1], ad, m, BH, st); });
+    GemmArgs at2 = args(L, m, kTile);
+    at2.b_kofs = 1;
+    at2.addend = X;
+    at2.ld_add = m;
+    at2.ld_out = m;
+    at2.out_hi = tt[0];
+    at2.out_lo = tt[1];
+    at2.rowsum = rowsum;
+    at2.side_hi = phq[0];
+    at2.side_lo = phq[1];
+    at2.ld_side = m;
+    run([&] { return launch_gemm_t<false, true, true, true, kEpiT>(mBm[0], mBm[1], mPhkT[0], mPhkT[1], at2, m, BH, st); });
+    // dQ = t W - Q rowsum(t)
+    GemmArgs aqq = args(L, d, m);
+    aqq.b_batched = 0;
+    aqq.ld_out = d;
+    aqq.out_f32 = dQ;
+    aqq.rowsum = rowsum;
+    aqq.side_hi = (const uint16_t *)Q;
+    aqq.ld_side = d;
+    run([&] { return launch_gemm_t<false, true, true, false, kEpiDX>(mT[0], mT[1], mW_n, mW_n, aqq, d, BH, st); });
+    // per-chunk query sums phi(Q_c)^T [g | s]_c, exclusive suffix images R_c
+    GemmArgs ar = args(m, Np, L);
+    ar.n_split = nc;
+    ar.kt_split = kTile / kGemmBK;
+    ar.ld_out = Np;
+    ar.out_f32 = part;
+    run([&] { return launch_gemm_t<true, true, true, true, kEpiPartial>(mPhqT[0], mPhqT[1], mGsT[0], mGsT[1], ar, Np, BH, st); });
+    run([&] { return launch_scan_image(part, nc, m, Np, 1, rimg[0], rimg[1], BH, st); });
+    // dV: phi(K_c) R_c[:, :d] into X, then A^T g_c + X
+    GemmArgs av = args(L, d, m);
+    av.b_chunk = 1;
+    av.n_chunks = nc;
+    av.ld_out = d;
+    av.out_f32 = X;
+    run([&] { return launch_gemm_t<false, false, true, true, kEpiF32>(mPhk[0], mPhk[1], mRK[0], mRK[1], av, d, BH, st); });
+    GemmArgs av2 = args(L, d, kTile);
+    av2.a_kofs = 1;
+    av2.a_mlocal = 1;
+    av2.b_kofs = 1;
+    av2.addend = X;
+    av2.ld_add = d;
+    av2.ld_out = d;
+    av2.out_f32 = dV;
+    run([&] { return launch_gemm_t<true, true, true, true, kEpiF32>(mAmT[0], mAmT[1], mGsT[0], mGsT[1], av2, d, BH, st); });
+    // dphi(K): [V | 1]_c R_c^T into X, then B^T phi(Q_c) + X -> t, rowsum(t)
+    GemmArgs ae = args(L, m, Np);
+    ae.a_ones = 1;
+    ae.b_chunk = 1;
+    ae.n_chunks = nc;
+    ae.ld_out = m;
+    ae.out_f32 = X;
+    run([&] { return launch_gemm_t<false, true, false, true, kEpiF32>(mV, mV, mRN[0], mRN[1], ae, m, BH, st); });
+    GemmArgs ak2 = args(L, m, kTile);
+    ak2.a_kofs = 1;
+    ak2.a_mlocal = 1;
+    ak2.b_kofs = 1;
+    ak2.addend = X;
+    ak2.ld_add = m;
+    ak2.ld_out = m;
+    ak2.out_hi = tt[0];
+    ak2.out_lo = tt[1];
+    ak2.rowsum = rowsum;
+    ak2.side_hi = phk[0];
+    ak2.side_lo = phk[1];
+    ak2.ld_side = m;
+    run([&] { return launch_gemm_t<true, true, true, true, kEpiT>(mBmT[0], mBmT[1], mPhqT[0], mPhqT[1], ak2, m, BH, st); });
+    // dK = t W - K rowsum(t)
+    GemmArgs akk = args(L, d, m);
+    akk.b_batched = 0;
+    akk.ld_out = d;
+    akk.out_f32 = dK;
+    akk.rowsum = rowsum;
+    akk.side_hi = (const uint16_t *)K;
+    akk.ld_side = d;
+    run([&] { return launch_gemm_t<false, true, true, false, kEpiDX>(mT[0], mT[1], mW_n, mW_n, akk, d, BH, st); });
+    return cuda_status(e);
+}
+
 }  // namespace
 }  // namespace favor
 
@@ -541,8 +971,14 @@ extern "C" const char *favor_status_string(favor_status st) {
 extern "C" size_t favor_workspace_size(const favor_shape *s, int causal, int backward, const favor_opts *o) {
     if (!shape_ok(s) || (causal != 0 && causal != 1)) return 0;
     if (shape_supported(s, causal, backward) != FAVOR_OK) return 0;
+    const int map = opt_feature_map(o);
+    if (map != FAVOR_MAP_POSITIVE) {
+        if (map != FAVOR_MAP_RELU && map != FAVOR_MAP_TRIG) return 0;
+        if (s->dtype != FAVOR_BF16 || causal || backward) return 0;
+        return map_layout(s, map).total;
+    }
     if (s->dtype == FAVOR_F32) return align256(f32_workspace_floats(s->B * s->H, s->L, s->d, s->m) * 4);
-    if (backward) return causal ? bf16_bwd_bytes(s) : bwd_layout(s).total;
+    if (backward) return causal ? causal_bwd_layout(s).total : bwd_layout(s).total;
     if (!causal) return bidir_layout(s, true).total;
     return bf16_layout(s, o, true, causal).total;
 }
@@ -562,6 +998,10 @@ extern "C" favor_status favor_fwd(const favor_shape *s, const void *Q, const voi
         return FAVOR_ERR_INVALID_ARG;
     const favor_status sup = shape_supported(s, causal, 0);
     if (sup != FAVOR_OK) return sup;
+    const int map = opt_feature_map(o);
+    if (map != FAVOR_MAP_POSITIVE &&
+        ((map != FAVOR_MAP_RELU && map != FAVOR_MAP_TRIG) || s->dtype != FAVOR_BF16 || causal))
+        return FAVOR_ERR_UNSUPPORTED;
     if (workspace == nullptr || ((uintptr_t)workspace & 255u) != 0) return FAVOR_ERR_WORKSPACE;
     if (ctx != nullptr && ((uintptr_t)ctx & 255u) != 0) return FAVOR_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
@@ -586,33 +1026,16 @@ extern "C" favor_status favor_bwd(const favor_shape *s, const void *Q, const voi
         return FAVOR_ERR_INVALID_ARG;
     const favor_status sup = shape_supported(s, causal, 1);
     if (sup != FAVOR_OK) return sup;
+    if (opt_feature_map(o) != FAVOR_MAP_POSITIVE) return FAVOR_ERR_UNSUPPORTED;
     if (workspace == nullptr || ((uintptr_t)workspace & 255u) != 0) return FAVOR_ERR_WORKSPACE;
     if (ws_bytes < favor_workspace_size(s, causal, 1, o)) return FAVOR_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
-    if (s->dtype == FAVOR_BF16 && !causal) {
+    if (s->dtype == FAVOR_BF16) {
         // the key reference of the forward's context keeps the backward's key features in range
         if (ctx == nullptr || ((uintptr_t)ctx & 255u) != 0) return FAVOR_ERR_WORKSPACE;
-        return bwd_bf16_bidir(s, Q, K, V, W, dout, ctx, dQ, dK, dV, (uint8_t *)workspace, ws_bytes, o, st);
-    }
-    if (s->dtype == FAVOR_BF16) {
-        const size_t n = (size_t)s->B * s->H * s->L * s->d;
         uint8_t *ws = (uint8_t *)workspace;
-        float *q = (float *)ws, *k = (float *)(ws + align256(n * 4)), *v = (float *)(ws + 2 * align256(n * 4));
-        float *g = (float *)(ws + 3 * align256(n * 4)), *w = (float *)(ws + 4 * align256(n * 4));
-        float *fws = (float *)(ws + 4 * align256(n * 4) + align256((size_t)s->m * s->d * 4));
-        const void *src[5] = {Q, K, V, dout, W};
-        float *dst[5] = {q, k, v, g, w};
-        for (int i = 0; i < 5; ++i) {
-            record_stage(o, 2 * i, st);
-            const cudaError_t e = launch_widen(src[i], dst[i], i == 4 ? (size_t)s->m * s->d : n, st);
-            record_stage(o, 2 * i + 1, st);
-            if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-        }
-        F32Params p{s->L, s->d, s->m, q, k, v, w, out, g, nullptr, dQ, dK, dV, fws};
-        record_stage(o, 10, st);
-        const cudaError_t e = launch_f32(p, s->B * s->H, causal != 0, true, st);
-        record_stage(o, 11, st);
-        return cuda_status(e);
+        return causal ? bwd_bf16_causal(s, Q, K, V, W, dout, ctx, dQ, dK, dV, ws, ws_bytes, o, st)
+                      : bwd_bf16_bidir(s, Q, K, V, W, dout, ctx, dQ, dK, dV, ws, ws_bytes, o, st);
     }
     F32Params p{s->L, s->d, s->m, (const float *)Q, (const float *)K, (const float *)V, (const float *)W,
                 out, (const float *)dout, nullptr, dQ, dK, dV, (float *)workspace};
@@ -646,6 +1069,118 @@ extern "C" favor_status favor_decode_step(const favor_shape *s, const void *q, c
         return FAVOR_ERR_UNSUPPORTED;
     DecodeParams p{s->B * s->H, s->m, s->dtype == FAVOR_BF16 ? 1 : 0, q, k, v, W, state, out};
     return cuda_status(launch_decode_step(p, s->d, (cudaStream_t)stream));
+}
+
+// ------------------------------------------------------------------ sequence-parallel forward
+
+namespace favor {
+namespace {
+
+favor_status sp_check(const favor_shape *s, const void *a, const void *b, const void *c, const void *d, const void *e,
+                      void *ws) {
+    if (!shape_ok(s) || a == nullptr || b == nullptr || c == nullptr || d == nullptr || e == nullptr)
+        return FAVOR_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(c) || !aligned16(d) || !aligned16(e)) return FAVOR_ERR_INVALID_ARG;
+    if (s->dtype != FAVOR_BF16 || (s->d != 64 && s->d != 128) || (s->m != 128 && s->m != 256) ||
+        (long long)s->B * s->H > 65535)
+        return FAVOR_ERR_UNSUPPORTED;
+    if (ws == nullptr || ((uintptr_t)ws & 255u) != 0) return FAVOR_ERR_WORKSPACE;
+    return FAVOR_OK;
+}
+
+GemmArgs sp_args(int M, int N, int Kd) {
+    GemmArgs a{};
+    a.M = M;
+    a.N = N;
+    a.K = Kd;
+    a.n_split = 1;
+    a.kt_split = (Kd + kGemmBK - 1) / kGemmBK;
+    a.a_batched = a.b_batched = 1;
+    return a;
+}
+
+}  // namespace
+}  // namespace favor
+
+extern "C" size_t favor_sp_state_size(const favor_shape *s) {
+    if (!shape_ok(s)) return 0;
+    return (size_t)s->B * s->H * s->m * (s->d + 64) * 4;
+}
+
+extern "C" size_t favor_sp_workspace_size(const favor_shape *s) {
+    if (!shape_ok(s) || s->dtype != FAVOR_BF16 || (s->d != 64 && s->d != 128) || (s->m != 128 && s->m != 256))
+        return 0;
+    return sp_layout(s).total;
+}
+
+extern "C" favor_status favor_sp_state(const favor_shape *s, const void *K, const void *V, const void *W, float *state,
+                                       void *workspace, size_t ws_bytes, void *stream) {
+    const favor_status chk = sp_check(s, K, V, W, state, K, workspace);
+    if (chk != FAVOR_OK) return chk;
+    const SpLayout l = sp_layout(s);
+    if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t *ws = (uint8_t *)workspace;
+    const int BH = l.BH, L = s->L, d = s->d, m = s->m, Np = l.Np;
+    float *c = (float *)(ws + l.off_c), *part = (float *)(ws + l.off_part);
+    uint16_t *phi[2] = {(uint16_t *)(ws + l.off_phi[0]), (uint16_t *)(ws + l.off_phi[1])};
+    CUtensorMap mK, mVn, mW, mPhT[2];
+    bool ok = make_map3(&mK, K, d, L, BH, 128) && make_map3(&mVn, V, d, L, BH, 64) && make_map3(&mW, W, d, m, 1, m);
+    for (int i = 0; ok && i < 2; ++i) ok = make_map3(&mPhT[i], phi[i], m, L, BH, 64);
+    if (!ok) return FAVOR_ERR_CUDA;
+    if (launch_feature_offsets(W, m, d, c, st) != cudaSuccess) return FAVOR_ERR_CUDA;
+    GemmArgs ak = sp_args(L, m, d);
+    ak.b_batched = 0;
+    ak.ld_out = m;
+    ak.out_hi = phi[0];
+    ak.out_lo = phi[1];
+    ak.colbias = c;
+    if (launch_gemm_t<false, false, false, false, kEpiPhiKey>(mK, mK, mW, mW, ak, m, BH, st) != cudaSuccess)
+        return FAVOR_ERR_CUDA;
+    GemmArgs as = sp_args(m, Np, L);
+    as.n_split = l.n_split;
+    as.kt_split = l.kt_split;
+    as.b_ones = 1;
+    as.ld_out = Np;
+    as.out_f32 = part;
+    if (launch_gemm_t<true, true, true, false, kEpiPartial>(mPhT[0], mPhT[1], mVn, mVn, as, Np, BH, st) != cudaSuccess)
+        return FAVOR_ERR_CUDA;
+    return cuda_status(launch_sum_partials(part, l.n_split, (size_t)m * Np, state, BH, st));
+}
+
+extern "C" favor_status favor_sp_output(const favor_shape *s, const void *Q, const void *W, const float *state,
+                                        float *out, void *workspace, size_t ws_bytes, void *stream) {
+    const favor_status chk = sp_check(s, Q, W, state, out, Q, workspace);
+    if (chk != FAVOR_OK) return chk;
+    const SpLayout l = sp_layout(s);
+    if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t *ws = (uint8_t *)workspace;
+    const int BH = l.BH, L = s->L, d = s->d, m = s->m, Np = l.Np;
+    float *c = (float *)(ws + l.off_c);
+    uint16_t *phi[2] = {(uint16_t *)(ws + l.off_phi[0]), (uint16_t *)(ws + l.off_phi[1])};
+    uint16_t *img[2] = {(uint16_t *)(ws + l.off_img[0]), (uint16_t *)(ws + l.off_img[1])};
+    CUtensorMap mQ, mW, mPh[2], mImg[2];
+    bool ok = make_map3(&mQ, Q, d, L, BH, 128) && make_map3(&mW, W, d, m, 1, m);
+    for (int i = 0; ok && i < 2; ++i)
+        ok = make_map3(&mPh[i], phi[i], m, L, BH, 128) && make_map3(&mImg[i], img[i], m, Np, BH, Np);
+    if (!ok) return FAVOR_ERR_CUDA;
+    if (launch_feature_offsets(W, m, d, c, st) != cudaSuccess) return FAVOR_ERR_CUDA;
+    if (launch_reduce_image(state, 1, m, Np, img[0], img[1], BH, st) != cudaSuccess) return FAVOR_ERR_CUDA;
+    GemmArgs aq = sp_args(L, m, d);
+    aq.b_batched = 0;
+    aq.ld_out = m;
+    aq.out_hi = phi[0];
+    aq.out_lo = phi[1];
+    aq.colbias = c;
+    if (launch_gemm_t<false, false, false, false, kEpiPhiQuery>(mQ, mQ, mW, mW, aq, m, BH, st) != cudaSuccess)
+        return FAVOR_ERR_CUDA;
+    GemmArgs ao = sp_args(L, Np, m);
+    ao.ld_out = d;
+    ao.out_f32 = out;
+    ao.d = d;
+    return cuda_status(
+        launch_gemm_t<false, false, true, true, kEpiOut>(mPh[0], mPh[1], mImg[0], mImg[1], ao, Np, BH, st));
 }
 
 extern "C" favor_status favor_selftest_bounded_wait(unsigned int limit_us, void *stream) {

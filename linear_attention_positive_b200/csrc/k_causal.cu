@@ -10,9 +10,9 @@
 // exclusive prefixes; k_causal_chunk walks each segment's tiles in order from that prefix:
 //   out_tile = ( phi(Q_t) S_<t + mask(phi(Q_t) phi(K_t)^T) V_t ) / ( phi(Q_t) z_<t + rowsum(mask(...)) ),
 //   S_<t+1 = S_<t + phi(K_t)^T V_t.
-// k_causal_prefix_* recompute the first tokens of every head in fp32 on CUDA cores: there the
-// output is a weighted mean of few values, its magnitude is far above the RMS of a long output,
-// and the 11-bit fp16 operands alone would use up the error budget.
+// The first tokens of every head are recomputed afterwards at split precision (bf16 hi + lo
+// operands, k_gemm.cu): there the output is a weighted mean of few values, its magnitude is far
+// above the RMS of a long output, and the 11-bit fp16 operands alone would use up the error budget.
 
 #include "common.cuh"
 
@@ -67,245 +67,6 @@ __global__ void __launch_bounds__(256) k_state_scan(ScanParams p) {
         run += a;
     }
 }
-
-struct PrefixParams {
-    int L, d, m, P;              // P = tokens per head recomputed exactly
-    int Ps;                      // row stride of the feature scratch: P rounded up to 32
-    const uint16_t *Q, *K, *V;   // bf16 [BH, L, d]
-    const uint16_t *W;           // bf16 [m, d]
-    const float *bias;           // [BH, L]  -|k|^2/2
-    const float *head_max;       // [BH]
-    float *phiQ, *phiK;          // [BH, m, Ps] fp32 scratch, feature-major
-    float *out;                  // fp32 [BH, L, d]
-};
-
-__device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
-
-// phi(q) = exp(w.q - max_r w.q) and phi(k) = exp(w.k - |k|^2/2 - C) in fp32 for the first P tokens
-// of each head. CTA per (32 tokens, head); the tokens' q and k rows are widened to fp32 in shared
-// memory once; thread r computes feature r (its W row in registers) token by token and stores its
-// 32 values as one contiguous run of its feature row; the per-token max over features goes through
-// shared memory.
-__global__ void __launch_bounds__(256) k_causal_prefix_features(PrefixParams p) {
-    // xq, xk [32][64] token rows; su [32][257] query logits then phi(q); sk [32][257] phi(k);
-    // smax, sbias [32]
-    extern __shared__ __align__(16) float fsm[];
-    float(*xq)[64] = (float(*)[64])fsm;
-    float(*xk)[64] = (float(*)[64])(fsm + 32 * 64);
-    float(*su)[257] = (float(*)[257])(fsm + 2 * 32 * 64);  // rows padded: token-wise reads stay conflict-free
-    float(*sk)[257] = (float(*)[257])(fsm + 2 * 32 * 64 + 32 * 257);
-    float *smax = fsm + 2 * 32 * 64 + 2 * 32 * 257, *sbias = smax + 32;
-    const int bh = blockIdx.y, j0 = blockIdx.x * 32, t = threadIdx.x;
-    {
-        // 32 token rows of q and k (64 bf16 each) as 16-byte loads, widened to fp32
-        const int a = t >> 3, e8 = (t & 7) * 8, j = j0 + a;
-        const size_t row = ((size_t)bh * p.L + j) * p.d + e8;
-        const uint4 rq = j < p.P ? *(const uint4 *)(p.Q + row) : make_uint4(0, 0, 0, 0);
-        const uint4 rk = j < p.P ? *(const uint4 *)(p.K + row) : make_uint4(0, 0, 0, 0);
-        const uint32_t wq[4] = {rq.x, rq.y, rq.z, rq.w}, wk[4] = {rk.x, rk.y, rk.z, rk.w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            xq[a][e8 + 2 * h] = __uint_as_float(wq[h] << 16);
-            xq[a][e8 + 2 * h + 1] = __uint_as_float(wq[h] & 0xFFFF0000u);
-            xk[a][e8 + 2 * h] = __uint_as_float(wk[h] << 16);
-            xk[a][e8 + 2 * h + 1] = __uint_as_float(wk[h] & 0xFFFF0000u);
-        }
-    }
-    if (t < 32) sbias[t] = j0 + t < p.P ? p.bias[(size_t)bh * p.L + j0 + t] - p.head_max[bh] : -INFINITY;
-    __syncthreads();
-    if (t < p.m) {
-        float w[64];
-        const uint4 *wr = (const uint4 *)(p.W + (size_t)t * p.d);
-#pragma unroll
-        for (int e = 0; e < 64; e += 8) {
-            const uint4 u = __ldg(wr + e / 8);
-            const uint32_t h4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                w[e + 2 * h] = __uint_as_float(h4[h] << 16);
-                w[e + 2 * h + 1] = __uint_as_float(h4[h] & 0xFFFF0000u);
-            }
-        }
-#pragma unroll 1
-        for (int a = 0; a < 32; ++a) {
-            float q0 = 0.f, q1 = 0.f, k0 = 0.f, k1 = 0.f;
-#pragma unroll
-            for (int e = 0; e < 64; e += 4) {
-                const float4 x4 = *(const float4 *)&xq[a][e], y4 = *(const float4 *)&xk[a][e];
-                q0 = fmaf(w[e], x4.x, q0);
-                q1 = fmaf(w[e + 1], x4.y, q1);
-                q0 = fmaf(w[e + 2], x4.z, q0);
-                q1 = fmaf(w[e + 3], x4.w, q1);
-                k0 = fmaf(w[e], y4.x, k0);
-                k1 = fmaf(w[e + 1], y4.y, k1);
-                k0 = fmaf(w[e + 2], y4.z, k0);
-                k1 = fmaf(w[e + 3], y4.w, k1);
-            }
-            su[a][t] = q0 + q1;
-            sk[a][t] = expf(k0 + k1 + sbias[a]);
-        }
-    }
-    __syncthreads();
-    {
-        const int warp = t >> 5, lane = t & 31;
-        for (int a = warp * 4; a < warp * 4 + 4; ++a) {
-            float mx = -INFINITY;
-            for (int r = lane; r < p.m; r += 32) mx = fmaxf(mx, su[a][r]);
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (lane == 0) smax[a] = mx;
-        }
-    }
-    __syncthreads();
-    if (t < p.m)
-#pragma unroll 4
-        for (int a = 0; a < 32; ++a) su[a][t] = j0 + a < p.P ? expf(su[a][t] - smax[a]) : 0.f;
-    __syncthreads();
-    {
-        // feature rows out: warp w writes rows f = w, w + 8, ...; lane = token (128-byte rows)
-        const int warp = t >> 5, lane = t & 31;
-        for (int f = warp; f < p.m; f += 8) {
-            const size_t o = ((size_t)bh * p.m + f) * p.Ps + j0 + lane;
-            p.phiK[o] = sk[lane][f];
-            p.phiQ[o] = su[lane][f];
-        }
-    }
-}
-
-// Masked attention over the first P tokens in fp32: 32-query blocks, two per CTA (below), 256 threads. The
-// queries' phi (all m features) stays in shared memory; per 64-key block up to the diagonal the
-// keys' phi is brought in 128-feature halves. Scores S = phi(Q) phi(K)^T (2 queries x 4 keys per
-// thread), the mask j <= i, then num += S V and den += rowsum(S) (2 queries x 4 values per
-// thread). Dynamic shared memory: qT [m][32], kT [128][64], V block [64][64], S [32][68].
-constexpr int kPrefixQ = 32;
-__device__ __forceinline__ void prefix_attn_block(const PrefixParams &p, int i0) {
-    extern __shared__ __align__(16) float psm[];
-    float *qT = psm;                         // [m][32]
-    float *kT = qT + (size_t)p.m * kPrefixQ;  // [128][64]
-    float *sv = kT + 128 * 64;               // [64][64]
-    float *ss = sv + 64 * 64;                // [32][68]
-    const int bh = blockIdx.y, t = threadIdx.x;
-    __syncthreads();  // the previous block's readers of the shared buffers are done
-    const float *phq = p.phiQ + (size_t)bh * p.m * p.Ps;
-    const float *phk = p.phiK + (size_t)bh * p.m * p.Ps;
-    // qT: m rows of 32 queries (i0 + 31 < Ps: rows of the scratch are padded to multiples of 32)
-    for (int idx = t; idx < p.m * (kPrefixQ / 4); idx += 256 * 4) {
-        float4 r[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int k = idx + 256 * u, f = k >> 3, a4 = (k & 7) * 4;
-            r[u] = k < p.m * (kPrefixQ / 4) ? *(const float4 *)(phq + (size_t)f * p.Ps + i0 + a4) : make_float4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int k = idx + 256 * u;
-            if (k < p.m * (kPrefixQ / 4)) *(float4 *)(qT + 4 * k) = r[u];
-        }
-    }
-    const int tq = (t >> 4) * 2, tk = (t & 15) * 4;  // scores: 2 queries x 4 keys
-    float num[2][4], den[2];
-#pragma unroll
-    for (int a = 0; a < 2; ++a) {
-        den[a] = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) num[a][c] = 0.f;
-    }
-    for (int j0 = 0; j0 < i0 + kPrefixQ && j0 < p.P; j0 += 64) {
-        float sc[2][4];
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) sc[a][b] = 0.f;
-        for (int f0 = 0; f0 < p.m; f0 += 128) {
-            __syncthreads();  // previous readers of kT / sv / ss are done
-            {
-                // kT: 128 feature rows of 64 keys as float4 (a float4 never crosses the padded row end;
-                // entries past P are zero in the scratch)
-                float4 r[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int k = t + 256 * u, f = k >> 4, a4 = (k & 15) * 4;
-                    r[u] = j0 + a4 < p.Ps ? *(const float4 *)(phk + (size_t)(f0 + f) * p.Ps + j0 + a4)
-                                          : make_float4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) *(float4 *)(kT + 4 * (t + 256 * u)) = r[u];
-            }
-            if (f0 == 0) {
-                // V block: 64 keys x 64 values (bf16, 8 per 16-byte load), zero past P
-                uint4 r[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int k = t + 256 * u, a = k >> 3, e8 = (k & 7) * 8;
-                    r[u] = j0 + a < p.P ? *(const uint4 *)(p.V + ((size_t)bh * p.L + j0 + a) * p.d + e8)
-                                        : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int k = t + 256 * u;
-                    const uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
-                    float *dst = sv + 8 * k;
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        dst[2 * h] = __uint_as_float(w[h] << 16);
-                        dst[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
-                    }
-                }
-            }
-            __syncthreads();
-#pragma unroll 4
-            for (int f = 0; f < 128; ++f) {
-                const float2 q2 = *(const float2 *)&qT[(f0 + f) * kPrefixQ + tq];
-                const float4 k4 = *(const float4 *)&kT[f * 64 + tk];
-                sc[0][0] = fmaf(q2.x, k4.x, sc[0][0]);
-                sc[0][1] = fmaf(q2.x, k4.y, sc[0][1]);
-                sc[0][2] = fmaf(q2.x, k4.z, sc[0][2]);
-                sc[0][3] = fmaf(q2.x, k4.w, sc[0][3]);
-                sc[1][0] = fmaf(q2.y, k4.x, sc[1][0]);
-                sc[1][1] = fmaf(q2.y, k4.y, sc[1][1]);
-                sc[1][2] = fmaf(q2.y, k4.z, sc[1][2]);
-                sc[1][3] = fmaf(q2.y, k4.w, sc[1][3]);
-            }
-        }
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) ss[(tq + a) * 68 + tk + b] = (j0 + tk + b <= i0 + tq + a) ? sc[a][b] : 0.f;
-        __syncthreads();
-        // num[2 queries][4 values] += S V over the block's 64 keys
-#pragma unroll 4
-        for (int j = 0; j < 64; ++j) {
-            const float4 v4 = *(const float4 *)&sv[j * 64 + tk];
-            const float s0 = ss[tq * 68 + j], s1 = ss[(tq + 1) * 68 + j];
-            num[0][0] = fmaf(s0, v4.x, num[0][0]);
-            num[0][1] = fmaf(s0, v4.y, num[0][1]);
-            num[0][2] = fmaf(s0, v4.z, num[0][2]);
-            num[0][3] = fmaf(s0, v4.w, num[0][3]);
-            num[1][0] = fmaf(s1, v4.x, num[1][0]);
-            num[1][1] = fmaf(s1, v4.y, num[1][1]);
-            num[1][2] = fmaf(s1, v4.z, num[1][2]);
-            num[1][3] = fmaf(s1, v4.w, num[1][3]);
-            den[0] += s0;
-            den[1] += s1;
-        }
-    }
-#pragma unroll
-    for (int a = 0; a < 2; ++a) {
-        const int i = i0 + tq + a;
-        if (i < p.P && i < p.L && tk < p.d) {
-            float *o = p.out + ((size_t)bh * p.L + i) * p.d + tk;
-            *(float4 *)o = make_float4(num[a][0] / den[a], num[a][1] / den[a], num[a][2] / den[a], num[a][3] / den[a]);
-        }
-    }
-}
-
-// Query blocks i and n - 1 - i share a CTA, so every CTA does about the same number of key blocks.
-__global__ void __launch_bounds__(256) k_causal_prefix_attn(PrefixParams p) {
-    const int nq = (p.P + kPrefixQ - 1) / kPrefixQ, qa = blockIdx.x, qb = nq - 1 - blockIdx.x;
-    prefix_attn_block(p, qb * kPrefixQ);
-    if (qa < qb) prefix_attn_block(p, qa * kPrefixQ);
-}
-
-static size_t prefix_attn_smem(int m) { return ((size_t)m * kPrefixQ + 128 * 64 + 64 * 64 + 32 * 68) * 4; }
 
 // ============================================================================ k_causal_chunk
 //
@@ -1136,20 +897,6 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
 cudaError_t launch_state_scan(const ScanParams &p, int BH, cudaStream_t st) {
     const size_t n = (size_t)p.m * p.d + p.m;
     k_state_scan<<<dim3((unsigned)((n + 255) / 256), BH), 256, 0, st>>>(p);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_causal_prefix(const PrefixParams &p, int BH, cudaStream_t st) {
-    if (p.P <= 0) return cudaSuccess;
-    const size_t fsm = (2 * 32 * 64 + 2 * 32 * 257 + 64) * 4;
-    cudaFuncSetAttribute(k_causal_prefix_features, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
-    k_causal_prefix_features<<<dim3((p.P + 31) / 32, BH), 256, fsm, st>>>(p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const size_t sm = prefix_attn_smem(p.m);
-    cudaFuncSetAttribute(k_causal_prefix_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    const int nq = (p.P + kPrefixQ - 1) / kPrefixQ;
-    k_causal_prefix_attn<<<dim3((nq + 1) / 2, BH), 256, sm, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -237,17 +237,6 @@ __global__ void __launch_bounds__(kF32Threads) k_f32_head(F32Params p) {
     }
 }
 
-// bf16 -> fp32 widening (exact), for running bf16 operands through the fp32 kernels.
-__global__ void k_widen_bf16(const uint16_t *__restrict__ src, float *__restrict__ dst, size_t n) {
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
-        dst[i] = __uint_as_float((uint32_t)src[i] << 16);
-}
-
-cudaError_t launch_widen(const void *src, float *dst, size_t n, cudaStream_t st) {
-    k_widen_bf16<<<592, 256, 0, st>>>((const uint16_t *)src, dst, n);
-    return cudaGetLastError();
-}
-
 size_t f32_workspace_floats(int BH, int L, int d, int m) {
     return (size_t)BH * (2 * (size_t)m * d + (size_t)L * (d + 2));
 }

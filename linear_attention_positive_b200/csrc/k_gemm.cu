@@ -33,7 +33,11 @@ enum GemmEpi : int {
     kEpiDX = 4,        // dx = acc - x * rowsum (x bf16 rows, rowsum fp32): fp32 rows
     kEpiF32 = 5,       // acc as fp32 rows
     kEpiPartial = 6,   // acc as fp32 rows of the split's partial tile [z][M][N]
-    kEpiMask = 7,      // causal mask inside the chunk (column j kept for j <= row i): hi/lo rows
+    kEpiMask = 7,      // causal mask (column j kept for j <= row i, both within the batch): hi/lo rows
+    kEpiOut = 8,       // [num | den]: out = num / den as fp32 rows
+    kEpiRelu = 9,      // phi = max(acc, 0) as hi/lo rows (generalised attention, f = ReLU)
+    kEpiTrigQ = 10,    // phi = [sin(acc), cos(acc)] as hi/lo rows of 2N (queries: exp(|q|^2/2) cancels)
+    kEpiTrigK = 11,    // phi = exp(|k|^2/2) [sin(acc), cos(acc)] as hi/lo rows of 2N (|k|^2 from the A tiles)
 };
 
 struct GemmArgs {
@@ -45,7 +49,7 @@ struct GemmArgs {
     int ld_out;               // row pitch (elements) of the epilogue's outputs
     uint16_t *out_hi, *out_lo;
     float *out_f32;
-    float *rowsum;            // [batch][M] (written by kEpiT, read by kEpiDX)
+    float *rowsum;            // [batch][M][2]: two partial row sums (written by kEpiT, read by kEpiDX)
     const uint16_t *side_hi, *side_lo;  // kEpiT: phi rows; kEpiGS / kEpiDX: dO / x rows (hi only)
     int ld_side;
     const float *kc;          // kEpiPhiKey: per-batch key reference (log2 units)
@@ -58,9 +62,12 @@ struct GemmArgs {
     int a_mlocal;             // M-major A: M coordinate local to the chunk (0..127), not the token
     const float *addend;      // NULL, or fp32 rows (pitch ld_add) added to the accumulator first
     int ld_add;
+    int out_rows;             // rows per batch of the outputs when they differ from M (else 0)
+    const float *colbias;     // kEpiPhiQuery / kEpiPhiKey: NULL, or a per-column exponent offset
+                              // (log2 units) added to the query logits / subtracted from the keys'
 };
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
 constexpr int kGemmBK = 64;
 
 struct GemmSmem {
@@ -131,12 +138,51 @@ __device__ __forceinline__ void acc_row32(uint32_t t_row, int c0, const GemmArgs
     }
 }
 
+// Position of one output tile: tile index t over (M tiles, N tiles, batch x split), M fastest.
+struct GemmTile {
+    int m0, n0, mt, batch, split, kt0, nk, ab, bb, a_k0, b_k0, b_n0;
+};
+
+__device__ __forceinline__ GemmTile gemm_tile(const GemmArgs &p, int BN, int t) {
+    GemmTile g;
+    const int Mt = (p.M + 127) / 128, Nt = (p.N + BN - 1) / BN;
+    g.mt = t % Mt;
+    const int nt = (t / Mt) % Nt, z = t / (Mt * Nt);
+    g.m0 = g.mt * 128;
+    g.n0 = nt * BN;
+    g.batch = z / p.n_split;
+    g.split = z % p.n_split;
+    const int kt_total = (p.K + kGemmBK - 1) / kGemmBK;
+    g.kt0 = g.split * p.kt_split;
+    g.nk = max(min(g.kt0 + p.kt_split, kt_total) - g.kt0, 0);
+    g.ab = p.a_batched ? g.batch : 0;
+    g.bb = p.b_chunk ? g.batch * p.n_chunks + g.mt : (p.b_batched ? g.batch : 0);
+    g.a_k0 = p.a_kofs ? g.m0 : 0;
+    g.b_k0 = p.b_kofs ? g.m0 : 0;
+    g.b_n0 = p.b_nofs ? g.m0 : g.n0;
+    return g;
+}
+
+__host__ __device__ inline int gemm_tiles(const GemmArgs &p, int BN, int batches) {
+    return ((p.M + 127) / 128) * ((p.N + BN - 1) / BN) * batches * p.n_split;
+}
+
+// Persistent CTAs (one per SM) walk the output tiles t = blockIdx.x, + gridDim.x, ...; the
+// accumulator is double-buffered in TMEM (2 x 256 columns), so the epilogue of one tile runs while
+// the next tile's operands stream in and its MMAs run. Warp roles (10 warps): 0 TMA, 1 MMA issue and
+// TMEM allocation, 2-9 the epilogue: warp w handles rows 32 (w % 4) .. + 31 of the tile (its TMEM
+// lane quarter) and the column half (w - 2) / 4. The two halves never wait on each other: a
+// row-wide statistic either is recomputed by each half from the accumulator (the query row maximum,
+// the dot product of s) or is written as two partial values (the row sums of t, added by the
+// consumer), so every wait in the kernel stays a bounded barrier wait.
 template <bool A_MN, bool B_MN, bool A_SPLIT, bool B_SPLIT, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
-       const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mB2, GemmArgs p, int BN) {
+       const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mB2, GemmArgs p, int BN,
+       int n_tiles) {
     constexpr int AP = A_SPLIT ? 2 : 1, BP = B_SPLIT ? 2 : 1;
-    constexpr bool NORM = EPI == kEpiPhiKey;
+    constexpr bool NORM = EPI == kEpiPhiKey || EPI == kEpiTrigK;
+    constexpr int kEpiWarps = 8;
     const GemmSmem plan = gemm_smem_plan(BN, AP, BP, gemm_const_bytes(p, BN));
     const int STAGES = plan.stages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -145,24 +191,16 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
     uint8_t *sOnesA = sStage + (size_t)STAGES * plan.stage_bytes;  // 16 KB, used when a_ones
     uint8_t *sOnesB = sOnesA + (p.a_ones ? 128 * 128 : 0);           // BN x 128 B, used when b_ones_k
     uint64_t *bars = (uint64_t *)(sOnesB + (p.b_ones_k ? BN * 128 : 0));
-    uint64_t *full = bars, *empty = full + 4, *acc_full = empty + 4;
-    uint32_t *tmem_slot = (uint32_t *)(acc_full + 1);
+    uint64_t *full = bars, *empty = full + 4, *acc_full = empty + 4, *acc_empty = acc_full + 2, *drain = acc_empty + 2;
+    uint32_t *tmem_slot = (uint32_t *)(drain + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * 128, n0 = blockIdx.y * BN;
-    const int batch = blockIdx.z / p.n_split, split = blockIdx.z % p.n_split;
     const int kt_total = (p.K + kGemmBK - 1) / kGemmBK;
-    const int kt0 = split * p.kt_split, kt1 = min(kt0 + p.kt_split, kt_total);
-    const int nk = max(kt1 - kt0, 0);
-    const int ab = p.a_batched ? batch : 0;
-    const int bb = p.b_chunk ? batch * p.n_chunks + (int)blockIdx.x : (p.b_batched ? batch : 0);
-    const int a_k0 = p.a_kofs ? m0 : 0;           // offset of A's K coordinate
-    const int b_k0 = p.b_kofs ? m0 : 0, b_n0 = p.b_nofs ? m0 : n0;
     const int nb_load = p.b_ones ? BN / 64 - 1 : BN / 64;  // N-major B blocks loaded by TMA
-    const int kt_ones = kt_total - 1;                      // the A ones block's K tile (a_ones)
+    const int kt_ones = kt_total - 1;                      // the ones blocks' K tile (a_ones, b_ones_k)
 
-    // Constant blocks: the B ones block of every stage, the A ones block.
+    // Constant blocks: the B ones block of every stage, the A ones block, the K-major B ones block.
     if (p.b_ones) {
         for (int i = threadIdx.x; i < STAGES * BP * 64; i += kGemmThreads) {
             const int s = i / (BP * 64), part = (i / 64) % BP, k = i % 64;
@@ -192,20 +230,29 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], NORM ? 5 : 1);
+            mbar_init(&empty[s], NORM ? 1 + kEpiWarps : 1);
         }
-        mbar_init(acc_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kEpiWarps);
+        }
+        mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Launched after the previous pass without waiting for it: everything above touched only this
+    // CTA's shared and tensor memory. Every global read and write below comes after the previous
+    // kernel has completed (and so, transitively, every kernel before it).
+    pdl_launch_dependents();
+    pdl_wait_prerequisites();
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
@@ -217,41 +264,45 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
         }
         __syncwarp();
         int issued = 0;
-        for (int i = 0; i < nk; ++i) {
-            const int s = i % STAGES, kt = kt0 + i, k0 = kt * kGemmBK;
-            if (!mbar_wait_lazy(&empty[s], ((i / STAGES) & 1) ^ 1, abort_flag)) break;
-            if (elect_one()) {
-                uint8_t *st = sStage + (size_t)s * plan.stage_bytes;
-                const bool a_const = p.a_ones && kt == kt_ones;
-                const bool b_const = p.b_ones_k && kt == kt_ones;
-                const uint32_t bytes = (a_const ? 0u : AP * plan.a_bytes) +
-                                       (b_const ? 0u : (B_MN ? BP * (uint32_t)nb_load * 8192u : BP * plan.b_bytes));
-                mbar_arrive_expect_tx(&full[s], bytes);
-                for (int part = 0; part < AP && !a_const; ++part) {
-                    const CUtensorMap *m = part ? &mA2 : &mA;
-                    uint8_t *dst = st + part * plan.a_bytes;
-                    if (A_MN) {
-                        const int am = p.a_mlocal ? 0 : m0;
-                        tma_load_3d(dst, m, &full[s], am, a_k0 + k0, ab);
-                        tma_load_3d(dst + 8192, m, &full[s], am + 64, a_k0 + k0, ab);
-                    } else {
-                        tma_load_3d(dst, m, &full[s], a_k0 + k0, m0, ab);
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+            const GemmTile g = gemm_tile(p, BN, t);
+            for (int i = 0; i < g.nk; ++i, ++issued) {
+                const int s = issued % STAGES, kt = g.kt0 + i, k0 = kt * kGemmBK;
+                if (!mbar_wait_lazy(&empty[s], ((issued / STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                if (elect_one()) {
+                    uint8_t *st = sStage + (size_t)s * plan.stage_bytes;
+                    const bool a_const = p.a_ones && kt == kt_ones;
+                    const bool b_const = p.b_ones_k && kt == kt_ones;
+                    const uint32_t bytes = (a_const ? 0u : AP * plan.a_bytes) +
+                                           (b_const ? 0u : (B_MN ? BP * (uint32_t)nb_load * 8192u : BP * plan.b_bytes));
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    for (int part = 0; part < AP && !a_const; ++part) {
+                        const CUtensorMap *m = part ? &mA2 : &mA;
+                        uint8_t *dst = st + part * plan.a_bytes;
+                        if (A_MN) {
+                            const int am = p.a_mlocal ? 0 : g.m0;
+                            tma_load_3d(dst, m, &full[s], am, g.a_k0 + k0, g.ab);
+                            tma_load_3d(dst + 8192, m, &full[s], am + 64, g.a_k0 + k0, g.ab);
+                        } else {
+                            tma_load_3d(dst, m, &full[s], g.a_k0 + k0, g.m0, g.ab);
+                        }
+                    }
+                    for (int part = 0; part < BP && !b_const; ++part) {
+                        const CUtensorMap *m = part ? &mB2 : &mB;
+                        uint8_t *dst = st + AP * plan.a_bytes + part * plan.b_bytes;
+                        if (B_MN) {
+                            for (int j = 0; j < nb_load; ++j)
+                                tma_load_3d(dst + j * 8192, m, &full[s], g.b_n0 + 64 * j, g.b_k0 + k0, g.bb);
+                        } else {
+                            tma_load_3d(dst, m, &full[s], g.b_k0 + k0, g.b_n0, g.bb);
+                        }
                     }
                 }
-                for (int part = 0; part < BP && !b_const; ++part) {
-                    const CUtensorMap *m = part ? &mB2 : &mB;
-                    uint8_t *dst = st + AP * plan.a_bytes + part * plan.b_bytes;
-                    if (B_MN) {
-                        for (int j = 0; j < nb_load; ++j)
-                            tma_load_3d(dst + j * 8192, m, &full[s], b_n0 + 64 * j, b_k0 + k0, bb);
-                    } else {
-                        tma_load_3d(dst, m, &full[s], b_k0 + k0, b_n0, bb);
-                    }
-                }
+                __syncwarp();
             }
-            __syncwarp();
-            ++issued;
         }
+        // every issued copy has landed before the CTA can exit
         volatile int no_abort = 0;
         for (int i = max(issued - STAGES, 0); i < issued; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, &no_abort);
     } else if (warp == 1) {
@@ -260,85 +311,156 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
         // K-step of 16: K-major operands advance 32 B, MN-major operands 16 rows of 128 B
         constexpr uint32_t a_step = A_MN ? 2048 / 16 : 2, b_step = B_MN ? 2048 / 16 : 2;
         const uint32_t a_lbo = A_MN ? 8192 : 16, b_lbo = B_MN ? 8192 : 16;
+        int consumed = 0, local = 0;
         bool ok = true;
-        for (int i = 0; i < nk; ++i) {
-            const int s = i % STAGES, kt = kt0 + i;
-            if (!mbar_wait_all(&full[s], (i / STAGES) & 1, abort_flag)) { ok = false; break; }
+        for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++local) {
+            const GemmTile g = gemm_tile(p, BN, t);
+            const int b = local & 1;
+            const uint32_t acc = tmem + (uint32_t)b * 256;
+            // the epilogue has drained this accumulator buffer (two tiles ago)
+            if (!mbar_wait_all(&acc_empty[b], ((local >> 1) & 1) ^ 1, abort_flag)) break;
             tc_fence_after();
-            const uint32_t st = smem_u32(sStage) + (uint32_t)s * plan.stage_bytes;
-            const bool a_const = p.a_ones && kt == kt_ones;
-            const bool b_const = p.b_ones_k && kt == kt_ones;
-            const uint32_t a_hi = a_const ? smem_u32(sOnesA) : st;
-            const uint32_t a_lo = st + plan.a_bytes;
-            const uint32_t b_hi = b_const ? smem_u32(sOnesB) : st + AP * plan.a_bytes, b_lo = b_hi + plan.b_bytes;
-            if (elect_one()) {
-                const uint32_t acc0 = i > 0 ? 1u : 0u;
-                mma_ss_x4(tmem, make_sdesc(a_hi, a_lbo, 1024), make_sdesc(b_hi, b_lbo, 1024), idesc, acc0, a_step, b_step);
-                if (A_SPLIT && !a_const)
-                    mma_ss_x4(tmem, make_sdesc(a_lo, a_lbo, 1024), make_sdesc(b_hi, b_lbo, 1024), idesc, 1u, a_step, b_step);
-                if (B_SPLIT && !b_const)
-                    mma_ss_x4(tmem, make_sdesc(a_hi, a_lbo, 1024), make_sdesc(b_lo, b_lbo, 1024), idesc, 1u, a_step, b_step);
-                mma_commit(&empty[s]);
+            for (int i = 0; i < g.nk; ++i, ++consumed) {
+                const int s = consumed % STAGES, kt = g.kt0 + i;
+                if (!mbar_wait_all(&full[s], (consumed / STAGES) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t st = smem_u32(sStage) + (uint32_t)s * plan.stage_bytes;
+                const bool a_const = p.a_ones && kt == kt_ones;
+                const bool b_const = p.b_ones_k && kt == kt_ones;
+                const uint32_t a_hi = a_const ? smem_u32(sOnesA) : st;
+                const uint32_t a_lo = st + plan.a_bytes;
+                const uint32_t b_hi = b_const ? smem_u32(sOnesB) : st + AP * plan.a_bytes, b_lo = b_hi + plan.b_bytes;
+                if (elect_one()) {
+                    const uint32_t acc0 = i > 0 ? 1u : 0u;
+                    mma_ss_x4(acc, make_sdesc(a_hi, a_lbo, 1024), make_sdesc(b_hi, b_lbo, 1024), idesc, acc0, a_step, b_step);
+                    if (A_SPLIT && !a_const)
+                        mma_ss_x4(acc, make_sdesc(a_lo, a_lbo, 1024), make_sdesc(b_hi, b_lbo, 1024), idesc, 1u, a_step, b_step);
+                    if (B_SPLIT && !b_const)
+                        mma_ss_x4(acc, make_sdesc(a_hi, a_lbo, 1024), make_sdesc(b_lo, b_lbo, 1024), idesc, 1u, a_step, b_step);
+                    mma_commit(&empty[s]);
+                }
+                __syncwarp();
             }
+            if (!ok) break;
+            if (elect_one()) mma_commit(&acc_full[b]);
             __syncwarp();
         }
-        if (elect_one()) mma_commit(acc_full);
+        // every MMA has completed before the TMEM is freed
+        if (elect_one()) mma_commit(drain);
         __syncwarp();
-        (void)ok;
+        volatile int no_abort = 0;
+        mbar_wait(drain, 0, &no_abort);
     } else {
         // ------------------------------------------------------------------ epilogue
         const int q = warp & 3;             // TMEM lane quarter
+        const int ch = (warp - 2) >> 2;     // column half
         const int r = q * 32 + lane;        // row of the tile
-        const int row = m0 + r;             // row of the output
-        const bool valid = row < p.M;
-        const uint32_t t_row = tmem + (((uint32_t)q * 32u) << 16);
-        float sq = 0.f;                     // |x|^2 of this row (key feature map)
-        if (NORM) {
-            // A K-major: row r of each A tile, 8 chunks of 16 B; the whole K range is in this CTA
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % STAGES;
-                if (!mbar_wait_all(&full[s], (i / STAGES) & 1, abort_flag)) break;
-                const uint8_t *tile = sStage + (size_t)s * plan.stage_bytes;
-                float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+        const int HB = BN / 2;              // columns per half
+        const int cb = ch * HB;             // first column of this half
+        int consumed = 0, local = 0;
+        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
+            const GemmTile g = gemm_tile(p, BN, t);
+            const int row = g.m0 + r;       // row of the output
+            const bool valid = row < p.M;
+            const int b = local & 1;
+            const uint32_t t_row = tmem + (uint32_t)b * 256 + (((uint32_t)q * 32u) << 16);
+            bool ok = true;
+            float sq = 0.f;                 // |x|^2 of this row (key feature map)
+            if (NORM) {
+                // A K-major: row r of each A tile, 8 chunks of 16 B; the whole K range is in this tile
+                for (int i = 0; i < g.nk; ++i, ++consumed) {
+                    const int s = consumed % STAGES;
+                    if (!mbar_wait_all(&full[s], (consumed / STAGES) & 1, abort_flag)) { ok = false; break; }
+                    const uint8_t *tile = sStage + (size_t)s * plan.stage_bytes;
+                    float acc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float x[8];
-                    load_bf16x8((const uint16_t *)(tile + sw128_offset(r, ch)), x);
+                    for (int c = 0; c < 8; ++c) {
+                        float x[8];
+                        load_bf16x8((const uint16_t *)(tile + sw128_offset(r, c)), x);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc4[e & 3] = fmaf(x[e], x[e], acc4[e & 3]);
+                        for (int e = 0; e < 8; ++e) acc4[e & 3] = fmaf(x[e], x[e], acc4[e & 3]);
+                    }
+                    sq += (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[s]);
                 }
-                sq += (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
             }
-        }
-        const bool have = nk > 0 && mbar_wait_all(acc_full, 0, abort_flag);
-        tc_fence_after();
-        const size_t orow = (size_t)batch * p.M + row;  // output row (batch-major)
-        if (have) {
+            if (!ok) break;
+            if (g.nk == 0) {
+                // an empty split contributes zeros (kEpiPartial only; nothing was accumulated)
+                if (EPI == kEpiPartial && valid)
+                    for (int c0 = cb; c0 < cb + HB; c0 += 4)
+                        *(float4 *)(p.out_f32 + (((size_t)g.batch * p.n_split + g.split) * p.M + row) * p.ld_out + g.n0 +
+                                    c0) = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (!mbar_wait_all(&acc_full[b], (local >> 1) & 1, abort_flag)) break;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
+                continue;
+            }
+            if (!mbar_wait_all(&acc_full[b], (local >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            const size_t orow = (size_t)g.batch * (p.out_rows > 0 ? p.out_rows : p.M) + row;  // output row
             if (EPI == kEpiPhiQuery || EPI == kEpiPhiKey) {
+                // logit in log2 units: acc log2e (+ column offset for queries, - for keys)
+                const float csign = EPI == kEpiPhiQuery ? 1.f : -1.f;
+                auto col_off = [&](int c) { return p.colbias != nullptr ? csign * p.colbias[g.n0 + c] : 0.f; };
                 float shift;
                 if (EPI == kEpiPhiQuery) {
-                    float mx = -INFINITY;
+                    float mx = -INFINITY;  // over the whole row (both halves read it)
                     for (int c0 = 0; c0 < BN; c0 += 32) {
                         float v[32];
                         tmem_ld32(t_row + c0, v);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fmaf(v[e], kLog2e, col_off(c0 + e)));
                     }
-                    shift = mx * kLog2e;
+                    shift = mx;
                 } else {
-                    shift = 0.5f * sq * kLog2e + p.kc[batch];
+                    shift = 0.5f * sq * kLog2e + (p.kc != nullptr ? p.kc[g.batch] : 0.f);
                 }
-                for (int c0 = 0; c0 < BN; c0 += 32) {
+                for (int c0 = cb; c0 < cb + HB; c0 += 32) {
                     float v[32];
                     tmem_ld32(t_row + c0, v);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = exp2f(fmaf(v[e], kLog2e, -shift));
+                    for (int e = 0; e < 32; ++e) v[e] = exp2f(fmaf(v[e], kLog2e, col_off(c0 + e) - shift));
                     if (valid) {
-                        const size_t o = orow * p.ld_out + n0 + c0;
+                        const size_t o = orow * p.ld_out + g.n0 + c0;
 #pragma unroll
                         for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
+                    }
+                }
+            } else if (EPI == kEpiRelu) {
+                for (int c0 = cb; c0 < cb + HB; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(t_row + c0, v);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = fmaxf(v[e], 0.f);
+                    if (valid) {
+                        const size_t o = orow * p.ld_out + g.n0 + c0;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
+                    }
+                }
+            } else if (EPI == kEpiTrigQ || EPI == kEpiTrigK) {
+                // columns [0, N) of the row hold sin, [N, 2N) cos, of the same projections
+                const float scale = EPI == kEpiTrigK ? exp2f(0.5f * sq * kLog2e) : 1.f;
+                for (int c0 = cb; c0 < cb + HB; c0 += 32) {
+                    float v[32], c[32];
+                    tmem_ld32(t_row + c0, v);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        float sn, cs;
+                        sincosf(v[e], &sn, &cs);
+                        v[e] = sn * scale;
+                        c[e] = cs * scale;
+                    }
+                    if (valid) {
+                        const size_t o = orow * p.ld_out + g.n0 + c0;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
+                            store_split8(p.out_hi + o + p.N + 8 * j, p.out_lo + o + p.N + 8 * j, &c[8 * j]);
+                        }
                     }
                 }
             } else if (EPI == kEpiGS) {
@@ -346,42 +468,57 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
                 float den = tmem_ld1(t_row + p.d);
                 if (p.addend != nullptr && valid) den += p.addend[orow * p.ld_add + p.d];
                 const float inv = 1.0f / den;
+                // the half that writes s (column d) takes the dot product over all d columns; the
+                // other half only forms g over its own columns
+                const bool owns_s = p.d >= cb && p.d < cb + HB;
                 float dot = 0.f;
                 const uint16_t *dO = p.side_hi + orow * p.ld_side;
-                for (int c0 = 0; c0 < p.d; c0 += 32) {
-                    float v[32], g[32];
+                for (int c0 = owns_s ? 0 : cb; c0 < min(cb + HB, p.d); c0 += 32) {
+                    float v[32], gg[32];
                     acc_row32(t_row, c0, p, orow, 0, valid, v);
                     if (valid) {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) load_bf16x8(dO + c0 + 8 * j, &g[8 * j]);
+                        for (int j = 0; j < 4; ++j) load_bf16x8(dO + c0 + 8 * j, &gg[8 * j]);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) g[e] = 0.f;
+                        for (int e = 0; e < 32; ++e) gg[e] = 0.f;
                     }
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        dot = fmaf(g[e], v[e] * inv, dot);
-                        g[e] *= inv;
+                        dot = fmaf(gg[e], v[e] * inv, dot);
+                        gg[e] *= inv;
                     }
-                    if (valid) {
+                    if (valid && c0 >= cb) {
                         const size_t o = orow * p.ld_out + c0;
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &g[8 * j]);
+                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &gg[8 * j]);
                     }
                 }
                 if (valid) {
-                    const float s = -dot * inv;
-                    for (int c0 = p.d; c0 < BN; c0 += 8) {
-                        float z[8] = {c0 == p.d ? s : 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    const float sv = -dot * inv;
+                    for (int c0 = max(cb, p.d); c0 < cb + HB; c0 += 8) {
+                        float z[8] = {c0 == p.d ? sv : 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                         store_split8(p.out_hi + orow * p.ld_out + c0, p.out_lo + orow * p.ld_out + c0, z);
+                    }
+                }
+            } else if (EPI == kEpiOut) {
+                const float inv = 1.0f / tmem_ld1(t_row + p.d);
+                for (int c0 = cb; c0 < min(cb + HB, p.d); c0 += 32) {
+                    float v[32];
+                    tmem_ld32(t_row + c0, v);
+                    if (valid) {
+                        float4 *o = (float4 *)(p.out_f32 + orow * p.ld_out + c0);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            o[j] = make_float4(v[4 * j] * inv, v[4 * j + 1] * inv, v[4 * j + 2] * inv, v[4 * j + 3] * inv);
                     }
                 }
             } else if (EPI == kEpiT) {
                 float tsum = 0.f;
-                const uint16_t *ph = p.side_hi + orow * p.ld_side + n0, *pl = p.side_lo + orow * p.ld_side + n0;
-                for (int c0 = 0; c0 < BN; c0 += 32) {
+                const uint16_t *ph = p.side_hi + orow * p.ld_side + g.n0, *pl = p.side_lo + orow * p.ld_side + g.n0;
+                for (int c0 = cb; c0 < cb + HB; c0 += 32) {
                     float v[32];
-                    acc_row32(t_row, c0, p, orow, n0, valid, v);
+                    acc_row32(t_row, c0, p, orow, g.n0, valid, v);
                     if (valid) {
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
@@ -394,18 +531,18 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
                                 tsum += v[8 * j + e];
                             }
                         }
-                        const size_t o = orow * p.ld_out + n0 + c0;
+                        const size_t o = orow * p.ld_out + g.n0 + c0;
 #pragma unroll
                         for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
                     }
                 }
-                if (valid) p.rowsum[orow] = tsum;
+                if (valid) p.rowsum[2 * orow + ch] = tsum;  // two partial sums per row
             } else if (EPI == kEpiDX) {
-                const float ts = valid ? p.rowsum[orow] : 0.f;
-                const uint16_t *x = p.side_hi + orow * p.ld_side + n0;
-                for (int c0 = 0; c0 < BN; c0 += 32) {
+                const float ts = valid ? p.rowsum[2 * orow] + p.rowsum[2 * orow + 1] : 0.f;
+                const uint16_t *x = p.side_hi + orow * p.ld_side + g.n0;
+                for (int c0 = cb; c0 < cb + HB; c0 += 32) {
                     float v[32];
-                    acc_row32(t_row, c0, p, orow, n0, valid, v);
+                    acc_row32(t_row, c0, p, orow, g.n0, valid, v);
                     if (valid) {
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
@@ -414,48 +551,49 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
 #pragma unroll
                             for (int e = 0; e < 8; ++e) v[8 * j + e] = fmaf(-xv[e], ts, v[8 * j + e]);
                         }
-                        float4 *o = (float4 *)(p.out_f32 + orow * p.ld_out + n0 + c0);
+                        float4 *o = (float4 *)(p.out_f32 + orow * p.ld_out + g.n0 + c0);
 #pragma unroll
                         for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
                     }
                 }
             } else if (EPI == kEpiMask) {
-                // A chunk's 128 x 128 tile: row r is the chunk's query r, column j its key j
-                for (int c0 = 0; c0 < BN; c0 += 32) {
+                // row = query index, column = key index (the chunk's own keys when b_nofs)
+                const int col0 = p.b_nofs ? g.m0 : g.n0;
+                for (int c0 = cb; c0 < cb + HB; c0 += 32) {
                     float v[32];
                     tmem_ld32(t_row + c0, v);
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        if (c0 + e > r) v[e] = 0.f;
+                        if (col0 + c0 + e > row) v[e] = 0.f;
                     if (valid) {
-                        const size_t o = orow * p.ld_out + c0;
+                        const size_t o = orow * p.ld_out + g.n0 + c0;
 #pragma unroll
                         for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
                     }
                 }
             } else {
                 // kEpiF32 (rows of batch) and kEpiPartial (rows of batch * n_split + split)
-                const size_t prow = EPI == kEpiPartial ? (size_t)blockIdx.z * p.M + row : orow;
-                for (int c0 = 0; c0 < BN; c0 += 32) {
+                const size_t prow = EPI == kEpiPartial ? ((size_t)g.batch * p.n_split + g.split) * p.M + row : orow;
+                for (int c0 = cb; c0 < cb + HB; c0 += 32) {
                     float v[32];
-                    acc_row32(t_row, c0, p, orow, n0, valid, v);
+                    acc_row32(t_row, c0, p, orow, g.n0, valid, v);
                     if (valid) {
-                        float4 *o = (float4 *)(p.out_f32 + prow * p.ld_out + n0 + c0);
+                        float4 *o = (float4 *)(p.out_f32 + prow * p.ld_out + g.n0 + c0);
 #pragma unroll
                         for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
                     }
                 }
             }
-        } else if (EPI == kEpiPartial && valid) {
-            // an empty split contributes zeros
-            for (int c0 = 0; c0 < BN; c0 += 4)
-                *(float4 *)(p.out_f32 + ((size_t)blockIdx.z * p.M + row) * p.ld_out + n0 + c0) = make_float4(0.f, 0.f, 0.f, 0.f);
+            // this warp has read its part of the accumulator buffer
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 256);
+    if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // Sums the n_split partial tiles of each batch ([batch][split][M][Np] fp32, M = m features,
@@ -487,6 +625,35 @@ __global__ void __launch_bounds__(256) k_gemm_reduce_image(const float *__restri
         *(uint32_t *)(img_hi + o) = h;
         *(uint32_t *)(img_lo + o) = l;
     }
+}
+
+// Sums the n_split partial tiles of each batch ([batch * n_split + s][M][Np] fp32) in split order
+// into [batch][M][Np] fp32. One thread per element.
+__global__ void __launch_bounds__(256) k_gemm_sum_partials(const float *__restrict__ part, int n_split, size_t per_batch,
+                                                           float *__restrict__ out) {
+    const size_t i = (size_t)blockIdx.x * 256 + threadIdx.x;
+    if (i >= per_batch) return;
+    const size_t b = blockIdx.y;
+    float acc = 0.f;
+    for (int s = 0; s < n_split; ++s) acc += part[(b * n_split + s) * per_batch + i];
+    out[b * per_batch + i] = acc;
+}
+
+// Per-feature exponent offsets of the sequence-parallel path, log2 units:
+// c_r = (|w_r|^2 / 2 - kSpKeyHeadroom) log2e. Since u_r(k) = w_r.k - |k|^2/2 <= |w_r|^2 / 2 for every
+// key, 2^(u_r log2e - c_r) <= e^kSpKeyHeadroom: no key feature can overflow, and the offsets depend
+// on W alone, so every rank's partial state is on the same scale.
+constexpr float kSpKeyHeadroom = 40.f;
+
+__global__ void k_feature_offsets(const uint16_t *__restrict__ W, int m, int d, float *__restrict__ c) {
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= m) return;
+    float acc = 0.f;
+    for (int e = 0; e < d; ++e) {
+        const float w = __uint_as_float((uint32_t)W[(size_t)r * d + e] << 16);
+        acc = fmaf(w, w, acc);
+    }
+    c[r] = (0.5f * acc - kSpKeyHeadroom) * kLog2e;
 }
 
 // Exclusive prefix (forward) or suffix (reverse) over the n_chunks per-chunk partial states of
@@ -535,14 +702,25 @@ static cudaError_t launch_gemm_t(const CUtensorMap &mA, const CUtensorMap &mA2, 
     const size_t smem = 1024 + (size_t)plan.stages * plan.stage_bytes + cb + 256;
     auto kern = k_gemm<A_MN, B_MN, A_SPLIT, B_SPLIT, EPI>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    const dim3 grid((p.M + 127) / 128, (p.N + BN - 1) / BN, batches * p.n_split);
-    kern<<<grid, kGemmThreads, smem, st>>>(mA, mA2, mB, mB2, p, BN);
-    return cudaGetLastError();
+    const int tiles = gemm_tiles(p, BN, batches);
+    const dim3 grid(std::max(1, std::min(tiles, num_sms())));
+    return launch_after_previous(kern, grid, dim3(kGemmThreads), smem, st, mA, mA2, mB, mB2, p, BN, tiles);
 }
 
 cudaError_t launch_scan_image(const float *part, int n_chunks, int m, int Np, int reverse, uint16_t *hi, uint16_t *lo,
                               int batches, cudaStream_t st) {
     k_gemm_scan_image<<<dim3(Np / 32, m / 64, batches), dim3(32, 8), 0, st>>>(part, n_chunks, m, Np, reverse, hi, lo);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sum_partials(const float *part, int n_split, size_t per_batch, float *out, int batches,
+                               cudaStream_t st) {
+    k_gemm_sum_partials<<<dim3((unsigned)((per_batch + 255) / 256), batches), 256, 0, st>>>(part, n_split, per_batch, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_feature_offsets(const void *W, int m, int d, float *c, cudaStream_t st) {
+    k_feature_offsets<<<(m + 127) / 128, 128, 0, st>>>((const uint16_t *)W, m, d, c);
     return cudaGetLastError();
 }
 

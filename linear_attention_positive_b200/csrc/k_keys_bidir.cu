@@ -213,6 +213,7 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
     uint32_t *tmem_slot = (uint32_t *)(drain + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
 
+    pdl_launch_dependents();  // the state image kernel may stage its launch meanwhile
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nt = p.f.nt;
     const int f0 = blockIdx.x * p.f.T, f1 = min(f0 + p.f.T, p.f.total);

@@ -18,6 +18,8 @@
 //
 // The causal path keeps the fp32 per-segment state blocks below (state_floats, state_image_offset).
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace favor {
@@ -65,6 +67,8 @@ __device__ __forceinline__ float pow2i(float e) {
 // fp16. Grid: (chunks / 128, heads).
 __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
     __shared__ float sC, sScale, sRed[kImageThreads / 32];
+    pdl_launch_dependents();   // the query kernel may start its projections meanwhile
+    pdl_wait_prerequisites();  // the key kernel's partial states are complete and visible
     const int bh = blockIdx.y;
     const int c_first = flat_first_cta(p.f, bh), c_last = flat_last_cta(p.f, bh);
     const int halves = p.m / 128, nhs = p.d / 64;
@@ -331,7 +335,9 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             mbar_wait(w_full, 0, &no_abort);
         } else if (warp == 14 && n_items > 0) {
             // State image of each (head, value half) group, once the previous group's output
-            // MMAs have finished with it.
+            // MMAs have finished with it. The image kernel (the launch before this one) must have
+            // completed first: only this warp reads its output.
+            pdl_wait_prerequisites();
             int groups = 0;
             for (int g = 0; g < n_items; ++g) {
                 const ItemInfo it = item_info<NH>(g, f0, f1, nt);
@@ -523,10 +529,28 @@ int num_sms() {
     return n;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled before the previous
+// kernel on the stream completes; it waits (griddepcontrol.wait) before reading that kernel's output.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_after_previous(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                         Args &&...args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_state_image(const ImageParams &p, int BH, cudaStream_t st) {
     const int chunks = (p.d / 64) * (p.m / 128) * 2 * kImgRows * 8;
-    k_state_image<<<dim3((chunks + kImageThreads - 1) / kImageThreads, BH), kImageThreads, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_after_previous(k_state_image, dim3((chunks + kImageThreads - 1) / kImageThreads, BH),
+                                 dim3(kImageThreads), 0, st, p);
 }
 
 // The register split of k_query_out (88 + 2 x 184 + 56 per warpgroup lane) adds up to the 128 per
@@ -546,8 +570,7 @@ static cudaError_t launch_query_t(const CUtensorMap &mQ, const CUtensorMap &mW, 
     if (checked < 0) return cudaErrorInvalidConfiguration;
     const size_t sm = query_smem<D>(p.m);
     cudaFuncSetAttribute(k_query_out<D, POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_query_out<D, POLY><<<grid, kQueryThreads, sm, st>>>(mQ, mW, mO, p);
-    return cudaGetLastError();
+    return launch_after_previous(k_query_out<D, POLY>, grid, dim3(kQueryThreads), sm, st, mQ, mW, mO, p);
 }
 
 // Persistent launch: at most one CTA per SM, each over a contiguous head-major range of tiles.

@@ -16,6 +16,15 @@ workloads the Performer pages describe):
    long sequences stand-in); Q, K then scaled by d^-1/4. W seed 4, data seed 14.
 5. ``bidir-bf16-L16384-d128-fwdbwd``: B=2, H=8, L=16384, d=128, m=256, bf16 forward + backward;
    upstream gradient dO iid N(0,1). W seed 5, data seed 15.
+
+Two more shapes measure the other feature maps (not among the method's five configurations):
+
+6. ``bidir-bf16-L4096-relu``: workload 2's shape and inputs, generalised attention with ReLU
+   features.
+7. ``bidir-bf16-L4096-trig``: workload 2's shape, trigonometric features, inputs 0.5 * N(0, 1)
+   (with unit-variance inputs the trigonometric normaliser crosses zero). Data seed 17.
+8. ``bidir-bf16-L4096-seqpar``: workload 2 through the sequence-parallel calls (partial state,
+   then outputs from the state) on one GPU.
 """
 
 from dataclasses import dataclass, replace
@@ -38,6 +47,8 @@ class Workload:
     data_seed: int
     scale: float = 1.0  # std of the Gaussian rows before the d^-1/4 scaling of Q and K
     rotated: bool = False
+    feature_map: str = "positive"  # "positive", "relu" or "trig"
+    sequence_parallel: bool = False  # through the state / output calls of the sequence-parallel path
 
     @property
     def tokens(self):
@@ -54,6 +65,11 @@ WORKLOADS = {
     4: Workload("causal-bf16-L65536-protein", 1, 16, 65536, 64, 256, True, "bf16", False, 4, 14,
                 scale=0.5, rotated=True),
     5: Workload("bidir-bf16-L16384-d128-fwdbwd", 2, 8, 16384, 128, 256, False, "bf16", True, 5, 15),
+    6: Workload("bidir-bf16-L4096-relu", 8, 8, 4096, 64, 256, False, "bf16", False, 2, 12, feature_map="relu"),
+    7: Workload("bidir-bf16-L4096-trig", 8, 8, 4096, 64, 256, False, "bf16", False, 2, 17, scale=0.5,
+                feature_map="trig"),
+    8: Workload("bidir-bf16-L4096-seqpar", 8, 8, 4096, 64, 256, False, "bf16", False, 2, 12,
+                sequence_parallel=True),
 }
 
 

@@ -165,3 +165,25 @@ def test_bf16_bidirectional_backward_requires_the_forward_context(favor_lib):
     p = ctypes.c_void_p(256)
     assert favor_lib.favor_bwd(ctypes.byref(sh), p, p, p, p, p, p, None, 0, p, p, p, p, ws, None, None) == \
         api.FAVOR_ERR_WORKSPACE
+
+
+def test_feature_map_workspace_and_refusals(favor_lib):
+    """Other feature maps are built for the bf16 bidirectional forward only; elsewhere the sizes are
+    zero and the calls refuse before any launch."""
+    sh = api.make_shape(1, 2, 1000, 64, 256, api.FAVOR_BF16)
+    relu, trig = api.make_opts(feature_map=api.FAVOR_MAP_RELU), api.make_opts(feature_map=api.FAVOR_MAP_TRIG)
+    wr, wt = api.workspace_size(sh, opts=relu), api.workspace_size(sh, opts=trig)
+    assert 0 < wr < wt and wr % 256 == 0  # the trigonometric map carries 2m features
+    assert api.workspace_size(sh, causal=True, opts=relu) == 0
+    assert api.workspace_size(sh, backward=True, opts=trig) == 0
+    f32 = api.make_shape(1, 2, 1000, 64, 256, api.FAVOR_F32)
+    assert api.workspace_size(f32, opts=relu) == 0
+    bad = api.make_opts(feature_map=7)
+    assert api.workspace_size(sh, opts=bad) == 0
+    p = ctypes.c_void_p(256)
+    assert favor_lib.favor_fwd(ctypes.byref(sh), p, p, p, p, 1, p, None, p, 1 << 30, ctypes.byref(relu), None) == \
+        api.FAVOR_ERR_UNSUPPORTED
+    assert favor_lib.favor_fwd(ctypes.byref(sh), p, p, p, p, 0, p, None, p, 1 << 30, ctypes.byref(bad), None) == \
+        api.FAVOR_ERR_UNSUPPORTED
+    assert favor_lib.favor_bwd(ctypes.byref(sh), p, p, p, p, p, p, p, 0, p, p, p, p, 1 << 30, ctypes.byref(relu),
+                               None) == api.FAVOR_ERR_UNSUPPORTED
