@@ -145,7 +145,9 @@ FAVOR_API size_t favor_ctx_size(const favor_shape *shape, int causal);
  *   W            : device, [m,d] in shape->dtype (the caller rounds the fp64 draw)
  *   causal       : 0 or 1
  *   out          : device, fp32 [B,H,L,d]; fully written
- *   ctx          : device, favor_ctx_size bytes, or NULL when no backward will follow
+ *   ctx          : device, favor_ctx_size bytes, or NULL when no backward will follow (the bf16
+ *                  forward writes the per-head key reference, and the causal path the per-key
+ *                  -|k|^2/2, into it)
  *   workspace    : device, >= favor_workspace_size(shape, causal, 0, opts) bytes, 256-B aligned
  *   stream       : cudaStream_t as void*
  * Numerics: query features are stabilised by their row maximum. Key features, bidirectional: each
@@ -163,12 +165,21 @@ FAVOR_API favor_status favor_fwd(const favor_shape *shape, const void *Q, const 
  * (Derived by the chain rule from the forward definition; the pages print no backward.)
  *
  *   Q, K, V, W   : as passed to favor_fwd
- *   out          : device, fp32 [B,H,L,d], the forward output (validated; the kernels recompute
- *                  out_i from the features and state they differentiate through)
+ *   out          : device, fp32 [B,H,L,d], the forward output (validated, not read: the kernels
+ *                  recompute out_i at the precision of the gradient passes)
  *   dout         : device, [B,H,L,d] in shape->dtype, upstream gradient
- *   ctx          : device, the context written by favor_fwd with the same inputs
+ *   ctx          : bf16: device, required, the context favor_fwd wrote for the same inputs and
+ *                  mask; the backward reads the per-head key reference from it (the largest key
+ *                  stabiliser of the forward), which keeps its key features below 2^19.
+ *                  fp32: not read (may be NULL); the fp32 kernels recompute everything.
  *   dQ, dK, dV   : device, fp32 [B,H,L,d]; fully written
  *   workspace    : device, >= favor_workspace_size(shape, causal, 1, opts) bytes
+ * bf16 arithmetic: every operand computed on the way (phi(Q), phi(K), the state, [g | s], the
+ * query-side sums, phi * dphi) is a pair of bf16 values hi + lo, and each product is three tcgen05
+ * MMAs (two where one side is an exact bf16 input), accumulated in fp32: the gradients' largest
+ * entries are 50-90x their RMS, beyond what single 16-bit operands resolve within 2e-2 x RMS.
+ * Returns FAVOR_ERR_WORKSPACE for a missing (bf16) context or short workspace, FAVOR_ERR_UNSUPPORTED
+ * for a feature map other than the positive one or an unsupported shape (bf16 causal: d = 64).
  */
 FAVOR_API favor_status favor_bwd(const favor_shape *shape, const void *Q, const void *K, const void *V,
                        const void *W, const float *out, const void *dout, const void *ctx,

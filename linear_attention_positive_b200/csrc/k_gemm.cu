@@ -75,13 +75,18 @@ struct GemmSmem {
     int stages;
 };
 
-// Stage ring that fits next to the constant blocks (const_bytes) in about 196 KB.
+// Epilogue staging: one 32-row x 32-column tile per epilogue warp (hi | lo bf16, or fp32), 4 KB.
+constexpr uint32_t kGemmStageOut = 4096;
+constexpr uint32_t kGemmSmemMax = 232448;  // dynamic shared memory per CTA on sm_100
+
+// Stage ring (2 to 4 stages) that fits next to the constant blocks and the epilogue staging.
 __host__ __device__ inline GemmSmem gemm_smem_plan(int BN, int a_parts, int b_parts, uint32_t const_bytes) {
     GemmSmem g;
     g.a_bytes = 128u * 128u;                      // 128 rows x 64 k x 2 B
     g.b_bytes = (uint32_t)BN * 128u;              // BN x 64 k x 2 B
     g.stage_bytes = a_parts * g.a_bytes + b_parts * g.b_bytes;
-    int s = (int)((196u * 1024u - const_bytes) / g.stage_bytes);
+    const uint32_t budget = kGemmSmemMax - 1024u - 512u - 8u * kGemmStageOut - const_bytes;
+    int s = (int)(budget / g.stage_bytes);
     g.stages = s < 2 ? 2 : (s > 4 ? 4 : s);
     return g;
 }
@@ -178,7 +183,8 @@ __host__ __device__ inline int gemm_tiles(const GemmArgs &p, int BN, int batches
 template <bool A_MN, bool B_MN, bool A_SPLIT, bool B_SPLIT, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
-       const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mB2, GemmArgs p, int BN,
+       const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mB2,
+       const __grid_constant__ CUtensorMap mO, const __grid_constant__ CUtensorMap mO2, GemmArgs p, int BN,
        int n_tiles) {
     constexpr int AP = A_SPLIT ? 2 : 1, BP = B_SPLIT ? 2 : 1;
     constexpr bool NORM = EPI == kEpiPhiKey || EPI == kEpiTrigK;
@@ -190,7 +196,8 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
     uint8_t *sStage = smem;
     uint8_t *sOnesA = sStage + (size_t)STAGES * plan.stage_bytes;  // 16 KB, used when a_ones
     uint8_t *sOnesB = sOnesA + (p.a_ones ? 128 * 128 : 0);           // BN x 128 B, used when b_ones_k
-    uint64_t *bars = (uint64_t *)(sOnesB + (p.b_ones_k ? BN * 128 : 0));
+    uint8_t *sOut = sOnesB + (p.b_ones_k ? BN * 128 : 0);           // 8 x kGemmStageOut
+    uint64_t *bars = (uint64_t *)(sOut + 8 * kGemmStageOut);
     uint64_t *full = bars, *empty = full + 4, *acc_full = empty + 4, *acc_empty = acc_full + 2, *drain = acc_empty + 2;
     uint32_t *tmem_slot = (uint32_t *)(drain + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
@@ -357,6 +364,49 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
         const int r = q * 32 + lane;        // row of the tile
         const int HB = BN / 2;              // columns per half
         const int cb = ch * HB;             // first column of this half
+        // Outputs leave through this warp's staging tile (its 32 rows x 32 columns) by TMA stores;
+        // rows past the output's extent are clipped by the tensor map.
+        uint8_t *stg = sOut + (size_t)(warp - 2) * kGemmStageOut;
+        if (lane == 0) {
+            prefetch_tensormap(&mO);
+            prefetch_tensormap(&mO2);
+        }
+        auto stage_free = [&]() {
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+        };
+        // this row's 32 values as hi and lo bf16 at (column, row block, batch coordinate) of the output
+        // staging layouts are the tensor maps' swizzles: 16-byte chunk j of row r at chunk
+        // j ^ ((r >> 1) & 3) of its 64-byte row (bf16), j ^ (r & 7) of its 128-byte row (fp32)
+        auto put_split = [&](const float *v, int col, int row0, int bz) {
+            stage_free();
+            uint8_t *h = stg + lane * 64, *l = stg + 2048 + lane * 64;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t off = (uint32_t)(j ^ ((lane >> 1) & 3)) << 4;
+                store_split8((uint16_t *)(h + off), (uint16_t *)(l + off), v + 8 * j);
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(&mO, stg, col, row0, bz);
+                tma_store_3d(&mO2, stg + 2048, col, row0, bz);
+                bulk_commit_group();
+            }
+        };
+        auto put_f32 = [&](const float *v, int col, int row0, int bz) {
+            stage_free();
+            uint8_t *o = stg + lane * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *(float4 *)(o + ((j ^ (lane & 7)) << 4)) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(&mO, stg, col, row0, bz);
+                bulk_commit_group();
+            }
+        };
         int consumed = 0, local = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
             const GemmTile g = gemm_tile(p, BN, t);
@@ -364,6 +414,8 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
             const bool valid = row < p.M;
             const int b = local & 1;
             const uint32_t t_row = tmem + (uint32_t)b * 256 + (((uint32_t)q * 32u) << 16);
+            const int row0 = g.m0 + q * 32;  // first row of this warp's block (within the batch)
+            const int bz = EPI == kEpiPartial ? g.batch * p.n_split + g.split : g.batch;  // output batch
             bool ok = true;
             float sq = 0.f;                 // |x|^2 of this row (key feature map)
             if (NORM) {
@@ -388,10 +440,12 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
             if (!ok) break;
             if (g.nk == 0) {
                 // an empty split contributes zeros (kEpiPartial only; nothing was accumulated)
-                if (EPI == kEpiPartial && valid)
-                    for (int c0 = cb; c0 < cb + HB; c0 += 4)
-                        *(float4 *)(p.out_f32 + (((size_t)g.batch * p.n_split + g.split) * p.M + row) * p.ld_out + g.n0 +
-                                    c0) = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (EPI == kEpiPartial) {
+                    float z[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) z[e] = 0.f;
+                    for (int c0 = cb; c0 < cb + HB; c0 += 32) put_f32(z, g.n0 + c0, row0, bz);
+                }
                 if (!mbar_wait_all(&acc_full[b], (local >> 1) & 1, abort_flag)) break;
                 tc_fence_before();
                 __syncwarp();
@@ -423,11 +477,7 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
                     tmem_ld32(t_row + c0, v);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] = exp2f(fmaf(v[e], kLog2e, col_off(c0 + e) - shift));
-                    if (valid) {
-                        const size_t o = orow * p.ld_out + g.n0 + c0;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
-                    }
+                    put_split(v, g.n0 + c0, row0, bz);
                 }
             } else if (EPI == kEpiRelu) {
                 for (int c0 = cb; c0 < cb + HB; c0 += 32) {
@@ -435,11 +485,7 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
                     tmem_ld32(t_row + c0, v);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] = fmaxf(v[e], 0.f);
-                    if (valid) {
-                        const size_t o = orow * p.ld_out + g.n0 + c0;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
-                    }
+                    put_split(v, g.n0 + c0, row0, bz);
                 }
             } else if (EPI == kEpiTrigQ || EPI == kEpiTrigK) {
                 // columns [0, N) of the row hold sin, [N, 2N) cos, of the same projections
@@ -454,14 +500,8 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
                         v[e] = sn * scale;
                         c[e] = cs * scale;
                     }
-                    if (valid) {
-                        const size_t o = orow * p.ld_out + g.n0 + c0;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
-                            store_split8(p.out_hi + o + p.N + 8 * j, p.out_lo + o + p.N + 8 * j, &c[8 * j]);
-                        }
-                    }
+                    put_split(v, g.n0 + c0, row0, bz);
+                    put_split(c, g.n0 + c0 + p.N, row0, bz);
                 }
             } else if (EPI == kEpiGS) {
                 // acc columns: num [0, d), den at d. Output [g | s | 0 ...] over BN columns.
@@ -488,17 +528,16 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
                         dot = fmaf(gg[e], v[e] * inv, dot);
                         gg[e] *= inv;
                     }
-                    if (valid && c0 >= cb) {
-                        const size_t o = orow * p.ld_out + c0;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &gg[8 * j]);
-                    }
+                    if (c0 >= cb) put_split(gg, c0, row0, bz);
                 }
-                if (valid) {
+                {
                     const float sv = -dot * inv;
-                    for (int c0 = max(cb, p.d); c0 < cb + HB; c0 += 8) {
-                        float z[8] = {c0 == p.d ? sv : 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        store_split8(p.out_hi + orow * p.ld_out + c0, p.out_lo + orow * p.ld_out + c0, z);
+                    for (int c0 = max(cb, p.d); c0 < cb + HB; c0 += 32) {
+                        float z[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) z[e] = 0.f;
+                        if (c0 == p.d) z[0] = sv;
+                        put_split(z, c0, row0, bz);
                     }
                 }
             } else if (EPI == kEpiOut) {
@@ -506,12 +545,9 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
                 for (int c0 = cb; c0 < min(cb + HB, p.d); c0 += 32) {
                     float v[32];
                     tmem_ld32(t_row + c0, v);
-                    if (valid) {
-                        float4 *o = (float4 *)(p.out_f32 + orow * p.ld_out + c0);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            o[j] = make_float4(v[4 * j] * inv, v[4 * j + 1] * inv, v[4 * j + 2] * inv, v[4 * j + 3] * inv);
-                    }
+                    for (int e = 0; e < 32; ++e) v[e] *= inv;
+                    put_f32(v, c0, row0, bz);
                 }
             } else if (EPI == kEpiT) {
                 float tsum = 0.f;
@@ -531,10 +567,8 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
                                 tsum += v[8 * j + e];
                             }
                         }
-                        const size_t o = orow * p.ld_out + g.n0 + c0;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
                     }
+                    put_split(v, g.n0 + c0, row0, bz);
                 }
                 if (valid) p.rowsum[2 * orow + ch] = tsum;  // two partial sums per row
             } else if (EPI == kEpiDX) {
@@ -551,10 +585,8 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
 #pragma unroll
                             for (int e = 0; e < 8; ++e) v[8 * j + e] = fmaf(-xv[e], ts, v[8 * j + e]);
                         }
-                        float4 *o = (float4 *)(p.out_f32 + orow * p.ld_out + g.n0 + c0);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
                     }
+                    put_f32(v, g.n0 + c0, row0, bz);
                 }
             } else if (EPI == kEpiMask) {
                 // row = query index, column = key index (the chunk's own keys when b_nofs)
@@ -565,23 +597,14 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
                         if (col0 + c0 + e > row) v[e] = 0.f;
-                    if (valid) {
-                        const size_t o = orow * p.ld_out + g.n0 + c0;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) store_split8(p.out_hi + o + 8 * j, p.out_lo + o + 8 * j, &v[8 * j]);
-                    }
+                    put_split(v, g.n0 + c0, row0, bz);
                 }
             } else {
                 // kEpiF32 (rows of batch) and kEpiPartial (rows of batch * n_split + split)
-                const size_t prow = EPI == kEpiPartial ? ((size_t)g.batch * p.n_split + g.split) * p.M + row : orow;
                 for (int c0 = cb; c0 < cb + HB; c0 += 32) {
                     float v[32];
                     acc_row32(t_row, c0, p, orow, g.n0, valid, v);
-                    if (valid) {
-                        float4 *o = (float4 *)(p.out_f32 + prow * p.ld_out + g.n0 + c0);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                    }
+                    put_f32(v, g.n0 + c0, row0, bz);
                 }
             }
             // this warp has read its part of the accumulator buffer
@@ -589,6 +612,9 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[b]);
         }
+        // every bulk store of this warp has completed before the CTA exits
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
@@ -694,17 +720,58 @@ __global__ void __launch_bounds__(256) k_gemm_scan_image(const float *__restrict
 
 // ------------------------------------------------------------------------------------ host side
 
+// Output tensor map of an epilogue: [batches][rows][ld] (bf16 or fp32) written from 32 x 32 x 1
+// staging boxes with 64-byte (bf16) or 128-byte (fp32) rows, in the matching swizzle.
+typedef CUresult (*GemmEncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static bool gemm_out_map(CUtensorMap *map, const void *base, bool f32, int ld, int rows, int batches) {
+    static GemmEncodeFn fn = nullptr;
+    if (fn == nullptr) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        fn = (GemmEncodeFn)ptr;
+    }
+    if (base == nullptr) return false;
+    const cuuint64_t es = f32 ? 4 : 2;
+    const cuuint64_t dims[3] = {(cuuint64_t)ld, (cuuint64_t)rows, (cuuint64_t)batches};
+    const cuuint64_t strides[2] = {(cuuint64_t)ld * es, (cuuint64_t)ld * rows * es};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base),
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool A_MN, bool B_MN, bool A_SPLIT, bool B_SPLIT, int EPI>
 static cudaError_t launch_gemm_t(const CUtensorMap &mA, const CUtensorMap &mA2, const CUtensorMap &mB,
                                  const CUtensorMap &mB2, const GemmArgs &p, int BN, int batches, cudaStream_t st) {
     const uint32_t cb = gemm_const_bytes(p, BN);
     const GemmSmem plan = gemm_smem_plan(BN, A_SPLIT ? 2 : 1, B_SPLIT ? 2 : 1, cb);
-    const size_t smem = 1024 + (size_t)plan.stages * plan.stage_bytes + cb + 256;
+    const size_t smem = 1024 + (size_t)plan.stages * plan.stage_bytes + cb + 8 * kGemmStageOut + 512;
+    // outputs: a row block past M would be written unless M fills its tiles or the output ends at M
+    const int rows = p.out_rows > 0 ? p.out_rows : p.M;
+    if (rows != p.M && p.M % 128 != 0) return cudaErrorInvalidValue;
+    constexpr bool F32OUT = EPI == kEpiDX || EPI == kEpiF32 || EPI == kEpiPartial || EPI == kEpiOut;
+    const int zb = EPI == kEpiPartial ? batches * p.n_split : batches;
+    CUtensorMap mO, mO2;
+    if (F32OUT) {
+        if (!gemm_out_map(&mO, p.out_f32, true, p.ld_out, rows, zb)) return cudaErrorInvalidValue;
+        mO2 = mO;
+    } else if (!gemm_out_map(&mO, p.out_hi, false, p.ld_out, rows, zb) ||
+               !gemm_out_map(&mO2, p.out_lo, false, p.ld_out, rows, zb)) {
+        return cudaErrorInvalidValue;
+    }
     auto kern = k_gemm<A_MN, B_MN, A_SPLIT, B_SPLIT, EPI>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const int tiles = gemm_tiles(p, BN, batches);
     const dim3 grid(std::max(1, std::min(tiles, num_sms())));
-    return launch_after_previous(kern, grid, dim3(kGemmThreads), smem, st, mA, mA2, mB, mB2, p, BN, tiles);
+    return launch_after_previous(kern, grid, dim3(kGemmThreads), smem, st, mA, mA2, mB, mB2, mO, mO2, p, BN, tiles);
 }
 
 cudaError_t launch_scan_image(const float *part, int n_chunks, int m, int Np, int reverse, uint16_t *hi, uint16_t *lo,
