@@ -177,6 +177,13 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// Issue forms. Every MMA / commit helper below has a warp-collective "_w" form: all 32 lanes of a
+// converged warp execute it and the lane elect.sync picks issues the instruction, predicated inside
+// the same asm block. Issued from a branch taken by one lane, a tcgen05.mma stalls the issuing
+// thread for about 60-90 cycles (measured on B200); the predicated form issues in a cycle or two and
+// leaves the MMAs queued behind each other, so small-N MMA chains run at the tensor pipe's rate.
+#define FAVOR_ELECT "elect.sync _|e, 0xffffffff;\n\t"
+
 // D[tmem] (+)= A[smem] * B[smem]; kind::f16 (bf16 operands), fp32 accumulation.
 __device__ __forceinline__ void mma_f16_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
@@ -251,6 +258,68 @@ __device__ __forceinline__ void mma_tf32_ss(uint32_t d, uint64_t a, uint64_t b, 
 // Arrive on an mbarrier once all previously issued tcgen05.mma of this thread have completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// ---- warp-collective forms (see "Issue forms" above): call from all 32 lanes of a converged warp.
+
+__device__ __forceinline__ void mma_f16_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t" FAVOR_ELECT
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_f16_ts_w(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t" FAVOR_ELECT
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_tf32_ts_w(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t" FAVOR_ELECT
+        "@e tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_tf32_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t" FAVOR_ELECT
+        "@e tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ss_x4_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                            uint32_t a_step, uint32_t b_step) {
+    const uint64_t a1 = a + a_step, b1 = b + b_step, a2 = a1 + a_step, b2 = b1 + b_step, a3 = a2 + a_step,
+                   b3 = b2 + b_step;
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\tsetp.ne.b32 p, %9, 0;\n\tsetp.eq.b32 t, %9, %9;\n\t" FAVOR_ELECT
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %8, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %8, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %8, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %10, %8, t;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "l"(a1), "l"(b1), "l"(a2), "l"(b2), "l"(a3), "r"(idesc), "r"(acc), "l"(b3)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ts_x4_w(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc,
+                                            uint32_t b_step) {
+    const uint64_t b1 = b + b_step, b2 = b1 + b_step, b3 = b2 + b_step;
+    asm volatile(
+        "{\n\t.reg .pred p, t, e;\n\tsetp.ne.b32 p, %6, 0;\n\tsetp.eq.b32 t, %6, %6;\n\t" FAVOR_ELECT
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %5, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %3, %5, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %4, %5, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%9], %10, %5, t;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "l"(b1), "l"(b2), "r"(idesc), "r"(acc), "r"(a_tmem + 8), "r"(a_tmem + 16),
+        "r"(a_tmem + 24), "l"(b3)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_w(uint64_t *bar) {
+    asm volatile("{\n\t.reg .pred e;\n\t" FAVOR_ELECT
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
                  : "memory");
 }
 

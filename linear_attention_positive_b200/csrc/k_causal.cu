@@ -243,37 +243,37 @@ __device__ __forceinline__ uint32_t desc_lo(uint32_t smem_addr, uint32_t lbo_byt
     return ((smem_addr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
 }
 // D (+)= sum over 4 K-steps of A_k B_k, A and B in shared memory (low descriptor words advancing by
-// a_step / b_step 16-byte units per step).
-__device__ __forceinline__ void mma_ss4(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, uint32_t acc,
-                                        uint32_t a_step, uint32_t b_step) {
+// a_step / b_step 16-byte units per step). Warp-collective: issued by the elect.sync lane.
+__device__ __forceinline__ void mma_ss4_w(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, uint32_t acc,
+                                          uint32_t a_step, uint32_t b_step) {
     asm volatile(
-        "{\n\t.reg .pred p, t;\n\t.reg .b32 al, bl;\n\t.reg .b64 ad, bd;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+        "{\n\t.reg .pred p, t, e;\n\t.reg .b32 al, bl;\n\t.reg .b64 ad, bd;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t" FAVOR_ELECT
         "mov.b64 ad, {%1, %7};\n\tmov.b64 bd, {%2, %7};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t"
         "add.u32 al, %1, %5;\n\tadd.u32 bl, %2, %6;\n\tmov.b64 ad, {al, %7};\n\tmov.b64 bd, {bl, %7};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, t;\n\t"
         "add.u32 al, al, %5;\n\tadd.u32 bl, bl, %6;\n\tmov.b64 ad, {al, %7};\n\tmov.b64 bd, {bl, %7};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, t;\n\t"
         "add.u32 al, al, %5;\n\tadd.u32 bl, bl, %6;\n\tmov.b64 ad, {al, %7};\n\tmov.b64 bd, {bl, %7};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, t;\n\t}" ::"r"(d),
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, t;\n\t}" ::"r"(d),
         "r"(a), "r"(b), "r"(idesc), "r"(acc), "r"(a_step), "r"(b_step), "r"(kDescHi)
         : "memory");
 }
 // The same with A in TMEM (8 columns per K-step).
-__device__ __forceinline__ void mma_ts4(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t idesc, uint32_t acc,
-                                        uint32_t b_step) {
+__device__ __forceinline__ void mma_ts4_w(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t idesc, uint32_t acc,
+                                          uint32_t b_step) {
     asm volatile(
-        "{\n\t.reg .pred p, t;\n\t.reg .b32 al, bl;\n\t.reg .b64 bd;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+        "{\n\t.reg .pred p, t, e;\n\t.reg .b32 al, bl;\n\t.reg .b64 bd;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t" FAVOR_ELECT
         "mov.b64 bd, {%2, %6};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %3, p;\n\t"
         "add.u32 al, %1, 8;\n\tadd.u32 bl, %2, %5;\n\tmov.b64 bd, {bl, %6};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [al], bd, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [al], bd, %3, t;\n\t"
         "add.u32 al, al, 8;\n\tadd.u32 bl, bl, %5;\n\tmov.b64 bd, {bl, %6};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [al], bd, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [al], bd, %3, t;\n\t"
         "add.u32 al, al, 8;\n\tadd.u32 bl, bl, %5;\n\tmov.b64 bd, {bl, %6};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [al], bd, %3, t;\n\t}" ::"r"(d),
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [al], bd, %3, t;\n\t}" ::"r"(d),
         "r"(a_tmem), "r"(b), "r"(idesc), "r"(acc), "r"(b_step), "r"(kDescHi)
         : "memory");
 }
@@ -434,11 +434,10 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                 if (ok && n > 0) {
                     ok = mbar_wait_all(&bar[B_FULL_QK], 0, abort_flag);
                     tc_fence_after();
-                    if (ok && elect_one()) {
-                        mma_ss4(tmem + T_P, dQK, dW, id_proj, 0u, 2, 2);
-                        mma_commit(&bar[B_PQ_FULL]);
+                    if (ok) {
+                        mma_ss4_w(tmem + T_P, dQK, dW, id_proj, 0u, 2, 2);
+                        mma_commit_w(&bar[B_PQ_FULL]);
                     }
-                    __syncwarp();
                 }
                 for (int g = 0; ok && g < n; ++g) {
                     const int s = g % STAGES;
@@ -446,23 +445,21 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                     // K projection of tile g, once the query warps have read P; frees the Q/K stage
                     if (!(ok = mbar_wait_all(&bar[B_PQ_FREE], ph, abort_flag))) break;
                     tc_fence_after();
-                    if (elect_one()) {
-                        mma_ss4(tmem + T_P, dW, dQK + (2 * s + 1) * kTileU, id_proj, 0u, 2, 2);
-                        mma_commit(&bar[B_PK_FULL]);
-                        mma_commit(&bar[B_EMPTY_QK + s]);
+                    {
+                        mma_ss4_w(tmem + T_P, dW, dQK + (2 * s + 1) * kTileU, id_proj, 0u, 2, 2);
+                        mma_commit_w(&bar[B_PK_FULL]);
+                        mma_commit_w(&bar[B_EMPTY_QK + s]);
                     }
-                    __syncwarp();
                     // Q projection of tile g + 1, once the key warps have read P
                     if (g + 1 < n) {
                         const int s1 = (g + 1) % STAGES;
                         if (!(ok = mbar_wait_all(&bar[B_FULL_QK + s1], ((g + 1) / STAGES) & 1, abort_flag))) break;
                         if (!(ok = mbar_wait_all(&bar[B_PK_FREE], ph, abort_flag))) break;
                         tc_fence_after();
-                        if (elect_one()) {
-                            mma_ss4(tmem + T_P, dQK + 2 * s1 * kTileU, dW, id_proj, 0u, 2, 2);
-                            mma_commit(&bar[B_PQ_FULL]);
+                        {
+                            mma_ss4_w(tmem + T_P, dQK + 2 * s1 * kTileU, dW, id_proj, 0u, 2, 2);
+                            mma_commit_w(&bar[B_PQ_FULL]);
                         }
-                        __syncwarp();
                     }
                 }
             } else {
@@ -475,14 +472,13 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                 auto issue_av = [&](int e) -> bool {
                     if (!mbar_wait_all(&bar[B_MASK_DONE], e & 1, abort_flag)) return false;
                     tc_fence_after();
-                    if (elect_one()) {
+                    {
                         const uint32_t tO = tmem + T_O + 64 * (e & 1), dV = dV0 + (e % STAGES) * kTileU;
-                        mma_ts4(tO, tmem + T_A, dV, id_64, 1u, kRow16);
-                        mma_ts4(tO, tmem + T_A + 32, dV + kHalfU, id_64, 1u, kRow16);
-                        mma_commit(&bar[B_O_FULL + (e & 1)]);
-                        mma_commit(&bar[B_EMPTY_V + e % STAGES]);
+                        mma_ts4_w(tO, tmem + T_A, dV, id_64, 1u, kRow16);
+                        mma_ts4_w(tO, tmem + T_A + 32, dV + kHalfU, id_64, 1u, kRow16);
+                        mma_commit_w(&bar[B_O_FULL + (e & 1)]);
+                        mma_commit_w(&bar[B_EMPTY_V + e % STAGES]);
                     }
-                    __syncwarp();
                     return true;
                 };
                 int g = 0;
@@ -495,39 +491,35 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                     if (!(ok = mbar_wait_all(&bar[B_PHIQ_FULL], ph, abort_flag))) break;
                     if (!(ok = mbar_wait_all(&bar[B_PHIK_FULL], ph, abort_flag))) break;
                     tc_fence_after();
-                    if (elect_one()) {
-                        mma_ts4(tmem + T_A, tmem + T_PHIQ, dKB, id_sc, 0u, kRow16);
-                        mma_ts4(tmem + T_A, tmem + T_PHIQ + 32, dKB + kHalfU, id_sc, 1u, kRow16);
-                        mma_commit(&bar[B_SC_FULL]);
+                    {
+                        mma_ts4_w(tmem + T_A, tmem + T_PHIQ, dKB, id_sc, 0u, kRow16);
+                        mma_ts4_w(tmem + T_A, tmem + T_PHIQ + 32, dKB + kHalfU, id_sc, 1u, kRow16);
+                        mma_commit_w(&bar[B_SC_FULL]);
                     }
-                    __syncwarp();
                     // O = phiq Simg
                     if (!(ok = mbar_wait_all(&bar[B_S_READY], ph, abort_flag))) break;
                     if (g >= 2 && !(ok = mbar_wait_all(&bar[B_O_EMPTY + b], ((g >> 1) - 1) & 1, abort_flag))) break;
                     tc_fence_after();
-                    if (elect_one()) {
+                    {
                         const uint32_t tO = tmem + T_O + 64 * b;
-                        mma_ts4(tO, tmem + T_PHIQ, dSimg, id_64, 0u, kRow16);
-                        mma_ts4(tO, tmem + T_PHIQ + 32, dSimg + kHalfU, id_64, 1u, kRow16);
-                        mma_commit(&bar[B_PHIQ_FREE]);
+                        mma_ts4_w(tO, tmem + T_PHIQ, dSimg, id_64, 0u, kRow16);
+                        mma_ts4_w(tO, tmem + T_PHIQ + 32, dSimg + kHalfU, id_64, 1u, kRow16);
+                        mma_commit_w(&bar[B_PHIQ_FREE]);
                     }
-                    __syncwarp();
                     // S += phik^T V'
                     if (!(ok = mbar_wait_all(&bar[B_CONV + s], (g / STAGES) & 1, abort_flag))) break;
                     tc_fence_after();
-                    if (elect_one()) {
+                    {
                         const uint32_t dV = dV0 + s * kTileU;
-                        mma_ss4(tmem + T_S, dKA, dV, id_64, 1u, 2, kRow16);
-                        mma_ss4(tmem + T_S, dKA + kTileU, dV + kHalfU, id_64, 1u, 2, kRow16);
-                        mma_commit(&bar[B_PHIK_FREE]);
-                        mma_commit(&bar[B_S_DONE]);
+                        mma_ss4_w(tmem + T_S, dKA, dV, id_64, 1u, 2, kRow16);
+                        mma_ss4_w(tmem + T_S, dKA + kTileU, dV + kHalfU, id_64, 1u, 2, kRow16);
+                        mma_commit_w(&bar[B_PHIK_FREE]);
+                        mma_commit_w(&bar[B_S_DONE]);
                     }
-                    __syncwarp();
                 }
                 if (ok && n > 0) issue_av(n - 1);
             }
-            if (elect_one()) mma_commit(&bar[B_DRAIN + (warp - 13)]);
-            __syncwarp();
+            mma_commit_w(&bar[B_DRAIN + (warp - 13)]);
             volatile int no_abort = 0;
             mbar_wait(&bar[B_DRAIN + (warp - 13)], 0, &no_abort);
         } else {

@@ -337,26 +337,21 @@ k_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorM
                 const uint32_t a_hi = a_const ? smem_u32(sOnesA) : st;
                 const uint32_t a_lo = st + plan.a_bytes;
                 const uint32_t b_hi = b_const ? smem_u32(sOnesB) : st + AP * plan.a_bytes, b_lo = b_hi + plan.b_bytes;
-                if (elect_one()) {
-                    const uint32_t acc0 = i > 0 ? 1u : 0u;
-                    mma_ss_x4(acc, make_sdesc(a_hi, a_lbo, 1024), make_sdesc(b_hi, b_lbo, 1024), idesc, acc0, a_step, b_step);
-                    if (A_SPLIT && !a_const)
-                        mma_ss_x4(acc, make_sdesc(a_lo, a_lbo, 1024), make_sdesc(b_hi, b_lbo, 1024), idesc, 1u, a_step, b_step);
-                    if (B_SPLIT && !b_const)
-                        mma_ss_x4(acc, make_sdesc(a_hi, a_lbo, 1024), make_sdesc(b_lo, b_lbo, 1024), idesc, 1u, a_step, b_step);
-                    mma_commit(&empty[s]);
-                }
-                __syncwarp();
+                const uint32_t acc0 = i > 0 ? 1u : 0u;
+                mma_ss_x4_w(acc, make_sdesc(a_hi, a_lbo, 1024), make_sdesc(b_hi, b_lbo, 1024), idesc, acc0, a_step, b_step);
+                if (A_SPLIT && !a_const)
+                    mma_ss_x4_w(acc, make_sdesc(a_lo, a_lbo, 1024), make_sdesc(b_hi, b_lbo, 1024), idesc, 1u, a_step, b_step);
+                if (B_SPLIT && !b_const)
+                    mma_ss_x4_w(acc, make_sdesc(a_hi, a_lbo, 1024), make_sdesc(b_lo, b_lbo, 1024), idesc, 1u, a_step, b_step);
+                mma_commit_w(&empty[s]);
             }
             if (!ok) break;
-            if (elect_one()) mma_commit(&acc_full[b]);
-            __syncwarp();
+            mma_commit_w(&acc_full[b]);
         }
         // every MMA has completed before the TMEM is freed
-        if (elect_one()) mma_commit(drain);
-        __syncwarp();
+        mma_commit_w(drain);
         volatile int no_abort = 0;
-        mbar_wait(drain, 0, &no_abort);
+        mbar_wait_all(drain, 0, &no_abort);
     } else {
         // ------------------------------------------------------------------ epilogue
         const int q = warp & 3;             // TMEM lane quarter

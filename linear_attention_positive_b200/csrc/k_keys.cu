@@ -99,28 +99,27 @@ k_key_logit_max(const __grid_constant__ CUtensorMap mapK, const __grid_constant_
             mbar_wait(w_full, 0, &no_abort_w);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc(kTile, p.m, kFmtBF16, 0, 0);
-            bool ok = mbar_wait(w_full, 0, abort_flag);
-            for (int it = 0; ok && it < n_tiles; ++it) {
-                const int s = it % STAGES, ab = it & 1;
-                if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag)) break;
-                if (!mbar_wait(&acc_empty[ab], ((it >> 1) & 1) ^ 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t a0 = smem_u32(sK + (size_t)s * TILE_BYTES), b0 = smem_u32(sW);
-                for (int k = 0; k < D / 16; ++k) {
-                    const int kb = k >> 2, kk = k & 3;
-                    const uint64_t ad = make_sdesc(a0 + kb * kTile * 128 + kk * 32, 16, 1024);
-                    const uint64_t bd = make_sdesc(b0 + kb * p.m * 128 + kk * 32, 16, 1024);
-                    mma_f16_ss(tmem + ab * p.m, ad, bd, idesc, k > 0);
-                }
-                mma_commit(&acc_full[ab]);
-                mma_commit(&empty[s]);
+        // MMA issue by the whole (converged) warp through the predicated issue forms.
+        const uint32_t idesc = make_idesc(kTile, p.m, kFmtBF16, 0, 0);
+        bool ok = mbar_wait_all(w_full, 0, abort_flag);
+        for (int it = 0; ok && it < n_tiles; ++it) {
+            const int s = it % STAGES, ab = it & 1;
+            if (!mbar_wait_all(&full[s], (it / STAGES) & 1, abort_flag)) break;
+            if (!mbar_wait_all(&acc_empty[ab], ((it >> 1) & 1) ^ 1, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sK + (size_t)s * TILE_BYTES), b0 = smem_u32(sW);
+            for (int k = 0; k < D / 16; ++k) {
+                const int kb = k >> 2, kk = k & 3;
+                const uint64_t ad = make_sdesc(a0 + kb * kTile * 128 + kk * 32, 16, 1024);
+                const uint64_t bd = make_sdesc(b0 + kb * p.m * 128 + kk * 32, 16, 1024);
+                mma_f16_ss_w(tmem + ab * p.m, ad, bd, idesc, k > 0);
             }
-            mma_commit(drain);
-            volatile int no_abort = 0;
-            mbar_wait(drain, 0, &no_abort);
+            mma_commit_w(&acc_full[ab]);
+            mma_commit_w(&empty[s]);
         }
+        mma_commit_w(drain);
+        volatile int no_abort = 0;
+        mbar_wait_all(drain, 0, &no_abort);
     } else {
         // Epilogue: warps 2..5 cover TMEM lane quarters 2,3,0,1; thread <-> token row.
         const int q = warp & 3, row = q * 32 + lane;
@@ -298,54 +297,53 @@ k_key_state(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CU
             mbar_wait(w_full, 0, &no_abort_w);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idesc_p = make_idesc(128, 64, kFmtBF16, 0, 0);
-            const uint32_t idesc_s = make_idesc(128, D, kFmtTF32, 0, 0);
-            bool ok = mbar_wait(w_full, 0, abort_flag);
-            // Projection of sub-tile u into D2 buffer u&1.
-            auto project = [&](int u) -> bool {
-                const int it = u >> 1, s = it % STAGES, hs = u & 1, b = u & 1;
-                if (hs == 0 && !mbar_wait(&full[s], (it / STAGES) & 1, abort_flag)) return false;
-                if (!mbar_wait(&d2_empty[b], ((u >> 1) & 1) ^ 1, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t kt = smem_u32(sK + (size_t)s * SM::K_TILE) + hs * 64 * 128;
-                for (int h = 0; h < halves; ++h) {
-                    const uint32_t wa = smem_u32(sW) + h * 128 * 128;
-                    for (int k = 0; k < D / 16; ++k) {
-                        const int kb = k >> 2, kk = k & 3;
-                        const uint64_t ad = make_sdesc(wa + kb * p.m * 128 + kk * 32, 16, 1024);
-                        const uint64_t bd = make_sdesc(kt + kb * kTile * 128 + kk * 32, 16, 1024);
-                        mma_f16_ss(tmem + b * d2_cols + h * 64, ad, bd, idesc_p, k > 0);
-                    }
+        // MMA issue by the whole (converged) warp through the predicated issue forms.
+        const uint32_t idesc_p = make_idesc(128, 64, kFmtBF16, 0, 0);
+        const uint32_t idesc_s = make_idesc(128, D, kFmtTF32, 0, 0);
+        bool ok = mbar_wait_all(w_full, 0, abort_flag);
+        // Projection of sub-tile u into D2 buffer u&1.
+        auto project = [&](int u) -> bool {
+            const int it = u >> 1, s = it % STAGES, hs = u & 1, b = u & 1;
+            if (hs == 0 && !mbar_wait_all(&full[s], (it / STAGES) & 1, abort_flag)) return false;
+            if (!mbar_wait_all(&d2_empty[b], ((u >> 1) & 1) ^ 1, abort_flag)) return false;
+            tc_fence_after();
+            const uint32_t kt = smem_u32(sK + (size_t)s * SM::K_TILE) + hs * 64 * 128;
+            for (int h = 0; h < halves; ++h) {
+                const uint32_t wa = smem_u32(sW) + h * 128 * 128;
+                for (int k = 0; k < D / 16; ++k) {
+                    const int kb = k >> 2, kk = k & 3;
+                    const uint64_t ad = make_sdesc(wa + kb * p.m * 128 + kk * 32, 16, 1024);
+                    const uint64_t bd = make_sdesc(kt + kb * kTile * 128 + kk * 32, 16, 1024);
+                    mma_f16_ss_w(tmem + b * d2_cols + h * 64, ad, bd, idesc_p, k > 0);
                 }
-                mma_commit(&d2_full[b]);
-                if (hs == 1) mma_commit(&empty[s]);
-                return true;
-            };
-            if (ok && n_sub > 0) ok = project(0);
-            for (int u = 0; ok && u < n_sub; ++u) {
-                if (u + 1 < n_sub && !project(u + 1)) break;
-                const int b = u & 1;
-                if (!mbar_wait(&phi_full[b], (u >> 1) & 1, abort_flag)) break;
-                if (!mbar_wait(&v_full[b], (u >> 1) & 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t vb = smem_u32(sV + b * SM::V32_SUB);
-                for (int h = 0; h < halves; ++h) {
-                    for (int ks = 0; ks < 8; ++ks) {
-                        // K-step of 8 tokens: block ks/4 of V^T, 32-byte offset inside its rows.
-                        const uint64_t bd = make_sdesc(vb + (ks >> 2) * (D * 128) + (ks & 3) * 32, 16, 1024);
-                        mma_tf32_ts(tmem + s_col + h * D, tmem + b * d2_cols + h * 64 + ks * 8, bd, idesc_s,
-                                    (u > 0 || ks > 0) ? 1u : 0u);
-                    }
-                }
-                mma_commit(&d2_empty[b]);
-                mma_commit(&v_empty[b]);
             }
-            mma_commit(state_done);
-            mma_commit(drain);
-            volatile int no_abort = 0;
-            mbar_wait(drain, 0, &no_abort);
+            mma_commit_w(&d2_full[b]);
+            if (hs == 1) mma_commit_w(&empty[s]);
+            return true;
+        };
+        if (ok && n_sub > 0) ok = project(0);
+        for (int u = 0; ok && u < n_sub; ++u) {
+            if (u + 1 < n_sub && !project(u + 1)) break;
+            const int b = u & 1;
+            if (!mbar_wait_all(&phi_full[b], (u >> 1) & 1, abort_flag)) break;
+            if (!mbar_wait_all(&v_full[b], (u >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t vb = smem_u32(sV + b * SM::V32_SUB);
+            for (int h = 0; h < halves; ++h) {
+                for (int ks = 0; ks < 8; ++ks) {
+                    // K-step of 8 tokens: block ks/4 of V^T, 32-byte offset inside its rows.
+                    const uint64_t bd = make_sdesc(vb + (ks >> 2) * (D * 128) + (ks & 3) * 32, 16, 1024);
+                    mma_tf32_ts_w(tmem + s_col + h * D, tmem + b * d2_cols + h * 64 + ks * 8, bd, idesc_s,
+                                (u > 0 || ks > 0) ? 1u : 0u);
+                }
+            }
+            mma_commit_w(&d2_empty[b]);
+            mma_commit_w(&v_empty[b]);
         }
+        mma_commit_w(state_done);
+        mma_commit_w(drain);
+        volatile int no_abort = 0;
+        mbar_wait_all(drain, 0, &no_abort);
     } else if (warp == 2 || warp == 3) {
         // V converter: the bf16 V rows of a 64-token sub-tile become the K-major tf32 operand
         // V^T: [2 blocks of 32 tokens][D value rows][32 fp32], 128-byte swizzled. Lane <-> token,

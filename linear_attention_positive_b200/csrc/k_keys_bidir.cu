@@ -63,10 +63,9 @@ __device__ __forceinline__ float key_sq_norm(const uint8_t *tile, int row) {
 //
 // Per key tile of 64 tokens, with the m features as 128-feature halves h, one per exponent
 // warpgroup, each with its own TMEM buffers (the halves never wait on each other):
-//   P_h^T = W_h K_tile^T - D_r ln2 (bf16 MMA accumulating onto a per-row value the warpgroup
-//           stored beforehand; TMEM lanes are features, columns are tokens)
+//   P_h^T = W_h K_tile^T (bf16 MMA; TMEM lanes are features, columns are tokens)
 //   -> warpgroup h: t = P_h^T log2e + B_j with B_j = -|k_j|^2/2 log2e + A + b_t, i.e.
-//      t = u_r(k_j) log2e - D_r + A + b_t; phi' = 2^t rounded to fp16 into TMEM
+//      t = u_r(k_j) log2e + A + b_t; phi' = 2^(t - D_r) rounded to fp16 into TMEM
 //   -> [S_h | z_h] += phi'_h [V'_t | 2^-b_t] (fp16 MMA, A from TMEM, B the converted V tile read
 //      MN-major plus one column holding 2^-b_t), accumulated in TMEM over the run.
 // Stabiliser D_r (integer): set on a run's first tile so that the row's largest t is in (A+b-1, A+b];
@@ -81,9 +80,8 @@ __device__ __forceinline__ float key_sq_norm(const uint8_t *tile, int row) {
 // exponentials of feature half 0 / 1 and the run-end write; 12 TMA; 13 MMA issue; 14 the tile's
 // largest |v|; 15 idle.
 // P_h^T is double-buffered where TMEM allows (d = 64): the projection of tile g+2 runs while tile g+1
-// is loaded and tile g's exponentials are computed. The -D_r ln2 it accumulates onto is written
-// when the buffer is released, two tiles ahead; the exponent warpgroup corrects by the difference
-// to the current D_r (zero unless D_r changed in between: a raise, or a run boundary).
+// is loaded and tile g's exponentials are computed. A buffer is released as soon as its load into
+// registers has completed.
 // TMEM columns: P_h^T [64 (NPB h + b), +64), phi'_h [T_PHI + 32h, +32) (fp16 pairs),
 // [S_h | z_h] [T_PHI + 64 + h*ON, +ON).
 
@@ -99,7 +97,6 @@ struct KeyStateParams2 {
 constexpr int kKeyThreads = 512;
 constexpr int kKeyTile = 64;            // tokens per key tile of k_key_partials
 constexpr float kKeyFeatureShift = 4.f;  // A: the run's largest phi' is about 2^(A + b_t)
-constexpr float kLn2 = 0.6931471805599453f;
 
 template <int D>
 struct KeyCfg {
@@ -129,10 +126,12 @@ __device__ __forceinline__ float key_logits(float (&v)[64], const float *bias) {
     return fmaxf(a, b);
 }
 
-// phi' = 2^t (in place), rounded to fp16 pairs. Per 32 columns the first 32 - POLY exponentials
-// go to MUFU ex2, the last POLY to the FMA-pipe polynomial.
+// phi' = 2^(t - D) (in place), rounded to fp16 pairs. Per 32 columns the first 32 - POLY
+// exponentials go to MUFU ex2, the last POLY to the FMA-pipe polynomial.
 template <int POLY>
-__device__ __forceinline__ void key_features(float (&v)[64], uint32_t (&hv)[32]) {
+__device__ __forceinline__ void key_features(float (&v)[64], float D, uint32_t (&hv)[32]) {
+#pragma unroll
+    for (int e = 0; e < 64; ++e) v[e] -= D;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
 #pragma unroll
@@ -150,17 +149,6 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&h)[3
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
         "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
         FAVOR_U16(h, 0), FAVOR_U16(h, 16)
-        : "memory");
-}
-
-// Fills 64 consecutive columns of this thread's TMEM lane with x (warp-collective; not waited).
-__device__ __forceinline__ void tmem_fill64(uint32_t taddr, float x) {
-    const uint32_t u = __float_as_uint(x);
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
-        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
-        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
-        "r"(u)
         : "memory");
 }
 
@@ -256,8 +244,6 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto first_of_run = [&](int g) { return g == 0 || (f0 + g) % nt == 0; };
-    auto last_of_run = [&](int g) { return g == n - 1 || (f0 + g + 1) % nt == 0; };
 
     if (warp >= 12) {
         regs_dec<56>();
@@ -314,9 +300,9 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 __syncwarp();
             }
         } else if (warp == 13 && n > 0) {
-            // MMA issue in a fixed order: the projections of tile g+1 as soon as each half's P has
-            // been read (and refilled with -D_r ln2), then the state MMAs of tile g once its V tile
-            // is converted and phi' is in TMEM.
+            // MMA issue by the whole (converged) warp through the predicated issue forms: per tile g,
+            // first the projection of tile g + NPB into the P buffer tile g has just been read out
+            // of, then the state MMAs of tile g once its V tile is converted and phi' is in TMEM.
             const uint32_t idesc1 = make_idesc(128, kKeyTile, kFmtBF16, 0, 0);
             const uint32_t idesc2 = make_idesc(128, ON, kFmtF16, 0, 1);
             const uint64_t dW = make_sdesc(smem_u32(sW), 16, 1024), dS = make_sdesc(smem_u32(sStage), 16, 1024);
@@ -326,63 +312,52 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 const uint64_t a = dW + (uint32_t)h * (128 * 128 / 16);
                 const uint64_t b = dS + (uint32_t)(g % STAGES) * (C::STAGE / 16);
                 const uint32_t d = tmem + (uint32_t)(h * NPB + g % NPB) * 64;
-                if (elect_one()) {
-                    // the first NPB projections have no stored -D_r ln2 to accumulate onto
-                    mma_ss_x4(d, a, b, idesc1, g >= NPB ? 1u : 0u, 2, 2);
-                    if (KB == 2) mma_ss_x4(d, a + (uint32_t)p.m * 8, b + kKeyTile * 128 / 16, idesc1, 1u, 2, 2);
-                    mma_commit(&p_full[h * 2 + g % NPB]);
-                }
-                __syncwarp();
+                mma_ss_x4_w(d, a, b, idesc1, 0u, 2, 2);
+                if (KB == 2) mma_ss_x4_w(d, a + (uint32_t)p.m * 8, b + kKeyTile * 128 / 16, idesc1, 1u, 2, 2);
+                mma_commit_w(&p_full[h * 2 + g % NPB]);
             };
-            int runs[2] = {0, 0};
             bool ok = mbar_wait_all(w_full, 0, abort_flag);
             for (int g = 0; ok && g < min(NPB, n); ++g) {
-                if (!mbar_wait_all(&full[g % STAGES], (g / STAGES) & 1, abort_flag)) { ok = false; break; }
+                ok = mbar_wait_all(&full[g % STAGES], (g / STAGES) & 1, abort_flag);
                 tc_fence_after();
-                for (int h = 0; h < halves; ++h) project(g, h);
+                for (int h = 0; ok && h < halves; ++h) project(g, h);
             }
-            // the projection of tile g2 into the buffer tile g2 - NPB used, once that is released
-            auto project_next = [&](int g2, int g) {
-                if (!mbar_wait_all(&full[g2 % STAGES], (g2 / STAGES) & 1, abort_flag)) return false;
-                for (int h = 0; h < halves; ++h) {
-                    if (!mbar_wait_all(&p_free[h * 2 + g % NPB], (g / NPB) & 1, abort_flag)) return false;
-                    tc_fence_after();
-                    project(g2, h);
-                }
-                return true;
-            };
+            int runs[2] = {0, 0};
+            int pos = f0 % nt;  // tile g's index within its head
             for (int g = 0; ok && g < n; ++g) {
                 const int s = g % STAGES;
-                // single-buffered P: the next projection goes ahead of this tile's state MMAs
-                if (NPB == 1 && g + 1 < n && !project_next(g + 1, g)) break;
-                if (!mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag)) break;
-                const bool first = first_of_run(g), last = last_of_run(g);
+                const bool first = g == 0 || pos == 0, last = g == n - 1 || pos == nt - 1;
+                pos = pos + 1 == nt ? 0 : pos + 1;
+                if (g + NPB < n) {
+                    const int g2 = g + NPB;
+                    ok = mbar_wait_all(&full[g2 % STAGES], (g2 / STAGES) & 1, abort_flag);
+                    for (int h = 0; ok && h < halves; ++h) {
+                        ok = mbar_wait_all(&p_free[h * 2 + g % NPB], (g / NPB) & 1, abort_flag);
+                        tc_fence_after();
+                        if (ok) project(g2, h);
+                    }
+                    if (!ok) break;
+                }
+                ok = mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag);
                 const uint64_t vd = dV + (uint32_t)s * (C::STAGE / 16);
                 for (int h = 0; ok && h < halves; ++h) {
-                    if (first && runs[h] > 0 && !mbar_wait_all(&acc_empty[h], (runs[h] - 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    if (!mbar_wait_all(&phi_full[h], g & 1, abort_flag)) { ok = false; break; }
+                    if (first && runs[h] > 0) ok = mbar_wait_all(&acc_empty[h], (runs[h] - 1) & 1, abort_flag);
+                    if (ok) ok = mbar_wait_all(&phi_full[h], g & 1, abort_flag);
+                    if (!ok) break;
                     tc_fence_after();
-                    if (elect_one()) {
-                        mma_ts_x4(tmem + C::T_S + h * ON, tmem + C::T_PHI + h * 32, vd, idesc2, first ? 0u : 1u, 2048 / 16);
-                        mma_commit(&phi_free[h]);
-                        if (last) mma_commit(&acc_full[h]);
+                    mma_ts_x4_w(tmem + C::T_S + h * ON, tmem + C::T_PHI + h * 32, vd, idesc2, first ? 0u : 1u, 2048 / 16);
+                    mma_commit_w(&phi_free[h]);
+                    if (last) {
+                        mma_commit_w(&acc_full[h]);
+                        ++runs[h];
                     }
-                    __syncwarp();
-                    if (last) ++runs[h];
                 }
                 if (!ok) break;
-                if (elect_one()) mma_commit(&empty[s]);
-                __syncwarp();
-                // double-buffered P: the projection two tiles ahead, into the buffer this tile used
-                if (NPB == 2 && g + 2 < n && !project_next(g + 2, g)) break;
+                mma_commit_w(&empty[s]);
             }
-            if (elect_one()) mma_commit(drain);
-            __syncwarp();
+            mma_commit_w(drain);
             volatile int no_abort = 0;
-            mbar_wait(drain, 0, &no_abort);
+            mbar_wait_all(drain, 0, &no_abort);
         }
     } else if (warp >= 4) {
         regs_inc<184>();
@@ -392,8 +367,8 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
             const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
             const uint32_t tP = tmem + lane_off + h * NPB * 64, tS = tmem + lane_off + C::T_S + h * ON;
             int runs = 0;
-            float Dr = 0.f;                        // this feature's stabiliser D_r in the current run
-            float fillD[2] = {0.f, 0.f};           // D_r the buffer's stored -D_r ln2 stands for
+            float Dr = 0.f;    // this feature's stabiliser D_r in the current run
+            int pos = f0 % nt;  // tile g's index within its head
             float v[64];
             if (n > 0 && mbar_wait_all(&p_full[h * 2], 0, abort_flag)) {
                 tc_fence_after();
@@ -401,37 +376,21 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
             }
             for (int g = 0; g < n; ++g) {
                 const int s = g % STAGES, b = g % NPB;
-                if (!mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag)) break;
+                const bool first = g == 0 || pos == 0, last = g == n - 1 || pos == nt - 1;
+                pos = pos + 1 == nt ? 0 : pos + 1;
                 asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32((&v[0])), FAVOR_RW32((&v[32]))::"memory");
-                const bool first = first_of_run(g), last = last_of_run(g);
+                // the logits are in registers: the buffer is free for the projection of tile g + NPB
+                tc_fence_before();
+                mbar_arrive(&p_free[h * 2 + b]);
+                if (!mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag)) break;
                 const float Dbase = first ? 0.f : Dr;
-                // the buffer's projection accumulated onto -fillD ln2; bring it to Dbase
-                const float corr = Dbase - fillD[b];
-                float tmax = key_logits(v, sBias + s * kKeyTile);
-                if (__any_sync(0xffffffffu, corr != 0.f)) {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) v[e] -= corr;
-                    tmax -= corr;
-                }
+                const float tmax = key_logits(v, sBias + s * kKeyTile) - Dbase;
                 const float lim = kKeyFeatureShift + (float)sShift[s];  // target for the row's largest t
                 // new stabiliser: on a run's first tile always, later only when 2^t would overflow fp16
                 const float delta = (first || tmax > 15.f) ? ceilf(tmax - lim) : 0.f;
-                if (__any_sync(0xffffffffu, delta != 0.f)) {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) v[e] -= delta;
-                }
                 Dr = Dbase + delta;
-                // release this buffer for tile g + NPB, with -D_r ln2 as the value it accumulates onto
-                // (0 if that tile starts a new run)
-                if (g + NPB < n) {
-                    fillD[b] = first_of_run(g + NPB) ? 0.f : Dr;
-                    tmem_fill64(tP + b * 64, -fillD[b] * kLn2);
-                    tmem_wait_st();
-                }
-                tc_fence_before();
-                mbar_arrive(&p_free[h * 2 + b]);
                 uint32_t hv[32];
-                key_features<POLY>(v, hv);
+                key_features<POLY>(v, Dr, hv);
                 // prefetch the next tile's logits (its projection ran meanwhile)
                 if (g + 1 < n) {
                     if (!mbar_wait_all(&p_full[h * 2 + (g + 1) % NPB], ((g + 1) / NPB) & 1, abort_flag)) break;

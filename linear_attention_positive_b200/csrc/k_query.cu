@@ -364,19 +364,15 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             const uint32_t w_kb = (uint32_t)p.m * 128 / 16;  // W k-block stride, 16-byte units
             auto project = [&](int g) {
                 const uint64_t a = dQ + (uint32_t)(g % STAGES) * (C::Q_TILE / 16);
-                if (elect_one()) {
-                    mma_ss_x4(tmem, a, dW, idesc1, 0u, 2, 2);
-                    if (KB == 2) mma_ss_x4(tmem, a + kTile * 128 / 16, dW + w_kb, idesc1, 1u, 2, 2);
-                    mma_commit(p_full);
-                }
-                __syncwarp();
+                mma_ss_x4_w(tmem, a, dW, idesc1, 0u, 2, 2);
+                if (KB == 2) mma_ss_x4_w(tmem, a + kTile * 128 / 16, dW + w_kb, idesc1, 1u, 2, 2);
+                mma_commit_w(p_full);
             };
             bool ok = mbar_wait_all(w_full, 0, abort_flag) && mbar_wait_all(&full[0], 0, abort_flag);
             if (ok) {
                 tc_fence_after();
                 project(0);
-                if (elect_one()) mma_commit(&empty[0]);
-                __syncwarp();
+                mma_commit_w(&empty[0]);
             }
             int bh = f0 / nt, nh = 0, t = f0 - bh * nt, group = 0;  // item g's place, advanced per item
             int run_end = min(f1, (bh + 1) * nt) - bh * nt;          // one past the last tile of this group
@@ -389,24 +385,20 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                     if (!mbar_wait_all(p_free, g & 1, abort_flag)) break;
                     tc_fence_after();
                     project(g + 1);
-                    if (elect_one()) mma_commit(&empty[s1]);
-                    __syncwarp();
+                    mma_commit_w(&empty[s1]);
                 }
                 if (first && !mbar_wait_all(img_full, group & 1, abort_flag)) break;
                 if (g > 0 && !mbar_wait_all(o_empty, (g - 1) & 1, abort_flag)) break;
                 if (!mbar_wait_all(phi_full, g & 1, abort_flag)) break;
                 tc_fence_after();
-                if (elect_one()) {
-                    for (int h = 0; h < halves; ++h) {
-                        const uint64_t b = dI + (uint32_t)h * (kImgHalf / 16);
-                        mma_ts_x4(tmem + kTmemO, tmem + kTmemPhi + h * 64, b, idesc2, h > 0 ? 1u : 0u, 2);
-                        mma_ts_x4(tmem + kTmemO, tmem + kTmemPhi + h * 64 + 32, b + kImgKBlock / 16, idesc2, 1u, 2);
-                    }
-                    mma_commit(phi_free);
-                    mma_commit(o_full);
-                    if (last) mma_commit(img_empty);
+                for (int h = 0; h < halves; ++h) {
+                    const uint64_t b = dI + (uint32_t)h * (kImgHalf / 16);
+                    mma_ts_x4_w(tmem + kTmemO, tmem + kTmemPhi + h * 64, b, idesc2, h > 0 ? 1u : 0u, 2);
+                    mma_ts_x4_w(tmem + kTmemO, tmem + kTmemPhi + h * 64 + 32, b + kImgKBlock / 16, idesc2, 1u, 2);
                 }
-                __syncwarp();
+                mma_commit_w(phi_free);
+                mma_commit_w(o_full);
+                if (last) mma_commit_w(img_empty);
                 // advance to item g + 1
                 if (!last) {
                     ++t;
@@ -422,10 +414,9 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                     run_end = min(f1, (bh + 1) * nt) - bh * nt;
                 }
             }
-            if (elect_one()) mma_commit(drain);
-            __syncwarp();
+            mma_commit_w(drain);
             volatile int no_abort = 0;
-            mbar_wait(drain, 0, &no_abort);
+            mbar_wait_all(drain, 0, &no_abort);
         }
     } else if (warp >= 4) {
         regs_inc<184>();
