@@ -442,6 +442,15 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
         "r"(h[o + 7]), "r"(h[o + 8]), "r"(h[o + 9]), "r"(h[o + 10]), "r"(h[o + 11]), "r"(h[o + 12]),           \
         "r"(h[o + 13]), "r"(h[o + 14]), "r"(h[o + 15])
 
+// Stores 16 consecutive 32-bit columns of this thread's TMEM lane (warp-collective; not waited).
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&h)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        FAVOR_U16(h, 0)
+        : "memory");
+}
+
 // Stores 64 consecutive 32-bit columns of this thread's TMEM lane (warp-collective; not waited).
 __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&h)[64]) {
     asm volatile(

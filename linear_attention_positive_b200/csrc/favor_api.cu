@@ -16,6 +16,7 @@
 #include "k_fp32.cu"
 #include "k_keys.cu"
 #include "k_keys_bidir.cu"
+#include "k_keys_wide.cu"
 #include "k_query.cu"
 #include "k_causal.cu"
 #include "k_gemm.cu"
@@ -124,15 +125,18 @@ Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_
 // Bidirectional bf16 forward: per-run key maxima, per-run partial states [S | z] (feature-major
 // columns), their largest magnitudes, and the per-head fp16 state images (unless a ctx holds them).
 struct BidirLayout {
-    Flat f;  // 64-token key tiles of k_key_partials
+    Flat f;  // key tiles of the key-state kernel (128 tokens for d = 64, else 64)
     int BH;
     size_t off_part, off_D, off_amax, off_Dmax, off_state, total;
 };
 
+// Tokens per key tile: k_key_partials_wide (d = 64) takes 128, k_key_partials (d = 128) 64.
+int bidir_key_tile(int d) { return d == 64 ? kWideTile : kKeyTile; }
+
 BidirLayout bidir_layout(const favor_shape *s, bool state_in_ws) {
     BidirLayout l{};
     l.BH = s->B * s->H;
-    l.f = make_flat(l.BH, s->L, num_sms(), kKeyTile);
+    l.f = make_flat(l.BH, s->L, num_sms(), bidir_key_tile(s->d));
     const size_t slots = (size_t)flat_slots(l.f, l.BH);
     size_t off = 0;
     l.off_part = off;
@@ -446,8 +450,8 @@ favor_status fwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, 
     const BidirLayout l = bidir_layout(s, ctx == nullptr);
     if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
     CUtensorMap mQ, mK64, mV64, mW, mO;
-    if (!make_token_map(&mQ, Q, l.BH, s->L, s->d) || !make_token_map(&mK64, K, l.BH, s->L, s->d, kKeyTile) ||
-        !make_token_map(&mV64, V, l.BH, s->L, s->d, kKeyTile) || !make_w_map(&mW, W, s->m, s->d) ||
+    if (!make_token_map(&mQ, Q, l.BH, s->L, s->d) || !make_token_map(&mK64, K, l.BH, s->L, s->d, bidir_key_tile(s->d)) ||
+        !make_token_map(&mV64, V, l.BH, s->L, s->d, bidir_key_tile(s->d)) || !make_w_map(&mW, W, s->m, s->d) ||
         !make_out_map(&mO, out, l.BH, s->L, s->d))
         return FAVOR_ERR_CUDA;
     float *part = (float *)(ws + l.off_part);
@@ -460,7 +464,8 @@ favor_status fwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, 
 
     KeyStateParams2 ks{s->L, s->m, l.f, part, partD, amax, Dmax};
     record_stage(o, 0, st);
-    cudaError_t e = launch_key_partials(mK64, mV64, mW, ks, s->d, opt_poly_pct(o), st);
+    cudaError_t e = s->d == 64 ? launch_key_partials_wide(mK64, mV64, mW, ks, opt_poly_pct(o), st)
+                               : launch_key_partials(mK64, mV64, mW, ks, s->d, opt_poly_pct(o), st);
     record_stage(o, 1, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     ImageParams ip{s->m, s->d, l.f, part, partD, amax, Dmax, state, stride, kref};

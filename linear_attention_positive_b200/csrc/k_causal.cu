@@ -218,14 +218,6 @@ __device__ __forceinline__ bool mbar_wait_cluster_all(uint64_t *bar, uint32_t pa
     return __all_sync(0xffffffffu, ok);
 }
 
-// Stores 16 consecutive 32-bit columns of this thread's TMEM lane (warp-collective; not waited).
-__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&h)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16};" ::"r"(taddr),
-        FAVOR_U16(h, 0)
-        : "memory");
-}
 
 // Bulk copy of `bytes` from this CTA's shared memory into another CTA of the cluster (destination
 // and its mbarrier as cluster addresses); completes as transaction bytes on that mbarrier.

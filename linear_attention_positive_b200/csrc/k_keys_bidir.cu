@@ -197,8 +197,8 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
     // p_full / p_free: one barrier per (half, P buffer), so no waiter can fall two phases behind
     uint64_t *w_full = conv_full + STAGES, *p_full = w_full + 1, *p_free = p_full + 4;
     uint64_t *phi_full = p_free + 4, *phi_free = phi_full + 2, *acc_full = phi_free + 2, *acc_empty = acc_full + 2;
-    uint64_t *drain = acc_empty + 2;
-    uint32_t *tmem_slot = (uint32_t *)(drain + 1);
+    uint64_t *drain = acc_empty + 2, *stagger = drain + 2;
+    uint32_t *tmem_slot = (uint32_t *)(stagger + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
 
     pdl_launch_dependents();  // the state image kernel may stage its launch meanwhile
@@ -216,7 +216,7 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], halves);  // one MMA commit per feature half
             mbar_init(&vmax_full[s], 1);
             mbar_init(&conv_full[s], 128);
         }
@@ -231,7 +231,9 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
             mbar_init(&acc_full[h], 1);
             mbar_init(&acc_empty[h], 128);
         }
-        mbar_init(drain, 1);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
+        mbar_init(stagger, 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -299,30 +301,33 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 }
                 __syncwarp();
             }
-        } else if (warp == 13 && n > 0) {
-            // MMA issue by the whole (converged) warp through the predicated issue forms: per tile g,
-            // first the projection of tile g + NPB into the P buffer tile g has just been read out
-            // of, then the state MMAs of tile g once its V tile is converted and phi' is in TMEM.
+        } else if ((warp == 13 || warp == 15) && n > 0 && (warp == 13 || halves == 2)) {
+            // MMA issue for feature half h (warp 13: h = 0, warp 15: h = 1), by the whole converged
+            // warp through the predicated issue forms, so the halves never wait on each other: per
+            // tile g, first the projection of tile g + NPB into the P buffer tile g has just been
+            // read out of, then the state MMA of tile g once its V tile is converted and phi' is in
+            // TMEM.
+            const int h = warp == 13 ? 0 : 1;
             const uint32_t idesc1 = make_idesc(128, kKeyTile, kFmtBF16, 0, 0);
             const uint32_t idesc2 = make_idesc(128, ON, kFmtF16, 0, 1);
-            const uint64_t dW = make_sdesc(smem_u32(sW), 16, 1024), dS = make_sdesc(smem_u32(sStage), 16, 1024);
+            const uint64_t dW = make_sdesc(smem_u32(sW), 16, 1024) + (uint32_t)h * (128 * 128 / 16);
+            const uint64_t dS = make_sdesc(smem_u32(sStage), 16, 1024);
             const uint64_t dV = make_sdesc(smem_u32(sStage) + C::TILE, kKeyTile * 128, 1024);
             constexpr int NPB = C::NPB;
-            auto project = [&](int g, int h) {
-                const uint64_t a = dW + (uint32_t)h * (128 * 128 / 16);
+            auto project = [&](int g) {
                 const uint64_t b = dS + (uint32_t)(g % STAGES) * (C::STAGE / 16);
                 const uint32_t d = tmem + (uint32_t)(h * NPB + g % NPB) * 64;
-                mma_ss_x4_w(d, a, b, idesc1, 0u, 2, 2);
-                if (KB == 2) mma_ss_x4_w(d, a + (uint32_t)p.m * 8, b + kKeyTile * 128 / 16, idesc1, 1u, 2, 2);
+                mma_ss_x4_w(d, dW, b, idesc1, 0u, 2, 2);
+                if (KB == 2) mma_ss_x4_w(d, dW + (uint32_t)p.m * 8, b + kKeyTile * 128 / 16, idesc1, 1u, 2, 2);
                 mma_commit_w(&p_full[h * 2 + g % NPB]);
             };
             bool ok = mbar_wait_all(w_full, 0, abort_flag);
             for (int g = 0; ok && g < min(NPB, n); ++g) {
                 ok = mbar_wait_all(&full[g % STAGES], (g / STAGES) & 1, abort_flag);
                 tc_fence_after();
-                for (int h = 0; ok && h < halves; ++h) project(g, h);
+                if (ok) project(g);
             }
-            int runs[2] = {0, 0};
+            int runs = 0;
             int pos = f0 % nt;  // tile g's index within its head
             for (int g = 0; ok && g < n; ++g) {
                 const int s = g % STAGES;
@@ -330,34 +335,29 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 pos = pos + 1 == nt ? 0 : pos + 1;
                 if (g + NPB < n) {
                     const int g2 = g + NPB;
-                    ok = mbar_wait_all(&full[g2 % STAGES], (g2 / STAGES) & 1, abort_flag);
-                    for (int h = 0; ok && h < halves; ++h) {
-                        ok = mbar_wait_all(&p_free[h * 2 + g % NPB], (g / NPB) & 1, abort_flag);
-                        tc_fence_after();
-                        if (ok) project(g2, h);
-                    }
+                    ok = mbar_wait_all(&full[g2 % STAGES], (g2 / STAGES) & 1, abort_flag) &&
+                         mbar_wait_all(&p_free[h * 2 + g % NPB], (g / NPB) & 1, abort_flag);
+                    tc_fence_after();
                     if (!ok) break;
+                    project(g2);
                 }
                 ok = mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag);
-                const uint64_t vd = dV + (uint32_t)s * (C::STAGE / 16);
-                for (int h = 0; ok && h < halves; ++h) {
-                    if (first && runs[h] > 0) ok = mbar_wait_all(&acc_empty[h], (runs[h] - 1) & 1, abort_flag);
-                    if (ok) ok = mbar_wait_all(&phi_full[h], g & 1, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    mma_ts_x4_w(tmem + C::T_S + h * ON, tmem + C::T_PHI + h * 32, vd, idesc2, first ? 0u : 1u, 2048 / 16);
-                    mma_commit_w(&phi_free[h]);
-                    if (last) {
-                        mma_commit_w(&acc_full[h]);
-                        ++runs[h];
-                    }
-                }
+                if (ok && first && runs > 0) ok = mbar_wait_all(&acc_empty[h], (runs - 1) & 1, abort_flag);
+                if (ok) ok = mbar_wait_all(&phi_full[h], g & 1, abort_flag);
                 if (!ok) break;
+                tc_fence_after();
+                mma_ts_x4_w(tmem + C::T_S + h * ON, tmem + C::T_PHI + h * 32, dV + (uint32_t)s * (C::STAGE / 16), idesc2,
+                            first ? 0u : 1u, 2048 / 16);
+                mma_commit_w(&phi_free[h]);
+                if (last) {
+                    mma_commit_w(&acc_full[h]);
+                    ++runs;
+                }
                 mma_commit_w(&empty[s]);
             }
-            mma_commit_w(drain);
+            mma_commit_w(&drain[h]);
             volatile int no_abort = 0;
-            mbar_wait_all(drain, 0, &no_abort);
+            mbar_wait_all(&drain[h], 0, &no_abort);
         }
     } else if (warp >= 4) {
         regs_inc<184>();
@@ -374,7 +374,11 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 tc_fence_after();
                 tmem_ld64_nowait(tP, v);
             }
-            for (int g = 0; g < n; ++g) {
+            // The second half starts once the first has reached its first exponentials, so the two
+            // warps sharing an SM sub-partition (one per half) alternate on the MUFU pipe.
+            bool go = true;
+            if (h == 1 && n > 0) go = mbar_wait_all(stagger, 0, abort_flag);
+            for (int g = 0; go && g < n; ++g) {
                 const int s = g % STAGES, b = g % NPB;
                 const bool first = g == 0 || pos == 0, last = g == n - 1 || pos == nt - 1;
                 pos = pos + 1 == nt ? 0 : pos + 1;
@@ -389,6 +393,7 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 // new stabiliser: on a run's first tile always, later only when 2^t would overflow fp16
                 const float delta = (first || tmax > 15.f) ? ceilf(tmax - lim) : 0.f;
                 Dr = Dbase + delta;
+                if (h == 0 && g == 0 && halves == 2) mbar_arrive(stagger);
                 uint32_t hv[32];
                 key_features<POLY>(v, Dr, hv);
                 // prefetch the next tile's logits (its projection ran meanwhile)

@@ -1,0 +1,496 @@
+// Key side of the bidirectional bf16 tensor-core path for d = 64, on 128-token key tiles
+// ("Fast Attention Via Positive Orthogonal Random Features", codewithpapers.app/method/favor: the
+// FA-part needs (K')^T V and (K')^T 1_L).
+//
+//   k_key_partials_wide : per run, the partial state [S | z] = sum_j phi'(k_j) [v_j | 1] with
+//                         phi'_r(k) = 2^(A - D_r) exp(u_r(k)), u_r(k) = w_r.k - |k|^2/2, D_r a
+//                         per-feature stabiliser (log2 units) and A = 4. The output format is the
+//                         one k_key_partials writes (same slots, same per-run maxima), so the state
+//                         image kernel serves both.
+//
+// Why a second key kernel: on 64-token tiles each exponent warp spends most of a tile in fixed
+// per-tile costs (barrier round trips, TMEM load latency, the stabiliser vote) rather than on the
+// MUFU. Here a tile is 128 tokens and, except on a run's first tile, the projection is read once:
+//   - P_h^T = W_h K_tile^T (M = 128 features of half h, N = 128 tokens, K = 64);
+//   - per 32-token chunk c: t = P log2e + B_j - D_r, phi' = 2^t in fp16 stored to TMEM (16 packed
+//     columns), z_r += 2^-b_t sum_j phi', and the chunk's largest t, which decides (by a warp vote)
+//     whether D_r must be raised and the chunk redone; the next chunk's TMEM load is in flight
+//     meanwhile;
+//   - [S_h] += phi'_h V'_t (fp16 MMA, A from TMEM, B the converted V tile read MN-major, N = 64).
+// z_r is kept in the exponent thread's registers instead of a ones column of the state MMA, which
+// frees the TMEM columns the wider tile needs: per half P (128) + phi' (64) + S (64) = 256 columns.
+//
+// Stabiliser D_r (integer, per feature and run): on a run's first tile a separate pass over P finds
+// the row's largest t and sets D_r so that it lands in (A+b-1, A+b]; on later tiles D_r is kept
+// unless a chunk's largest t - D_r exceeds 15 (fp16 holds 2^t only below 2^16), in which case D_r
+// is raised, the row's accumulated [S | z] and the tile's already stored phi' chunks are scaled by
+// 2^-delta, and the chunk's exponentials are recomputed before they are stored. Typical inputs
+// raise it rarely. V'_t = V_t 2^-b_t as in k_key_partials.
+//
+// Warp roles (16 warps): 0-3 convert V, write the biases B_j (thread j = token j of the tile);
+// 4-7 / 8-11 exponentials of feature half 0 / 1 and the run-end write; 12 TMA; 13 / 15 MMA issue
+// for half 0 / 1; 14 the tile's largest |v|.
+
+#include "common.cuh"
+
+namespace favor {
+
+constexpr int kWideTile = 128;  // tokens per key tile of k_key_partials_wide
+
+struct WideCfg {
+    static constexpr int D = 64;
+    static constexpr int STAGES = 4;
+    static constexpr uint32_t TILE = kWideTile * 128;  // K or V tile: 128 rows of 64 bf16
+    static constexpr uint32_t STAGE = 2 * TILE;        // K tile | V tile
+    // TMEM columns of half h (base h * 256): P [0, 128), phi' [128, 192), [S_h] [192, 256)
+    static constexpr uint32_t T_P = 0, T_PHI = 128, T_S = 192, T_HALF = 256;
+};
+
+// Loads 32 consecutive fp32 columns of this thread's TMEM lane without waiting (warp-collective).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : FAVOR_REG32(v)
+        : "r"(taddr));
+}
+// Waits for this thread's outstanding TMEM loads; names v so no use of it moves above the wait.
+__device__ __forceinline__ void tmem_wait_ld32(float (&v)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32(v)::"memory");
+}
+// Loads 16 consecutive 32-bit columns of this thread's TMEM lane and waits for them.
+__device__ __forceinline__ void tmem_ld16u(uint32_t taddr, uint32_t (&h)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]), "=r"(h[4]), "=r"(h[5]), "=r"(h[6]), "=r"(h[7]), "=r"(h[8]),
+          "=r"(h[9]), "=r"(h[10]), "=r"(h[11]), "=r"(h[12]), "=r"(h[13]), "=r"(h[14]), "=r"(h[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(h[0]), "+r"(h[1]), "+r"(h[2]), "+r"(h[3]), "+r"(h[4]), "+r"(h[5]), "+r"(h[6]), "+r"(h[7]),
+                   "+r"(h[8]), "+r"(h[9]), "+r"(h[10]), "+r"(h[11]), "+r"(h[12]), "+r"(h[13]), "+r"(h[14]),
+                   "+r"(h[15])::"memory");
+}
+
+// Largest t = v log2e + B_j over a 32-token chunk (v the projection, bias the chunk's B_j).
+__device__ __forceinline__ float chunk_tmax(const float (&v)[32], const float *bias) {
+    float a = -INFINITY, b = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+        const float4 b4 = *(const float4 *)(bias + e);
+        a = fmax3(a, fmaf(v[e], kLog2e, b4.x), fmaf(v[e + 1], kLog2e, b4.y));
+        b = fmax3(b, fmaf(v[e + 2], kLog2e, b4.z), fmaf(v[e + 3], kLog2e, b4.w));
+    }
+    return fmaxf(a, b);
+}
+
+// t = v log2e + B_j - D for a 32-token chunk, in place; returns the chunk's largest t.
+__device__ __forceinline__ float chunk_shift(float (&v)[32], const float *bias, float D) {
+    float a = -INFINITY, b = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+        const float4 b4 = *(const float4 *)(bias + e);
+        v[e] = fmaf(v[e], kLog2e, b4.x) - D;
+        v[e + 1] = fmaf(v[e + 1], kLog2e, b4.y) - D;
+        v[e + 2] = fmaf(v[e + 2], kLog2e, b4.z) - D;
+        v[e + 3] = fmaf(v[e + 3], kLog2e, b4.w) - D;
+        a = fmax3(a, v[e], v[e + 1]);
+        b = fmax3(b, v[e + 2], v[e + 3]);
+    }
+    return fmaxf(a, b);
+}
+
+// phi' = 2^t for a 32-token chunk (t kept), rounded to fp16 pairs; returns the fp32 sum of phi'.
+// The first 32 - POLY exponentials go to MUFU ex2, the last POLY to the FMA-pipe polynomial.
+template <int POLY>
+__device__ __forceinline__ float chunk_exp(const float (&t)[32], uint32_t (&hv)[16]) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        float e0, e1;
+        if (e < 32 - POLY) {
+            e0 = ex2_approx(t[e]);
+            e1 = ex2_approx(t[e + 1]);
+        } else {
+            exp2_poly_pair(t[e], t[e + 1], e0, e1);
+        }
+        hv[e >> 1] = pack_f16x2(e0, e1);
+        s0 += e0;
+        s1 += e1;
+    }
+    return s0 + s1;
+}
+
+// The two fp16 halves of a 32-bit word as fp32 (low half first).
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t h) {
+    float lo, hi;
+    asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h));
+    return make_float2(lo, hi);
+}
+
+// Multiplies the fp16 pairs in 16 TMEM columns of this thread's lane by s (a power of two), in place.
+__device__ __forceinline__ void tmem_scale_f16x16(uint32_t taddr, float s) {
+    uint32_t h[16];
+    tmem_ld16u(taddr, h);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 f = unpack_f16x2(h[i]);
+        h[i] = pack_f16x2(f.x * s, f.y * s);
+    }
+    tmem_st16u(taddr, h);
+    tmem_wait_st();
+}
+
+template <int POLY>
+__global__ void __launch_bounds__(kKeyThreads, 1)
+k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                    const __grid_constant__ CUtensorMap mapW, KeyStateParams2 p) {
+    using C = WideCfg;
+    constexpr int STAGES = C::STAGES, D = C::D;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int halves = p.m / 128;
+    uint8_t *sW = smem;                                              // m rows of 128 B
+    uint8_t *sStage = sW + (size_t)p.m * 128;                        // [STAGES] K tile | V tile
+    float *sBias = (float *)(sStage + (size_t)STAGES * C::STAGE);   // [STAGES][128]
+    int *sShift = (int *)(sBias + STAGES * kWideTile);               // [STAGES] (16-int slot)
+    uint64_t *bars = (uint64_t *)(sShift + 16);
+    uint64_t *full = bars, *empty = full + STAGES, *vmax_full = empty + STAGES, *conv_full = vmax_full + STAGES;
+    // per feature half h: p_full / p_free (the P buffer), phi_full / phi_free (the phi' buffer),
+    // acc_full / acc_empty ([S_h] at a run's end), drain (the half's MMAs at exit)
+    uint64_t *w_full = conv_full + STAGES, *p_full = w_full + 1, *p_free = p_full + 2, *phi_full = p_free + 2;
+    uint64_t *phi_free = phi_full + 2, *acc_full = phi_free + 2, *acc_empty = acc_full + 2, *drain = acc_empty + 2;
+    uint32_t *tmem_slot = (uint32_t *)(drain + 2);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+
+    pdl_launch_dependents();  // the state image kernel may stage its launch meanwhile
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nt = p.f.nt;
+    const int f0 = blockIdx.x * p.f.T, f1 = min(f0 + p.f.T, p.f.total);
+    const int n = max(f1 - f0, 0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], halves);  // one MMA commit per feature half
+            mbar_init(&vmax_full[s], 1);
+            mbar_init(&conv_full[s], 128);
+        }
+        mbar_init(w_full, 1);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&p_full[h], 1);
+            mbar_init(&p_free[h], 128);
+            mbar_init(&phi_full[h], 128);
+            mbar_init(&phi_free[h], 1);
+            mbar_init(&acc_full[h], 1);
+            mbar_init(&acc_empty[h], 128);
+            mbar_init(&drain[h], 1);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 13) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp >= 12) {
+        regs_dec<88>();
+        if (warp == 12 && n > 0) {
+            if (elect_one()) {
+                prefetch_tensormap(&mapK);
+                prefetch_tensormap(&mapV);
+                prefetch_tensormap(&mapW);
+                mbar_arrive_expect_tx(w_full, p.m * 128);
+                tma_load_2d(sW, &mapW, w_full, 0, 0);
+            }
+            __syncwarp();
+            int issued = 0;
+            for (int g = 0; g < n; ++g) {
+                const int s = g % STAGES, fl = f0 + g;
+                if (!mbar_wait_lazy(&empty[s], ((g / STAGES) & 1) ^ 1, abort_flag)) break;
+                if (elect_one()) {
+                    uint8_t *st = sStage + (size_t)s * C::STAGE;
+                    mbar_arrive_expect_tx(&full[s], 2 * C::TILE);
+                    tma_load_3d(st, &mapK, &full[s], 0, (fl % nt) * kWideTile, fl / nt);
+                    tma_load_3d(st + C::TILE, &mapV, &full[s], 0, (fl % nt) * kWideTile, fl / nt);
+                }
+                __syncwarp();
+                ++issued;
+            }
+            volatile int no_abort = 0;
+            for (int i = max(issued - STAGES, 0); i < issued; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, &no_abort);
+            mbar_wait(w_full, 0, &no_abort);
+        } else if (warp == 14 && n > 0) {
+            // Largest |v| of each V tile (bf16 magnitudes compared as integers) -> b_t.
+            for (int g = 0; g < n; ++g) {
+                const int s = g % STAGES;
+                if (!mbar_wait_lazy(&full[s], (g / STAGES) & 1, abort_flag)) break;
+                const uint8_t *vt = sStage + (size_t)s * C::STAGE + C::TILE;
+                uint32_t mx = 0;
+#pragma unroll 4
+                for (int q = lane; q < (int)(C::TILE / 16); q += 32) {
+                    const uint4 w = *(const uint4 *)(vt + q * 16);
+                    mx = __vmaxu2(mx, w.x & 0x7FFF7FFFu);
+                    mx = __vmaxu2(mx, w.y & 0x7FFF7FFFu);
+                    mx = __vmaxu2(mx, w.z & 0x7FFF7FFFu);
+                    mx = __vmaxu2(mx, w.w & 0x7FFF7FFFu);
+                }
+                mx = max(mx & 0xFFFFu, mx >> 16);
+                for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                if (lane == 0) {
+                    const int e = (int)(mx >> 7) - 127;  // exponent of the largest |v| (-127 for an all-zero tile)
+                    sShift[s] = min(max(e - 7, -8), 7);
+                    mbar_arrive(&vmax_full[s]);
+                }
+                __syncwarp();
+            }
+        } else if ((warp == 13 || (warp == 15 && halves == 2)) && n > 0) {
+            // MMA issue for feature half h by the whole converged warp (predicated issue forms): per
+            // tile g, the projection of tile g + 1 once the exponent warps have read P(g), then the
+            // state MMA of tile g once its V tile is converted and phi'(g) is in TMEM.
+            const int h = warp == 13 ? 0 : 1;
+            const uint32_t tH = tmem + (uint32_t)h * C::T_HALF;
+            const uint32_t idesc_p = make_idesc(128, kWideTile, kFmtBF16, 0, 0);
+            const uint32_t idesc_s = make_idesc(128, D, kFmtF16, 0, 1);
+            const uint64_t dW = make_sdesc(smem_u32(sW) + (uint32_t)h * 128 * 128, 16, 1024);
+            const uint64_t dK = make_sdesc(smem_u32(sStage), 16, 1024);
+            const uint64_t dV = make_sdesc(smem_u32(sStage) + C::TILE, C::TILE, 1024);
+            auto project = [&](int g) {
+                mma_ss_x4_w(tH + C::T_P, dW, dK + (uint32_t)(g % STAGES) * (C::STAGE / 16), idesc_p, 0u, 2, 2);
+                mma_commit_w(&p_full[h]);
+            };
+            bool ok = mbar_wait_all(w_full, 0, abort_flag) && mbar_wait_all(&full[0], 0, abort_flag);
+            tc_fence_after();
+            if (ok) project(0);
+            int runs = 0;
+            int pos = f0 % nt;  // tile g's index within its head
+            for (int g = 0; ok && g < n; ++g) {
+                const int s = g % STAGES;
+                const bool first = g == 0 || pos == 0, last = g == n - 1 || pos == nt - 1;
+                pos = pos + 1 == nt ? 0 : pos + 1;
+                if (g + 1 < n) {
+                    ok = mbar_wait_all(&full[(g + 1) % STAGES], ((g + 1) / STAGES) & 1, abort_flag) &&
+                         mbar_wait_all(&p_free[h], g & 1, abort_flag);
+                    tc_fence_after();
+                    if (!ok) break;
+                    project(g + 1);
+                }
+                ok = mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag);
+                if (ok && first && runs > 0) ok = mbar_wait_all(&acc_empty[h], (runs - 1) & 1, abort_flag);
+                if (ok) ok = mbar_wait_all(&phi_full[h], g & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t vd = dV + (uint32_t)s * (C::STAGE / 16);
+                mma_ts_x4_w(tH + C::T_S, tH + C::T_PHI, vd, idesc_s, first ? 0u : 1u, 2048 / 16);
+                mma_ts_x4_w(tH + C::T_S, tH + C::T_PHI + 32, vd + 8192 / 16, idesc_s, 1u, 2048 / 16);
+                mma_commit_w(&phi_free[h]);
+                if (last) {
+                    mma_commit_w(&acc_full[h]);
+                    ++runs;
+                }
+                mma_commit_w(&empty[s]);
+            }
+            mma_commit_w(&drain[h]);
+            volatile int no_abort = 0;
+            mbar_wait_all(&drain[h], 0, &no_abort);
+        }
+    } else if (warp >= 4) {
+        regs_inc<160>();
+        const int h = (warp - 4) >> 2, row = (warp & 3) * 32 + lane;
+        if (h < halves && n > 0) {
+            const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
+            const uint32_t tH = tmem + lane_off + (uint32_t)h * C::T_HALF;
+            const uint32_t tP = tH + C::T_P, tPHI = tH + C::T_PHI, tS = tH + C::T_S;
+            int runs = 0;
+            float Dr = 0.f;  // this feature's stabiliser D_r in the current run
+            float z = 0.f;   // this feature's normaliser entry z_r of the current run (2^-b_t scale)
+            int pos = f0 % nt;
+            float va[32], vb[32], vc[32];
+            for (int g = 0; g < n; ++g) {
+                const int s = g % STAGES;
+                const bool first = g == 0 || pos == 0, last = g == n - 1 || pos == nt - 1;
+                pos = pos + 1 == nt ? 0 : pos + 1;
+                if (!mbar_wait_all(&p_full[h], g & 1, abort_flag) ||
+                    !mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag))
+                    break;
+                tc_fence_after();
+                const float *bias = sBias + s * kWideTile;
+                const int bt = sShift[s];
+                const float lim = kKeyFeatureShift + (float)bt;  // target for a run's largest t
+                if (first) {
+                    // a run's first tile: D_r from the row's largest t over the whole tile
+                    tmem_ld32_nowait(tP, va);
+                    tmem_wait_ld32(va);
+                    tmem_ld32_nowait(tP + 32, vb);
+                    float tm = chunk_tmax(va, bias);
+                    tmem_wait_ld32(vb);
+                    tmem_ld32_nowait(tP + 64, va);
+                    tm = fmaxf(tm, chunk_tmax(vb, bias + 32));
+                    tmem_wait_ld32(va);
+                    tmem_ld32_nowait(tP + 96, vb);
+                    tm = fmaxf(tm, chunk_tmax(va, bias + 64));
+                    tmem_wait_ld32(vb);
+                    tm = fmaxf(tm, chunk_tmax(vb, bias + 96));
+                    Dr = ceilf(tm - lim);
+                    z = 0.f;
+                }
+                float zs = 0.f;  // this tile's sum of phi'
+                // One 32-token chunk: t, phi' and the chunk's largest t (in parallel); on a later tile of
+                // the run, a chunk that would overflow fp16 raises D_r (rescaling what already carries
+                // the old D_r) and is redone. phi'(g) overwrites phi'(g - 1), so before the first store
+                // the state MMA of tile g - 1 must have read it (which also makes [S] safe to rescale).
+                auto chunk = [&](float(&v)[32], int c) -> bool {
+                    const float cm = chunk_shift(v, bias + 32 * c, Dr);
+                    uint32_t hv[16];
+                    float cs = chunk_exp<POLY>(v, hv);
+                    if (c == 0) {
+                        if (g > 0 && !mbar_wait_all(&phi_free[h], (g - 1) & 1, abort_flag)) return false;
+                        tc_fence_after();
+                    }
+                    if (!first && __any_sync(0xffffffffu, cm > 15.f)) {
+                        const float delta = cm > 15.f ? ceilf(cm - lim) : 0.f;
+                        const float sc = __uint_as_float((uint32_t)(127 - (int)delta) << 23);  // 2^-delta
+                        tmem_wait_st();
+                        tmem_scale_row(tS, D, sc);
+                        for (int cc = 0; cc < c; ++cc) tmem_scale_f16x16(tPHI + 16 * cc, sc);
+                        z *= sc;
+                        zs *= sc;
+                        Dr += delta;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] -= delta;
+                        cs = chunk_exp<POLY>(v, hv);
+                    }
+                    zs += cs;
+                    tmem_st16u(tPHI + 16 * c, hv);
+                    return true;
+                };
+                tmem_ld32_nowait(tP, va);
+                tmem_wait_ld32(va);
+                tmem_ld32_nowait(tP + 32, vb);
+                if (!chunk(va, 0)) break;
+                tmem_wait_ld32(vb);
+                tmem_ld32_nowait(tP + 64, va);
+                chunk(vb, 1);
+                tmem_wait_ld32(va);
+                tmem_ld32_nowait(tP + 96, vb);
+                chunk(va, 2);
+                tmem_wait_ld32(vb);
+                // P(g) is in registers: the buffer is free for the projection of tile g + 1
+                tc_fence_before();
+                mbar_arrive(&p_free[h]);
+                chunk(vb, 3);
+                z = fmaf(zs, __uint_as_float((uint32_t)(127 - bt) << 23), z);  // z_r += 2^-b_t sum_j phi'
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&phi_full[h]);
+                if (last) {
+                    if (!mbar_wait_all(&acc_full[h], runs & 1, abort_flag)) break;
+                    tc_fence_after();
+                    const int bh = (f0 + g) / nt;
+                    const size_t rs = (size_t)blockIdx.x + bh;
+                    float *dst = p.part + rs * (D + 1) * p.m + h * 128 + row;
+                    float amax = fabsf(z);
+#pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        tmem_ld32(tS + c0, va);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            dst[(size_t)(c0 + c) * p.m] = va[c];
+                            amax = fmaxf(amax, fabsf(va[c]));
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&acc_empty[h]);
+                    dst[(size_t)D * p.m] = z;
+                    p.part_D[rs * p.m + h * 128 + row] = Dr;
+                    float dmax = Dr;
+                    for (int o = 16; o > 0; o >>= 1) {
+                        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                        dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+                    }
+                    if (lane == 0) {
+                        p.part_amax[rs * 8 + h * 4 + (warp & 3)] = amax;
+                        p.part_Dmax[rs * 8 + h * 4 + (warp & 3)] = dmax;
+                    }
+                    ++runs;
+                }
+            }
+        }
+    } else {
+        regs_dec<88>();
+        // Converter warpgroup: thread j handles token j of each tile (its |k_j|^2 and bias) and
+        // converts 8 of the V tile's 16-byte chunks.
+        const int j = threadIdx.x;
+        for (int g = 0; g < n; ++g) {
+            const int s = g % STAGES, t = (f0 + g) % nt;
+            if (!mbar_wait_lazy(&vmax_full[s], (g / STAGES) & 1, abort_flag)) break;
+            uint8_t *st = sStage + (size_t)s * C::STAGE;
+            const int b = sShift[s];
+            const float scale = __uint_as_float((uint32_t)(127 - b) << 23);  // 2^-b
+#pragma unroll
+            for (int i = 0; i < (int)(C::TILE / 16 / 128); ++i) {
+                uint4 *q = (uint4 *)(st + C::TILE + (size_t)(j + 128 * i) * 16);
+                uint4 w = *q;
+                uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    u[k] = pack_f16x2(__uint_as_float(u[k] << 16) * scale, __uint_as_float(u[k] & 0xFFFF0000u) * scale);
+                *q = make_uint4(u[0], u[1], u[2], u[3]);
+            }
+            const bool valid = t * kWideTile + j < p.L;
+            const float k2 = key_sq_norm<1, kWideTile>(st, j);
+            sBias[s * kWideTile + j] = valid ? fmaf(-0.5f * k2, kLog2e, kKeyFeatureShift + (float)b) : -INFINITY;
+            fence_async_smem();
+            mbar_arrive(&conv_full[s]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 13) tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================ host launchers
+
+static size_t key_wide_smem(int m) {
+    using C = WideCfg;
+    return 1024 + (size_t)m * 128 + (size_t)C::STAGES * C::STAGE + C::STAGES * kWideTile * 4 + 64 + 512;
+}
+
+// The register split (88 + 2 x 160 + 88 per warpgroup lane) fits the 128 per thread the kernel is
+// launched with; the launch is refused unless the kernel carries exactly 128.
+template <int POLY>
+static cudaError_t launch_key_wide_t(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mW,
+                                     const KeyStateParams2 &p, cudaStream_t st) {
+    static int checked = 0;
+    if (checked == 0) {
+        cudaFuncAttributes a{};
+        checked = (cudaFuncGetAttributes(&a, k_key_partials_wide<POLY>) == cudaSuccess && a.numRegs == 128) ? 1 : -1;
+    }
+    if (checked < 0) return cudaErrorInvalidConfiguration;
+    const size_t sm = key_wide_smem(p.m);
+    cudaFuncSetAttribute(k_key_partials_wide<POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_key_partials_wide<POLY><<<p.f.n_cta, kKeyThreads, sm, st>>>(mK, mV, mW, p);
+    return cudaGetLastError();
+}
+
+// d = 64 only; K and V maps with 128-row boxes, p.f built on 128-token tiles.
+cudaError_t launch_key_partials_wide(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mW,
+                                     const KeyStateParams2 &p, int poly_pct, cudaStream_t st) {
+    const int poly = poly_pct < 13 ? 0 : poly_pct < 31 ? 8 : poly_pct < 44 ? 12 : 16;
+    switch (poly) {
+        case 0: return launch_key_wide_t<0>(mK, mV, mW, p, st);
+        case 8: return launch_key_wide_t<8>(mK, mV, mW, p, st);
+        case 12: return launch_key_wide_t<12>(mK, mV, mW, p, st);
+        default: return launch_key_wide_t<16>(mK, mV, mW, p, st);
+    }
+}
+
+}  // namespace favor

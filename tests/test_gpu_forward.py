@@ -114,6 +114,30 @@ def test_bf16_key_stabiliser_raised_within_a_range(cuda_device):
     assert rel_max_err(out, oracle_fwd(x, W64, False)) <= TOL["bf16"]
 
 
+def test_bf16_key_stabiliser_raised_inside_a_wide_tile(cuda_device):
+    # d = 64 runs on 128-token key tiles read in 32-token chunks. Keys k_j = a_q w_0 + noise with a_q
+    # rising from 0.2 to 1.0 over 12 consecutive 32-token chunks (three tiles) and then falling back:
+    # inside a CTA's range the stabiliser set on its first tile is raised in the middle of later
+    # tiles, so chunks already stored with the old value are rescaled along with the state.
+    L = 128 * 600
+    w = Workload("t", 1, 1, L, 64, 256, False, "bf16", False, 2, 59)
+    x = make_inputs(w)
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    w0 = W64[0].astype(np.float32)[None, :]
+    q = (np.arange(L) // 32) % 12
+    a = (0.2 + 0.8 * q / 11.0).astype(np.float32)[:, None]
+    x["K"][0, 0] = a * w0 + 0.3 * x["K"][0, 0]
+    x["Q"][0, 0] = 0.1 * w0 + x["Q"][0, 0]
+    x["K"] = round_to_bf16(x["K"])
+    x["Q"] = round_to_bf16(x["Q"])
+    K64 = x["K"][0, 0].astype(np.float64)
+    u0 = K64 @ W64[0] - 0.5 * (K64 ** 2).sum(1)
+    assert u0[352:384].max() - u0[:32].max() > 12.0  # nats: more than the 2^15 headroom of fp16
+    out = run_fwd(w, x, Wr, cuda_device, causal=False)
+    assert np.isfinite(out).all()
+    assert rel_max_err(out, oracle_fwd(x, W64, False)) <= TOL["bf16"]
+
+
 def test_bf16_value_tiles_of_very_different_magnitude(cuda_device):
     # One key tile's values near 3e4 and another's near 1e-5: the per-tile power-of-two scaling
     # of V keeps both inside fp16's normal range.
