@@ -34,7 +34,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TF32_PER_BF16 = 1.1 / 2.25   # nominal dense tf32 : bf16 tensor rate
 L2_FLUSH_BYTES = 256 << 20
 
-# Kernels favor_fwd launches for the bf16 path, in launch order (stage k <-> events 2k, 2k+1).
+# Kernels favor_fwd launches for the bf16 path, in launch order (stage k <-> events 2k, 2k+1); for
+# d = 64 the key-state kernel is k_key_partials_wide (128-token key tiles).
 FWD_STAGES = ["k_key_partials", "k_state_image", "k_query_out"]
 CAUSAL_STAGES = ["k_key_logit_max", "k_key_state", "k_state_scan", "k_causal_chunk", "gemm_causal_prefix"]
 # Kernels favor_bwd launches (bf16 bidirectional: split-precision GEMM passes and two reductions).
@@ -62,7 +63,7 @@ def stage_work(name, w, n_sms=148):
     BH = w.B * w.H
     if name == "k_key_max":            # read K
         return t * 2 * d, 2 * m * d * t, 0
-    if name == "k_key_partials":       # read K, V; MMAs K W^T and phi'(K)^T [V | 1]
+    if name in ("k_key_partials", "k_key_partials_wide"):  # read K, V; MMAs K W^T and phi'(K)^T [V | 1]
         return t * 4 * d, 2 * m * d * t + 2 * m * (d + 1) * t, 0
     if name == "k_state_image":        # read the per-run partial states and stabilisers, write the fp16 images
         runs = n_sms + BH - 1
@@ -344,6 +345,8 @@ def stage_names(w):
     if w.dtype != "bf16":
         return ["k_f32_head"] + (["k_f32_head_bwd"] if w.backward else [])
     names = list(CAUSAL_STAGES if w.causal else FWD_STAGES)
+    if not w.causal and w.d == 64:
+        names[0] = "k_key_partials_wide"
     if w.backward:
         names += BWD_CAUSAL_STAGES if w.causal else BWD_STAGES
     return names
