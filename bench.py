@@ -352,13 +352,38 @@ def stage_names(w):
     return names
 
 
-def stage_roofline(name, w, ms, peaks, peak_src, n_sms, traffic_key=None):
+def stage_exps(name, w):
+    """MUFU transcendental evaluations (exp2; sin and cos for the trigonometric map) of one launch."""
+    t, m = w.tokens, w.m
+    per_feature = 0 if w.feature_map == "relu" else (2 if w.feature_map == "trig" else 1)
+    if name in ("k_key_partials", "k_key_partials_wide", "k_query_out", "k_key_state", "gemm_phi_k",
+                "gemm_phi_q"):
+        return per_feature * m * t
+    if name in ("k_causal_chunk", "sp_state+sp_output"):
+        return 2 * per_feature * m * t
+    return 0
+
+
+def stage_roofline(name, w, ms, peaks, peak_src, n_sms, clk=None, traffic_key=None):
+    """The launch against the slowest of its three bounds: HBM bytes at the copy bandwidth, tensor
+    FLOPs at the bf16 rate, and MUFU exponentials at 16 per clock per SM at the sampled SM clock
+    (reported as "alu": the special-function unit is the arithmetic unit that binds)."""
     nbytes, f_bf16, f_tf32 = stage_work(name, w, n_sms)
+    exps = stage_exps(name, w)
     sec = ms * 1e-3
     hbm_peak, tc_peak = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    mhz = clk["sm_mhz"] if clk and clk.get("sm_mhz") else 1965.0
+    mufu_peak = 16 * n_sms * mhz * 1e6 / 1e9   # G ex2 / s
     t_hbm = nbytes / (hbm_peak * 1e9)
     t_tc = f_bf16 / (tc_peak * 1e12) + f_tf32 / (tc_peak * TF32_PER_BF16 * 1e12)
+    t_mufu = exps / (mufu_peak * 1e9)
     traffic = measured_traffic(name, traffic_key or w.name)
+    if t_mufu > max(t_tc, t_hbm):
+        return {"kernel": name, "bound": "alu", "achieved": exps / sec / 1e9, "peak": mufu_peak, "unit": "Gexp2/s",
+                "frac": (exps / sec / 1e9) / mufu_peak, "traffic": traffic, "algorithmic_exps": exps,
+                "note": f"MUFU ex2 at 16 per clock per SM x {n_sms} SMs at {mhz:.0f} MHz; the tensor bound "
+                        f"({t_tc * 1e6:.1f} us) and the HBM bound ({t_hbm * 1e6:.1f} us, {peak_src} copy "
+                        f"bandwidth) are lower"}
     if t_tc > t_hbm:
         eq = f_bf16 + f_tf32 / TF32_PER_BF16
         return {"kernel": name, "bound": "tensor", "achieved": eq / sec / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
@@ -372,8 +397,8 @@ def stage_roofline(name, w, ms, peaks, peak_src, n_sms, traffic_key=None):
 
 def path_roofline(w, ms_per_step, peaks, clk, n_sm):
     """Path-level fractions (work of the definition, not of the kernels): Q, K, V (and dO) bf16 read,
-    out (and dQ, dK, dV) fp32 written, at the measured copy bandwidth; 6 L m d FLOPs per head for the
-    forward (twice that again for the backward) at the measured bf16 rate; 2 m exponentials per
+    out (and dQ, dK, dV) fp32 written, at the copy bandwidth; 6 L m d FLOPs per head for the
+    forward (twice that again for the backward) at the bf16 rate; 2 m exponentials per
     token per pass at 16 MUFU ex2 per clock per SM, at the SM clock sampled during the timed steps."""
     bwd = 1 if w.backward else 0
     path_bytes = w.tokens * ((6 * w.d + 4 * w.d) + bwd * (8 * w.d + 12 * w.d))
@@ -385,8 +410,9 @@ def path_roofline(w, ms_per_step, peaks, clk, n_sm):
     return {"hbm_bytes_per_step": path_bytes, "hbm_frac": path_bytes / step_s / (peaks["hbm_gbs"] * 1e9),
             "tensor_flops_per_step": path_flops, "tensor_frac": path_flops / step_s / (peaks["bf16_tflops"] * 1e12),
             "exps_per_step": path_exps, "mufu_frac": path_exps / step_s / (16 * n_sm * sm_hz),
-            "note": "hbm: bf16 inputs + fp32 outputs; tensor: 6 L m d per head forward, 12 L m d backward, "
-                    "at the measured bf16 peak; mufu: 2 m ex2 per token per pass at 16 per clock per SM"}
+            "note": "hbm: bf16 inputs + fp32 outputs at the copy bandwidth; tensor: 6 L m d per head forward, "
+                    "12 L m d backward, at the bf16 peak (peaks: MEASURED_PEAKS.json when present, else the "
+                    "fallback); mufu: 2 m ex2 per token per pass at 16 per clock per SM"}
 
 
 class Runner:
@@ -536,7 +562,7 @@ def workload_summary(r, step_ms_list, stage_ms, peaks, peak_src, clk, n_sm, worl
            "stage_ms": {k: round(v, 5) for k, v in stage_ms.items()}}
     if w.dtype == "bf16":
         dom = max(stage_ms, key=stage_ms.get)
-        rec["roofline"] = stage_roofline(dom.split("#")[0], w, stage_ms[dom], peaks, peak_src, n_sm)
+        rec["roofline"] = stage_roofline(dom.split("#")[0], w, stage_ms[dom], peaks, peak_src, n_sm, clk)
         rec["path_roofline"] = path_roofline(w, ms_per_step, peaks, clk, n_sm)
     return rec
 
@@ -590,7 +616,10 @@ def run_ours(args, w):
     clk = clocks.stop()
     for k, rec in others.items():  # MUFU fractions at the clock sampled over all timed loops
         if "path_roofline" in rec:
-            rec["path_roofline"] = path_roofline(WORKLOADS[int(k)], rec["ms_per_step"], peaks, clk, n_sm)
+            wk = WORKLOADS[int(k)]
+            rec["path_roofline"] = path_roofline(wk, rec["ms_per_step"], peaks, clk, n_sm)
+            dom = max(rec["stage_ms"], key=rec["stage_ms"].get)
+            rec["roofline"] = stage_roofline(dom.split("#")[0], wk, rec["stage_ms"][dom], peaks, peak_src, n_sm, clk)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -611,7 +640,7 @@ def run_ours(args, w):
     if w.dtype == "bf16":
         line["stage_ms"] = {k: round(v, 5) for k, v in headline_stage_ms.items()}
         dom = max(headline_stage_ms, key=headline_stage_ms.get)
-        line["roofline"] = stage_roofline(dom.split("#")[0], w, headline_stage_ms[dom], peaks, peak_src, n_sm)
+        line["roofline"] = stage_roofline(dom.split("#")[0], w, headline_stage_ms[dom], peaks, peak_src, n_sm, clk)
         line["path_roofline"] = path_roofline(w, ms_per_step, peaks, clk, n_sm)
     if clk is not None:
         line["clocks"] = clk
