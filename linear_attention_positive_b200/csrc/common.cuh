@@ -382,6 +382,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32(v)::"memory");
 }
 
+// Loads 32 consecutive fp32 columns of this thread's TMEM lane without waiting (warp-collective).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : FAVOR_REG32(v)
+        : "r"(taddr));
+}
+// Waits for this thread's outstanding TMEM loads; names v so no use of it moves above the wait.
+__device__ __forceinline__ void tmem_wait_ld32(float (&v)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32(v)::"memory");
+}
+
 // Stores 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective; not waited).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
     asm volatile(

@@ -46,18 +46,6 @@ struct WideCfg {
     static constexpr uint32_t T_P = 0, T_PHI = 128, T_S = 192, T_HALF = 256;
 };
 
-// Loads 32 consecutive fp32 columns of this thread's TMEM lane without waiting (warp-collective).
-__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float (&v)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : FAVOR_REG32(v)
-        : "r"(taddr));
-}
-// Waits for this thread's outstanding TMEM loads; names v so no use of it moves above the wait.
-__device__ __forceinline__ void tmem_wait_ld32(float (&v)[32]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" : FAVOR_RW32(v)::"memory");
-}
 // Loads 16 consecutive 32-bit columns of this thread's TMEM lane and waits for them.
 __device__ __forceinline__ void tmem_ld16u(uint32_t taddr, uint32_t (&h)[16]) {
     asm volatile(
@@ -84,16 +72,18 @@ __device__ __forceinline__ float chunk_tmax(const float (&v)[32], const float *b
     return fmaxf(a, b);
 }
 
-// t = v log2e + B_j - D for a 32-token chunk, in place; returns the chunk's largest t.
+// t = v log2e + B_j - D for a 32-token chunk, in place (paired FMA-pipe instructions); returns the
+// chunk's largest t.
 __device__ __forceinline__ float chunk_shift(float (&v)[32], const float *bias, float D) {
     float a = -INFINITY, b = -INFINITY;
 #pragma unroll
     for (int e = 0; e < 32; e += 4) {
         const float4 b4 = *(const float4 *)(bias + e);
-        v[e] = fmaf(v[e], kLog2e, b4.x) - D;
-        v[e + 1] = fmaf(v[e + 1], kLog2e, b4.y) - D;
-        v[e + 2] = fmaf(v[e + 2], kLog2e, b4.z) - D;
-        v[e + 3] = fmaf(v[e + 3], kLog2e, b4.w) - D;
+        float c0, c1, c2, c3;
+        ffma2(b4.x, b4.y, 1.f, 1.f, -D, -D, c0, c1);  // B_j - D
+        ffma2(b4.z, b4.w, 1.f, 1.f, -D, -D, c2, c3);
+        ffma2(v[e], v[e + 1], kLog2e, kLog2e, c0, c1, v[e], v[e + 1]);
+        ffma2(v[e + 2], v[e + 3], kLog2e, kLog2e, c2, c3, v[e + 2], v[e + 3]);
         a = fmax3(a, v[e], v[e + 1]);
         b = fmax3(b, v[e + 2], v[e + 3]);
     }
@@ -115,8 +105,7 @@ __device__ __forceinline__ float chunk_exp(const float (&t)[32], uint32_t (&hv)[
             exp2_poly_pair(t[e], t[e + 1], e0, e1);
         }
         hv[e >> 1] = pack_f16x2(e0, e1);
-        s0 += e0;
-        s1 += e1;
+        ffma2(e0, e1, 1.f, 1.f, s0, s1, s0, s1);
     }
     return s0 + s1;
 }

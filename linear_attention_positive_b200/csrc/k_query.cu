@@ -232,7 +232,7 @@ __device__ __forceinline__ void query_features(float (&v)[128], float cl, uint32
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int e = c * 32; e < c * 32 + 32; ++e) v[e] = fmaf(v[e], kLog2e, -cl);
+        for (int e = c * 32; e < c * 32 + 32; e += 2) ffma2(v[e], v[e + 1], kLog2e, kLog2e, -cl, -cl, v[e], v[e + 1]);
 #pragma unroll
         for (int e = c * 32; e < c * 32 + 32 - POLY; ++e) v[e] = ex2_approx(v[e]);
 #pragma unroll
