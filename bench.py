@@ -37,7 +37,7 @@ L2_FLUSH_BYTES = 256 << 20
 # Kernels favor_fwd launches for the bf16 path, in launch order (stage k <-> events 2k, 2k+1); for
 # d = 64 the key-state kernel is k_key_partials_wide (128-token key tiles).
 FWD_STAGES = ["k_key_partials", "k_state_image", "k_query_out"]
-CAUSAL_STAGES = ["k_key_logit_max", "k_key_state", "k_state_scan", "k_causal_chunk", "gemm_causal_prefix"]
+CAUSAL_STAGES = ["k_key_partials_wide", "k_segment_scan", "k_causal_chunk", "gemm_causal_prefix"]
 # Kernels favor_bwd launches (bf16 bidirectional: split-precision GEMM passes and two reductions).
 BWD_STAGES = ["gemm_phi_k", "gemm_state_partial", "reduce_state", "gemm_phi_q", "gemm_gs", "gemm_t_q", "gemm_dq",
               "gemm_G_partial", "reduce_G", "gemm_dv", "gemm_t_k", "gemm_dk"]
@@ -61,19 +61,18 @@ def stage_work(name, w, n_sms=148):
     """Algorithmic HBM bytes and tensor FLOPs (bf16/fp16 rate, tf32 rate) of one launch of a stage."""
     t, d, m = w.tokens, w.d, w.m
     BH = w.B * w.H
-    if name == "k_key_max":            # read K
-        return t * 2 * d, 2 * m * d * t, 0
     if name in ("k_key_partials", "k_key_partials_wide"):  # read K, V; MMAs K W^T and phi'(K)^T [V | 1]
+        if w.causal:                   # the causal instantiation also writes -|k|^2/2 per key
+            return t * (4 * d + 4), 2 * m * d * t + 2 * m * (d + 1) * t, 0
         return t * 4 * d, 2 * m * d * t + 2 * m * (d + 1) * t, 0
     if name == "k_state_image":        # read the per-run partial states and stabilisers, write the fp16 images
         runs = n_sms + BH - 1
         return runs * (d + 2) * m * 4 + BH * (d // 64) * (m // 128) * 20480, 0, 0
+    if name == "k_segment_scan":       # read the per-segment states and stabilisers, write the prefixes
+        n_seg = BH * ((((w.L + 127) // 128) + 7) // 8)
+        return n_seg * m * (2 * (d + 1) + 1) * 4, 0, 0
     if name == "k_query_out":          # read Q; write fp32 out; MMAs Q W^T and phi(Q) [S | z]
         return t * (2 * d + 4 * d), 2 * m * d * t + 2 * m * (d + 1) * t, 0
-    if name == "k_key_logit_max":      # read K; write -|k|^2/2
-        return t * (2 * d + 4), 2 * m * d * t, 0
-    if name == "k_key_state":          # read K, V, -|k|^2/2
-        return t * (4 * d + 4), 2 * m * d * t, 2 * m * d * t
     # Backward passes: the bytes each launch must move given the materialised hi/lo bf16
     # intermediates (4 B per element: phi(K), phi(Q), t are m wide, [g | s] is d + 64 wide) and the
     # tensor FLOPs of its split products (3 MMAs when both operands are split, 2 when one is exact).
@@ -356,7 +355,7 @@ def stage_exps(name, w):
     """MUFU transcendental evaluations (exp2; sin and cos for the trigonometric map) of one launch."""
     t, m = w.tokens, w.m
     per_feature = 0 if w.feature_map == "relu" else (2 if w.feature_map == "trig" else 1)
-    if name in ("k_key_partials", "k_key_partials_wide", "k_query_out", "k_key_state", "gemm_phi_k",
+    if name in ("k_key_partials", "k_key_partials_wide", "k_query_out", "gemm_phi_k",
                 "gemm_phi_q"):
         return per_feature * m * t
     if name in ("k_causal_chunk", "sp_state+sp_output"):

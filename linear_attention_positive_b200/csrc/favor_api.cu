@@ -14,10 +14,9 @@
 #include "common.cuh"
 
 #include "k_fp32.cu"
-#include "k_keys.cu"
 #include "k_keys_bidir.cu"
-#include "k_keys_wide.cu"
 #include "k_query.cu"
+#include "k_keys_wide.cu"
 #include "k_causal.cu"
 #include "k_gemm.cu"
 #include "k_selftest.cu"
@@ -77,46 +76,50 @@ constexpr int kCausalExactPrefix = 512;
 // Key columns of the prefix's masked score matrix: P rounded up to the 128-wide GEMM tile.
 int prefix_cols(int P) { return (P + 127) & ~127; }
 
+// Causal bf16 forward: per-key -|k|^2/2, the per-segment partial states of k_key_partials_wide
+// ([S' | z'] columns feature-minor, per-feature stabilisers, per-warp maxima), the exclusive
+// segment prefixes at the head reference, and the exact prefix's features and scores.
 struct Bf16Layout {
-    int BH, n_tiles, tiles_per_split, n_split, P_exact, Ppad;
-    size_t off_bias, off_split_max, off_head_max, off_part_S, off_part_z, off_state, off_seg_S, off_seg_z,
+    int BH, n_tiles, tiles_per_split, n_split, n_seg, P_exact, Ppad;
+    size_t off_bias, off_head_max, off_part, off_part_D, off_part_amax, off_part_umax, off_seg_S, off_seg_z,
         off_kref, off_pq[2], off_pk[2], off_pa[2], total;
 };
 
-Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o, bool state_in_ws, int causal = 0) {
+Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o) {
     Bf16Layout l{};
     l.BH = s->B * s->H;
     l.n_tiles = (s->L + kTile - 1) / kTile;
     l.tiles_per_split = opt_split_tiles(o);
     l.n_split = (l.n_tiles + l.tiles_per_split - 1) / l.tiles_per_split;
+    l.n_seg = l.BH * l.n_split;
     size_t off = 0;
     l.off_bias = off;
     off += align256((size_t)l.BH * s->L * 4);
-    l.off_split_max = off;
-    off += align256((size_t)l.BH * l.n_split * 4);
     l.off_head_max = off;
     off += align256((size_t)l.BH * 4);
-    l.off_part_S = off;
-    off += align256((size_t)l.BH * l.n_split * s->m * s->d * 4);
-    l.off_part_z = off;
-    off += align256((size_t)l.BH * l.n_split * s->m * 4);
-    l.off_state = off;
-    if (state_in_ws) off += align256((size_t)l.BH * state_floats(s->m, s->d) * 4);
-    l.P_exact = causal ? std::min(s->L, kCausalExactPrefix) : 0;
+    l.off_part = off;
+    off += align256((size_t)l.n_seg * (s->d + 1) * s->m * 4);
+    l.off_part_D = off;
+    off += align256((size_t)l.n_seg * s->m * 4);
+    l.off_part_amax = off;
+    off += align256((size_t)l.n_seg * 8 * 4);
+    l.off_part_umax = off;
+    off += align256((size_t)l.n_seg * 8 * 4);
+    l.P_exact = std::min(s->L, kCausalExactPrefix);
     l.off_seg_S = off;
-    if (causal) off += align256((size_t)l.BH * l.n_split * s->m * s->d * 4);
+    off += align256((size_t)l.n_seg * s->m * s->d * 4);
     l.off_seg_z = off;
-    if (causal) off += align256((size_t)l.BH * l.n_split * s->m * 4);
+    off += align256((size_t)l.n_seg * s->m * 4);
     l.Ppad = prefix_cols(l.P_exact);
     l.off_kref = off;
-    if (causal) off += align256((size_t)l.BH * 4);
+    off += align256((size_t)l.BH * 4);
     for (int i = 0; i < 2; ++i) {
         l.off_pq[i] = off;
-        if (causal) off += align256((size_t)l.BH * l.P_exact * s->m * 2);
+        off += align256((size_t)l.BH * l.P_exact * s->m * 2);
         l.off_pk[i] = off;
-        if (causal) off += align256((size_t)l.BH * l.P_exact * s->m * 2);
+        off += align256((size_t)l.BH * l.P_exact * s->m * 2);
         l.off_pa[i] = off;
-        if (causal) off += align256((size_t)l.BH * l.P_exact * l.Ppad * 2);
+        off += align256((size_t)l.BH * l.P_exact * l.Ppad * 2);
     }
     l.total = off;
     return l;
@@ -418,7 +421,7 @@ favor_status causal_prefix(const favor_shape *s, const Bf16Layout &l, const void
     ak.out_hi = pk[0];
     ak.out_lo = pk[1];
     ak.kc = kref;
-    record_stage(o, 8, st);
+    record_stage(o, 6, st);
     cudaError_t e = launch_gemm_t<false, false, false, false, kEpiPhiKey>(mK, mK, mW, mW, ak, m, BH, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     GemmArgs aq = args(P, m, d);
@@ -441,7 +444,7 @@ favor_status causal_prefix(const favor_shape *s, const Bf16Layout &l, const void
     ao.out_rows = L;
     ao.d = d;
     e = launch_gemm_t<false, true, true, false, kEpiOut>(mPa[0], mPa[1], mVn, mVn, ao, Np, BH, st);
-    record_stage(o, 9, st);
+    record_stage(o, 7, st);
     return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
 
@@ -562,7 +565,7 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     const int map = opt_feature_map(o);
     if (map != FAVOR_MAP_POSITIVE) return fwd_bf16_map(s, map, Q, K, V, W, out, ws, ws_bytes, o, st);
     if (!causal) return fwd_bf16_bidir(s, Q, K, V, W, out, ctx, ws, ws_bytes, o, st);
-    const Bf16Layout l = bf16_layout(s, o, ctx == nullptr, causal);
+    const Bf16Layout l = bf16_layout(s, o);
     if (ws_bytes < l.total) return FAVOR_ERR_WORKSPACE;
     CUtensorMap mQ, mK, mV, mW, mW128;
     if (!make_token_map(&mQ, Q, l.BH, s->L, s->d) || !make_token_map(&mK, K, l.BH, s->L, s->d) ||
@@ -571,36 +574,39 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
         return FAVOR_ERR_CUDA;
     // Per-key -|k|^2/2 goes straight into the context (after the state blocks) when one is kept.
     float *bias = ctx ? (float *)((uint8_t *)ctx + ctx_layout(s).off_bias) : (float *)(ws + l.off_bias);
-    float *split_max = (float *)(ws + l.off_split_max);
     float *head_max = (float *)(ws + l.off_head_max);
-    float *part_S = (float *)(ws + l.off_part_S);
-    float *part_z = (float *)(ws + l.off_part_z);
     float *seg_S = (float *)(ws + l.off_seg_S);
     float *seg_z = (float *)(ws + l.off_seg_z);
-
-    KeyMaxParams km{s->L, s->d, s->m, l.n_split, l.tiles_per_split, bias, split_max};
-    record_stage(o, 0, st);
-    cudaError_t e = launch_key_logit_max(mK, mW, km, l.BH, st);
-    record_stage(o, 1, st);
-    if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     // the head's key reference in log2 units, for the exact prefix and (in the context) the backward
     float *kref = ctx ? (float *)((uint8_t *)ctx + ctx_layout(s).off_kref) : (float *)(ws + l.off_kref);
-    KeyStateParams ks{s->L, s->d, s->m, l.n_split, l.tiles_per_split, (const uint16_t *)V, bias, split_max,
-                      part_S, part_z, head_max, kref};
-    record_stage(o, 2, st);
-    e = launch_key_state(mK, mW, ks, l.BH, st);
-    record_stage(o, 3, st);
+
+    // per-segment states (one pass over K and V; 128-token tiles, per-feature stabilisers)
+    CUtensorMap mK128, mV128;
+    if (!make_token_map(&mK128, K, l.BH, s->L, s->d, kWideTile) || !make_token_map(&mV128, V, l.BH, s->L, s->d, kWideTile))
+        return FAVOR_ERR_CUDA;
+    const int segs_per_cta = (l.n_seg + num_sms() - 1) / num_sms();
+    Flat f{};
+    f.nt = l.n_tiles;
+    f.total = l.BH * l.n_tiles;
+    float *part = (float *)(ws + l.off_part);
+    KeyStateParams2 ks{s->L, s->m, f, part, (float *)(ws + l.off_part_D), (float *)(ws + l.off_part_amax),
+                       (float *)(ws + l.off_part_umax)};
+    const WideSegParams sgp{l.n_split, l.tiles_per_split, l.n_seg, segs_per_cta, bias};
+    record_stage(o, 0, st);
+    cudaError_t e = launch_key_segments(mK128, mV128, mW, ks, sgp, opt_poly_pct(o), st);
+    record_stage(o, 1, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
-    ScanParams sp{s->m, s->d, l.n_split, 1.f * (1 << (int)kChunkKeyShift), part_S, part_z, seg_S, seg_z};
-    record_stage(o, 4, st);
-    e = launch_state_scan(sp, l.BH, st);
-    record_stage(o, 5, st);
+    SegScanParams sp{s->m, l.n_split, s->m / 128, part, (float *)(ws + l.off_part_D), (float *)(ws + l.off_part_umax),
+                     seg_S, seg_z, head_max, kref};
+    record_stage(o, 2, st);
+    e = launch_segment_scan(sp, l.BH, st);
+    record_stage(o, 3, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     ChunkParams cp{s->L, s->m, l.n_split, l.tiles_per_split, l.P_exact, l.BH * l.n_split, bias, head_max,
                    seg_S, seg_z, out};
-    record_stage(o, 6, st);
+    record_stage(o, 4, st);
     e = launch_causal_chunk(mQ, mK, mV, mW128, cp, opt_poly_pct(o), st);
-    record_stage(o, 7, st);
+    record_stage(o, 5, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     return causal_prefix(s, l, Q, K, V, W, kref, out, ws, o, st);
 }
@@ -985,7 +991,7 @@ extern "C" size_t favor_workspace_size(const favor_shape *s, int causal, int bac
     if (s->dtype == FAVOR_F32) return align256(f32_workspace_floats(s->B * s->H, s->L, s->d, s->m) * 4);
     if (backward) return causal ? causal_bwd_layout(s).total : bwd_layout(s).total;
     if (!causal) return bidir_layout(s, true).total;
-    return bf16_layout(s, o, true, causal).total;
+    return bf16_layout(s, o).total;
 }
 
 extern "C" size_t favor_ctx_size(const favor_shape *s, int causal) {

@@ -6,8 +6,9 @@
 //   out_i = phi(q_i)^T S_i / phi(q_i)^T z_i,   S_i = sum_{j<=i} phi(k_j) v_j^T,  z_i = sum_{j<=i} phi(k_j).
 //
 // Sequence parallelism: the sequence of each head is cut into segments (runs of 128-token
-// tiles). k_key_state gives each segment's aggregate [S | z]; k_state_scan turns them into
-// exclusive prefixes; k_causal_chunk walks each segment's tiles in order from that prefix:
+// tiles). k_key_partials_wide (its causal instantiation, k_keys_wide.cu) gives each segment's
+// aggregate [S | z] and the per-key -|k|^2/2; k_segment_scan turns them into exclusive prefixes at
+// the head's key reference C; k_causal_chunk walks each segment's tiles in order from that prefix:
 //   out_tile = ( phi(Q_t) S_<t + mask(phi(Q_t) phi(K_t)^T) V_t ) / ( phi(Q_t) z_<t + rowsum(mask(...)) ),
 //   S_<t+1 = S_<t + phi(K_t)^T V_t.
 // The first tokens of every head are recomputed afterwards at split precision (bf16 hi + lo
@@ -17,56 +18,6 @@
 #include "common.cuh"
 
 namespace favor {
-
-// ============================================================================ k_state_scan
-
-struct ScanParams {
-    int m, d, n_split;
-    float scale;            // factor on the prefixes (the key shift 2^A of k_causal_chunk)
-    const float *part_S;    // [BH, n_split, m, d]
-    const float *part_z;    // [BH, n_split, m]
-    float *seg_S;           // [BH, n_split, m, d]: exclusive prefix of S per segment, times scale
-    float *seg_z;           // [BH, n_split, m]
-};
-
-// One thread per element of [S | z] (coalesced across the segment records), walking the segments
-// in order with the loads of eight segments in flight (grid: element blocks x heads).
-__global__ void __launch_bounds__(256) k_state_scan(ScanParams p) {
-    const int bh = blockIdx.y;
-    const size_t md = (size_t)p.m * p.d;
-    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const float *src;
-    float *dst;
-    size_t stride;
-    if (i < md) {
-        src = p.part_S + (size_t)bh * p.n_split * md + i;
-        dst = p.seg_S + (size_t)bh * p.n_split * md + i;
-        stride = md;
-    } else if (i < md + p.m) {
-        src = p.part_z + (size_t)bh * p.n_split * p.m + (i - md);
-        dst = p.seg_z + (size_t)bh * p.n_split * p.m + (i - md);
-        stride = p.m;
-    } else {
-        return;
-    }
-    float run = 0.f;
-    int sg = 0;
-    for (; sg + 8 <= p.n_split; sg += 8) {
-        float a[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) a[k] = src[(size_t)(sg + k) * stride];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            dst[(size_t)(sg + k) * stride] = run * p.scale;
-            run += a[k];
-        }
-    }
-    for (; sg < p.n_split; ++sg) {
-        const float a = src[(size_t)sg * stride];
-        dst[(size_t)sg * stride] = run * p.scale;
-        run += a;
-    }
-}
 
 // ============================================================================ k_causal_chunk
 //
@@ -105,7 +56,7 @@ struct ChunkParams {
     int n_seg;                 // BH * n_split
     const float *bias;         // [BH, L]: -|k_j|^2/2
     const float *head_max;     // [BH]: C
-    const float *seg_S;        // [BH, n_split, m, 64]: exclusive prefix of S per segment, times 2^A
+    const float *seg_S;        // [BH, n_split, 64, m]: exclusive prefix of S per segment, times 2^A
     const float *seg_z;        // [BH, n_split, m]: the same for z
     float *out;                // fp32 [BH, L, 64]
 };
@@ -613,18 +564,13 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                 mbar_arrive(&bar[B_Z_FULL + b]);
                 if (g > 0 && !mbar_wait_all(&bar[B_S_DONE], (g - 1) & 1, abort_flag)) break;
                 tc_fence_after();
-                const float4 *src = (const float4 *)(p.seg_S + srow * 64);
+                // feature-minor rows: thread f reads column c at p.seg_S[(seg * 64 + c) * m + fg]
+                const float *src = p.seg_S + (size_t)it.seg * 64 * p.m + fg;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     float w[32];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const float4 a = __ldg(src + 8 * h + c);
-                        w[4 * c] = a.x;
-                        w[4 * c + 1] = a.y;
-                        w[4 * c + 2] = a.z;
-                        w[4 * c + 3] = a.w;
-                    }
+                    for (int c = 0; c < 32; ++c) w[c] = __ldg(src + (size_t)(32 * h + c) * p.m);
                     tmem_st32(tmem + lane_off + T_S + 32 * h, w);
                 }
                 tmem_wait_st();
@@ -878,11 +824,6 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
 
 // ============================================================================ host launchers
 
-cudaError_t launch_state_scan(const ScanParams &p, int BH, cudaStream_t st) {
-    const size_t n = (size_t)p.m * p.d + p.m;
-    k_state_scan<<<dim3((unsigned)((n + 255) / 256), BH), 256, 0, st>>>(p);
-    return cudaGetLastError();
-}
 
 // The register split of k_causal_chunk (208 + 104 + 128 + 72 per warpgroup lane) fits the 128 per
 // thread it is launched with; the launch is refused unless the kernel carries exactly 128.

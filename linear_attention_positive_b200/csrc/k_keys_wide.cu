@@ -31,6 +31,8 @@
 // 4-7 / 8-11 exponentials of feature half 0 / 1 and the run-end write; 12 TMA; 13 / 15 MMA issue
 // for half 0 / 1; 14 the tile's largest |v|.
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace favor {
@@ -132,11 +134,71 @@ __device__ __forceinline__ void tmem_scale_f16x16(uint32_t taddr, float s) {
     tmem_wait_st();
 }
 
-template <int POLY>
+// Causal use of the kernel: the runs are the (head, segment) blocks of tps consecutive key tiles the
+// causal scan works on (the last segment of a head may be shorter); each CTA takes whole segments.
+struct WideSegParams {
+    int n_split;       // segments per head
+    int tps;           // tiles per segment
+    int n_seg;         // BH * n_split
+    int segs_per_cta;  // 0: bidirectional use (runs are the parts of heads inside CTA ranges)
+    float *bias;       // [BH, L]: -|k_j|^2/2 per key (causal use), else NULL
+};
+
+// The key tiles of one CTA in order, with their run boundaries and run slot.
+struct FlatWalk {  // bidirectional: tiles cta * T .. of the head-major flat order
+    int bh, t, g, n, nt, cta;
+    __device__ FlatWalk(const Flat &f, const WideSegParams &, int cta_) : nt(f.nt), cta(cta_) {
+        const int fl = cta_ * f.T;
+        n = max(min(fl + f.T, f.total) - fl, 0);
+        bh = fl / f.nt;
+        t = fl - bh * f.nt;
+        g = 0;
+    }
+    __device__ bool first() const { return g == 0 || t == 0; }
+    __device__ bool last() const { return g == n - 1 || t == nt - 1; }
+    __device__ int slot() const { return cta + bh; }  // distinct for distinct (CTA, head) runs
+    __device__ void next() {
+        ++g;
+        if (++t == nt) {
+            t = 0;
+            ++bh;
+        }
+    }
+};
+struct SegWalk {  // causal: whole segments of the CTA's range, one run each
+    int sg, j, len, n, nt, n_split, tps, bh, t;
+    __device__ int seg_len(int q) const { return min(tps, nt - (q % n_split) * tps); }
+    __device__ SegWalk(const Flat &f, const WideSegParams &sp, int cta) : nt(f.nt), n_split(sp.n_split), tps(sp.tps) {
+        const int s0 = cta * sp.segs_per_cta, s1 = min(s0 + sp.segs_per_cta, sp.n_seg);
+        n = 0;
+        for (int q = s0; q < s1; ++q) n += seg_len(q);
+        sg = s0;
+        j = 0;
+        len = seg_len(sg);
+        bh = sg / n_split;
+        t = (sg - bh * n_split) * tps;
+    }
+    __device__ bool first() const { return j == 0; }
+    __device__ bool last() const { return j == len - 1; }
+    __device__ int slot() const { return sg; }
+    __device__ void next() {
+        ++t;
+        if (++j == len) {
+            ++sg;
+            j = 0;
+            len = seg_len(sg);
+            bh = sg / n_split;
+            t = (sg - bh * n_split) * tps;
+        }
+    }
+};
+
+template <int POLY, bool SEG>
 __global__ void __launch_bounds__(kKeyThreads, 1)
 k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
-                    const __grid_constant__ CUtensorMap mapW, KeyStateParams2 p) {
+                    const __grid_constant__ CUtensorMap mapW, KeyStateParams2 p, WideSegParams sp) {
     using C = WideCfg;
+    using Walk = typename std::conditional<SEG, SegWalk, FlatWalk>::type;
     constexpr int STAGES = C::STAGES, D = C::D;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -156,9 +218,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
 
     pdl_launch_dependents();  // the state image kernel may stage its launch meanwhile
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nt = p.f.nt;
-    const int f0 = blockIdx.x * p.f.T, f1 = min(f0 + p.f.T, p.f.total);
-    const int n = max(f1 - f0, 0);
+    const int n = Walk(p.f, sp, blockIdx.x).n;  // key tiles of this CTA
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -201,14 +261,15 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
             }
             __syncwarp();
             int issued = 0;
-            for (int g = 0; g < n; ++g) {
-                const int s = g % STAGES, fl = f0 + g;
+            Walk wk(p.f, sp, blockIdx.x);
+            for (int g = 0; g < n; ++g, wk.next()) {
+                const int s = g % STAGES;
                 if (!mbar_wait_lazy(&empty[s], ((g / STAGES) & 1) ^ 1, abort_flag)) break;
                 if (elect_one()) {
                     uint8_t *st = sStage + (size_t)s * C::STAGE;
                     mbar_arrive_expect_tx(&full[s], 2 * C::TILE);
-                    tma_load_3d(st, &mapK, &full[s], 0, (fl % nt) * kWideTile, fl / nt);
-                    tma_load_3d(st + C::TILE, &mapV, &full[s], 0, (fl % nt) * kWideTile, fl / nt);
+                    tma_load_3d(st, &mapK, &full[s], 0, wk.t * kWideTile, wk.bh);
+                    tma_load_3d(st + C::TILE, &mapV, &full[s], 0, wk.t * kWideTile, wk.bh);
                 }
                 __syncwarp();
                 ++issued;
@@ -259,11 +320,10 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
             tc_fence_after();
             if (ok) project(0);
             int runs = 0;
-            int pos = f0 % nt;  // tile g's index within its head
-            for (int g = 0; ok && g < n; ++g) {
+            Walk wk(p.f, sp, blockIdx.x);
+            for (int g = 0; ok && g < n; ++g, wk.next()) {
                 const int s = g % STAGES;
-                const bool first = g == 0 || pos == 0, last = g == n - 1 || pos == nt - 1;
-                pos = pos + 1 == nt ? 0 : pos + 1;
+                const bool first = wk.first(), last = wk.last();
                 if (g + 1 < n) {
                     ok = mbar_wait_all(&full[(g + 1) % STAGES], ((g + 1) / STAGES) & 1, abort_flag) &&
                          mbar_wait_all(&p_free[h], g & 1, abort_flag);
@@ -300,12 +360,12 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
             int runs = 0;
             float Dr = 0.f;  // this feature's stabiliser D_r in the current run
             float z = 0.f;   // this feature's normaliser entry z_r of the current run (2^-b_t scale)
-            int pos = f0 % nt;
-            float va[32], vb[32], vc[32];
-            for (int g = 0; g < n; ++g) {
+            float umax = -INFINITY;  // the run's largest t - b_t = u log2e + A (causal use)
+            Walk wk(p.f, sp, blockIdx.x);
+            float va[32], vb[32];
+            for (int g = 0; g < n; ++g, wk.next()) {
                 const int s = g % STAGES;
-                const bool first = g == 0 || pos == 0, last = g == n - 1 || pos == nt - 1;
-                pos = pos + 1 == nt ? 0 : pos + 1;
+                const bool first = wk.first(), last = wk.last();
                 if (!mbar_wait_all(&p_full[h], g & 1, abort_flag) ||
                     !mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag))
                     break;
@@ -329,6 +389,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                     tm = fmaxf(tm, chunk_tmax(vb, bias + 96));
                     Dr = ceilf(tm - lim);
                     z = 0.f;
+                    umax = tm - (float)bt;
                 }
                 float zs = 0.f;  // this tile's sum of phi'
                 // One 32-token chunk: t, phi' and the chunk's largest t (in parallel); on a later tile of
@@ -337,6 +398,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                 // the state MMA of tile g - 1 must have read it (which also makes [S] safe to rescale).
                 auto chunk = [&](float(&v)[32], int c) -> bool {
                     const float cm = chunk_shift(v, bias + 32 * c, Dr);
+                    if (SEG && !first) umax = fmaxf(umax, cm + Dr - (float)bt);
                     uint32_t hv[16];
                     float cs = chunk_exp<POLY>(v, hv);
                     if (c == 0) {
@@ -382,8 +444,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                 if (last) {
                     if (!mbar_wait_all(&acc_full[h], runs & 1, abort_flag)) break;
                     tc_fence_after();
-                    const int bh = (f0 + g) / nt;
-                    const size_t rs = (size_t)blockIdx.x + bh;
+                    const size_t rs = (size_t)wk.slot();
                     float *dst = p.part + rs * (D + 1) * p.m + h * 128 + row;
                     float amax = fabsf(z);
 #pragma unroll
@@ -399,7 +460,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                     mbar_arrive(&acc_empty[h]);
                     dst[(size_t)D * p.m] = z;
                     p.part_D[rs * p.m + h * 128 + row] = Dr;
-                    float dmax = Dr;
+                    float dmax = SEG ? umax : Dr;
                     for (int o = 16; o > 0; o >>= 1) {
                         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                         dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
@@ -417,8 +478,9 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
         // Converter warpgroup: thread j handles token j of each tile (its |k_j|^2 and bias) and
         // converts 8 of the V tile's 16-byte chunks.
         const int j = threadIdx.x;
-        for (int g = 0; g < n; ++g) {
-            const int s = g % STAGES, t = (f0 + g) % nt;
+        Walk wk(p.f, sp, blockIdx.x);
+        for (int g = 0; g < n; ++g, wk.next()) {
+            const int s = g % STAGES, t = wk.t;
             if (!mbar_wait_lazy(&vmax_full[s], (g / STAGES) & 1, abort_flag)) break;
             uint8_t *st = sStage + (size_t)s * C::STAGE;
             const int b = sShift[s];
@@ -436,6 +498,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
             const bool valid = t * kWideTile + j < p.L;
             const float k2 = key_sq_norm<1, kWideTile>(st, j);
             sBias[s * kWideTile + j] = valid ? fmaf(-0.5f * k2, kLog2e, kKeyFeatureShift + (float)b) : -INFINITY;
+            if (SEG && valid) sp.bias[(size_t)wk.bh * p.L + t * kWideTile + j] = -0.5f * k2;
             fence_async_smem();
             mbar_arrive(&conv_full[s]);
         }
@@ -455,31 +518,133 @@ static size_t key_wide_smem(int m) {
 
 // The register split (88 + 2 x 160 + 88 per warpgroup lane) fits the 128 per thread the kernel is
 // launched with; the launch is refused unless the kernel carries exactly 128.
-template <int POLY>
+template <int POLY, bool SEG>
 static cudaError_t launch_key_wide_t(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mW,
-                                     const KeyStateParams2 &p, cudaStream_t st) {
+                                     const KeyStateParams2 &p, const WideSegParams &sp, int n_cta, cudaStream_t st) {
     static int checked = 0;
     if (checked == 0) {
         cudaFuncAttributes a{};
-        checked = (cudaFuncGetAttributes(&a, k_key_partials_wide<POLY>) == cudaSuccess && a.numRegs == 128) ? 1 : -1;
+        checked = (cudaFuncGetAttributes(&a, k_key_partials_wide<POLY, SEG>) == cudaSuccess && a.numRegs == 128) ? 1 : -1;
     }
     if (checked < 0) return cudaErrorInvalidConfiguration;
     const size_t sm = key_wide_smem(p.m);
-    cudaFuncSetAttribute(k_key_partials_wide<POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_key_partials_wide<POLY><<<p.f.n_cta, kKeyThreads, sm, st>>>(mK, mV, mW, p);
+    cudaFuncSetAttribute(k_key_partials_wide<POLY, SEG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_key_partials_wide<POLY, SEG><<<n_cta, kKeyThreads, sm, st>>>(mK, mV, mW, p, sp);
     return cudaGetLastError();
 }
 
-// d = 64 only; K and V maps with 128-row boxes, p.f built on 128-token tiles.
-cudaError_t launch_key_partials_wide(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mW,
-                                     const KeyStateParams2 &p, int poly_pct, cudaStream_t st) {
+template <bool SEG>
+static cudaError_t launch_key_wide_poly(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mW,
+                                        const KeyStateParams2 &p, const WideSegParams &sp, int n_cta, int poly_pct,
+                                        cudaStream_t st) {
     const int poly = poly_pct < 13 ? 0 : poly_pct < 31 ? 8 : poly_pct < 44 ? 12 : 16;
     switch (poly) {
-        case 0: return launch_key_wide_t<0>(mK, mV, mW, p, st);
-        case 8: return launch_key_wide_t<8>(mK, mV, mW, p, st);
-        case 12: return launch_key_wide_t<12>(mK, mV, mW, p, st);
-        default: return launch_key_wide_t<16>(mK, mV, mW, p, st);
+        case 0: return launch_key_wide_t<0, SEG>(mK, mV, mW, p, sp, n_cta, st);
+        case 8: return launch_key_wide_t<8, SEG>(mK, mV, mW, p, sp, n_cta, st);
+        case 12: return launch_key_wide_t<12, SEG>(mK, mV, mW, p, sp, n_cta, st);
+        default: return launch_key_wide_t<16, SEG>(mK, mV, mW, p, sp, n_cta, st);
     }
+}
+
+// Bidirectional use, d = 64: K and V maps with 128-row boxes, p.f built on 128-token tiles.
+cudaError_t launch_key_partials_wide(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mW,
+                                     const KeyStateParams2 &p, int poly_pct, cudaStream_t st) {
+    const WideSegParams none{0, 0, 0, 0, nullptr};
+    return launch_key_wide_poly<false>(mK, mV, mW, p, none, p.f.n_cta, poly_pct, st);
+}
+
+// Causal use, d = 64: one run per (head, segment of sp.tps tiles), each CTA taking sp.segs_per_cta
+// whole segments; slot = segment index (head-major). p.part_Dmax receives, per (slot, half, warp),
+// the run's largest u log2e + A instead of its largest D_r, and sp.bias the per-key -|k|^2/2.
+cudaError_t launch_key_segments(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mW,
+                                const KeyStateParams2 &p, const WideSegParams &sp, int poly_pct, cudaStream_t st) {
+    const int n_cta = (sp.n_seg + sp.segs_per_cta - 1) / sp.segs_per_cta;
+    return launch_key_wide_poly<true>(mK, mV, mW, p, sp, n_cta, poly_pct, st);
+}
+
+// ============================================================================ k_segment_scan
+//
+// Causal use: the exclusive prefix over a head's segments of the state the chunked scan starts
+// each segment from, at the head's key reference. Segment sg of k_key_partials_wide holds
+// [S'_r | z'_r] = 2^(A - D_r) sum_j e^(u_r(k_j)) [v_j | 1] (A the key shift 4, D_r its per-feature
+// stabiliser); with C = max over the head's keys and features of u (nats), taken from the segments'
+// largest u log2e + A, the prefix of segment sp is 2^8 sum_{sg < sp} 2^(D_r - A - C log2e) [S' | z']
+// = 2^8 sum_j e^(u_r(k_j) - C) [v_j | 1] over the keys before the segment: the form k_causal_chunk
+// reads (keys 2^8 below fp16's limit under C). One thread per element (value column c, feature r),
+// feature-minor like the partial states, so reads and writes are coalesced; eight segments' loads
+// in flight.
+
+struct SegScanParams {
+    int m, n_split, halves;
+    const float *part;       // [n_seg][65][m]
+    const float *part_D;     // [n_seg][m]
+    const float *part_umax;  // [n_seg][8]: per (half, warp) largest u log2e + A
+    float *seg_S;            // [BH][n_split][64][m]
+    float *seg_z;            // [BH][n_split][m]
+    float *head_max;         // [BH]: C (nats)
+    float *key_ref;          // NULL or [BH]: C log2e
+};
+
+__global__ void __launch_bounds__(256) k_segment_scan(SegScanParams p) {
+    constexpr int D = 64, NC = D + 1;
+    __shared__ float sRed[8];
+    const int bh = blockIdx.y;
+    pdl_wait_prerequisites();  // the key kernel's segments are complete and visible
+    // the head's reference: the largest u log2e + A over its segments
+    float mx = -INFINITY;
+    for (int i = threadIdx.x; i < p.n_split * 8; i += 256)
+        if ((i & 7) < 4 * p.halves) mx = fmaxf(mx, p.part_umax[((size_t)bh * p.n_split + (i >> 3)) * 8 + (i & 7)]);
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) sRed[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = sRed[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) mx = fmaxf(mx, sRed[i]);
+    const float kref = mx - kKeyFeatureShift;  // C log2e
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        p.head_max[bh] = kref / kLog2e;
+        if (p.key_ref) p.key_ref[bh] = kref;
+    }
+    const size_t i = (size_t)blockIdx.x * 256 + threadIdx.x;
+    if (i >= (size_t)NC * p.m) return;
+    const int c = (int)(i / p.m), r = (int)(i - (size_t)c * p.m);
+    const size_t seg0 = (size_t)bh * p.n_split;
+    const float *src = p.part + seg0 * NC * p.m + i;
+    const float *dsrc = p.part_D + seg0 * p.m + r;
+    const size_t sstride = (size_t)NC * p.m;
+    float *dst;
+    size_t dstride;
+    if (c < D) {
+        dst = p.seg_S + seg0 * D * p.m + (size_t)c * p.m + r;
+        dstride = (size_t)D * p.m;
+    } else {
+        dst = p.seg_z + seg0 * p.m + r;
+        dstride = p.m;
+    }
+    const float off = kKeyFeatureShift + kref;
+    float run = 0.f;
+    int sp = 0;
+    for (; sp + 8 <= p.n_split; sp += 8) {
+        float a[8], dd[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            a[k] = src[(size_t)(sp + k) * sstride];
+            dd[k] = dsrc[(size_t)(sp + k) * p.m];
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            dst[(size_t)(sp + k) * dstride] = run * 256.f;  // exclusive prefix, times 2^8
+            run = fmaf(exp2f(dd[k] - off), a[k], run);
+        }
+    }
+    for (; sp < p.n_split; ++sp) {
+        dst[(size_t)sp * dstride] = run * 256.f;
+        run = fmaf(exp2f(dsrc[(size_t)sp * p.m] - off), src[(size_t)sp * sstride], run);
+    }
+}
+
+cudaError_t launch_segment_scan(const SegScanParams &p, int BH, cudaStream_t st) {
+    return launch_after_previous(k_segment_scan, dim3((65 * p.m + 255) / 256, BH), dim3(256), 0, st, p);
 }
 
 }  // namespace favor
