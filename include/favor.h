@@ -189,8 +189,10 @@ FAVOR_API favor_status favor_bwd(const favor_shape *shape, const void *Q, const 
 /*
  * favor_sync_status -- synchronise the stream, then return and clear the device status word
  * (FAVOR_ERR_TIMEOUT if a bounded wait inside a kernel gave up since the last call;
- * FAVOR_ERR_UNSUPPORTED if the causal bf16 forward met a V entry of magnitude 2^16 or more, or a
- * non-finite one: its tensor-core operands are fp16, and such outputs are not valid), or
+ * FAVOR_ERR_UNSUPPORTED if a bf16 forward met a V entry of magnitude 2^23 or more, or a non-finite
+ * one: the values reach the fp16 tensor-core operands scaled by at most 2^-7 per key tile (the
+ * causal path scales each 1024-key segment further, by 2^-b, b as needed), and such outputs are not
+ * valid), or
  * FAVOR_ERR_CUDA if the stream reports an error.
  */
 FAVOR_API favor_status favor_sync_status(void *stream);

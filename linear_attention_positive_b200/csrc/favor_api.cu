@@ -81,8 +81,8 @@ int prefix_cols(int P) { return (P + 127) & ~127; }
 // segment prefixes at the head reference, and the exact prefix's features and scores.
 struct Bf16Layout {
     int BH, n_tiles, tiles_per_split, n_split, n_seg, P_exact, Ppad;
-    size_t off_bias, off_head_max, off_part, off_part_D, off_part_amax, off_part_umax, off_seg_S, off_seg_z,
-        off_kref, off_pq[2], off_pk[2], off_pa[2], total;
+    size_t off_bias, off_head_max, off_part, off_part_D, off_part_amax, off_part_umax, off_seg_vmax, off_seg_S,
+        off_seg_z, off_kref, off_pq[2], off_pk[2], off_pa[2], total;
 };
 
 Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o) {
@@ -105,6 +105,8 @@ Bf16Layout bf16_layout(const favor_shape *s, const favor_opts *o) {
     off += align256((size_t)l.n_seg * 8 * 4);
     l.off_part_umax = off;
     off += align256((size_t)l.n_seg * 8 * 4);
+    l.off_seg_vmax = off;
+    off += align256((size_t)l.n_seg * 4);
     l.P_exact = std::min(s->L, kCausalExactPrefix);
     l.off_seg_S = off;
     off += align256((size_t)l.n_seg * s->m * s->d * 4);
@@ -591,7 +593,8 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     float *part = (float *)(ws + l.off_part);
     KeyStateParams2 ks{s->L, s->m, f, part, (float *)(ws + l.off_part_D), (float *)(ws + l.off_part_amax),
                        (float *)(ws + l.off_part_umax)};
-    const WideSegParams sgp{l.n_split, l.tiles_per_split, l.n_seg, segs_per_cta, bias};
+    uint32_t *seg_vmax = (uint32_t *)(ws + l.off_seg_vmax);
+    const WideSegParams sgp{l.n_split, l.tiles_per_split, l.n_seg, segs_per_cta, bias, seg_vmax};
     record_stage(o, 0, st);
     cudaError_t e = launch_key_segments(mK128, mV128, mW, ks, sgp, opt_poly_pct(o), st);
     record_stage(o, 1, st);
@@ -603,7 +606,7 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     record_stage(o, 3, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     ChunkParams cp{s->L, s->m, l.n_split, l.tiles_per_split, l.P_exact, l.BH * l.n_split, bias, head_max,
-                   seg_S, seg_z, out};
+                   seg_S, seg_z, seg_vmax, out};
     record_stage(o, 4, st);
     e = launch_causal_chunk(mQ, mK, mV, mW128, cp, opt_poly_pct(o), st);
     record_stage(o, 5, st);

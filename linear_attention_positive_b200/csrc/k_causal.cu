@@ -43,8 +43,10 @@ namespace favor {
 // C is the per-(batch, head) key maximum, so phik <= 2^A with A = 8 (fp16 headroom for keys far
 // below the maximum); every product phik v carries the same 2^A, which cancels in the ratio.
 // sigma_t keeps the scaled S below 2^15, and with phik <= 2^8 over 128 features the scaled scores
-// stay below 2^15 too. V entries must fit fp16 (magnitude below 2^16): larger or non-finite
-// entries are reported as FAVOR_ERR_UNSUPPORTED through the device status word.
+// stay below 2^15 too. V enters as fp16 scaled by 2^-b per segment (b = max(0, e - 14), e the
+// exponent of the segment's largest |v|, recorded by the key pass); the numerator is scaled back by
+// 2^b with 2^sigma_t. Non-finite entries are reported as FAVOR_ERR_UNSUPPORTED through the device
+// status word.
 // Warp roles (16 warps): 0-3 query exponentials and den_q; 4-7 key exponentials, z and the state
 // image; 8-11 masking and the output epilogue (one tile behind); 12 TMA and the key terms beta_j;
 // 13 projection MMAs; 14 scores, state term, state update and masked A V MMAs; 15 V conversion.
@@ -58,10 +60,17 @@ struct ChunkParams {
     const float *head_max;     // [BH]: C
     const float *seg_S;        // [BH, n_split, 64, m]: exclusive prefix of S per segment, times 2^A
     const float *seg_z;        // [BH, n_split, m]: the same for z
+    const uint32_t *seg_vmax;  // [BH, n_split]: the segment's largest |v| (bf16 bits)
     float *out;                // fp32 [BH, L, 64]
 };
 
 constexpr int kChunkThreads = 512;
+
+// Power-of-two shift b of a segment's values (V' = V 2^-b in fp16): 0 while its largest |v| is
+// below 2^15, else enough to bring it there; the output numerator is scaled back by 2^b.
+__device__ __forceinline__ int segment_value_shift(uint32_t vmax_bits) {
+    return max(0, (int)(vmax_bits >> 7) - 127 - 14);
+}
 constexpr float kChunkKeyShift = 8.f;
 
 namespace chunk {
@@ -466,12 +475,14 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
             volatile int no_abort = 0;
             mbar_wait(&bar[B_DRAIN + (warp - 13)], 0, &no_abort);
         } else {
-            // ---- V tiles bf16 -> fp16 in place (entries beyond the fp16 range are reported)
+            // ---- V tiles bf16 -> fp16 in place, times 2^-b of their segment (non-finite entries are
+            // reported)
             int g = 0;
             for (ChunkSteps it(p, cid, n_cl); it.ok; it.next(p), ++g) {
                 const int s = g % STAGES;
                 if (!mbar_wait_lazy(&bar[B_FULL_V + s], (g / STAGES) & 1, abort_flag)) break;
                 uint8_t *vt = smem + OFF_V + s * TILE;
+                const float vsc = pow2i((float)-segment_value_shift(__ldg(p.seg_vmax + it.seg)));
                 uint32_t mx = 0;
 #pragma unroll 4
                 for (int q = lane; q < (int)(TILE / 16); q += 32) {
@@ -485,11 +496,11 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                     uint32_t h[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        h[k] = pack_f16x2(__uint_as_float(u[k] << 16), __uint_as_float(u[k] & 0xFFFF0000u));
+                        h[k] = pack_f16x2(__uint_as_float(u[k] << 16) * vsc, __uint_as_float(u[k] & 0xFFFF0000u) * vsc);
                     *pq = make_uint4(h[0], h[1], h[2], h[3]);
                 }
-                // bf16 magnitudes from 2^16 up (and inf / nan) do not fit fp16
-                if (max(mx & 0xFFFFu, mx >> 16) >= 0x4780u) record_status(FAVOR_ERR_UNSUPPORTED);
+                // inf / nan entries (bf16 exponent field all ones) have no scaled fp16 form
+                if (max(mx & 0xFFFFu, mx >> 16) >= 0x7F80u) record_status(FAVOR_ERR_UNSUPPORTED);
                 fence_async_smem();
                 mbar_arrive(&bar[B_CONV + s]);
             }
@@ -564,13 +575,15 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                 mbar_arrive(&bar[B_Z_FULL + b]);
                 if (g > 0 && !mbar_wait_all(&bar[B_S_DONE], (g - 1) & 1, abort_flag)) break;
                 tc_fence_after();
-                // feature-minor rows: thread f reads column c at p.seg_S[(seg * 64 + c) * m + fg]
+                // feature-minor rows: thread f reads column c at p.seg_S[(seg * 64 + c) * m + fg]; the
+                // prefix takes the segment's value scale 2^-b
                 const float *src = p.seg_S + (size_t)it.seg * 64 * p.m + fg;
+                const float vsc = pow2i((float)-segment_value_shift(__ldg(p.seg_vmax + it.seg)));
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     float w[32];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) w[c] = __ldg(src + (size_t)(32 * h + c) * p.m);
+                    for (int c = 0; c < 32; ++c) w[c] = __ldg(src + (size_t)(32 * h + c) * p.m) * vsc;
                     tmem_st32(tmem + lane_off + T_S + 32 * h, w);
                 }
                 tmem_wait_st();
@@ -768,7 +781,8 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                 }
                 if (g >= 2 && !mbar_wait_all(&bar[B_O_EMPTY + b], ((g >> 1) - 1) & 1, abort_flag)) break;
                 sf[F_DENA + b * 128 + row] = rs0 + rs1;
-                if (row == 0) sf[F_SIGE + b] = (float)sig;
+                // the output's scale back: 2^sigma of the scores and 2^b of the segment's values
+                if (row == 0) sf[F_SIGE + b] = (float)(sig + segment_value_shift(__ldg(p.seg_vmax + it.seg)));
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bar[B_MASK_DONE]);

@@ -297,6 +297,8 @@ k_key_partials(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
                 if (lane == 0) {
                     const int e = (int)(mx >> 7) - 127;  // exponent of the largest |v| (-127 for an all-zero tile)
                     sShift[s] = min(max(e - 7, -8), 7);
+                    // V' = V 2^-b_t is an fp16 operand: from 2^23 on (and for inf / nan) it would overflow
+                    if (mx >= 0x4B00u) record_status(FAVOR_ERR_UNSUPPORTED);
                     mbar_arrive(&vmax_full[s]);
                 }
                 __syncwarp();

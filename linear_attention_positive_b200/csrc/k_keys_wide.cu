@@ -142,6 +142,7 @@ struct WideSegParams {
     int n_seg;         // BH * n_split
     int segs_per_cta;  // 0: bidirectional use (runs are the parts of heads inside CTA ranges)
     float *bias;       // [BH, L]: -|k_j|^2/2 per key (causal use), else NULL
+    uint32_t *vmax;    // [n_seg]: the segment's largest |v| as bf16 bits (causal use), else NULL
 };
 
 // The key tiles of one CTA in order, with their run boundaries and run slot.
@@ -278,8 +279,11 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
             for (int i = max(issued - STAGES, 0); i < issued; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, &no_abort);
             mbar_wait(w_full, 0, &no_abort);
         } else if (warp == 14 && n > 0) {
-            // Largest |v| of each V tile (bf16 magnitudes compared as integers) -> b_t.
-            for (int g = 0; g < n; ++g) {
+            // Largest |v| of each V tile (bf16 magnitudes compared as integers) -> b_t; in causal use
+            // also each segment's largest |v|.
+            Walk wk(p.f, sp, blockIdx.x);
+            uint32_t run_mx = 0;
+            for (int g = 0; g < n; ++g, wk.next()) {
                 const int s = g % STAGES;
                 if (!mbar_wait_lazy(&full[s], (g / STAGES) & 1, abort_flag)) break;
                 const uint8_t *vt = sStage + (size_t)s * C::STAGE + C::TILE;
@@ -297,7 +301,16 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                 if (lane == 0) {
                     const int e = (int)(mx >> 7) - 127;  // exponent of the largest |v| (-127 for an all-zero tile)
                     sShift[s] = min(max(e - 7, -8), 7);
+                    // V' = V 2^-b_t is an fp16 operand: from 2^23 on (and for inf / nan) it would overflow
+                    if (mx >= 0x4B00u) record_status(FAVOR_ERR_UNSUPPORTED);
                     mbar_arrive(&vmax_full[s]);
+                    if (SEG) {
+                        run_mx = max(run_mx, mx);
+                        if (wk.last()) {
+                            sp.vmax[wk.slot()] = run_mx;
+                            run_mx = 0;
+                        }
+                    }
                 }
                 __syncwarp();
             }
@@ -549,7 +562,7 @@ static cudaError_t launch_key_wide_poly(const CUtensorMap &mK, const CUtensorMap
 // Bidirectional use, d = 64: K and V maps with 128-row boxes, p.f built on 128-token tiles.
 cudaError_t launch_key_partials_wide(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mW,
                                      const KeyStateParams2 &p, int poly_pct, cudaStream_t st) {
-    const WideSegParams none{0, 0, 0, 0, nullptr};
+    const WideSegParams none{0, 0, 0, 0, nullptr, nullptr};
     return launch_key_wide_poly<false>(mK, mV, mW, p, none, p.f.n_cta, poly_pct, st);
 }
 

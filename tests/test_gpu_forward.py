@@ -158,6 +158,27 @@ def test_bf16_value_tiles_of_very_different_magnitude(cuda_device):
     assert rel_max_err(out2, oracle_fwd(x2, W64, False)) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_bf16_bidirectional_values_beyond_range_are_reported(cuda_device, d):
+    """The bidirectional key kernels scale each key tile's values by at most 2^-7 into fp16
+    operands: values near 2^22 still give valid outputs, an entry of 2^23 (or a non-finite one) is
+    reported as FAVOR_ERR_UNSUPPORTED instead of a silently wrong output."""
+    w = Workload("t", 1, 1, 640, d, 256, False, "bf16", False, 2, 61)
+    x = make_inputs(w)
+    x["V"][0, 0, 128:256] *= 1.0e6
+    x["V"] = round_to_bf16(x["V"])
+    Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
+    out = run_fwd(w, x, Wr, cuda_device, causal=False)
+    assert rel_max_err(out, oracle_fwd(x, W64, False)) <= TOL["bf16"]
+    Q, K = (to_torch(x[k], w.dtype, cuda_device) for k in "QK")
+    for bad in (np.inf, 2.0 ** 23):
+        V = x["V"].copy()
+        V[0, 0, 300, 3] = bad
+        api.fwd(Q, K, to_torch(V, w.dtype, cuda_device), to_torch(Wr, w.dtype, cuda_device))
+        assert api.sync_status() == api.FAVOR_ERR_UNSUPPORTED, bad
+        assert api.sync_status() == api.FAVOR_OK
+
+
 @pytest.mark.parametrize("split_tiles", [1, 3, 64])
 def test_bf16_split_choice_does_not_change_result(cuda_device, split_tiles):
     w = Workload("t", 1, 2, 1500, 64, 256, False, "bf16", False, 2, 33)
@@ -278,24 +299,39 @@ def test_bf16_causal_config4_full_size_all_rows(cuda_device):
     assert max(errs) / rms <= TOL["bf16"]
 
 
-def test_bf16_causal_values_beyond_fp16_range_are_reported(cuda_device):
-    """The causal bf16 path feeds V to fp16 tensor-core operands: a value entry of magnitude 2^16 or
-    more cannot be represented there, and the call reports FAVOR_ERR_UNSUPPORTED through the device
-    status word instead of returning a silently wrong output. Entries just below the limit pass."""
-    w = Workload("t", 1, 1, 700, 64, 256, True, "bf16", False, 3, 41)
+def test_bf16_causal_values_beyond_fp16_range(cuda_device):
+    """The causal bf16 path feeds V to fp16 tensor-core operands; a segment (8 tiles of 128 keys)
+    whose values exceed fp16's range is scaled by a power of two for the fp16 operands and the
+    output scaled back. Segments of values up to ~1.2e6 and near 1e-4 beside ordinary ones, against
+    the fp64 oracle. Entries from 2^23 on (beyond what the key side's per-tile scaling keeps in fp16)
+    and non-finite ones are reported as FAVOR_ERR_UNSUPPORTED."""
+    w = Workload("t", 1, 2, 3 * 1024 + 200, 64, 256, True, "bf16", False, 3, 41)
     x = make_inputs(w)
+    x["V"][0, 0, 1024:2048] *= 3.0e5     # the second segment of head 0
+    x["V"][0, 1, 2048:3072] *= 1.0e-4    # the third segment of head 1
+    x["V"] = round_to_bf16(x["V"])
     Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
-    Q, K = (to_torch(x[k], w.dtype, cuda_device) for k in "QK")
-    Wt = to_torch(Wr, w.dtype, cuda_device)
+    out = run_fwd(w, x, Wr, cuda_device, causal=True)
+    assert np.isfinite(out).all()
+    ref = oracle_fwd(x, W64, True)
+    for h in range(2):  # each head against its own RMS: head 0's outputs after 1024 are ~1e6 larger
+        assert rel_max_err(out[0, h], ref[0, h]) <= TOL["bf16"], h
+    # one entry of 7e4 (past fp16's range; its segment shifted by 2^-2): finite, and the rows it
+    # dominates within the fp16 operands' relative precision
     V = x["V"].copy()
-    V[0, 0, 600, 5] = 60000.0      # bf16 rounds it to 59904: inside the fp16 range
-    out = api.fwd(Q, K, to_torch(V, w.dtype, cuda_device), Wt, causal=True)
-    assert api.sync_status() == api.FAVOR_OK
-    assert np.isfinite(out.cpu().numpy()).all()
-    V[0, 0, 600, 5] = 70000.0      # beyond it
-    api.fwd(Q, K, to_torch(V, w.dtype, cuda_device), Wt, causal=True)
-    assert api.sync_status() == api.FAVOR_ERR_UNSUPPORTED
-    assert api.sync_status() == api.FAVOR_OK  # the status word is cleared by the read
+    V[0, 1, 3100, 7] = 7.0e4
+    x2 = dict(x, V=round_to_bf16(V))
+    out2 = run_fwd(w, x2, Wr, cuda_device, causal=True)
+    ref2 = oracle_fwd(x2, W64, True)
+    assert np.isfinite(out2).all()
+    assert np.abs(out2[0, 1, 3100:, 7] - ref2[0, 1, 3100:, 7]).max() <= 2e-3 * np.abs(ref2[0, 1, 3100:, 7]).max()
+    Q, K = (to_torch(x[k], w.dtype, cuda_device) for k in "QK")
+    for bad in (np.inf, 2.0 ** 23):
+        V = x["V"].copy()
+        V[0, 0, 600, 5] = bad
+        api.fwd(Q, K, to_torch(V, w.dtype, cuda_device), to_torch(Wr, w.dtype, cuda_device), causal=True)
+        assert api.sync_status() == api.FAVOR_ERR_UNSUPPORTED, bad
+        assert api.sync_status() == api.FAVOR_OK  # the status word is cleared by the read
 
 
 @pytest.mark.parametrize("poly_pct", [25, 50, 100])
