@@ -443,18 +443,21 @@ class Runner:
         self.fmap = MAP_CODES[w.feature_map]
         self.base_opts = api.make_opts(exp_poly_pct=exp_poly_pct, feature_map=self.fmap)
 
-    def step(self, T=None, fwd_opts=None, bwd_opts=None):
+    def step(self, T=None, fwd_opts=None, bwd_opts=None, outs=None):
+        """One pass of the path on the current stream; ``outs`` = [out (, dQ, dK, dV)] to write into
+        other buffers than the runner's own."""
         api, w = self.api, self.w
         T = T or self.T
+        out, grads = (outs[0], outs[1:]) if outs else (self.out, self.grads)
         if w.sequence_parallel:
             # one rank's two calls; a multi-GPU run adds the all-reduce of the state in between
             api.sp_state(T["K"], T["V"], self.Wt, state=self.sp_state, workspace=self.sp_ws)
-            api.sp_output(T["Q"], self.Wt, self.sp_state, out=self.out, workspace=self.sp_ws)
+            api.sp_output(T["Q"], self.Wt, self.sp_state, out=out, workspace=self.sp_ws)
             return
-        api.fwd(T["Q"], T["K"], T["V"], self.Wt, causal=w.causal, out=self.out, ctx=self.ctx, workspace=self.ws,
+        api.fwd(T["Q"], T["K"], T["V"], self.Wt, causal=w.causal, out=out, ctx=self.ctx, workspace=self.ws,
                 opts=fwd_opts or self.base_opts)
         if w.backward:
-            api.bwd_into(T["Q"], T["K"], T["V"], self.Wt, self.out, T["dO"], *self.grads, ctx=self.ctx,
+            api.bwd_into(T["Q"], T["K"], T["V"], self.Wt, out, T["dO"], *grads, ctx=self.ctx,
                          causal=w.causal, workspace=self.ws, opts=bwd_opts)
 
     def n_fwd_stages(self):
@@ -516,32 +519,51 @@ class Runner:
         return step_ms, stage_ms, status
 
     def e2e(self, steps, flush, world, dist):
-        """Through the public API: pinned host inputs in, fp32 output (and gradients) back, every step."""
+        """Through the public API: every step, the inputs come in from pinned host memory and the fp32
+        output (and gradients) go back. The copies run on their own streams and are double-buffered
+        against the compute, so a step's inputs stream in while the previous step computes and the
+        one before it streams out (the job's throughput is set by the slower copy direction); the
+        time is from the first input copy to the last output copy."""
         torch = self.torch
-        stream = torch.cuda.current_stream()
+        comp = torch.cuda.current_stream()
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
         pin = {k: torch.from_numpy(self.x[k]).to(self.tdt).pin_memory() for k in self.x}
-        outs = [self.out] + (self.grads or [])
-        outs_h = [torch.empty(o.shape, dtype=torch.float32).pin_memory() for o in outs]
-        dT = {k: torch.empty_like(self.T[k]) for k in self.T}
-        evs = []
+        nb = 2
+        dT = [{k: torch.empty_like(self.T[k]) for k in self.T} for _ in range(nb)]
+        outs = [[torch.empty_like(o) for o in [self.out] + (self.grads or [])] for _ in range(nb)]
+        outs_h = [[torch.empty(o.shape, dtype=torch.float32).pin_memory() for o in outs[0]] for _ in range(nb)]
+        ev_in = [torch.cuda.Event() for _ in range(nb)]
+        ev_comp = [torch.cuda.Event() for _ in range(nb)]
+        ev_out = [torch.cuda.Event() for _ in range(nb)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        for _ in range(steps):
+        start.record(s_in)
+        for k in range(steps):
+            b = k % nb
+            with torch.cuda.stream(s_in):
+                if k >= nb:
+                    s_in.wait_event(ev_comp[b])  # step k - 2 has finished reading these buffers
+                for name in dT[b]:
+                    dT[b][name].copy_(pin[name], non_blocking=True)
+                ev_in[b].record(s_in)
+            comp.wait_event(ev_in[b])
+            if k >= nb:
+                comp.wait_event(ev_out[b])  # step k - 2's outputs have left
             flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for name in dT:
-                dT[name].copy_(pin[name], non_blocking=True)
-            self.step(T=dT)
-            for o, oh in zip(outs, outs_h):
-                oh.copy_(o, non_blocking=True)
-            b.record(stream)
-            evs.append((a, b))
+            self.step(T=dT[b], outs=outs[b])
+            ev_comp[b].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[b])
+                for o, oh in zip(outs[b], outs_h[b]):
+                    oh.copy_(o, non_blocking=True)
+                ev_out[b].record(s_out)
+        end.record(s_out)
         torch.cuda.synchronize()
-        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        ms = start.elapsed_time(end) / steps
         h2d = sum(pin[k].numel() * pin[k].element_size() for k in pin)
-        d2h = sum(oh.numel() * 4 for oh in outs_h)
+        d2h = sum(oh.numel() * 4 for oh in outs_h[0])
         return ms, h2d, d2h
 
     def launches_per_step(self):
