@@ -1,5 +1,7 @@
-// Key side of the bidirectional bf16 tensor-core path ("Fast Attention Via Positive Orthogonal
-// Random Features", codewithpapers.app/method/favor: the FA-part needs (K')^T V and (K')^T 1_L).
+// Key side of the bidirectional bf16 tensor-core path for d = 128 on 64-token key tiles ("Fast
+// Attention Via Positive Orthogonal Random Features", codewithpapers.app/method/favor: the FA-part
+// needs (K')^T V and (K')^T 1_L). d = 64 runs on k_key_partials_wide (k_keys_wide.cu), which also
+// uses this file's shared pieces (Flat, key_sq_norm, KeyStateParams2, tmem_scale_row).
 //
 //   k_key_partials : per run, the partial state [S | z] = sum_j phi'(k_j) [v_j | 1] with
 //                    phi'_r(k) = 2^(A - D_r) exp(u_r(k)), u_r(k) = w_r.k - |k|^2/2, where D_r is a
@@ -517,17 +519,11 @@ static cudaError_t launch_key_partials_t(const CUtensorMap &mK, const CUtensorMa
     return cudaGetLastError();
 }
 
+// d = 128 (d = 64 runs on k_key_partials_wide, 128-token tiles).
 cudaError_t launch_key_partials(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mW,
                                 const KeyStateParams2 &p, int d, int poly_pct, cudaStream_t st) {
+    if (d != 128) return cudaErrorInvalidValue;
     const int poly = poly_pct < 13 ? 0 : poly_pct < 31 ? 8 : poly_pct < 44 ? 12 : 16;
-    if (d == 64) {
-        switch (poly) {
-            case 0: return launch_key_partials_t<64, 0>(mK, mV, mW, p, st);
-            case 8: return launch_key_partials_t<64, 8>(mK, mV, mW, p, st);
-            case 12: return launch_key_partials_t<64, 12>(mK, mV, mW, p, st);
-            default: return launch_key_partials_t<64, 16>(mK, mV, mW, p, st);
-        }
-    }
     switch (poly) {
         case 0: return launch_key_partials_t<128, 0>(mK, mV, mW, p, st);
         case 8: return launch_key_partials_t<128, 8>(mK, mV, mW, p, st);
