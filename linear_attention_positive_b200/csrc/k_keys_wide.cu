@@ -11,11 +11,15 @@
 // Why a second key kernel: on 64-token tiles each exponent warp spends most of a tile in fixed
 // per-tile costs (barrier round trips, TMEM load latency, the stabiliser vote) rather than on the
 // MUFU. Here a tile is 128 tokens and, except on a run's first tile, the projection is read once:
-//   - P_h^T = W_h K_tile^T (M = 128 features of half h, N = 128 tokens, K = 64);
+//   - P_h^T = W_h K_tile^T (M = 128 features of half h, K = 64), issued as two N = 64 MMAs, one per
+//     64-token half of the tile, so that each half of the P buffer is handed to the next tile's
+//     projection as soon as the exponent warps are done with it;
 //   - per 32-token chunk c: t = P log2e + B_j - D_r, phi' = 2^t in fp16 stored to TMEM (16 packed
-//     columns), z_r += 2^-b_t sum_j phi', and the chunk's largest t, which decides (by a warp vote)
-//     whether D_r must be raised and the chunk redone; the next chunk's TMEM load is in flight
-//     meanwhile;
+//     columns) and z_r += 2^-b_t sum_j phi'; the next chunk's TMEM load is in flight meanwhile. A
+//     warp vote on the chunk's fp32 sum of phi' (below the largest fp16 value no element can
+//     overflow) sends the rare chunk that may overflow to an out-of-line redo, which re-reads its
+//     P columns and raises D_r where its largest t passes 15 (the causal use votes on every chunk's
+//     largest t, which its head reference needs anyway);
 //   - [S_h] += phi'_h V'_t (fp16 MMA, A from TMEM, B the converted V tile read MN-major, N = 64).
 // z_r is kept in the exponent thread's registers instead of a ones column of the state MMA, which
 // frees the TMEM columns the wider tile needs: per half P (128) + phi' (64) + S (64) = 256 columns.
@@ -27,9 +31,9 @@
 // 2^-delta, and the chunk's exponentials are recomputed before they are stored. Typical inputs
 // raise it rarely. V'_t = V_t 2^-b_t as in k_key_partials.
 //
-// Warp roles (16 warps): 0-3 convert V, write the biases B_j (thread j = token j of the tile);
-// 4-7 / 8-11 exponentials of feature half 0 / 1 and the run-end write; 12 TMA; 13 / 15 MMA issue
-// for half 0 / 1; 14 the tile's largest |v|.
+// Warp roles (16 warps): 0-3 the tile's largest |v| and b_t, convert V, write the biases B_j (thread
+// j = token j of the tile); 4-7 / 8-11 exponentials of feature half 0 / 1 and the run-end write;
+// 12 TMA; 13 / 15 MMA issue for half 0 / 1; 14 idle.
 
 #include <type_traits>
 
@@ -75,7 +79,8 @@ __device__ __forceinline__ float chunk_tmax(const float (&v)[32], const float *b
 }
 
 // t = v log2e + B_j - D for a 32-token chunk, in place (paired FMA-pipe instructions); returns the
-// chunk's largest t.
+// chunk's largest t when MAX is set (else 0).
+template <bool MAX>
 __device__ __forceinline__ float chunk_shift(float (&v)[32], const float *bias, float D) {
     float a = -INFINITY, b = -INFINITY;
 #pragma unroll
@@ -86,11 +91,16 @@ __device__ __forceinline__ float chunk_shift(float (&v)[32], const float *bias, 
         ffma2(b4.z, b4.w, 1.f, 1.f, -D, -D, c2, c3);
         ffma2(v[e], v[e + 1], kLog2e, kLog2e, c0, c1, v[e], v[e + 1]);
         ffma2(v[e + 2], v[e + 3], kLog2e, kLog2e, c2, c3, v[e + 2], v[e + 3]);
-        a = fmax3(a, v[e], v[e + 1]);
-        b = fmax3(b, v[e + 2], v[e + 3]);
+        if (MAX) {
+            a = fmax3(a, v[e], v[e + 1]);
+            b = fmax3(b, v[e + 2], v[e + 3]);
+        }
     }
-    return fmaxf(a, b);
+    return MAX ? fmaxf(a, b) : 0.f;
 }
+
+// Largest finite fp16 value: a chunk whose phi' sum stays below it has no element that overflows.
+constexpr float kF16Max = 65504.f;
 
 // phi' = 2^t for a 32-token chunk (t kept), rounded to fp16 pairs; returns the fp32 sum of phi'.
 // The first 32 - POLY exponentials go to MUFU ex2, the last POLY to the FMA-pipe polynomial.
@@ -132,6 +142,40 @@ __device__ __forceinline__ void tmem_scale_f16x16(uint32_t taddr, float s) {
     }
     tmem_st16u(taddr, h);
     tmem_wait_st();
+}
+
+// Rare path of the exponent warps (warp-collective; out of line so that the common path's code
+// stays compact): chunk c of the current tile, whose phi' may overflow fp16, is redone from its
+// projection (tP: the chunk's P columns, still unreleased; bias: its B_j). Where the chunk's largest
+// t passes 15, D_r is raised so that it lands at lim, and what already carries the old D_r -- the
+// row's [S_h] (64 columns at tS), the tile's earlier phi' chunks, z and this tile's sum zs -- is
+// scaled by 2^-delta. Stores the chunk's phi' and returns the updated scalars with its phi' sum.
+struct KeyRaise {
+    float Dr, z, zs, cs;
+};
+template <int POLY>
+__device__ __noinline__ KeyRaise key_chunk_raise(uint32_t tP, uint32_t tPHI, uint32_t tS, const float *bias, int c,
+                                                 float Dr, float z, float zs, float lim) {
+    float v[32];
+    tmem_ld32_nowait(tP, v);
+    tmem_wait_ld32(v);
+    const float cm = chunk_shift<true>(v, bias, Dr);
+    if (__any_sync(0xffffffffu, cm > 15.f)) {
+        const float delta = cm > 15.f ? ceilf(cm - lim) : 0.f;
+        const float sc = __uint_as_float((uint32_t)(127 - (int)delta) << 23);  // 2^-delta
+        tmem_wait_st();
+        tmem_scale_row(tS, WideCfg::D, sc);
+        for (int cc = 0; cc < c; ++cc) tmem_scale_f16x16(tPHI + 16 * cc, sc);
+        z *= sc;
+        zs *= sc;
+        Dr += delta;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] -= delta;
+    }
+    uint32_t hv[16];
+    const float cs = chunk_exp<POLY>(v, hv);
+    tmem_st16u(tPHI + 16 * c, hv);
+    return KeyRaise{Dr, z, zs, cs};
 }
 
 // Causal use of the kernel: the runs are the (head, segment) blocks of tps consecutive key tiles the
@@ -207,12 +251,12 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
     uint8_t *sW = smem;                                              // m rows of 128 B
     uint8_t *sStage = sW + (size_t)p.m * 128;                        // [STAGES] K tile | V tile
     float *sBias = (float *)(sStage + (size_t)STAGES * C::STAGE);   // [STAGES][128]
-    int *sShift = (int *)(sBias + STAGES * kWideTile);               // [STAGES] (16-int slot)
+    int *sShift = (int *)(sBias + STAGES * kWideTile);               // [STAGES] b_t; [8, 16) converter scratch
     uint64_t *bars = (uint64_t *)(sShift + 16);
-    uint64_t *full = bars, *empty = full + STAGES, *vmax_full = empty + STAGES, *conv_full = vmax_full + STAGES;
-    // per feature half h: p_full / p_free (the P buffer), phi_full / phi_free (the phi' buffer),
-    // acc_full / acc_empty ([S_h] at a run's end), drain (the half's MMAs at exit)
-    uint64_t *w_full = conv_full + STAGES, *p_full = w_full + 1, *p_free = p_full + 2, *phi_full = p_free + 2;
+    uint64_t *full = bars, *empty = full + STAGES, *conv_full = empty + STAGES;
+    // per feature half h: p_full / p_free [2h + q] (P columns of token half q), phi_full / phi_free
+    // (the phi' buffer), acc_full / acc_empty ([S_h] at a run's end), drain (the half's MMAs at exit)
+    uint64_t *w_full = conv_full + STAGES, *p_full = w_full + 1, *p_free = p_full + 4, *phi_full = p_free + 4;
     uint64_t *phi_free = phi_full + 2, *acc_full = phi_free + 2, *acc_empty = acc_full + 2, *drain = acc_empty + 2;
     uint32_t *tmem_slot = (uint32_t *)(drain + 2);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
@@ -225,13 +269,14 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], halves);  // one MMA commit per feature half
-            mbar_init(&vmax_full[s], 1);
             mbar_init(&conv_full[s], 128);
         }
         mbar_init(w_full, 1);
+        for (int q = 0; q < 4; ++q) {
+            mbar_init(&p_full[q], 1);
+            mbar_init(&p_free[q], 128);
+        }
         for (int h = 0; h < 2; ++h) {
-            mbar_init(&p_full[h], 1);
-            mbar_init(&p_free[h], 128);
             mbar_init(&phi_full[h], 128);
             mbar_init(&phi_free[h], 1);
             mbar_init(&acc_full[h], 1);
@@ -265,6 +310,9 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
             Walk wk(p.f, sp, blockIdx.x);
             for (int g = 0; g < n; ++g, wk.next()) {
                 const int s = g % STAGES;
+                // the later stages' first loads wait until tile 0 has landed: at launch every CTA asks
+                // for its first tile alone, so that it arrives sooner
+                if (g == 1 && !mbar_wait_all(&full[0], 0, abort_flag)) break;
                 if (!mbar_wait_lazy(&empty[s], ((g / STAGES) & 1) ^ 1, abort_flag)) break;
                 if (elect_one()) {
                     uint8_t *st = sStage + (size_t)s * C::STAGE;
@@ -278,60 +326,30 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
             volatile int no_abort = 0;
             for (int i = max(issued - STAGES, 0); i < issued; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, &no_abort);
             mbar_wait(w_full, 0, &no_abort);
-        } else if (warp == 14 && n > 0) {
-            // Largest |v| of each V tile (bf16 magnitudes compared as integers) -> b_t; in causal use
-            // also each segment's largest |v|.
-            Walk wk(p.f, sp, blockIdx.x);
-            uint32_t run_mx = 0;
-            for (int g = 0; g < n; ++g, wk.next()) {
-                const int s = g % STAGES;
-                if (!mbar_wait_lazy(&full[s], (g / STAGES) & 1, abort_flag)) break;
-                const uint8_t *vt = sStage + (size_t)s * C::STAGE + C::TILE;
-                uint32_t mx = 0;
-#pragma unroll 4
-                for (int q = lane; q < (int)(C::TILE / 16); q += 32) {
-                    const uint4 w = *(const uint4 *)(vt + q * 16);
-                    mx = __vmaxu2(mx, w.x & 0x7FFF7FFFu);
-                    mx = __vmaxu2(mx, w.y & 0x7FFF7FFFu);
-                    mx = __vmaxu2(mx, w.z & 0x7FFF7FFFu);
-                    mx = __vmaxu2(mx, w.w & 0x7FFF7FFFu);
-                }
-                mx = max(mx & 0xFFFFu, mx >> 16);
-                for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                if (lane == 0) {
-                    const int e = (int)(mx >> 7) - 127;  // exponent of the largest |v| (-127 for an all-zero tile)
-                    sShift[s] = min(max(e - 7, -8), 7);
-                    // V' = V 2^-b_t is an fp16 operand: from 2^23 on (and for inf / nan) it would overflow
-                    if (mx >= 0x4B00u) record_status(FAVOR_ERR_UNSUPPORTED);
-                    mbar_arrive(&vmax_full[s]);
-                    if (SEG) {
-                        run_mx = max(run_mx, mx);
-                        if (wk.last()) {
-                            sp.vmax[wk.slot()] = run_mx;
-                            run_mx = 0;
-                        }
-                    }
-                }
-                __syncwarp();
-            }
         } else if ((warp == 13 || (warp == 15 && halves == 2)) && n > 0) {
             // MMA issue for feature half h by the whole converged warp (predicated issue forms): per
-            // tile g, the projection of tile g + 1 once the exponent warps have read P(g), then the
-            // state MMA of tile g once its V tile is converted and phi'(g) is in TMEM.
+            // tile g, the projection of tile g + 1's first 64 tokens once the exponent warps are done
+            // with P(g)'s columns 0-63, the state MMA of tile g once its V tile is converted and
+            // phi'(g) is in TMEM, then the projection of tile g + 1's last 64 tokens.
             const int h = warp == 13 ? 0 : 1;
             const uint32_t tH = tmem + (uint32_t)h * C::T_HALF;
-            const uint32_t idesc_p = make_idesc(128, kWideTile, kFmtBF16, 0, 0);
+            const uint32_t idesc_p = make_idesc(128, kWideTile / 2, kFmtBF16, 0, 0);
             const uint32_t idesc_s = make_idesc(128, D, kFmtF16, 0, 1);
             const uint64_t dW = make_sdesc(smem_u32(sW) + (uint32_t)h * 128 * 128, 16, 1024);
             const uint64_t dK = make_sdesc(smem_u32(sStage), 16, 1024);
             const uint64_t dV = make_sdesc(smem_u32(sStage) + C::TILE, C::TILE, 1024);
-            auto project = [&](int g) {
-                mma_ss_x4_w(tH + C::T_P, dW, dK + (uint32_t)(g % STAGES) * (C::STAGE / 16), idesc_p, 0u, 2, 2);
-                mma_commit_w(&p_full[h]);
+            // token half q of tile g (K rows 64q.., 64 swizzled rows = 8 KB) into P columns 64q..
+            auto project = [&](int g, int q) {
+                const uint64_t kd = dK + (uint32_t)(g % STAGES) * (C::STAGE / 16) + (uint32_t)q * (8192 / 16);
+                mma_ss_x4_w(tH + C::T_P + 64 * q, dW, kd, idesc_p, 0u, 2, 2);
+                mma_commit_w(&p_full[2 * h + q]);
             };
             bool ok = mbar_wait_all(w_full, 0, abort_flag) && mbar_wait_all(&full[0], 0, abort_flag);
             tc_fence_after();
-            if (ok) project(0);
+            if (ok) {
+                project(0, 0);
+                project(0, 1);
+            }
             int runs = 0;
             Walk wk(p.f, sp, blockIdx.x);
             for (int g = 0; ok && g < n; ++g, wk.next()) {
@@ -339,10 +357,10 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                 const bool first = wk.first(), last = wk.last();
                 if (g + 1 < n) {
                     ok = mbar_wait_all(&full[(g + 1) % STAGES], ((g + 1) / STAGES) & 1, abort_flag) &&
-                         mbar_wait_all(&p_free[h], g & 1, abort_flag);
+                         mbar_wait_all(&p_free[2 * h], g & 1, abort_flag);
                     tc_fence_after();
                     if (!ok) break;
-                    project(g + 1);
+                    project(g + 1, 0);
                 }
                 ok = mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag);
                 if (ok && first && runs > 0) ok = mbar_wait_all(&acc_empty[h], (runs - 1) & 1, abort_flag);
@@ -358,6 +376,12 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                     ++runs;
                 }
                 mma_commit_w(&empty[s]);
+                if (g + 1 < n) {
+                    ok = mbar_wait_all(&p_free[2 * h + 1], g & 1, abort_flag);
+                    tc_fence_after();
+                    if (!ok) break;
+                    project(g + 1, 1);
+                }
             }
             mma_commit_w(&drain[h]);
             volatile int no_abort = 0;
@@ -379,7 +403,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
             for (int g = 0; g < n; ++g, wk.next()) {
                 const int s = g % STAGES;
                 const bool first = wk.first(), last = wk.last();
-                if (!mbar_wait_all(&p_full[h], g & 1, abort_flag) ||
+                if (!mbar_wait_all(&p_full[2 * h], g & 1, abort_flag) ||
                     !mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag))
                     break;
                 tc_fence_after();
@@ -393,6 +417,8 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                     tmem_ld32_nowait(tP + 32, vb);
                     float tm = chunk_tmax(va, bias);
                     tmem_wait_ld32(vb);
+                    if (!mbar_wait_all(&p_full[2 * h + 1], g & 1, abort_flag)) break;
+                    tc_fence_after();
                     tmem_ld32_nowait(tP + 64, va);
                     tm = fmaxf(tm, chunk_tmax(vb, bias + 32));
                     tmem_wait_ld32(va);
@@ -405,51 +431,57 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                     umax = tm - (float)bt;
                 }
                 float zs = 0.f;  // this tile's sum of phi'
-                // One 32-token chunk: t, phi' and the chunk's largest t (in parallel); on a later tile of
-                // the run, a chunk that would overflow fp16 raises D_r (rescaling what already carries
-                // the old D_r) and is redone. phi'(g) overwrites phi'(g - 1), so before the first store
-                // the state MMA of tile g - 1 must have read it (which also makes [S] safe to rescale).
-                auto chunk = [&](float(&v)[32], int c) -> bool {
-                    const float cm = chunk_shift(v, bias + 32 * c, Dr);
+                // One 32-token chunk: t and phi'. On a later tile of the run, a chunk that may overflow
+                // fp16 is redone out of line (key_chunk_raise: D_r raised where a largest t passes 15).
+                // The vote takes the chunk's fp32 sum of phi' (below the largest fp16 value no element
+                // can overflow), or in causal use its largest t, which the head reference needs anyway.
+                // phi'(g) overwrites phi'(g - 1), so before the first store the state MMA of tile g - 1
+                // must have read it (which also makes [S] safe to rescale). `pend` is the buffer whose
+                // TMEM load is in flight: the rare path completes it before the call.
+                auto chunk = [&](float(&v)[32], float(&pend)[32], bool has_pend, int c) -> bool {
+                    const float cm = SEG ? chunk_shift<true>(v, bias + 32 * c, Dr) : chunk_shift<false>(v, bias + 32 * c, Dr);
                     if (SEG && !first) umax = fmaxf(umax, cm + Dr - (float)bt);
                     uint32_t hv[16];
-                    float cs = chunk_exp<POLY>(v, hv);
+                    const float cs = chunk_exp<POLY>(v, hv);
                     if (c == 0) {
                         if (g > 0 && !mbar_wait_all(&phi_free[h], (g - 1) & 1, abort_flag)) return false;
                         tc_fence_after();
                     }
-                    if (!first && __any_sync(0xffffffffu, cm > 15.f)) {
-                        const float delta = cm > 15.f ? ceilf(cm - lim) : 0.f;
-                        const float sc = __uint_as_float((uint32_t)(127 - (int)delta) << 23);  // 2^-delta
-                        tmem_wait_st();
-                        tmem_scale_row(tS, D, sc);
-                        for (int cc = 0; cc < c; ++cc) tmem_scale_f16x16(tPHI + 16 * cc, sc);
-                        z *= sc;
-                        zs *= sc;
-                        Dr += delta;
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] -= delta;
-                        cs = chunk_exp<POLY>(v, hv);
+                    if (!first && __any_sync(0xffffffffu, SEG ? cm > 15.f : cs >= kF16Max)) {
+                        if (has_pend) tmem_wait_ld32(pend);
+                        const KeyRaise r = key_chunk_raise<POLY>(tP + 32 * c, tPHI, tS, bias + 32 * c, c, Dr, z, zs, lim);
+                        Dr = r.Dr;
+                        z = r.z;
+                        zs = r.zs + r.cs;
+                    } else {
+                        zs += cs;
+                        tmem_st16u(tPHI + 16 * c, hv);
                     }
-                    zs += cs;
-                    tmem_st16u(tPHI + 16 * c, hv);
                     return true;
                 };
+                // P columns 0-63 (token half 0) stay readable until chunks 0 and 1 are done (a redo
+                // reads them again), columns 64-127 until chunk 3 is done; each half is then handed to
+                // the projection of tile g + 1.
                 tmem_ld32_nowait(tP, va);
                 tmem_wait_ld32(va);
                 tmem_ld32_nowait(tP + 32, vb);
-                if (!chunk(va, 0)) break;
+                if (!chunk(va, vb, true, 0)) break;
                 tmem_wait_ld32(vb);
+                if (!first) {
+                    if (!mbar_wait_all(&p_full[2 * h + 1], g & 1, abort_flag)) break;
+                    tc_fence_after();
+                }
                 tmem_ld32_nowait(tP + 64, va);
-                chunk(vb, 1);
+                chunk(vb, va, true, 1);
+                tc_fence_before();
+                mbar_arrive(&p_free[2 * h]);
                 tmem_wait_ld32(va);
                 tmem_ld32_nowait(tP + 96, vb);
-                chunk(va, 2);
+                chunk(va, vb, true, 2);
                 tmem_wait_ld32(vb);
-                // P(g) is in registers: the buffer is free for the projection of tile g + 1
+                chunk(vb, va, false, 3);
                 tc_fence_before();
-                mbar_arrive(&p_free[h]);
-                chunk(vb, 3);
+                mbar_arrive(&p_free[2 * h + 1]);
                 z = fmaf(zs, __uint_as_float((uint32_t)(127 - bt) << 23), z);  // z_r += 2^-b_t sum_j phi'
                 tmem_wait_st();
                 tc_fence_before();
@@ -488,25 +520,61 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
         }
     } else {
         regs_dec<88>();
-        // Converter warpgroup: thread j handles token j of each tile (its |k_j|^2 and bias) and
-        // converts 8 of the V tile's 16-byte chunks.
+        // Converter warpgroup: thread j handles token j of each tile (its |k_j|^2 and bias) and 8 of
+        // the V tile's 16-byte chunks. The largest |v| of the tile (bf16 magnitudes compared as
+        // integers, reduced over the warpgroup) gives b_t; the chunks are then rewritten as fp16
+        // V' = V 2^-b_t. In causal use thread 0 also records each segment's largest |v|.
         const int j = threadIdx.x;
+        uint32_t *sRed = (uint32_t *)(sShift + 8);  // [2 tile parities][4 warps]
+        uint32_t run_mx = 0;
         Walk wk(p.f, sp, blockIdx.x);
         for (int g = 0; g < n; ++g, wk.next()) {
             const int s = g % STAGES, t = wk.t;
-            if (!mbar_wait_lazy(&vmax_full[s], (g / STAGES) & 1, abort_flag)) break;
+            // the first tile is on every CTA's critical path: poll it without sleeping
+            const bool ok = g == 0 ? mbar_wait_all(&full[0], 0, abort_flag)
+                                   : mbar_wait_lazy(&full[s], (g / STAGES) & 1, abort_flag);
+            if (!ok) break;
             uint8_t *st = sStage + (size_t)s * C::STAGE;
-            const int b = sShift[s];
+            uint4 vw[C::TILE / 16 / 128];
+            uint32_t mx = 0;
+#pragma unroll
+            for (int i = 0; i < (int)(C::TILE / 16 / 128); ++i) {
+                vw[i] = *(const uint4 *)(st + C::TILE + (size_t)(j + 128 * i) * 16);
+                mx = __vmaxu2(mx, vw[i].x & 0x7FFF7FFFu);
+                mx = __vmaxu2(mx, vw[i].y & 0x7FFF7FFFu);
+                mx = __vmaxu2(mx, vw[i].z & 0x7FFF7FFFu);
+                mx = __vmaxu2(mx, vw[i].w & 0x7FFF7FFFu);
+            }
+            mx = max(mx & 0xFFFFu, mx >> 16);
+            for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if ((j & 31) == 0) sRed[(g & 1) * 4 + (j >> 5)] = mx;
+            named_bar_sync(1, 128);
+            mx = max(max(sRed[(g & 1) * 4], sRed[(g & 1) * 4 + 1]), max(sRed[(g & 1) * 4 + 2], sRed[(g & 1) * 4 + 3]));
+            const int e = (int)(mx >> 7) - 127;  // exponent of the largest |v| (-127 for an all-zero tile)
+            const int b = min(max(e - 7, -8), 7);
+            if (j == 0) {
+                sShift[s] = b;
+                // V' = V 2^-b_t is an fp16 operand: from 2^23 on (and for inf / nan) it would overflow
+                if (mx >= 0x4B00u) record_status(FAVOR_ERR_UNSUPPORTED);
+                if (SEG) {
+                    run_mx = max(run_mx, mx);
+                    if (wk.last()) {
+                        sp.vmax[wk.slot()] = run_mx;
+                        run_mx = 0;
+                    }
+                }
+            }
             const float scale = __uint_as_float((uint32_t)(127 - b) << 23);  // 2^-b
 #pragma unroll
             for (int i = 0; i < (int)(C::TILE / 16 / 128); ++i) {
-                uint4 *q = (uint4 *)(st + C::TILE + (size_t)(j + 128 * i) * 16);
-                uint4 w = *q;
-                uint32_t u[4] = {w.x, w.y, w.z, w.w};
+                uint32_t u[4] = {vw[i].x, vw[i].y, vw[i].z, vw[i].w};
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    u[k] = pack_f16x2(__uint_as_float(u[k] << 16) * scale, __uint_as_float(u[k] & 0xFFFF0000u) * scale);
-                *q = make_uint4(u[0], u[1], u[2], u[3]);
+                for (int k = 0; k < 4; ++k) {
+                    float lo, hi;
+                    ffma2(__uint_as_float(u[k] << 16), __uint_as_float(u[k] & 0xFFFF0000u), scale, scale, 0.f, 0.f, lo, hi);
+                    u[k] = pack_f16x2(lo, hi);
+                }
+                *(uint4 *)(st + C::TILE + (size_t)(j + 128 * i) * 16) = make_uint4(u[0], u[1], u[2], u[3]);
             }
             const bool valid = t * kWideTile + j < p.L;
             const float k2 = key_sq_norm<1, kWideTile>(st, j);
