@@ -17,6 +17,7 @@ namespace favor {
 
 constexpr int kTile = 128;               // tokens per tile (MMA M for token-major operands)
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s per wait
 
 // Device status word (FAVOR_OK or FAVOR_ERR_TIMEOUT), read and cleared by favor_sync_status.
@@ -344,6 +345,25 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t smem_addr, uint32_t lbo_
     d |= (uint64_t)1 << 46;  // descriptor version for sm_100
     d |= (uint64_t)2 << 61;  // SWIZZLE_128B
     return d;
+}
+
+// Shared-memory matrix descriptor without swizzle (interleaved core matrices of 8 rows x 16 bytes,
+// each 128 contiguous bytes), K-major: LBO = byte stride between core matrices along K, SBO = byte
+// stride between 8-row groups along M/N.
+__device__ __forceinline__ uint64_t make_sdesc_interleaved(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version for sm_100; layout type 0 (no swizzle)
+    return d;
+}
+
+// fp32 -> bf16 bits, round to nearest even.
+__device__ __forceinline__ uint32_t bf16_bits_rn(float x) {
+    unsigned short h;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(x));
+    return (uint32_t)h;
 }
 
 // Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a 128-byte-swizzled tile

@@ -11,15 +11,18 @@
 // Why a second key kernel: on 64-token tiles each exponent warp spends most of a tile in fixed
 // per-tile costs (barrier round trips, TMEM load latency, the stabiliser vote) rather than on the
 // MUFU. Here a tile is 128 tokens and, except on a run's first tile, the projection is read once:
-//   - P_h^T = W_h K_tile^T (M = 128 features of half h, K = 64), issued as two N = 64 MMAs, one per
-//     64-token half of the tile, so that each half of the P buffer is handed to the next tile's
-//     projection as soon as the exponent warps are done with it;
-//   - per 32-token chunk c: t = P log2e + B_j - D_r, phi' = 2^t in fp16 stored to TMEM (16 packed
-//     columns) and z_r += 2^-b_t sum_j phi'; the next chunk's TMEM load is in flight meanwhile. A
-//     warp vote on the chunk's fp32 sum of phi' (below the largest fp16 value no element can
-//     overflow) sends the rare chunk that may overflow to an out-of-line redo, which re-reads its
-//     P columns and raises D_r where its largest t passes 15 (the causal use votes on every chunk's
-//     largest t, which its head reference needs anyway);
+//   - P'_h^T = W_h K_tile^T + B'_j (M = 128 features of half h), issued as two N = 64 MMA groups,
+//     one per 64-token half of the tile, so that each half of the P buffer is handed to the next
+//     tile's projection as soon as the exponent warps are done with it. Each group is K = 64 of
+//     W K^T plus one K = 16 extension step that adds the key's bias B'_j = B_j / log2e =
+//     -|k_j|^2/2 + (A + b_t) ln 2: the converter warps write it as three bf16 parts (hi + mid + lo,
+//     fp32's precision in sum) into the key row's extension, against three ones columns of W's;
+//   - per 32-token chunk c: t = P' log2e - D_r (one paired FMA per two tokens), phi' = 2^t in fp16
+//     stored to TMEM (16 packed columns) and z_r += 2^-b_t sum_j phi'; the next chunk's TMEM load is
+//     in flight meanwhile. A warp vote on the chunk's fp32 sum of phi' (below the largest fp16
+//     value no element can overflow) sends the rare chunk that may overflow to an out-of-line redo,
+//     which re-reads its P columns and raises D_r where its largest t passes 15 (the causal use
+//     votes on every chunk's largest t, which its head reference needs anyway);
 //   - [S_h] += phi'_h V'_t (fp16 MMA, A from TMEM, B the converted V tile read MN-major, N = 64).
 // z_r is kept in the exponent thread's registers instead of a ones column of the state MMA, which
 // frees the TMEM columns the wider tile needs: per half P (128) + phi' (64) + S (64) = 256 columns.
@@ -31,9 +34,9 @@
 // 2^-delta, and the chunk's exponentials are recomputed before they are stored. Typical inputs
 // raise it rarely. V'_t = V_t 2^-b_t as in k_key_partials.
 //
-// Warp roles (16 warps): 0-3 the tile's largest |v| and b_t, convert V, write the biases B_j (thread
-// j = token j of the tile); 4-7 / 8-11 exponentials of feature half 0 / 1 and the run-end write;
-// 12 TMA; 13 / 15 MMA issue for half 0 / 1; 14 idle.
+// Warp roles (16 warps): 0-3 the tile's largest |v| and b_t, convert V, write the key rows'
+// extensions (thread j = token j of the tile); 4-7 / 8-11 exponentials of feature half 0 / 1 and
+// the run-end write; 12 TMA; 13 / 15 MMA issue for half 0 / 1; 14 idle.
 
 #include <type_traits>
 
@@ -48,6 +51,8 @@ struct WideCfg {
     static constexpr int STAGES = 4;
     static constexpr uint32_t TILE = kWideTile * 128;  // K or V tile: 128 rows of 64 bf16
     static constexpr uint32_t STAGE = 2 * TILE;        // K tile | V tile
+    // key-row extension of a stage (interleaved, 128 rows x 32 bytes): B'_j in three bf16 parts
+    static constexpr uint32_t KX = kWideTile * 32;
     // TMEM columns of half h (base h * 256): P [0, 128), phi' [128, 192), [S_h] [192, 256)
     static constexpr uint32_t T_P = 0, T_PHI = 128, T_S = 192, T_HALF = 256;
 };
@@ -66,31 +71,27 @@ __device__ __forceinline__ void tmem_ld16u(uint32_t taddr, uint32_t (&h)[16]) {
                    "+r"(h[15])::"memory");
 }
 
-// Largest t = v log2e + B_j over a 32-token chunk (v the projection, bias the chunk's B_j).
-__device__ __forceinline__ float chunk_tmax(const float (&v)[32], const float *bias) {
+// Largest value of a 32-token chunk.
+__device__ __forceinline__ float chunk_vmax(const float (&v)[32]) {
     float a = -INFINITY, b = -INFINITY;
 #pragma unroll
     for (int e = 0; e < 32; e += 4) {
-        const float4 b4 = *(const float4 *)(bias + e);
-        a = fmax3(a, fmaf(v[e], kLog2e, b4.x), fmaf(v[e + 1], kLog2e, b4.y));
-        b = fmax3(b, fmaf(v[e + 2], kLog2e, b4.z), fmaf(v[e + 3], kLog2e, b4.w));
+        a = fmax3(a, v[e], v[e + 1]);
+        b = fmax3(b, v[e + 2], v[e + 3]);
     }
     return fmaxf(a, b);
 }
 
-// t = v log2e + B_j - D for a 32-token chunk, in place (paired FMA-pipe instructions); returns the
-// chunk's largest t when MAX is set (else 0).
+// t = P' log2e - D for a 32-token chunk, in place (paired FMA-pipe instructions; P' carries the
+// key's B_j through the projection's extension step); returns the chunk's largest t when MAX is set
+// (else 0).
 template <bool MAX>
-__device__ __forceinline__ float chunk_shift(float (&v)[32], const float *bias, float D) {
+__device__ __forceinline__ float chunk_shift(float (&v)[32], float D) {
     float a = -INFINITY, b = -INFINITY;
 #pragma unroll
     for (int e = 0; e < 32; e += 4) {
-        const float4 b4 = *(const float4 *)(bias + e);
-        float c0, c1, c2, c3;
-        ffma2(b4.x, b4.y, 1.f, 1.f, -D, -D, c0, c1);  // B_j - D
-        ffma2(b4.z, b4.w, 1.f, 1.f, -D, -D, c2, c3);
-        ffma2(v[e], v[e + 1], kLog2e, kLog2e, c0, c1, v[e], v[e + 1]);
-        ffma2(v[e + 2], v[e + 3], kLog2e, kLog2e, c2, c3, v[e + 2], v[e + 3]);
+        ffma2(v[e], v[e + 1], kLog2e, kLog2e, -D, -D, v[e], v[e + 1]);
+        ffma2(v[e + 2], v[e + 3], kLog2e, kLog2e, -D, -D, v[e + 2], v[e + 3]);
         if (MAX) {
             a = fmax3(a, v[e], v[e + 1]);
             b = fmax3(b, v[e + 2], v[e + 3]);
@@ -146,7 +147,7 @@ __device__ __forceinline__ void tmem_scale_f16x16(uint32_t taddr, float s) {
 
 // Rare path of the exponent warps (warp-collective; out of line so that the common path's code
 // stays compact): chunk c of the current tile, whose phi' may overflow fp16, is redone from its
-// projection (tP: the chunk's P columns, still unreleased; bias: its B_j). Where the chunk's largest
+// projection (tP: the chunk's P columns, still unreleased). Where the chunk's largest
 // t passes 15, D_r is raised so that it lands at lim, and what already carries the old D_r -- the
 // row's [S_h] (64 columns at tS), the tile's earlier phi' chunks, z and this tile's sum zs -- is
 // scaled by 2^-delta. Stores the chunk's phi' and returns the updated scalars with its phi' sum.
@@ -154,12 +155,12 @@ struct KeyRaise {
     float Dr, z, zs, cs;
 };
 template <int POLY>
-__device__ __noinline__ KeyRaise key_chunk_raise(uint32_t tP, uint32_t tPHI, uint32_t tS, const float *bias, int c,
-                                                 float Dr, float z, float zs, float lim) {
+__device__ __noinline__ KeyRaise key_chunk_raise(uint32_t tP, uint32_t tPHI, uint32_t tS, int c, float Dr, float z,
+                                                 float zs, float lim) {
     float v[32];
     tmem_ld32_nowait(tP, v);
     tmem_wait_ld32(v);
-    const float cm = chunk_shift<true>(v, bias, Dr);
+    const float cm = chunk_shift<true>(v, Dr);
     if (__any_sync(0xffffffffu, cm > 15.f)) {
         const float delta = cm > 15.f ? ceilf(cm - lim) : 0.f;
         const float sc = __uint_as_float((uint32_t)(127 - (int)delta) << 23);  // 2^-delta
@@ -250,8 +251,9 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
     const int halves = p.m / 128;
     uint8_t *sW = smem;                                              // m rows of 128 B
     uint8_t *sStage = sW + (size_t)p.m * 128;                        // [STAGES] K tile | V tile
-    float *sBias = (float *)(sStage + (size_t)STAGES * C::STAGE);   // [STAGES][128]
-    int *sShift = (int *)(sBias + STAGES * kWideTile);               // [STAGES] b_t; [8, 16) converter scratch
+    uint8_t *sKx = sStage + (size_t)STAGES * C::STAGE;               // [STAGES] key-row extensions
+    uint8_t *sWx = sKx + (size_t)STAGES * C::KX;                     // m feature rows x 32 B: 1, 1, 1, 0...
+    int *sShift = (int *)(sWx + (size_t)p.m * 32);                   // [STAGES] b_t; [8, 16) converter scratch
     uint64_t *bars = (uint64_t *)(sShift + 16);
     uint64_t *full = bars, *empty = full + STAGES, *conv_full = empty + STAGES;
     // per feature half h: p_full / p_free [2h + q] (P columns of token half q), phi_full / phi_free
@@ -290,6 +292,19 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
+    // Projection extension (one K = 16 step, interleaved layout: row r's 16-byte core-matrix row at
+    // (r / 8) 256 + (k / 8) 128 + (r % 8) 16): W's rows get three ones columns, every key row's
+    // second core matrix is zero (the first is written per tile by the converter warps).
+    for (int i = threadIdx.x; i < p.m * 2; i += kKeyThreads) {
+        const int r = i >> 1, kc = i & 1;
+        *(uint4 *)(sWx + (r >> 3) * 256 + kc * 128 + (r & 7) * 16) =
+            kc == 0 ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int i = threadIdx.x; i < STAGES * kWideTile; i += kKeyThreads) {
+        const int st = i / kWideTile, r = i % kWideTile;
+        *(uint4 *)(sKx + st * C::KX + (r >> 3) * 256 + 128 + (r & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -339,12 +354,19 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
             const uint64_t dK = make_sdesc(smem_u32(sStage), 16, 1024);
             const uint64_t dV = make_sdesc(smem_u32(sStage) + C::TILE, C::TILE, 1024);
             // token half q of tile g (K rows 64q.., 64 swizzled rows = 8 KB) into P columns 64q..
+            // plus the extension step: B'_j of token half q against W's ones columns
+            const uint64_t dWx = make_sdesc_interleaved(smem_u32(sWx) + (uint32_t)h * 4096, 128, 256);
+            const uint64_t dKx = make_sdesc_interleaved(smem_u32(sKx), 128, 256);
             auto project = [&](int g, int q) {
                 const uint64_t kd = dK + (uint32_t)(g % STAGES) * (C::STAGE / 16) + (uint32_t)q * (8192 / 16);
                 mma_ss_x4_w(tH + C::T_P + 64 * q, dW, kd, idesc_p, 0u, 2, 2);
+                const uint64_t xd = dKx + (uint32_t)(g % STAGES) * (C::KX / 16) + (uint32_t)q * (2048 / 16);
+                mma_f16_ss_w(tH + C::T_P + 64 * q, dWx, xd, idesc_p, 1u);
                 mma_commit_w(&p_full[2 * h + q]);
             };
-            bool ok = mbar_wait_all(w_full, 0, abort_flag) && mbar_wait_all(&full[0], 0, abort_flag);
+            // a projection reads the tile's key rows (TMA) and their extension (converter warps)
+            bool ok = mbar_wait_all(w_full, 0, abort_flag) && mbar_wait_all(&full[0], 0, abort_flag) &&
+                      mbar_wait_all(&conv_full[0], 0, abort_flag);
             tc_fence_after();
             if (ok) {
                 project(0, 0);
@@ -357,6 +379,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                 const bool first = wk.first(), last = wk.last();
                 if (g + 1 < n) {
                     ok = mbar_wait_all(&full[(g + 1) % STAGES], ((g + 1) / STAGES) & 1, abort_flag) &&
+                         mbar_wait_all(&conv_full[(g + 1) % STAGES], ((g + 1) / STAGES) & 1, abort_flag) &&
                          mbar_wait_all(&p_free[2 * h], g & 1, abort_flag);
                     tc_fence_after();
                     if (!ok) break;
@@ -407,7 +430,6 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                     !mbar_wait_all(&conv_full[s], (g / STAGES) & 1, abort_flag))
                     break;
                 tc_fence_after();
-                const float *bias = sBias + s * kWideTile;
                 const int bt = sShift[s];
                 const float lim = kKeyFeatureShift + (float)bt;  // target for a run's largest t
                 if (first) {
@@ -415,17 +437,18 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                     tmem_ld32_nowait(tP, va);
                     tmem_wait_ld32(va);
                     tmem_ld32_nowait(tP + 32, vb);
-                    float tm = chunk_tmax(va, bias);
+                    float pm = chunk_vmax(va);
                     tmem_wait_ld32(vb);
                     if (!mbar_wait_all(&p_full[2 * h + 1], g & 1, abort_flag)) break;
                     tc_fence_after();
                     tmem_ld32_nowait(tP + 64, va);
-                    tm = fmaxf(tm, chunk_tmax(vb, bias + 32));
+                    pm = fmaxf(pm, chunk_vmax(vb));
                     tmem_wait_ld32(va);
                     tmem_ld32_nowait(tP + 96, vb);
-                    tm = fmaxf(tm, chunk_tmax(va, bias + 64));
+                    pm = fmaxf(pm, chunk_vmax(va));
                     tmem_wait_ld32(vb);
-                    tm = fmaxf(tm, chunk_tmax(vb, bias + 96));
+                    pm = fmaxf(pm, chunk_vmax(vb));
+                    const float tm = pm * kLog2e;  // the rounding of t = P' log2e is monotone
                     Dr = ceilf(tm - lim);
                     z = 0.f;
                     umax = tm - (float)bt;
@@ -439,7 +462,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                 // must have read it (which also makes [S] safe to rescale). `pend` is the buffer whose
                 // TMEM load is in flight: the rare path completes it before the call.
                 auto chunk = [&](float(&v)[32], float(&pend)[32], bool has_pend, int c) -> bool {
-                    const float cm = SEG ? chunk_shift<true>(v, bias + 32 * c, Dr) : chunk_shift<false>(v, bias + 32 * c, Dr);
+                    const float cm = SEG ? chunk_shift<true>(v, Dr) : chunk_shift<false>(v, Dr);
                     if (SEG && !first) umax = fmaxf(umax, cm + Dr - (float)bt);
                     uint32_t hv[16];
                     const float cs = chunk_exp<POLY>(v, hv);
@@ -449,7 +472,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
                     }
                     if (!first && __any_sync(0xffffffffu, SEG ? cm > 15.f : cs >= kF16Max)) {
                         if (has_pend) tmem_wait_ld32(pend);
-                        const KeyRaise r = key_chunk_raise<POLY>(tP + 32 * c, tPHI, tS, bias + 32 * c, c, Dr, z, zs, lim);
+                        const KeyRaise r = key_chunk_raise<POLY>(tP + 32 * c, tPHI, tS, c, Dr, z, zs, lim);
                         Dr = r.Dr;
                         z = r.z;
                         zs = r.zs + r.cs;
@@ -520,7 +543,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
         }
     } else {
         regs_dec<88>();
-        // Converter warpgroup: thread j handles token j of each tile (its |k_j|^2 and bias) and 8 of
+        // Converter warpgroup: thread j handles token j of each tile (its |k_j|^2 and extension) and 8 of
         // the V tile's 16-byte chunks. The largest |v| of the tile (bf16 magnitudes compared as
         // integers, reduced over the warpgroup) gives b_t; the chunks are then rewritten as fp16
         // V' = V 2^-b_t. In causal use thread 0 also records each segment's largest |v|.
@@ -578,7 +601,18 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
             }
             const bool valid = t * kWideTile + j < p.L;
             const float k2 = key_sq_norm<1, kWideTile>(st, j);
-            sBias[s * kWideTile + j] = valid ? fmaf(-0.5f * k2, kLog2e, kKeyFeatureShift + (float)b) : -INFINITY;
+            // B'_j = B_j / log2e = -|k_j|^2 / 2 + (A + b_t) ln 2 as three bf16 parts (hi, mid, lo: their
+            // sum carries fp32's precision) in key row j's extension; a key past L gets -inf
+            uint4 xb = make_uint4(0xFF80u, 0u, 0u, 0u);
+            if (valid) {
+                const float Bp = fmaf(-0.5f, k2, (kKeyFeatureShift + (float)b) * kLn2);
+                const uint32_t hi = bf16_bits_rn(Bp);
+                const float r1 = Bp - __uint_as_float(hi << 16);
+                const uint32_t mid = bf16_bits_rn(r1);
+                const uint32_t lo = bf16_bits_rn(r1 - __uint_as_float(mid << 16));
+                xb = make_uint4(hi | (mid << 16), lo, 0u, 0u);
+            }
+            *(uint4 *)(sKx + s * C::KX + (j >> 3) * 256 + (j & 7) * 16) = xb;
             if (SEG && valid) sp.bias[(size_t)wk.bh * p.L + t * kWideTile + j] = -0.5f * k2;
             fence_async_smem();
             mbar_arrive(&conv_full[s]);
@@ -594,7 +628,7 @@ k_key_partials_wide(const __grid_constant__ CUtensorMap mapK, const __grid_const
 
 static size_t key_wide_smem(int m) {
     using C = WideCfg;
-    return 1024 + (size_t)m * 128 + (size_t)C::STAGES * C::STAGE + C::STAGES * kWideTile * 4 + 64 + 512;
+    return 1024 + (size_t)m * 128 + (size_t)C::STAGES * (C::STAGE + C::KX) + (size_t)m * 32 + 64 + 512;
 }
 
 // The register split (88 + 2 x 160 + 88 per warpgroup lane) fits the 128 per thread the kernel is
