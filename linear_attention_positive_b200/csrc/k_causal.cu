@@ -520,7 +520,7 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
             mbar_arrive(&bar[B_PQ_FREE]);
             const float cl = row_max128(v) * kLog2e;
 #pragma unroll
-            for (int e = 0; e < 128; ++e) v[e] = fmaf(v[e], kLog2e, -cl);
+            for (int e = 0; e < 128; e += 2) ffma2(v[e], v[e + 1], kLog2e, kLog2e, -cl, -cl, v[e], v[e + 1]);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -535,10 +535,8 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
 #pragma unroll
             for (int e = 0; e < 128; e += 4) {
                 const float4 z4 = *(const float4 *)(z + e);
-                d0 = fmaf(v[e], z4.x, d0);
-                d1 = fmaf(v[e + 1], z4.y, d1);
-                d0 = fmaf(v[e + 2], z4.z, d0);
-                d1 = fmaf(v[e + 3], z4.w, d1);
+                ffma2(v[e], v[e + 1], z4.x, z4.y, d0, d1, d0, d1);
+                ffma2(v[e + 2], v[e + 3], z4.z, z4.w, d0, d1, d0, d1);
             }
             if (g > 0 && !mbar_wait_all(&bar[B_PHIQ_FREE], (g - 1) & 1, abort_flag)) break;
             tc_fence_after();
@@ -614,10 +612,8 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
                     const float4 b4 = *(const float4 *)(beta + 32 * c + e);
-                    v[e] = fmaf(v[e], kLog2e, b4.x);
-                    v[e + 1] = fmaf(v[e + 1], kLog2e, b4.y);
-                    v[e + 2] = fmaf(v[e + 2], kLog2e, b4.z);
-                    v[e + 3] = fmaf(v[e + 3], kLog2e, b4.w);
+                    ffma2(v[e], v[e + 1], kLog2e, kLog2e, b4.x, b4.y, v[e], v[e + 1]);
+                    ffma2(v[e + 2], v[e + 3], kLog2e, kLog2e, b4.z, b4.w, v[e + 2], v[e + 3]);
                 }
 #pragma unroll
                 for (int e = 0; e < 32 - POLY; ++e) v[e] = ex2_approx(v[e]);
@@ -626,8 +622,7 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                 uint32_t hv[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    zs0 += v[e];
-                    zs1 += v[e + 1];
+                    ffma2(v[e], v[e + 1], 1.f, 1.f, zs0, zs1, zs0, zs1);
                     hv[e >> 1] = pack_f16x2(v[e], v[e + 1]);
                 }
                 // tokens 32c .. 32c + 31: block c >> 1, 16-byte chunks 4 (c & 1) .. + 3
@@ -730,8 +725,12 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                     __syncwarp();
                     float *srow = (float *)(smem + OFF_SEND) + (row & 63) * RECV_ROW;
 #pragma unroll
-                    for (int c = 0; c < 64; c += 4)
-                        *(float4 *)(srow + c) = make_float4(o[c] * up, o[c + 1] * up, o[c + 2] * up, o[c + 3] * up);
+                    for (int c = 0; c < 64; c += 4) {
+                        float4 w;
+                        ffma2(o[c], o[c + 1], up, up, 0.f, 0.f, w.x, w.y);
+                        ffma2(o[c + 2], o[c + 3], up, up, 0.f, 0.f, w.z, w.w);
+                        *(float4 *)(srow + c) = w;
+                    }
                     *(float4 *)(srow + 64) = make_float4(den, cq, 0.f, 0.f);
                     fence_async_smem();
                     __syncwarp();
@@ -769,9 +768,10 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                         }
 #pragma unroll
                         for (int c = 0; c < 32; c += 2) {
-                            rs0 += a[c];
-                            rs1 += a[c + 1];
-                            h[c >> 1] = pack_f16x2(a[c] * sc, a[c + 1] * sc);
+                            float s0, s1;
+                            ffma2(a[c], a[c + 1], 1.f, 1.f, rs0, rs1, rs0, rs1);
+                            ffma2(a[c], a[c + 1], sc, sc, 0.f, 0.f, s0, s1);
+                            h[c >> 1] = pack_f16x2(s0, s1);
                         }
                     } else {
 #pragma unroll
@@ -797,8 +797,12 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                     const float inv = up * rcp_approx(den);
                     if (store)
 #pragma unroll
-                        for (int c = 0; c < 64; c += 4)
-                            *(float4 *)(dst + c) = make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv);
+                        for (int c = 0; c < 64; c += 4) {
+                            float4 w;
+                            ffma2(o[c], o[c + 1], inv, inv, 0.f, 0.f, w.x, w.y);
+                            ffma2(o[c + 2], o[c + 3], inv, inv, 0.f, 0.f, w.z, w.w);
+                            *(float4 *)(dst + c) = w;
+                        }
                 } else {
                     if (!mbar_wait_cluster_all(&bar[B_RECV_FULL + eb], (e >> 1) & 1, abort_flag)) break;
                     const float *slot = (const float *)(smem + OFF_RECV + eb * RECV_SLOT) + (row & 63) * RECV_ROW;
@@ -810,10 +814,11 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
 #pragma unroll
                     for (int c = 0; c < 64; c += 4) {
                         const float4 r4 = *(const float4 *)(slot + c);
-                        o[c] = fmaf(o[c], sa, r4.x * sb);
-                        o[c + 1] = fmaf(o[c + 1], sa, r4.y * sb);
-                        o[c + 2] = fmaf(o[c + 2], sa, r4.z * sb);
-                        o[c + 3] = fmaf(o[c + 3], sa, r4.w * sb);
+                        float t0, t1, t2, t3;
+                        ffma2(r4.x, r4.y, sb, sb, 0.f, 0.f, t0, t1);
+                        ffma2(r4.z, r4.w, sb, sb, 0.f, 0.f, t2, t3);
+                        ffma2(o[c], o[c + 1], sa, sa, t0, t1, o[c], o[c + 1]);
+                        ffma2(o[c + 2], o[c + 3], sa, sa, t2, t3, o[c + 2], o[c + 3]);
                     }
                     mbar_arrive_remote(cluster_map(smem_u32(&bar[B_RECV_FREE + eb]), partner));
                     if (store)
