@@ -495,8 +495,11 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                     const uint32_t u[4] = {w.x, w.y, w.z, w.w};
                     uint32_t h[4];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        h[k] = pack_f16x2(__uint_as_float(u[k] << 16) * vsc, __uint_as_float(u[k] & 0xFFFF0000u) * vsc);
+                    for (int k = 0; k < 4; ++k) {
+                        float lo, hi;
+                        ffma2(__uint_as_float(u[k] << 16), __uint_as_float(u[k] & 0xFFFF0000u), vsc, vsc, 0.f, 0.f, lo, hi);
+                        h[k] = pack_f16x2(lo, hi);
+                    }
                     *pq = make_uint4(h[0], h[1], h[2], h[3]);
                 }
                 // inf / nan entries (bf16 exponent field all ones) have no scaled fp16 form

@@ -50,11 +50,13 @@ __device__ __forceinline__ float key_sq_norm(const uint8_t *tile, int row) {
         for (int ch = 0; ch < 8; ++ch) {
             const uint4 w = *(const uint4 *)(tile + kb * (ROWS * 128) + sw128_offset(row, ch));
             const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+            // acc[i] += lo_i^2, then hi_i^2, two accumulators per paired FMA-pipe instruction
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float lo = __uint_as_float(u[i] << 16), hi = __uint_as_float(u[i] & 0xFFFF0000u);
-                acc[i] = fmaf(lo, lo, acc[i]);
-                acc[i] = fmaf(hi, hi, acc[i]);
+            for (int i = 0; i < 4; i += 2) {
+                const float lo0 = __uint_as_float(u[i] << 16), hi0 = __uint_as_float(u[i] & 0xFFFF0000u);
+                const float lo1 = __uint_as_float(u[i + 1] << 16), hi1 = __uint_as_float(u[i + 1] & 0xFFFF0000u);
+                ffma2(lo0, lo1, lo0, lo1, acc[i], acc[i + 1], acc[i], acc[i + 1]);
+                ffma2(hi0, hi1, hi0, hi1, acc[i], acc[i + 1], acc[i], acc[i + 1]);
             }
         }
     }

@@ -502,7 +502,10 @@ k_query_out(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
                     const float *q = &o[cb * 32 + 4 * ch];
-                    *(float4 *)(rowp + ((ch ^ (lane & 7)) << 4)) = make_float4(q[0] * inv, q[1] * inv, q[2] * inv, q[3] * inv);
+                    float4 w;
+                    ffma2(q[0], q[1], inv, inv, 0.f, 0.f, w.x, w.y);
+                    ffma2(q[2], q[3], inv, inv, 0.f, 0.f, w.z, w.w);
+                    *(float4 *)(rowp + ((ch ^ (lane & 7)) << 4)) = w;
                 }
             }
             fence_async_smem();
