@@ -680,11 +680,14 @@ k_causal_chunk(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__
                 tmem_ld32(tmem + lane_off + T_S + 32 * h, w);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
+                    float x[8];
+#pragma unroll
+                    for (int i = 0; i < 8; i += 2) ffma2(w[8 * c + i], w[8 * c + i + 1], sc, sc, 0.f, 0.f, x[i], x[i + 1]);
                     uint4 u;
-                    u.x = pack_f16x2(w[8 * c] * sc, w[8 * c + 1] * sc);
-                    u.y = pack_f16x2(w[8 * c + 2] * sc, w[8 * c + 3] * sc);
-                    u.z = pack_f16x2(w[8 * c + 4] * sc, w[8 * c + 5] * sc);
-                    u.w = pack_f16x2(w[8 * c + 6] * sc, w[8 * c + 7] * sc);
+                    u.x = pack_f16x2(x[0], x[1]);
+                    u.y = pack_f16x2(x[2], x[3]);
+                    u.z = pack_f16x2(x[4], x[5]);
+                    u.w = pack_f16x2(x[6], x[7]);
                     *(uint4 *)(simg + (((4 * h + c) ^ (f & 7)) << 4)) = u;
                 }
             }
