@@ -64,11 +64,7 @@ __device__ __forceinline__ float pow2i(float e) {
 // reference stabiliser C (the largest D over its runs and features): each run's feature row r is
 // weighted by 2^(D_r - C), exactly, and summed in CTA order. The sums are scaled by 2^(15 - e),
 // 2^e exceeding the bound sum_runs max_warp amax 2^(Dmax - C) on their magnitude, and rounded to
-// fp16. Grid: (chunks / 128, heads). Every load a thread needs -- its run statistics and its chunk
-// of the first kImageRunsAhead runs -- is issued before the block reductions, so the kernel pays
-// about one round trip to L2 (heads over more CTAs load the remaining runs afterwards).
-constexpr int kImageRunsAhead = 4;
-
+// fp16. Grid: (chunks / 128, heads).
 __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
     __shared__ float sC, sScale, sRed[kImageThreads / 32];
     pdl_launch_dependents();   // the query kernel may start its projections meanwhile
@@ -77,45 +73,15 @@ __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
     const int c_first = flat_first_cta(p.f, bh), c_last = flat_last_cta(p.f, bh);
     const int halves = p.m / 128, nhs = p.d / 64;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    // per-(run, warp) statistics, one per thread (a head spans at most a few runs)
     const int nstat = (c_last - c_first + 1) * 8;
-
-    // this thread's chunk: (value half nh, feature half h, k-block kb, image row, 16-byte chunk pch)
-    const int chunks = nhs * halves * 2 * kImgRows * 8;
-    const int q = blockIdx.x * kImageThreads + threadIdx.x;
-    const bool active = q < chunks;
-    const int pch = q & 7, row = (q >> 3) % kImgRows, blk = (q >> 3) / kImgRows;  // blk = (nh*H + h)*2 + kb
-    const int kb = blk & 1, h = (blk >> 1) % halves, nh = (blk >> 1) / halves;
-    const bool has_data = active && row <= 64;
-    const int col = row < 64 ? nh * 64 + row : p.d;
-    const int r0 = h * 128 + kb * 64 + 8 * (pch ^ (row & 7));
-    auto src_of = [&](int c) { return (const float4 *)(p.part + ((size_t)(c + bh) * (p.d + 1) + col) * p.m + r0); };
-    auto d_of = [&](int c) { return (const float4 *)(p.part_D + (size_t)(c + bh) * p.m + r0); };
-
-    // loads in flight together: the statistics (one per thread while a head spans at most 16 runs)
-    // and the first runs' partial states and stabilisers of this chunk
-    float st_d = -INFINITY, st_a = 0.f;
-    const bool st_mine = threadIdx.x < nstat && (threadIdx.x & 7) < 4 * halves;
-    if (st_mine) {
-        const size_t k = (size_t)(c_first + (threadIdx.x >> 3) + bh) * 8 + (threadIdx.x & 7);
-        st_d = p.part_Dmax[k];
-        st_a = p.part_amax[k];
-    }
-    float4 a[kImageRunsAhead], b[kImageRunsAhead], da[kImageRunsAhead], db[kImageRunsAhead];
-#pragma unroll
-    for (int i = 0; i < kImageRunsAhead; ++i) {
-        const int c = c_first + i;
-        if (has_data && c <= c_last) {
-            a[i] = src_of(c)[0];
-            b[i] = src_of(c)[1];
-            da[i] = d_of(c)[0];
-            db[i] = d_of(c)[1];
+    float dm = -INFINITY, am = 0.f;
+    for (int i = threadIdx.x; i < nstat; i += kImageThreads) {
+        if ((i & 7) < 4 * halves) {
+            const size_t k = (size_t)(c_first + (i >> 3) + bh) * 8 + (i & 7);
+            dm = fmaxf(dm, p.part_Dmax[k]);
         }
     }
-
-    // C: the largest per-run statistic D over the head
-    float dm = st_d;
-    for (int i = threadIdx.x + kImageThreads; i < nstat; i += kImageThreads)
-        if ((i & 7) < 4 * halves) dm = fmaxf(dm, p.part_Dmax[(size_t)(c_first + (i >> 3) + bh) * 8 + (i & 7)]);
     for (int o = 16; o > 0; o >>= 1) dm = fmaxf(dm, __shfl_xor_sync(0xffffffffu, dm, o));
     if (lane == 0) sRed[wid] = dm;
     __syncthreads();
@@ -128,24 +94,24 @@ __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
     }
     __syncthreads();
     const float C = sC;
-    // the bound: per run the max over its warps' amax 2^(Dmax - C), summed over runs; every run's
-    // warps are taken by consecutive threads (8 per run)
-    float am = st_mine ? st_a * pow2i(st_d - C) : 0.f;
-    for (int i = threadIdx.x + kImageThreads; i < nstat; i += kImageThreads)
+    for (int i = threadIdx.x; i < nstat; i += kImageThreads)
         if ((i & 7) < 4 * halves) {
             const size_t k = (size_t)(c_first + (i >> 3) + bh) * 8 + (i & 7);
-            am = fmaxf(am, p.part_amax[k] * pow2i(p.part_Dmax[k] - C));
+            am = fmaxf(am, p.part_amax[k] * pow2i(p.part_Dmax[k] - C));  // per run the max over warps...
         }
+    // ... summed over runs: every run's warps are taken by consecutive threads (8 per run), so the
+    // bound is the sum over runs of the max over that run's 8 threads' values
     for (int o = 4; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
     float bsum = (threadIdx.x & 7) == 0 ? am : 0.f;
     for (int o = 16; o > 0; o >>= 1) bsum += __shfl_xor_sync(0xffffffffu, bsum, o);
+    __syncthreads();
     if (lane == 0) sRed[wid] = bsum;
     __syncthreads();
     if (threadIdx.x == 0) {
         float bound = 0.f;
         for (int w = 0; w < kImageThreads / 32; ++w) bound += sRed[w];
         // runs beyond the first kImageThreads / 8 (very short heads over many CTAs) were folded by
-        // the strided loops into those threads' maxima: adding them per run keeps the bound valid
+        // the strided loop into those threads' maxima: adding them per run keeps the bound valid
         if (nstat > kImageThreads) bound *= (float)((nstat + kImageThreads - 1) / kImageThreads);
         int ex = 0;
         frexpf(bound, &ex);  // bound < 2^ex
@@ -153,24 +119,30 @@ __global__ void __launch_bounds__(kImageThreads) k_state_image(ImageParams p) {
     }
     __syncthreads();
     const float scale = sScale;
-    if (!active) return;
 
+    const int chunks = nhs * halves * 2 * kImgRows * 8;
+    const int q = blockIdx.x * kImageThreads + threadIdx.x;
+    if (q >= chunks) return;
+    const int pch = q & 7, row = (q >> 3) % kImgRows, blk = (q >> 3) / kImgRows;  // blk = (nh*H + h)*2 + kb
+    const int kb = blk & 1, h = (blk >> 1) % halves, nh = (blk >> 1) / halves;
     float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    auto add = [&](const float4 &x, const float4 &y, const float4 &dx, const float4 &dy) {
-        v[0] = fmaf(x.x, pow2i(dx.x - C), v[0]);
-        v[1] = fmaf(x.y, pow2i(dx.y - C), v[1]);
-        v[2] = fmaf(x.z, pow2i(dx.z - C), v[2]);
-        v[3] = fmaf(x.w, pow2i(dx.w - C), v[3]);
-        v[4] = fmaf(y.x, pow2i(dy.x - C), v[4]);
-        v[5] = fmaf(y.y, pow2i(dy.y - C), v[5]);
-        v[6] = fmaf(y.z, pow2i(dy.z - C), v[6]);
-        v[7] = fmaf(y.w, pow2i(dy.w - C), v[7]);
-    };
-    if (has_data) {
-#pragma unroll
-        for (int i = 0; i < kImageRunsAhead; ++i)
-            if (c_first + i <= c_last) add(a[i], b[i], da[i], db[i]);
-        for (int c = c_first + kImageRunsAhead; c <= c_last; ++c) add(src_of(c)[0], src_of(c)[1], d_of(c)[0], d_of(c)[1]);
+    if (row <= 64) {
+        const int col = row < 64 ? nh * 64 + row : p.d;
+        const int r0 = h * 128 + kb * 64 + 8 * (pch ^ (row & 7));
+        for (int c = c_first; c <= c_last; ++c) {
+            const size_t slot = (size_t)(c + bh);
+            const float4 *src = (const float4 *)(p.part + (slot * (p.d + 1) + col) * p.m + r0);
+            const float4 *dd = (const float4 *)(p.part_D + slot * p.m + r0);
+            const float4 a = src[0], b = src[1], da = dd[0], db = dd[1];
+            v[0] = fmaf(a.x, pow2i(da.x - C), v[0]);
+            v[1] = fmaf(a.y, pow2i(da.y - C), v[1]);
+            v[2] = fmaf(a.z, pow2i(da.z - C), v[2]);
+            v[3] = fmaf(a.w, pow2i(da.w - C), v[3]);
+            v[4] = fmaf(b.x, pow2i(db.x - C), v[4]);
+            v[5] = fmaf(b.y, pow2i(db.y - C), v[5]);
+            v[6] = fmaf(b.z, pow2i(db.z - C), v[6]);
+            v[7] = fmaf(b.w, pow2i(db.w - C), v[7]);
+        }
     }
     uint4 u;
     u.x = pack_f16x2(v[0] * scale, v[1] * scale);
