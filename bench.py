@@ -689,7 +689,8 @@ def main():
     ap.add_argument("--workload", type=int, default=2, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--exp-poly-pct", type=int, default=0,
-                    help="percent of feature exponentials on the FMA-pipe polynomial (0: library default)")
+                    help="percent of feature exponentials on the FMA-pipe polynomial (0: each kernel's "
+                         "library default; negative: all on MUFU)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle sample after the timed region (for profiler runs)")
     ap.add_argument("--headline-only", action="store_true",

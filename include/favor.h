@@ -75,9 +75,10 @@ typedef struct {
  *   split_tiles : 128-token tiles per causal segment (the unit of the causal key-side reduction
  *                 and of the chunked scan; default 8); the bidirectional path spreads its key
  *                 tiles over the SMs by itself
- *   exp_poly_pct: percent (0..100) of feature exponentials evaluated by the FMA-pipe
- *                 polynomial instead of the MUFU ex2 unit (bf16 path); 0 (the default) puts
- *                 all of them on MUFU
+ *   exp_poly_pct: percent (1..100) of feature exponentials evaluated by the FMA-pipe
+ *                 polynomial instead of the MUFU ex2 unit (bf16 path), in every kernel; a
+ *                 negative value puts all of them on MUFU; 0 takes each kernel's default (a
+ *                 quarter in the d = 64 query output kernel, none elsewhere)
  *   feature_map : the random-feature map (bf16 bidirectional forward only; other calls refuse a
  *                 non-default map with FAVOR_ERR_UNSUPPORTED):
  *                 FAVOR_MAP_POSITIVE (0, default): phi(x) = exp(Wx - |x|^2/2)/sqrt(m), FAVOR+;

@@ -51,12 +51,17 @@ favor_status shape_supported(const favor_shape *s, int causal, int backward) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Share of feature exponentials on the FMA-pipe polynomial (percent); 0 takes the default, all on
-// MUFU (measured fastest on B200 for every kernel: the kernels are latency-bound, not MUFU-bound).
-int opt_poly_pct(const favor_opts *o) {
+// Share of feature exponentials on the FMA-pipe polynomial (percent) for a kernel whose default is
+// dflt: 0 (or no opts) takes that default, 1..100 is used as given, a negative value puts every
+// exponential on MUFU. Defaults measured on B200 (bidirectional d = 64, L = 4096): the query output
+// kernel runs 1 us faster (of 40) with a quarter on the polynomial, the key kernel is best with none
+// (and both lose from 37 % on); the other kernels keep everything on MUFU.
+int opt_poly_pct(const favor_opts *o, int dflt) {
     const int v = o ? o->exp_poly_pct : 0;
+    if (v == 0) return dflt;
     return v > 0 ? std::min(v, 100) : 0;
 }
+constexpr int kQueryPolyPct = 25;  // k_query_out, d = 64
 
 int opt_feature_map(const favor_opts *o) { return o ? o->feature_map : FAVOR_MAP_POSITIVE; }
 
@@ -469,8 +474,8 @@ favor_status fwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, 
 
     KeyStateParams2 ks{s->L, s->m, l.f, part, partD, amax, Dmax};
     record_stage(o, 0, st);
-    cudaError_t e = s->d == 64 ? launch_key_partials_wide(mK64, mV64, mW, ks, opt_poly_pct(o), st)
-                               : launch_key_partials(mK64, mV64, mW, ks, s->d, opt_poly_pct(o), st);
+    cudaError_t e = s->d == 64 ? launch_key_partials_wide(mK64, mV64, mW, ks, opt_poly_pct(o, 0), st)
+                               : launch_key_partials(mK64, mV64, mW, ks, s->d, opt_poly_pct(o, 0), st);
     record_stage(o, 1, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     ImageParams ip{s->m, s->d, l.f, part, partD, amax, Dmax, state, stride, kref};
@@ -480,7 +485,7 @@ favor_status fwd_bf16_bidir(const favor_shape *s, const void *Q, const void *K, 
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     QueryParams qp{s->L, s->d, s->m, l.BH, 0, state, stride};
     record_stage(o, 4, st);
-    e = launch_query_out(mQ, mW, mO, qp, opt_poly_pct(o), st);
+    e = launch_query_out(mQ, mW, mO, qp, opt_poly_pct(o, s->d == 64 ? kQueryPolyPct : 0), st);
     record_stage(o, 5, st);
     return e == cudaSuccess ? FAVOR_OK : FAVOR_ERR_CUDA;
 }
@@ -596,7 +601,7 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     uint32_t *seg_vmax = (uint32_t *)(ws + l.off_seg_vmax);
     const WideSegParams sgp{l.n_split, l.tiles_per_split, l.n_seg, segs_per_cta, bias, seg_vmax};
     record_stage(o, 0, st);
-    cudaError_t e = launch_key_segments(mK128, mV128, mW, ks, sgp, opt_poly_pct(o), st);
+    cudaError_t e = launch_key_segments(mK128, mV128, mW, ks, sgp, opt_poly_pct(o, 0), st);
     record_stage(o, 1, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     SegScanParams sp{s->m, l.n_split, s->m / 128, part, (float *)(ws + l.off_part_D), (float *)(ws + l.off_part_umax),
@@ -608,7 +613,7 @@ favor_status fwd_bf16(const favor_shape *s, const void *Q, const void *K, const 
     ChunkParams cp{s->L, s->m, l.n_split, l.tiles_per_split, l.P_exact, l.BH * l.n_split, bias, head_max,
                    seg_S, seg_z, seg_vmax, out};
     record_stage(o, 4, st);
-    e = launch_causal_chunk(mQ, mK, mV, mW128, cp, opt_poly_pct(o), st);
+    e = launch_causal_chunk(mQ, mK, mV, mW128, cp, opt_poly_pct(o, 0), st);
     record_stage(o, 5, st);
     if (e != cudaSuccess) return FAVOR_ERR_CUDA;
     return causal_prefix(s, l, Q, K, V, W, kref, out, ws, o, st);

@@ -334,12 +334,13 @@ def test_bf16_causal_values_beyond_fp16_range(cuda_device):
         assert api.sync_status() == api.FAVOR_OK  # the status word is cleared by the read
 
 
-@pytest.mark.parametrize("poly_pct", [25, 50, 100])
+@pytest.mark.parametrize("poly_pct", [25, 50, 100, -1])
 @pytest.mark.parametrize("causal,d", [(False, 64), (False, 128), (True, 64)])
 def test_bf16_exponentials_on_the_fma_polynomial(cuda_device, poly_pct, causal, d):
     """favor_opts.exp_poly_pct moves a share of the feature exponentials from MUFU ex2 to the
-    FMA-pipe polynomial (every kernel instantiates each share); outputs stay within tolerance."""
-    w = Workload("t", 1, 2, 1100, d, 256, causal, "bf16", False, 3 if causal else 2, 90 + poly_pct)
+    FMA-pipe polynomial (every kernel instantiates each share; -1 puts all of them on MUFU, 0 --
+    the other tests -- takes the kernels' defaults); outputs stay within tolerance."""
+    w = Workload("t", 1, 2, 1100, d, 256, causal, "bf16", False, 3 if causal else 2, 90 + abs(poly_pct))
     x = make_inputs(w)
     Wr, W64 = features_for(w.w_seed, w.m, w.d, "bf16")
     out = run_fwd(w, x, Wr, cuda_device, causal, opts=api.make_opts(exp_poly_pct=poly_pct))
